@@ -1,0 +1,278 @@
+/*
+ * CPU ORACLE of the Mixtral-style sparse mixture-of-experts feed-forward layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke check
+ * and the benchmark's CPU-baseline leg may load or run this code.  It shares
+ * no code, header, table or helper with the GPU path, and the GPU path never
+ * calls it.
+ *
+ * Every step is the plain definition, computed in double precision from the
+ * same bf16 / fp32 input bytes the GPU consumes, in the order the pages state
+ * it; nothing is blocked, fused or reordered.  Sources (web pages, by title):
+ *
+ *  [P1] "How Mixtral 8x7B uses mixture of experts" (n4n.ai)
+ *       - "The architecture in one diagram": router logits -> softmax -> top-2
+ *         -> renormalise; outputs weighted and summed.
+ *       - "Routing without auxiliary loss": capacity factor; excess tokens are
+ *         dropped; "sort tokens by router probability for each expert, keep ...
+ *         up to capacity".
+ *  [P2] "Mixtral and Mixture-of-Experts, Explained" (automatone.win)
+ *       - "How it works": G(x) = Softmax(TopK(x . W_g)), logits outside the
+ *         top-k set to -inf; y = sum_i G(x)_i . Expert_i(x).
+ *  [P3] "Mixtral" (vanos001.github.io)
+ *       - "MoE Layer": MixtralMoE.forward (top-k of logits, softmax over the
+ *         k kept logits) and MixtralExpert.forward: w2(silu(w1 x) * w3 x),
+ *         all nn.Linear without bias.
+ *       - "SwiGLU Experts": SwiGLU(x) = SiLU(x W1) (.) (x W3), output @ W2.
+ *       - "MixtralBlock": the MoE output is added to the residual stream.
+ *  [P4] "Mixtral 8x7B" (interview.clozo.ai)
+ *       - "Step 2: A router picks 2 experts and mixes their outputs": the
+ *         worked example (scores 2.1 0.3 1.4 -0.5 0.0 0.9 -1.2 0.2 -> weights
+ *         0.6682 / 0.3318).
+ *
+ * Readings taken where the pages are silent or disagree (each is also tested):
+ *  - Gate: [P1] (softmax over all E, top-k, renormalise), [P2] (-inf mask then
+ *    softmax) and [P3] (softmax of the k largest logits) are the same function
+ *    except under exact ties; this file computes the [P3] form.
+ *  - Top-k order and ties: slot j = 0 holds the largest logit; equal logits
+ *    are ordered by the smaller expert index.
+ *  - Experts are numbered from 0 ([P4]'s "expert 1 and 3" are indices 0, 2).
+ *  - SiLU(a) = a * sigmoid(a) = a / (1 + exp(-a)).
+ *  - Capacity per expert = floor(cf * T * k / E) (the pages' cf * T / E per
+ *    slot of top-k); cf <= 0 means no capacity limit (dropless).
+ *  - Which slots overflow: policy 0 keeps, per expert, the `cap` slots with
+ *    the largest full-softmax router probability ([P1] "sort tokens by router
+ *    probability"), ties to the smaller token index; policy 1 keeps the first
+ *    `cap` slots in token order.
+ *  - A dropped slot contributes zero (the token passes on the residual path,
+ *    [P3] MixtralBlock); the remaining gate weights are not renormalised.
+ *
+ * Layouts (row-major): x [T, d] bf16 bits; Wg [E, d] fp32 (logit = x . Wg[e]);
+ * W1, W3 [E, f, d] bf16 bits; W2 [E, d, f] bf16 bits.  Slot s = t * k + j.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* Router logits [P2] "How it works" (x . W_g) with [P3] "MoE Layer" storage
+ * (nn.Linear(d_model, num_experts, bias=False) keeps W as [E, d]):
+ * logits[t, e] = sum_i x[t, i] * Wg[e, i], summed in index order. */
+void oracle_router_logits(int64_t T, int32_t d, int32_t E, const uint16_t *x, const float *Wg,
+                          double *logits) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    for (int32_t e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int32_t i = 0; i < d; ++i)
+        acc += bf16_to_double(x[t * d + i]) * (double)Wg[(int64_t)e * d + i];
+      logits[t * E + e] = acc;
+    }
+  }
+}
+
+/* Top-k [P3] "MoE Layer" (router_logits.topk(top_k)): the k experts with the
+ * largest logits, slot j = 0 the largest; equal logits -> smaller index first.
+ * Plain selection: k passes, each taking the best expert not yet chosen. */
+void oracle_topk(int64_t T, int32_t E, int32_t k, const double *logits, int32_t *idx) {
+  for (int64_t t = 0; t < T; ++t) {
+    const double *l = logits + t * E;
+    for (int32_t j = 0; j < k; ++j) {
+      int32_t best = -1;
+      for (int32_t e = 0; e < E; ++e) {
+        int taken = 0;
+        for (int32_t q = 0; q < j; ++q) taken |= (idx[t * k + q] == e);
+        if (taken) continue;
+        if (best < 0 || l[e] > l[best]) best = e; /* strict: ties keep smaller e */
+      }
+      idx[t * k + j] = best;
+    }
+  }
+}
+
+/* Gate weights [P3] "MoE Layer": softmax over the k kept logits,
+ *   w_j = exp(l_j - m) / sum_{q<k} exp(l_q - m),  m = l_{idx_0}.
+ * Router probability [P1] "The architecture in one diagram" (softmax over all
+ * E logits) of each chosen expert, used as the capacity priority:
+ *   p_j = exp(l_j - M) / sum_{e<E} exp(l_e - M),  M = max_e l_e. */
+void oracle_gates(int64_t T, int32_t E, int32_t k, const double *logits, const int32_t *idx,
+                  double *w, double *p) {
+  for (int64_t t = 0; t < T; ++t) {
+    const double *l = logits + t * E;
+    double m = l[idx[t * k]];
+    double zk = 0.0;
+    for (int32_t q = 0; q < k; ++q) zk += exp(l[idx[t * k + q]] - m);
+    double M = l[0];
+    for (int32_t e = 1; e < E; ++e)
+      if (l[e] > M) M = l[e];
+    double zE = 0.0;
+    for (int32_t e = 0; e < E; ++e) zE += exp(l[e] - M);
+    for (int32_t j = 0; j < k; ++j) {
+      w[t * k + j] = exp(l[idx[t * k + j]] - m) / zk;
+      p[t * k + j] = exp(l[idx[t * k + j]] - M) / zE;
+    }
+  }
+}
+
+typedef struct {
+  double p;
+  int64_t t;
+  int64_t s;
+} prio_t;
+
+/* (p descending, then t ascending) */
+static int prio_cmp(const void *a, const void *b) {
+  const prio_t *x = (const prio_t *)a, *y = (const prio_t *)b;
+  if (x->p > y->p) return -1;
+  if (x->p < y->p) return 1;
+  return (x->t < y->t) ? -1 : (x->t > y->t);
+}
+
+/* Capacity [P1] "Routing without auxiliary loss": each expert takes at most
+ * cap = floor(cf * T * k / E) slots; the excess is dropped.  policy 0 keeps
+ * the cap slots of highest router probability p (ties: smaller token first),
+ * policy 1 keeps the first cap slots in token order.  cf <= 0: keep all.
+ * kept[s] = 1 / 0.  Returns cap, or -1 when dropless. */
+int64_t oracle_capacity(int64_t T, int32_t E, int32_t k, double cf, int32_t policy,
+                        const int32_t *idx, const double *p, uint8_t *kept) {
+  int64_t S = T * k;
+  if (cf <= 0.0) {
+    for (int64_t s = 0; s < S; ++s) kept[s] = 1;
+    return -1;
+  }
+  int64_t cap = (int64_t)floor(cf * (double)T * (double)k / (double)E);
+  prio_t *list = (prio_t *)malloc(sizeof(prio_t) * (size_t)(S > 0 ? S : 1));
+  for (int64_t s = 0; s < S; ++s) kept[s] = 0;
+  for (int32_t e = 0; e < E; ++e) {
+    int64_t n = 0;
+    for (int64_t s = 0; s < S; ++s)
+      if (idx[s] == e) {
+        list[n].p = p[s];
+        list[n].t = s / k;
+        list[n].s = s;
+        ++n;
+      }
+    if (policy == 0) qsort(list, (size_t)n, sizeof(prio_t), prio_cmp);
+    /* policy 1: list is already in token order */
+    for (int64_t r = 0; r < n && r < cap; ++r) kept[list[r].s] = 1;
+  }
+  free(list);
+  return cap;
+}
+
+/* Grouping of slots by expert [P1] "The architecture in one diagram" (batch
+ * tokens by expert, run the experts, scatter back): for e = 0..E-1, the kept
+ * slots routed to e in ascending token order form rows offsets[e] ..
+ * offsets[e+1]-1 of the grouped layout.  counts[e] = routed slots (the
+ * per-expert histogram), kept_counts[e] = kept slots, perm_slot[row] = slot,
+ * slot_pos[slot] = row or -1 when dropped. */
+void oracle_permute(int64_t T, int32_t E, int32_t k, const int32_t *idx, const uint8_t *kept,
+                    int32_t *counts, int32_t *kept_counts, int32_t *offsets, int32_t *perm_slot,
+                    int32_t *slot_pos) {
+  int64_t S = T * k;
+  int64_t row = 0;
+  offsets[0] = 0;
+  for (int32_t e = 0; e < E; ++e) {
+    counts[e] = 0;
+    kept_counts[e] = 0;
+    for (int64_t s = 0; s < S; ++s) {
+      if (idx[s] != e) continue;
+      counts[e] += 1;
+      if (kept[s]) {
+        kept_counts[e] += 1;
+        perm_slot[row] = (int32_t)s;
+        slot_pos[s] = (int32_t)row;
+        ++row;
+      } else {
+        slot_pos[s] = -1;
+      }
+    }
+    offsets[e + 1] = (int32_t)row;
+  }
+}
+
+/* One expert on one token [P3] "MoE Layer" (MixtralExpert.forward) and
+ * "SwiGLU Experts":  a = W1 x,  b = W3 x,  h = SiLU(a) * b,  o = W2 h,
+ * SiLU(a) = a / (1 + exp(-a)).  W1e, W3e [f, d]; W2e [d, f].  h [f], o [d]. */
+void oracle_expert_row(int32_t d, int32_t f, const uint16_t *xrow, const uint16_t *W1e,
+                       const uint16_t *W3e, const uint16_t *W2e, double *h, double *o) {
+  for (int32_t n = 0; n < f; ++n) {
+    double a = 0.0, b = 0.0;
+    for (int32_t i = 0; i < d; ++i) {
+      double xi = bf16_to_double(xrow[i]);
+      a += bf16_to_double(W1e[(int64_t)n * d + i]) * xi;
+      b += bf16_to_double(W3e[(int64_t)n * d + i]) * xi;
+    }
+    h[n] = a / (1.0 + exp(-a)) * b;
+  }
+  for (int32_t c = 0; c < d; ++c) {
+    double acc = 0.0;
+    for (int32_t n = 0; n < f; ++n) acc += bf16_to_double(W2e[(int64_t)c * f + n]) * h[n];
+    o[c] = acc;
+  }
+}
+
+/* Layer output [P2] "How it works": y = sum_i G(x)_i * Expert_i(x), G zero off
+ * the top-k; with capacity, a dropped slot adds nothing.  Computed for the
+ * tokens listed in rows[0..n_rows): y[r, :] for token rows[r].
+ * Optional outputs (may be NULL): h_out [n_rows, k, f] and o_out
+ * [n_rows, k, d], the expert hidden state and output of each slot (zeros for
+ * a dropped slot). */
+void oracle_layer_rows(int64_t T, int32_t d, int32_t f, int32_t E, int32_t k, const uint16_t *x,
+                       const uint16_t *W1, const uint16_t *W3, const uint16_t *W2,
+                       const int32_t *idx, const double *w, const uint8_t *kept, int64_t n_rows,
+                       const int64_t *rows, double *y, double *h_out, double *o_out) {
+  (void)T;
+  (void)E;
+#pragma omp parallel
+  {
+    double *h = (double *)malloc(sizeof(double) * (size_t)f);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t t = rows[r];
+      double *yr = y + r * d;
+      for (int32_t c = 0; c < d; ++c) yr[c] = 0.0;
+      for (int32_t j = 0; j < k; ++j) {
+        int64_t s = t * k + j;
+        double *hs = h_out ? h_out + (r * k + j) * (int64_t)f : NULL;
+        double *os = o_out ? o_out + (r * k + j) * (int64_t)d : NULL;
+        if (!kept[s]) {
+          if (hs) memset(hs, 0, sizeof(double) * (size_t)f);
+          if (os) memset(os, 0, sizeof(double) * (size_t)d);
+          continue;
+        }
+        int64_t e = idx[s];
+        oracle_expert_row(d, f, x + t * d, W1 + e * f * d, W3 + e * f * d, W2 + e * d * f, h, o);
+        for (int32_t c = 0; c < d; ++c) yr[c] += w[s] * o[c];
+        if (hs) memcpy(hs, h, sizeof(double) * (size_t)f);
+        if (os) memcpy(os, o, sizeof(double) * (size_t)d);
+      }
+    }
+    free(h);
+    free(o);
+  }
+}
+
+/* Number of OpenMP threads the oracle runs with (reported with its timing). */
+int oracle_num_threads(void) {
+  int n = 1;
+#pragma omp parallel
+  {
+#pragma omp single
+    {
+#ifdef _OPENMP
+      extern int omp_get_num_threads(void);
+      n = omp_get_num_threads();
+#endif
+    }
+  }
+  return n;
+}

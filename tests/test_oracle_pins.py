@@ -1,0 +1,122 @@
+"""The CPU oracle against its pins, and the pins against planted mistakes.
+
+The second half compiles copies of the oracle source with one plausible
+mistake each (a dropped term, a wrong sign, a swapped operand, a wrong index
+or tie rule) and checks that at least one pin fails on every such copy.
+"""
+import os
+import shutil
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+import pins
+import synth
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.Oracle()
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_pin(o, pin):
+    pin(o)
+
+
+# (description, text in moe_oracle.c, replacement) -- each is a mistake that
+# a restatement of the layer could plausibly contain.
+MUTANTS = [
+    ("silu sign", "h[n] = a / (1.0 + exp(-a)) * b;", "h[n] = a / (1.0 + exp(a)) * b;"),
+    ("silu dropped", "h[n] = a / (1.0 + exp(-a)) * b;", "h[n] = a * b;"),
+    ("W1/W3 swapped in gate", "h[n] = a / (1.0 + exp(-a)) * b;", "h[n] = b / (1.0 + exp(-b)) * a;"),
+    ("W2 transposed", "acc += bf16_to_double(W2e[(int64_t)c * f + n]) * h[n];",
+     "acc += bf16_to_double(W2e[(int64_t)n * d + c]) * h[n];"),
+    ("topk ties to larger index", "if (best < 0 || l[e] > l[best]) best = e;",
+     "if (best < 0 || l[e] >= l[best]) best = e;"),
+    ("gate max not subtracted consistently", "w[t * k + j] = exp(l[idx[t * k + j]] - m) / zk;",
+     "w[t * k + j] = exp(l[idx[t * k + j]]) / zk;"),
+    ("gate over all experts (no renormalise)", "w[t * k + j] = exp(l[idx[t * k + j]] - m) / zk;",
+     "w[t * k + j] = exp(l[idx[t * k + j]] - M) / zE;"),
+    ("capacity without k", "cap = (int64_t)floor(cf * (double)T * (double)k / (double)E);",
+     "cap = (int64_t)floor(cf * (double)T / (double)E);"),
+    ("capacity ties to larger token", "return (x->t < y->t) ? -1 : (x->t > y->t);",
+     "return (x->t > y->t) ? -1 : (x->t < y->t);"),
+    ("capacity keeps lowest prob", "if (x->p > y->p) return -1;\n  if (x->p < y->p) return 1;",
+     "if (x->p < y->p) return -1;\n  if (x->p > y->p) return 1;"),
+    ("router skips last feature", "for (int32_t i = 0; i < d; ++i)\n        acc += bf16_to_double(x[t * d + i])",
+     "for (int32_t i = 0; i < d - 1; ++i)\n        acc += bf16_to_double(x[t * d + i])"),
+    ("combine ignores gate", "yr[c] += w[s] * o[c];", "yr[c] += o[c];"),
+    ("dropped slot still added", "if (!kept[s]) {", "if (0) {"),
+    ("grouping in reverse token order", "for (int64_t s = 0; s < S; ++s) {\n      if (idx[s] != e) continue;",
+     "for (int64_t s = S - 1; s >= 0; --s) {\n      if (idx[s] != e) continue;"),
+]
+
+
+@pytest.mark.parametrize("desc,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(desc, old, new):
+    src = open(oracle._SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found once: {desc}"
+    tmpdir = tempfile.mkdtemp(prefix="oracle_mutant_")
+    try:
+        msrc = os.path.join(tmpdir, "mutant.c")
+        with open(msrc, "w") as fh:
+            fh.write(src.replace(old, new))
+        lib = oracle._bind(oracle.build(force=True, src=msrc, out=os.path.join(tmpdir, "libm.so")))
+        m = oracle.Oracle(lib)
+        caught = []
+        for pin in pins.ALL_PINS:
+            try:
+                pin(m)
+            except AssertionError:
+                caught.append(pin.__name__)
+            except Exception as exc:  # a crash also counts as caught
+                caught.append(f"{pin.__name__}:{type(exc).__name__}")
+        assert caught, f"no pin caught the planted mistake: {desc}"
+    finally:
+        shutil.rmtree(tmpdir, ignore_errors=True)
+
+
+def test_generator_definition():
+    """The input generator follows its stated definition: splitmix64 words,
+    Box-Muller, round-to-nearest-even bf16; moments of a large draw."""
+    G = 0x9E3779B97F4A7C15
+    M = (1 << 64) - 1
+
+    def mix(z):
+        z ^= z >> 30
+        z = (z * 0xBF58476D1CE4E5B9) & M
+        z ^= z >> 27
+        z = (z * 0x94D049BB133111EB) & M
+        return z ^ (z >> 31)
+
+    seed, tid = 3, 4
+    base = mix(mix((seed + G) & M) ^ ((tid * 0xD1B54A32D192ED03) & M))
+    want = [mix((base + (n + 1) * G) & M) for n in range(6)]
+    assert synth.words(seed, tid, 6).tolist() == want
+    import math
+    u1 = ((want[0] >> 11) + 1) * 2.0 ** -53
+    u2 = (want[1] >> 11) * 2.0 ** -53
+    z0 = math.sqrt(-2 * math.log(u1)) * math.cos(2 * math.pi * u2)
+    v = synth.normal_f32(seed, tid, 1)
+    assert abs(float(v[0]) - z0) <= 1e-6 * max(1.0, abs(z0))
+    b = synth.normal_bf16(seed, tid, 1)
+    assert abs(float(synth.bf16_to_f32(b)[0]) - z0) <= abs(z0) * 2.0 ** -8
+    big = synth.normal_f32(0, 9, 1 << 20).astype(np.float64)
+    assert abs(big.mean()) < 5e-3 and abs(big.std() - 1.0) < 5e-3
+    # bf16 rounding is nearest-even
+    assert synth.f32_to_bf16(np.array([1.0 + 2 ** -8], np.float32))[0] == 0x3F80
+    assert synth.f32_to_bf16(np.array([1.0 + 3 * 2 ** -8], np.float32))[0] == 0x3F82
+
+
+def test_skew_recipe_share():
+    """The skewed workload's constant feature and router bias send close to
+    40 % of top-2 slots to expert 0 (sampled on 2048 tokens)."""
+    wl = synth.workload("skew", T=2048)
+    wl.generate(weights=False)
+    o = oracle.Oracle()
+    idx = o.topk(o.router_logits(wl.x, wl.Wg), 2)
+    share = float((idx == 0).sum()) / idx.size
+    assert 0.37 < share < 0.43, share
