@@ -1,0 +1,396 @@
+"""Benchmark of the sparse MoE layer on B200: one JSON line on rank 0.
+
+A step is one whole forward of the layer (router, top-2 gate, grouping by
+expert, grouped SwiGLU expert GEMMs, combine) over one batch of synthetic
+Mixtral-shaped input (d_model 4096, d_ff 14336, 8 experts, top-2, seed 0
+weights; every rank draws its own tokens).  The headline workload is prefill,
+T = 4096 tokens, on the tensor-core roofline; the decode workload, T = 16, is
+reported beside it on the HBM roofline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU runs (torchrun, one rank per GPU) shard the tokens: each rank runs
+the same layer on its own batch with no data-path collective (weak scaling);
+the step time is the max over ranks.  ``--impl reference`` times the CPU
+oracle on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; % bf16 TC peak (T=4096) and % HBM BW (T=16)"
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            pk = json.load(fh)
+        return dict(hbm=float(pk["hbm_gbs"]), bf16=float(pk["bf16_tflops"]),
+                    bf16_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=FALLBACK_BF16_TFLOPS,
+                    source="fallback")
+
+
+def traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, only while the
+    kernel's source is unchanged since the capture (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as fh:
+            recs = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    src = os.path.join(ROOT, "sparse_mixture_experts_13_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(src, name), "rb") as fh:
+                h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    for r in recs:
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is busy."""
+    QUERY = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, pci_bus_id: str | None):
+        self.pci = (pci_bus_id or "").lower()
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
+        self.proc.terminate()
+        self.proc.wait()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [list(map(str.strip, ln.split(","))) for ln in self.file.read().splitlines() if ln.strip()]
+        os.unlink(self.file.name)
+        bus = {r[1].lower() for r in rows}
+        if len(bus) > 1 and self.pci:
+            rows = [r for r in rows if r[1].lower().endswith(self.pci[-12:])]
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        power = [float(r[4]) for r in rows if r[4].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v.strip().lower() == "active"})
+        return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(mx) if mx else None,
+                    power_w_max=max(power) if power else None, reasons=reasons, samples=len(sm))
+
+
+# ---------------------------------------------------------------- helpers
+
+def to_dev_bf16(a, torch):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def time_steps(fn, steps, torch, dist=None):
+    """K steps between a barrier + synchronize on both sides; CUDA events on
+    the current stream; max over ranks."""
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        fn()
+    end.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+class Run:
+    """One workload on this rank's GPU."""
+
+    def __init__(self, wl, weights_dev, torch, moe):
+        self.wl, self.torch, self.moe = wl, torch, moe
+        Wg, W1, W3, W2 = weights_dev
+        self.layer = moe.MoELayer(torch.from_numpy(wl.Wg).cuda() if Wg is None else Wg, W1, W3, W2, k=wl.k,
+                                  capacity_factor=wl.capacity_factor, drop_policy=wl.drop_policy)
+        self.x = to_dev_bf16(wl.x, torch)
+        self.y = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+        self.counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+
+    def step(self):
+        self.layer.forward(self.x, self.y)
+
+    def kept_and_touched(self):
+        self.layer.forward(self.x, self.y, counts=self.counts)
+        c = self.counts.cpu().numpy()
+        cap = self.wl.capacity
+        kept = np.minimum(c, cap) if cap is not None else c
+        return int(kept.sum()), int((kept > 0).sum())
+
+    def profiled(self, steps):
+        """Average duration (ms) of each stage over `steps` instrumented forwards."""
+        torch, moe = self.torch, self.moe
+        sums = np.zeros(5)
+        sh = self.layer.shape(self.wl.T)
+        ws = self.layer.workspace(self.wl.T)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            st = moe.moe_layer_forward_profiled(sh, self.x, self.layer.Wg, self.layer.W1, self.layer.W3,
+                                                self.layer.W2, self.y, evs[i], ws, ws.numel())
+            moe.check(st, "moe_layer_forward_profiled")
+        torch.cuda.synchronize()
+        for i in range(steps):
+            sums += [evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
+        return dict(zip(["router", "capacity_and_permute", "gemm1_swiglu", "gemm2", "combine"],
+                        (sums / steps).tolist()))
+
+    def e2e(self, steps, dist):
+        """Tokens/s through moe_layer_forward_host: pinned host x in, y out."""
+        torch = self.torch
+        xh = torch.from_numpy(np.ascontiguousarray(self.wl.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+        yh = torch.empty(self.wl.T, self.wl.d, dtype=torch.bfloat16).pin_memory()
+        for _ in range(2):
+            self.layer.forward_host(xh, yh)
+        ms = time_steps(lambda: self.layer.forward_host(xh, yh), steps, torch, dist)
+        nbytes = self.wl.T * self.wl.d * 2
+        return ms, nbytes, nbytes
+
+
+def expert_bytes(d, f):
+    return 3 * d * f * 2
+
+
+def cpu_baseline(wl, n_sample=48):
+    """The oracle on the host cores: routing of every token plus the expert
+    FFN of a seeded sample of tokens; tokens/s scaled to the whole batch."""
+    import oracle
+    o = oracle.Oracle()
+    t0 = time.perf_counter()
+    r = o.route(wl.x, wl.Wg, wl.k, wl.capacity_factor, wl.drop_policy)
+    t_route = time.perf_counter() - t0
+    rows = np.random.default_rng(123).choice(wl.T, size=min(n_sample, wl.T), replace=False)
+    t0 = time.perf_counter()
+    o.layer_rows(wl.x, wl.W1, wl.W3, wl.W2, r, rows)
+    t_ffn = time.perf_counter() - t0
+    n = len(rows)
+    per_token = t_ffn / n + t_route / wl.T
+    return dict(value=1.0 / per_token, unit="tokens/s", cores=o.num_threads(), kind="oracle",
+                sample=f"routing of all {wl.T} tokens ({t_route:.2f} s) + expert FFN of {n} seeded tokens "
+                       f"({t_ffn:.2f} s), fp64, {wl.name}; tokens/s = 1 / (t_ffn/{n} + t_route/{wl.T})")
+
+
+def make_workload(name, rank, T=None):
+    wl = synth.workload(name, T=T)
+    wl.seed = 0
+    wl.generate(weights=False)
+    if rank:
+        # every rank routes its own tokens (same weights)
+        wl.x = synth.normal_bf16(1000 + rank, synth.TID_X, (wl.T, wl.d))
+    return wl
+
+
+def workload_desc(wl):
+    cap = "dropless" if wl.capacity_factor <= 0 else f"capacity factor {wl.capacity_factor}"
+    return f"{wl.name}: T={wl.T} d_model={wl.d} d_ff={wl.f} E={wl.E} top-{wl.k} {cap}"
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args):
+    """The CPU oracle as it stands, on rank 0; other ranks exit 0."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = synth.workload("prefill")
+    wl.generate(weights=True)
+    import oracle
+    o = oracle.Oracle()
+    n_sample = 8
+    rng = np.random.default_rng(7)
+
+    def one_step():
+        """Seconds per token of the oracle on this step's sample."""
+        t0 = time.perf_counter()
+        r = o.route(wl.x, wl.Wg, wl.k, wl.capacity_factor, wl.drop_policy)
+        t_route = time.perf_counter() - t0
+        rows = rng.choice(wl.T, size=n_sample, replace=False)
+        t0 = time.perf_counter()
+        o.layer_rows(wl.x, wl.W1, wl.W3, wl.W2, r, rows)
+        t_ffn = time.perf_counter() - t0
+        return t_ffn / n_sample + t_route / wl.T
+
+    for _ in range(args.warmup):
+        one_step()
+    t_steps = [one_step() for _ in range(args.steps)]
+    per_token = float(np.mean(t_steps))
+    value = 1.0 / per_token
+    sample = (f"per step: routing of all {wl.T} tokens + expert FFN of {n_sample} seeded tokens (fp64 oracle); "
+              f"tokens/s = 1 / (t_ffn/{n_sample} + t_route/{wl.T})")
+    line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=per_token * wl.T * 1e3, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
+                config=dict(workload=workload_desc(wl), T=wl.T, d_model=wl.d, d_ff=wl.f, E=wl.E, k=wl.k,
+                            l2="CPU run"),
+                cpu_baseline=dict(value=value, unit="tokens/s", cores=o.num_threads(), kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    import sparse_mixture_experts_13_b200 as moe
+    moe.lib()  # fails loudly if the CUDA library is missing
+    peaks = load_peaks()
+
+    # shared seed-0 expert weights
+    wl0 = synth.workload("prefill")
+    W1 = synth.normal_bf16(0, synth.TID_W1, (8, wl0.f, wl0.d), 0.0, 1.0 / np.sqrt(wl0.d))
+    W3 = synth.normal_bf16(0, synth.TID_W3, (8, wl0.f, wl0.d), 0.0, 1.0 / np.sqrt(wl0.d))
+    W2 = synth.normal_bf16(0, synth.TID_W2, (8, wl0.d, wl0.f), 0.0, 1.0 / np.sqrt(wl0.f))
+    Wd = (None, to_dev_bf16(W1, torch), to_dev_bf16(W3, torch), to_dev_bf16(W2, torch))
+
+    props = torch.cuda.get_device_properties(local)
+    sampler = ClockSampler(getattr(props, "pci_bus_id", None) if hasattr(props, "pci_bus_id") else None)
+    sampler.start()
+
+    out = {}
+    for name in ("prefill", "decode"):
+        wl = make_workload(name, rank)
+        run = Run(wl, Wd, torch, moe)
+        N, touched = run.kept_and_touched()
+        for _ in range(args.warmup):
+            run.step()
+        ms = time_steps(run.step, args.steps, torch, dist) / args.steps
+        stages = run.profiled(args.steps)
+        e2e_ms, h2d, d2h = run.e2e(args.steps, dist)
+        out[name] = dict(wl=wl, ms=ms, stages=stages, N=N, touched=touched, e2e_ms=e2e_ms / args.steps,
+                         h2d=h2d, d2h=d2h)
+        del run
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+
+    line = None
+    if rank == 0:
+        p = out["prefill"]
+        wl = p["wl"]
+        d, f, E = wl.d, wl.f, wl.E
+        flops_layer = 6.0 * p["N"] * d * f + 2.0 * wl.T * d * E
+        g1_flops = 4.0 * p["N"] * d * f
+        g1_ms = p["stages"]["gemm1_swiglu"]
+        long_run = args.steps * p["ms"] > 1000.0
+        peak_tf = peaks["bf16_sustained"] if long_run else peaks["bf16"]
+        achieved_tf = g1_flops / (g1_ms * 1e-3) / 1e12
+        tr = traffic_record("expert_gemm_kernel<0,256>", "prefill")
+        value = world * wl.T / (p["ms"] * 1e-3)
+
+        q = out["decode"]
+        wq = q["wl"]
+        g1_bytes_dec = q["touched"] * 2 * d * f * 2 + q["N"] * d * 2 + q["N"] * f * 2
+        layer_bytes_dec = q["touched"] * expert_bytes(d, f) + wq.T * d * 2 * 2 + E * d * 4 + 2 * q["N"] * f * 2
+        dec_g1_ms = q["stages"]["gemm1_swiglu"]
+        dec = dict(workload=workload_desc(wq), value=world * wq.T / (q["ms"] * 1e-3), unit="tokens/s",
+                   ms_per_step=q["ms"], stage_ms=q["stages"],
+                   layer_gbs=layer_bytes_dec / (q["ms"] * 1e-3) / 1e9,
+                   layer_frac_hbm=layer_bytes_dec / (q["ms"] * 1e-3) / 1e9 / peaks["hbm"],
+                   roofline=dict(bound="hbm", kernel="gate/up-projection GEMM (SwiGLU fused)",
+                                 achieved=g1_bytes_dec / (dec_g1_ms * 1e-3) / 1e9, peak=peaks["hbm"], unit="GB/s",
+                                 frac=g1_bytes_dec / (dec_g1_ms * 1e-3) / 1e9 / peaks["hbm"],
+                                 traffic=traffic_record("expert_gemm_kernel<2,16>", "decode"),
+                                 peak_source=f"{peaks['source']} HBM copy bandwidth"),
+                   e2e=dict(value=world * wq.T / (q["e2e_ms"] * 1e-3), unit="tokens/s",
+                            h2d_bytes_per_step=q["h2d"], d2h_bytes_per_step=q["d2h"]),
+                   experts_touched=q["touched"])
+        kernels_per_step = 5 + (1 if (wl.capacity_factor > 0 and wl.drop_policy == 0) else 0)
+        line = dict(
+            metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+            ms_per_step=p["ms"], higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+            data="synthetic (seeded counter-based N(0,1) tokens, random-init Mixtral-shaped expert weights)",
+            config=dict(workload=workload_desc(wl), T=wl.T, d_model=d, d_ff=f, E=E, k=wl.k,
+                        parallelism=f"dp{world} (token shards, weights replicated)" if world > 1 else "single GPU",
+                        l2="inputs larger than L2: 2.82 GB of expert weights streamed every step"),
+            tflops=flops_layer / (p["ms"] * 1e-3) / 1e12,
+            frac_layer_of_peak=flops_layer / (p["ms"] * 1e-3) / 1e12 / peak_tf,
+            stage_ms=p["stages"],
+            roofline=dict(bound="tensor", kernel="gate/up-projection GEMM (SwiGLU fused)", achieved=achieved_tf,
+                          peak=peak_tf, unit="TFLOP/s", frac=achieved_tf / peak_tf, traffic=tr,
+                          peak_source=f"{peaks['source']} bf16 dense "
+                                      f"({'sustained' if long_run else 'burst'})"),
+            e2e=dict(value=world * wl.T / (p["e2e_ms"] * 1e-3), unit="tokens/s", h2d_bytes_per_step=p["h2d"],
+                     d2h_bytes_per_step=p["d2h"]),
+            gpu_launches=kernels_per_step * args.steps,
+            clocks=clocks,
+            decode=dec,
+        )
+        if world == 1 and not args.no_cpu_baseline:
+            wl.W1, wl.W3, wl.W2 = W1, W3, W2
+            line["cpu_baseline"] = cpu_baseline(wl)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse mixture-of-experts layer.
+ *
+ * The layer (Mixtral style): for each token x_t (a row of x),
+ *   logits_t = x_t . Wg^T                     (fp32 router, E experts)
+ *   idx_t    = the k experts of largest logit (k = 2 for Mixtral)
+ *   w_t      = softmax over those k logits    (gate weights, sum to 1)
+ *   y_t      = sum_j w_tj * Expert_{idx_tj}(x_t),
+ *   Expert_e(v) = W2_e (SiLU(W1_e v) * (W3_e v)),  SiLU(a) = a * sigmoid(a)
+ * with an optional per-expert capacity: at most floor(cf * T * k / E) slots
+ * per expert, an overflowed slot contributing zero (the token passes through
+ * on the residual path outside this layer).
+ *
+ * Sources (web pages, by title and section):
+ *   "Mixtral and Mixture-of-Experts, Explained", "How it works" -- the gate
+ *       G(x) = Softmax(TopK(x . W_g)) and y = sum_i G(x)_i Expert_i(x).
+ *   "How Mixtral 8x7B uses mixture of experts", "The architecture in one
+ *       diagram" (top-2 of the router softmax, renormalised; batch tokens by
+ *       expert, run experts, scatter back) and "Routing without auxiliary
+ *       loss" (capacity factor; excess tokens dropped; sorted by router
+ *       probability per expert).
+ *   "Mixtral" (vanos001), "MoE Layer" (MixtralMoE / MixtralExpert: bias-free
+ *       nn.Linear router [E, d]; expert w2(silu(w1 x) * w3 x)) and "SwiGLU
+ *       Experts".
+ *
+ * Conventions for every entry point
+ *   - Layouts are row-major.  x [T, d]; Wg [E, d] (fp32); W1, W3 [E, f, d];
+ *     W2 [E, d, f]; slot s = t * k + j, j = 0 the larger logit.
+ *   - Matrices of bf16 are passed as raw 16-bit patterns (moe_bf16).
+ *   - All pointers are DEVICE pointers unless the name ends in _host.  The
+ *     caller allocates every buffer, including the workspace; the library
+ *     allocates no memory and keeps no state between calls apart from cached
+ *     device attributes and driver entry points.
+ *   - Calls are asynchronous on `stream`; none synchronises except
+ *     moe_read_device_status.  A workspace may serve one call in flight at a
+ *     time.
+ *   - Arguments are checked before any work is queued; on failure the call
+ *     returns the status and queues nothing.  T == 0 is a no-op (MOE_OK).
+ *     Requirements: 1 <= E <= 32, 1 <= k <= min(E, 4), d_model and d_ff
+ *     multiples of 64 in [64, 65536], T * k < 2^30, finite capacity_factor,
+ *     bf16 / fp32 matrices 16-byte aligned, int32 arrays 4-byte aligned,
+ *     workspace 256-byte aligned and at least moe_workspace_size() bytes.
+ *   - A queued kernel that fails to launch gives MOE_ERR_CUDA.  Device-side
+ *     waits are bounded; one that gives up writes MOE_ERR_TIMEOUT into the
+ *     workspace's status word (read it with moe_read_device_status) and the
+ *     kernel returns without trapping.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same handle as cudaStream_t */
+typedef uint16_t moe_bf16;                /* raw bfloat16 bits */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or enum */
+  MOE_ERR_UNSUPPORTED = 2, /* valid request this build does not handle (e.g. not sm_100) */
+  MOE_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up */
+} moe_status;
+
+/* Which slots an overfull expert drops (capacity mode only). */
+typedef enum {
+  MOE_DROP_BY_PROB = 0, /* keep the cap slots of highest router probability
+                           (full softmax over E), ties to the smaller token */
+  MOE_DROP_BY_ORDER = 1 /* keep the first cap slots in token order */
+} moe_drop_policy;
+
+/* Expert-GEMM schedule.  Both compute the same function. */
+typedef enum {
+  MOE_VARIANT_AUTO = 0,   /* STREAM when T <= 128, TILED otherwise */
+  MOE_VARIANT_TILED = 1,  /* 128-token x 256-column tiles: compute-bound sizes */
+  MOE_VARIANT_STREAM = 2  /* weights as the 128-row MMA operand, tokens as N,
+                             split-K on the down projection: weight-streaming sizes */
+} moe_gemm_variant;
+
+typedef struct {
+  int64_t T;               /* tokens (rows of x) */
+  int32_t d_model;         /* d: hidden size */
+  int32_t d_ff;            /* f: expert inner size */
+  int32_t E;               /* experts */
+  int32_t k;               /* experts per token */
+  float capacity_factor;   /* <= 0: dropless (default); else cap = floor(cf*T*k/E) */
+  int32_t drop_policy;     /* moe_drop_policy */
+  int32_t gemm_variant;    /* moe_gemm_variant */
+} moe_shape;
+
+/* Bytes of workspace every entry point below accepts for this shape
+ * (moe_layer_forward needs all of it; the stage entry points use parts).
+ * Returns 0 if the shape is invalid. */
+MOE_API size_t moe_workspace_size(const moe_shape *shape);
+
+/* Router and gate.  Source: "Mixtral and Mixture-of-Experts, Explained",
+ * "How it works" (G(x) = Softmax(TopK(x . W_g))); "Mixtral", "MoE Layer"
+ * (topk of the logits, softmax over the k kept ones).
+ *   x [T, d] bf16, Wg [E, d] fp32                                   (in)
+ *   logits [T, E] fp32, may be NULL                                  (out)
+ *   topk_idx [T, k] int32: experts by descending logit, equal logits
+ *            ordered by the smaller index                            (out)
+ *   topk_w [T, k] fp32: softmax over the k kept logits               (out)
+ *   topk_p [T, k] fp32: softmax over all E logits at the kept experts
+ *            (the capacity priority)                                 (out)
+ *   counts [E] int32: slots routed to each expert (histogram)        (out)
+ * Logits are accumulated in fp32. */
+MOE_API moe_status moe_router_topk(const moe_shape *shape, const moe_bf16 *x, const float *Wg,
+                           float *logits, int32_t *topk_idx, float *topk_w, float *topk_p,
+                           int32_t *counts, moe_stream_t stream);
+
+/* Capacity and grouping of slots by expert.  Source: "How Mixtral 8x7B uses
+ * mixture of experts", "The architecture in one diagram" (batch tokens by
+ * expert) and "Routing without auxiliary loss" (capacity, drop).
+ *   x [T, d], topk_idx [T, k], counts [E] (from moe_router_topk)    (in)
+ *   topk_p [T, k]: read only in capacity mode with MOE_DROP_BY_PROB,
+ *            may be NULL otherwise                                   (in)
+ *   offsets [E + 1]: rows of expert e are offsets[e] .. offsets[e+1]-1;
+ *            offsets[E] = kept slots N                               (out)
+ *   slot_pos [T * k]: row of slot s, or -1 if dropped                (out)
+ *   perm_slot [T * k]: slot of row r for r < N (rest untouched)      (out)
+ *   x_perm [T * k, d]: x_perm[r] = x[perm_slot[r] / k] for r < N     (out)
+ * Rows of one expert are in ascending token order. */
+MOE_API moe_status moe_permute(const moe_shape *shape, const moe_bf16 *x, const int32_t *topk_idx,
+                       const float *topk_p, const int32_t *counts, int32_t *offsets,
+                       int32_t *slot_pos, int32_t *perm_slot, moe_bf16 *x_perm, void *ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped SwiGLU experts on tensor cores.  Source: "Mixtral", "MoE Layer"
+ * (MixtralExpert.forward) and "SwiGLU Experts".  For each expert e and row r
+ * in offsets[e] .. offsets[e+1]-1:
+ *   h[r]      = SiLU(x_perm[r] . W1[e]^T) * (x_perm[r] . W3[e]^T)   [f] bf16
+ *   y_perm[r] = h[r] . W2[e]^T                                        [d] bf16
+ * bf16 operands, fp32 accumulation, results rounded to bf16 (nearest even).
+ * Rows r >= offsets[E] of h and y_perm are left untouched. */
+MOE_API moe_status moe_grouped_swiglu(const moe_shape *shape, const moe_bf16 *x_perm,
+                              const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
+                              const moe_bf16 *W2, moe_bf16 *h, moe_bf16 *y_perm, void *ws,
+                              size_t ws_bytes, moe_stream_t stream);
+
+/* Gate-weighted combine.  Source: "Mixtral and Mixture-of-Experts,
+ * Explained", "How it works" (y = sum_i G(x)_i Expert_i(x)).
+ *   y[t] = sum over j with slot_pos[t*k+j] >= 0 of
+ *          topk_w[t, j] * y_perm[slot_pos[t*k+j]]
+ * accumulated in fp32 in slot order, stored bf16; y[t] = 0 when every slot
+ * of t was dropped.  The remaining weights are not renormalised. */
+MOE_API moe_status moe_combine(const moe_shape *shape, const moe_bf16 *y_perm, const int32_t *slot_pos,
+                       const float *topk_w, moe_bf16 *y, moe_stream_t stream);
+
+/* The whole layer: router, capacity, grouping, experts, combine, all
+ * intermediates in the workspace.  y [T, d] bf16 (out).  topk_idx_out
+ * [T, k] and counts_out [E] (both may be NULL) receive the routing. */
+MOE_API moe_status moe_layer_forward(const moe_shape *shape, const moe_bf16 *x, const float *Wg,
+                             const moe_bf16 *W1, const moe_bf16 *W3, const moe_bf16 *W2,
+                             moe_bf16 *y, int32_t *topk_idx_out, int32_t *counts_out, void *ws,
+                             size_t ws_bytes, moe_stream_t stream);
+
+/* moe_layer_forward, also recording CUDA events on `stream` between its
+ * kernels, for timing each kernel inside a real forward pass.  events[6]
+ * are cudaEvent_t handles the caller created (timing enabled):
+ *   [0] before the router        [1] after the router
+ *   [2] after capacity selection and grouping by expert
+ *   [3] after the gate/up-projection GEMM (SiLU * mul fused)
+ *   [4] after the down-projection GEMM    [5] after the combine.
+ * Same arguments and results as moe_layer_forward otherwise. */
+MOE_API moe_status moe_layer_forward_profiled(const moe_shape *shape, const moe_bf16 *x,
+                                              const float *Wg, const moe_bf16 *W1,
+                                              const moe_bf16 *W3, const moe_bf16 *W2, moe_bf16 *y,
+                                              void *const *events, void *ws, size_t ws_bytes,
+                                              moe_stream_t stream);
+
+/* The whole layer with the activations in HOST memory: copies x_host
+ * [T, d] to the device (inside the workspace), runs moe_layer_forward and
+ * copies y back to y_host [T, d], all queued on `stream`.  Weights are
+ * device pointers.  Use page-locked host buffers for asynchronous copies;
+ * y_host is valid once the stream has been synchronised. */
+MOE_API moe_status moe_layer_forward_host(const moe_shape *shape, const moe_bf16 *x_host,
+                                  const float *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
+                                  const moe_bf16 *W2, moe_bf16 *y_host, void *ws,
+                                  size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, then returns the device status word of the last
+ * call that used this workspace (MOE_OK or MOE_ERR_TIMEOUT), or
+ * MOE_ERR_CUDA if the stream reports an error. */
+MOE_API moe_status moe_read_device_status(const void *ws, moe_stream_t stream);
+
+/* Static English text of a status code. */
+MOE_API const char *moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

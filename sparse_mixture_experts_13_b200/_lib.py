@@ -1,0 +1,149 @@
+"""ctypes binding of ``libmoe.so`` (the C ABI in include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  Tensors are passed by ``data_ptr()``; ``None`` becomes NULL;
+plain integers are taken as addresses.  Each wrapper returns the library's
+``moe_status`` code (0 = MOE_OK); ``check()`` turns a non-zero code into
+``MoeError``.  There is no fallback: if the library is missing the first call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+MOE_DROP_BY_PROB, MOE_DROP_BY_ORDER = 0, 1
+MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM = 0, 1, 2
+
+EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
+            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_read_device_status", "moe_status_string")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
+                ("drop_policy", ctypes.c_int32), ("gemm_variant", ctypes.c_int32)]
+
+
+def make_shape(T, d_model, d_ff, E=8, k=2, capacity_factor=0.0, drop_policy=0, gemm_variant=0) -> moe_shape:
+    return moe_shape(int(T), int(d_model), int(d_ff), int(E), int(k), float(capacity_factor),
+                     int(drop_policy), int(gemm_variant))
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so is not built ({LIB_PATH}); run the package build first")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, st = ctypes.c_void_p, ctypes.POINTER(moe_shape), ctypes.c_int
+        sz = ctypes.c_size_t
+        L.moe_workspace_size.argtypes = [S]
+        L.moe_workspace_size.restype = sz
+        L.moe_router_topk.argtypes = [S, P, P, P, P, P, P, P, P]
+        L.moe_permute.argtypes = [S, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_combine.argtypes = [S, P, P, P, P, P]
+        L.moe_layer_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_layer_forward_host.argtypes = [S, P, P, P, P, P, P, P, sz, P]
+        L.moe_layer_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_read_device_status.argtypes = [P, P]
+        L.moe_status_string.argtypes = [st]
+        L.moe_status_string.restype = ctypes.c_char_p
+        for name in EXPORTED[1:-1]:
+            getattr(L, name).restype = st
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def check(status: int, what: str = "moe") -> None:
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def moe_workspace_size(shape: moe_shape) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(shape)))
+
+
+def moe_router_topk(shape, x, Wg, logits, topk_idx, topk_w, topk_p, counts, stream=None) -> int:
+    return lib().moe_router_topk(ctypes.byref(shape), _p(x), _p(Wg), _p(logits), _p(topk_idx), _p(topk_w),
+                                 _p(topk_p), _p(counts), _stream(stream))
+
+
+def moe_permute(shape, x, topk_idx, topk_p, counts, offsets, slot_pos, perm_slot, x_perm, ws, ws_bytes,
+                stream=None) -> int:
+    return lib().moe_permute(ctypes.byref(shape), _p(x), _p(topk_idx), _p(topk_p), _p(counts), _p(offsets),
+                             _p(slot_pos), _p(perm_slot), _p(x_perm), _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_grouped_swiglu(shape, x_perm, offsets, W1, W3, W2, h, y_perm, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_grouped_swiglu(ctypes.byref(shape), _p(x_perm), _p(offsets), _p(W1), _p(W3), _p(W2), _p(h),
+                                    _p(y_perm), _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_combine(shape, y_perm, slot_pos, topk_w, y, stream=None) -> int:
+    return lib().moe_combine(ctypes.byref(shape), _p(y_perm), _p(slot_pos), _p(topk_w), _p(y), _stream(stream))
+
+
+def moe_layer_forward(shape, x, Wg, W1, W3, W2, y, topk_idx_out, counts_out, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_layer_forward(ctypes.byref(shape), _p(x), _p(Wg), _p(W1), _p(W3), _p(W2), _p(y),
+                                   _p(topk_idx_out), _p(counts_out), _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_layer_forward_host(shape, x_host, Wg, W1, W3, W2, y_host, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_layer_forward_host(ctypes.byref(shape), _p(x_host), _p(Wg), _p(W1), _p(W3), _p(W2),
+                                        _p(y_host), _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_layer_forward_profiled(shape, x, Wg, W1, W3, W2, y, events, ws, ws_bytes, stream=None) -> int:
+    """events: six torch.cuda.Event(enable_timing=True) objects (or raw handles)."""
+    handles = []
+    for ev in events:
+        if isinstance(ev, int):
+            handles.append(ev)
+        else:
+            if ev.cuda_event == 0:
+                ev.record()  # creates the underlying event
+            handles.append(ev.cuda_event)
+    arr = (ctypes.c_void_p * 6)(*handles)
+    return lib().moe_layer_forward_profiled(ctypes.byref(shape), _p(x), _p(Wg), _p(W1), _p(W3), _p(W2), _p(y), arr,
+                                            _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_read_device_status(ws, stream=None) -> int:
+    return lib().moe_read_device_status(_p(ws), _stream(stream))

@@ -1,0 +1,122 @@
+// Gate-weighted combine (un-permute).
+//
+// Source: "Mixtral and Mixture-of-Experts, Explained", section "How it works"
+// (y = sum_i G(x)_i . Expert_i(x)), and "How Mixtral 8x7B uses mixture of
+// experts", section "The architecture in one diagram" (out += weight *
+// expert_out, scattered back to the tokens).
+//
+//   y[t] = sum over kept slots j of t (slot_pos >= 0) of w[t, j] * o_j
+//
+// where o_j is the expert output row slot_pos[t*k+j] of y_perm (bf16), or the
+// sum in split order of the fp32 split-K partials of that row.  fp32
+// accumulation in slot order, one bf16 rounding at the end; no atomics, so
+// the result is bit-reproducible.  One warp per token, 16-byte vectors.
+#include <cstdint>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ void bf16x8_unpack(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int nvec = a.d >> 3;
+  for (int64_t t = warp_global; t < a.T; t += nwarps) {
+    int32_t pos[4];
+    float w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      pos[j] = -1;
+      w[j] = 0.f;
+      if (j < a.k) {
+        pos[j] = __ldg(a.slot_pos + t * a.k + j);
+        w[j] = __ldg(a.topk_w + t * a.k + j);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(a.y + t * a.d);
+    for (int v = lane; v < nvec; v += 32) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (pos[j] < 0) continue;
+        float o[8];
+        if (a.y_perm) {
+          bf16x8_unpack(__ldg(reinterpret_cast<const uint4*>(a.y_perm + (int64_t)pos[j] * a.d) + v), o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = 0.f;
+          for (int sp = 0; sp < a.splits; ++sp) {
+            const float4* src =
+                reinterpret_cast<const float4*>(a.partials + sp * a.part_stride + (int64_t)pos[j] * a.d) + 2 * v;
+            const float4 p0 = __ldg(src), p1 = __ldg(src + 1);
+            o[0] += p0.x; o[1] += p0.y; o[2] += p0.z; o[3] += p0.w;
+            o[4] += p1.x; o[5] += p1.y; o[6] += p1.z; o[7] += p1.w;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], o[i], acc[i]);
+      }
+      dst[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                          pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+  }
+}
+
+cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
+  const int64_t warps_needed = a.T;
+  int64_t blocks = (warps_needed + 7) / 8;
+  const int64_t cap = (int64_t)num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  combine_kernel<<<(unsigned)blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// y_perm[r] = bf16(sum over splits of partials[sp][r]) for rows r < offsets[E].
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partials, int32_t splits,
+                                                            int64_t part_stride, const int32_t* __restrict__ offsets,
+                                                            int32_t E, uint16_t* __restrict__ y_perm, int32_t d) {
+  const int64_t rows = offsets[E];
+  const int nvec = d >> 3;
+  const int64_t total = rows * nvec;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / nvec;
+    const int v = (int)(i % nvec);
+    float o[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) o[q] = 0.f;
+    for (int sp = 0; sp < splits; ++sp) {
+      const float4* src = reinterpret_cast<const float4*>(partials + sp * part_stride + r * d) + 2 * v;
+      const float4 p0 = __ldg(src), p1 = __ldg(src + 1);
+      o[0] += p0.x; o[1] += p0.y; o[2] += p0.z; o[3] += p0.w;
+      o[4] += p1.x; o[5] += p1.y; o[6] += p1.z; o[7] += p1.w;
+    }
+    reinterpret_cast<uint4*>(y_perm + r * d)[v] =
+        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+  }
+}
+
+cudaError_t launch_splitk_reduce(const float* partials, int32_t splits, int64_t part_stride, const int32_t* offsets,
+                                 int32_t E, uint16_t* y_perm, int64_t S, int32_t d, int num_sms, cudaStream_t s) {
+  int64_t blocks = (S * (d / 8) + 255) / 256;
+  const int64_t cap = (int64_t)num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(partials, splits, part_stride, offsets, E, y_perm, d);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

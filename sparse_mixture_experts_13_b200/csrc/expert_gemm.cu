@@ -1,0 +1,577 @@
+// Grouped SwiGLU expert GEMMs on the 5th-generation tensor cores.
+//
+// Source: "Mixtral", sections "MoE Layer" (MixtralExpert.forward:
+// w2(silu(w1 x) * w3 x), bias-free) and "SwiGLU Experts"
+// (SwiGLU(x) = SiLU(x W1) (.) (x W3), output = SwiGLU(x) W2).
+//
+// For each expert e the rows offsets[e] .. offsets[e+1]-1 of the grouped
+// activations are multiplied by that expert's weights:
+//   GEMM1: h[r]      = SiLU(x_perm[r] . W1[e]^T) * (x_perm[r] . W3[e]^T)
+//   GEMM2: y_perm[r] = h[r] . W2[e]^T
+// Both use one persistent, warp-specialised kernel (one CTA per SM):
+//   warp 0     one thread issues TMA tile loads into a STAGES-deep ring of
+//              shared-memory buffers (128-byte swizzle, K-major);
+//   warp 1     allocates tensor memory and one thread issues
+//              tcgen05.mma (kind::f16, bf16 in, fp32 accumulate, M = 128,
+//              N = BN, K = 16) into one of two TMEM accumulators;
+//   warps 2-5  epilogue: tcgen05.ld the accumulator, apply SiLU * mul or a
+//              plain conversion, store bf16 (or fp32 split-K partials).
+// The accumulators are double-buffered so the epilogue of one tile overlaps
+// the main loop of the next.  Tiles are enumerated per expert from the
+// device-resident offsets (no host synchronisation) and distributed
+// round-robin over the CTAs.
+//
+// Two schedules compute the same function:
+//   TILED  (token-rich): A = 128 activation rows, B = weight rows.  GEMM1's
+//          B tile stacks 128 rows of W1 over the same 128 rows of W3 (N = 256)
+//          so accumulator columns c and c + 128 hold the two projections of
+//          one output column; GEMM2's B tile is 256 rows of W2.
+//   STREAM (token-poor, bound by reading the weights): A = weight rows,
+//          B = the expert's (up to BN) tokens.  GEMM1's A tile stacks 64 rows
+//          of W1 over the same 64 rows of W3 (accumulator lanes r and r + 64);
+//          GEMM2's A tile is 128 rows of W2 and its K range is split so that
+//          there are enough tiles to stream the weights on every SM; the
+//          fp32 partials are summed by the combine (or a reduce kernel).
+// Rows past an expert's end (next expert's rows, or zero fill past the
+// buffer) are computed but never stored; weight rows past d_ff / d_model are
+// zero-filled by the 3-D tensor maps.
+#include <cstdint>
+#include <cstdio>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+constexpr int BM = 128;  // MMA M: rows of the A operand
+constexpr int BK = 64;   // K elements per stage: 128 bytes of bf16, one swizzle span
+constexpr int kGemmThreads = 192;
+constexpr int A_BYTES = BM * BK * 2;
+
+enum : int { EPI_TILED_SWIGLU = 0, EPI_TILED_STORE = 1, EPI_STREAM_SWIGLU = 2, EPI_STREAM_PARTIAL = 3 };
+
+struct GemmParams {
+  const int32_t* offsets;
+  uint32_t* status;
+  void* out;            // bf16 h / y_perm, or fp32 partials
+  int64_t out_ld;       // elements between output rows
+  int64_t part_stride;  // elements between split-K partial buffers
+  int32_t E;
+  int32_t num_kb;       // K / 64
+  int32_t n_out;        // valid output columns (d_ff or d_model)
+  int32_t n_blocks;     // weight blocks per expert
+  int32_t splits;       // K splits (STREAM partial), else 1
+  int32_t kb_per_split;
+};
+
+__host__ __device__ constexpr bool epi_is_tiled(int epi) { return epi <= EPI_TILED_STORE; }
+
+template <int EPI, int BN>
+struct GemmCfg {
+  static constexpr bool kTiled = epi_is_tiled(EPI);
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = kTiled ? 4 : ((192 * 1024) / STAGE_BYTES > 10 ? 10 : (192 * 1024) / STAGE_BYTES);
+  // TMEM columns: two accumulators of BN fp32 columns, power of two >= 32.
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int XBUF_BYTES = (EPI == EPI_STREAM_SWIGLU) ? 64 * 16 * 4 : 0;
+  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + XBUF_BYTES + BAR_BYTES;
+  // rows of the weight operand per tile (n-extent of one weight block)
+  static constexpr int W_ROWS = (EPI == EPI_TILED_SWIGLU) ? 128 : (EPI == EPI_TILED_STORE) ? 256 : (EPI == EPI_STREAM_SWIGLU) ? 64 : 128;
+  static constexpr uint32_t IDESC = make_idesc_bf16(BM, BN);
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+struct Tile {
+  int32_t e, row0, m_valid, n0, split, kb0, kb1;
+};
+
+template <int EPI, int BN>
+__device__ __forceinline__ bool decode_tile(const GemmParams& p, const int32_t* s_off,
+                                            const int32_t* s_base, int32_t tile, Tile& t) {
+  using C = GemmCfg<EPI, BN>;
+  int e = 0;
+  while (e < p.E && tile >= s_base[e + 1]) ++e;
+  if (e >= p.E) return false;
+  const int32_t local = tile - s_base[e];
+  const int32_t M_e = s_off[e + 1] - s_off[e];
+  t.e = e;
+  if (C::kTiled) {
+    const int32_t mb_count = (M_e + BM - 1) / BM;
+    const int32_t nb = local / mb_count, mb = local % mb_count;
+    t.row0 = s_off[e] + mb * BM;
+    t.m_valid = min(BM, M_e - mb * BM);
+    t.n0 = nb * C::W_ROWS;
+    t.split = 0;
+    t.kb0 = 0;
+    t.kb1 = p.num_kb;
+  } else {
+    const int32_t tb_count = (M_e + BN - 1) / BN;
+    const int32_t tb = local % tb_count;
+    const int32_t rest = local / tb_count;
+    t.split = rest % p.splits;
+    const int32_t wb = rest / p.splits;
+    t.row0 = s_off[e] + tb * BN;
+    t.m_valid = min(BN, M_e - tb * BN);
+    t.n0 = wb * C::W_ROWS;
+    t.kb0 = t.split * p.kb_per_split;
+    t.kb1 = min(p.num_kb, t.kb0 + p.kb_per_split);
+  }
+  return true;
+}
+
+template <int EPI, int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap map_act,
+                       const __grid_constant__ CUtensorMap map_wa,
+                       const __grid_constant__ CUtensorMap map_wb, GemmParams p) {
+  using C = GemmCfg<EPI, BN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_epi_fail;
+  __shared__ int32_t s_off[33];
+  __shared__ int32_t s_base[33];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  float* xbuf = reinterpret_cast<float*>(sB + STAGES * C::B_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES + C::XBUF_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* tfull_bar = bars + 2 * STAGES;
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    tma_prefetch_desc(&map_act);
+    tma_prefetch_desc(&map_wa);
+    if (EPI == EPI_TILED_SWIGLU || EPI == EPI_STREAM_SWIGLU) tma_prefetch_desc(&map_wb);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 4);
+    }
+    mbar_init(drain_bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 64) {
+    s_abort = 0;
+    s_epi_fail = 0;
+    int32_t acc = 0;
+    s_base[0] = 0;
+    for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+    for (int e = 0; e < p.E; ++e) {
+      const int32_t M_e = s_off[e + 1] - s_off[e];
+      int32_t n = 0;
+      if (M_e > 0) {
+        if (C::kTiled) n = ((M_e + BM - 1) / BM) * p.n_blocks;
+        else n = ((M_e + BN - 1) / BN) * p.n_blocks * p.splits;
+      }
+      acc += n;
+      s_base[e + 1] = acc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s_tmem;
+  const int32_t total = s_base[p.E];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int32_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        Tile t;
+        decode_tile<EPI, BN>(p, s_off, s_base, tile, t);
+        for (int32_t kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &s_abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          uint8_t* a_dst = sA + stage * A_BYTES;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+          const int32_t kx = kb * BK;
+          if (EPI == EPI_TILED_SWIGLU) {
+            tma_load_2d(&map_act, &full_bar[stage], a_dst, kx, t.row0);
+            tma_load_3d(&map_wa, &full_bar[stage], b_dst, kx, t.n0, t.e);
+            tma_load_3d(&map_wb, &full_bar[stage], b_dst + 128 * 128, kx, t.n0, t.e);
+          } else if (EPI == EPI_TILED_STORE) {
+            tma_load_2d(&map_act, &full_bar[stage], a_dst, kx, t.row0);
+            tma_load_3d(&map_wa, &full_bar[stage], b_dst, kx, t.n0, t.e);
+          } else if (EPI == EPI_STREAM_SWIGLU) {
+            tma_load_3d(&map_wa, &full_bar[stage], a_dst, kx, t.n0, t.e);
+            tma_load_3d(&map_wb, &full_bar[stage], a_dst + 64 * 128, kx, t.n0, t.e);
+            tma_load_2d(&map_act, &full_bar[stage], b_dst, kx, t.row0);
+          } else {
+            tma_load_3d(&map_wa, &full_bar[stage], a_dst, kx, t.n0, t.e);
+            tma_load_2d(&map_act, &full_bar[stage], b_dst, kx, t.row0);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        s_abort = 1;
+      }
+      // Let every load this thread issued land before the CTA may exit.
+      for (int s = 0; s < STAGES; ++s) {
+        if (s < issued) {
+          const int64_t uses = (issued - s + STAGES - 1) / STAGES;
+          mbar_wait(&full_bar[s], (uint32_t)((uses - 1) & 1), nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t iter = 0;
+      bool ok = true;
+      for (int32_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++iter) {
+        Tile t;
+        decode_tile<EPI, BN>(p, s_off, s_base, tile, t);
+        const uint32_t acc = iter & 1, use = iter >> 1;
+        if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+        for (int32_t kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            umma_bf16(d_tmem, make_sdesc_sw128(a_addr + kk * 32), make_sdesc_sw128(b_addr + kk * 32),
+                      C::IDESC, (kb > t.kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[acc]);
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        s_abort = 1;
+      }
+      // Wait for every MMA this thread issued before tensor memory is freed.
+      umma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;      // accumulator lane (row of the MMA's M)
+    uint32_t iter = 0;
+    for (int32_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++iter) {
+      Tile t;
+      decode_tile<EPI, BN>(p, s_off, s_base, tile, t);
+      const uint32_t acc = iter & 1, use = iter >> 1;
+      // The four epilogue warps decide together whether to go on, so that a
+      // wait that gives up in one warp never leaves the others at a barrier.
+      if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort)) s_epi_fail = 1;
+      named_bar_sync(2, 128);
+      if (s_epi_fail) {
+        record_status(p.status, kStatusTimeout);
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_acc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+
+      if (EPI == EPI_TILED_SWIGLU) {
+        uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
+        const bool row_ok = r < t.m_valid;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t va[32], vb[32];
+          tmem_ld_32x32b_x32(t_acc + c0, va);
+          tmem_ld_32x32b_x32(t_acc + 128 + c0, vb);
+          tmem_ld_wait();
+          if (row_ok && t.n0 + c0 < p.n_out) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f32(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
+              const float h1 = silu_f32(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
+              packed[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(t.row0 + r) * p.out_ld + t.n0 + c0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
+        }
+      } else if (EPI == EPI_TILED_STORE) {
+        uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
+        const bool row_ok = r < t.m_valid;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_acc + c0, v);
+          tmem_ld_wait();
+          if (row_ok && t.n0 + c0 < p.n_out) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(t.row0 + r) * p.out_ld + t.n0 + c0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
+        }
+      } else if (EPI == EPI_STREAM_SWIGLU) {
+        // lanes 0..63: W1 projection of output column n0 + r; lanes 64..127:
+        // W3 projection of column n0 + r - 64.  Columns of TMEM are tokens.
+        uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_acc + c0, v);
+          tmem_ld_wait();
+          if (r >= 64) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xbuf[j * 64 + (r - 64)] = __uint_as_float(v[j]);
+          }
+          named_bar_sync(1, 128);
+          if (r < 64 && t.n0 + r < p.n_out) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int tok = c0 + j;
+              if (tok < t.m_valid) {
+                const float hv = silu_f32(__uint_as_float(v[j])) * xbuf[j * 64 + r];
+                out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] =
+                    (uint16_t)(pack_bf16x2(hv, 0.f) & 0xFFFFu);
+              }
+            }
+          }
+          named_bar_sync(1, 128);
+        }
+      } else {
+        // fp32 split-K partial: lane r is output column n0 + r; TMEM columns are tokens.
+        float* out = reinterpret_cast<float*>(p.out) + (int64_t)t.split * p.part_stride;
+        const bool col_ok = t.n0 + r < p.n_out;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_acc + c0, v);
+          tmem_ld_wait();
+          if (col_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int tok = c0 + j;
+              if (tok < t.m_valid) out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] = __uint_as_float(v[j]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over a [rows, cols] row-major matrix, box {64, box_rows}.
+static bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over [E, rows, cols] row-major, box {64, box_rows, 1}.
+static bool encode_3d(CUtensorMap* m, const void* base, int64_t E, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)(rows * cols * 2)};
+  cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI, int BN>
+static cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& wa, const CUtensorMap& wb,
+                              const GemmParams& p, int num_sms, cudaStream_t s) {
+  using C = GemmCfg<EPI, BN>;
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_kernel<EPI, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  expert_gemm_kernel<EPI, BN><<<num_sms, kGemmThreads, C::SMEM_BYTES, s>>>(act, wa, wb, p);
+  return cudaGetLastError();
+}
+
+void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
+  int64_t b = ((T + 15) / 16) * 16;
+  if (b < 16) b = 16;
+  if (b > 128) b = 128;
+  if (b > 64) b = 128;
+  else if (b > 32) b = 64;
+  else if (b > 16) b = 32;
+  *bn = (int32_t)b;
+  // Split K of the down projection so that (experts x 128-row blocks x
+  // splits) tiles fill whole waves of the SMs as evenly as possible.
+  const int32_t num_kb = f / BK;
+  const int64_t base = (int64_t)E * ((d + 127) / 128);
+  int32_t best = 1;
+  double best_eff = 0.0;
+  for (int32_t sp = 1; sp <= 16 && sp <= num_kb; ++sp) {
+    const int32_t kbps = (num_kb + sp - 1) / sp;
+    const int32_t real = (num_kb + kbps - 1) / kbps;
+    const int64_t tiles = base * real;
+    const int64_t waves = (tiles + num_sms - 1) / num_sms;
+    const double eff = (double)(base * num_kb) / (double)(waves * num_sms * kbps);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = real;
+    }
+  }
+  *splits = best;
+}
+
+template <int BN>
+static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
+  CUtensorMap mx, mw1, mw3, mh, mw2;
+  if (!encode_2d(&mx, a.x_perm, a.S, a.d, BN) || !encode_3d(&mw1, a.W1, a.E, a.f, a.d, 64) ||
+      !encode_3d(&mw3, a.W3, a.E, a.f, a.d, 64) || !encode_2d(&mh, a.h, a.S, a.f, BN) ||
+      !encode_3d(&mw2, a.W2, a.E, a.d, a.f, 128))
+    return cudaErrorInvalidValue;
+  GemmParams p1{};
+  p1.offsets = a.offsets;
+  p1.status = a.status;
+  p1.out = a.h;
+  p1.out_ld = a.f;
+  p1.part_stride = 0;
+  p1.E = a.E;
+  p1.num_kb = a.d / BK;
+  p1.n_out = a.f;
+  p1.n_blocks = a.f / 64;
+  p1.splits = 1;
+  p1.kb_per_split = p1.num_kb;
+  cudaError_t err = launch_one<EPI_STREAM_SWIGLU, BN>(mx, mw1, mw3, p1, a.num_sms, s);
+  if (err != cudaSuccess) return err;
+  if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
+  GemmParams p2{};
+  p2.offsets = a.offsets;
+  p2.status = a.status;
+  p2.out = a.partials;
+  p2.out_ld = a.d;
+  p2.part_stride = a.S * (int64_t)a.d;
+  p2.E = a.E;
+  p2.num_kb = a.f / BK;
+  p2.n_out = a.d;
+  p2.n_blocks = (a.d + 127) / 128;
+  p2.kb_per_split = (p2.num_kb + a.splits - 1) / a.splits;
+  p2.splits = (p2.num_kb + p2.kb_per_split - 1) / p2.kb_per_split;
+  return launch_one<EPI_STREAM_PARTIAL, BN>(mh, mw2, mw2, p2, a.num_sms, s);
+}
+
+static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
+  CUtensorMap mx, mw1, mw3, mh, mw2;
+  if (!encode_2d(&mx, a.x_perm, a.S, a.d, 128) || !encode_3d(&mw1, a.W1, a.E, a.f, a.d, 128) ||
+      !encode_3d(&mw3, a.W3, a.E, a.f, a.d, 128) || !encode_2d(&mh, a.h, a.S, a.f, 128) ||
+      !encode_3d(&mw2, a.W2, a.E, a.d, a.f, 256))
+    return cudaErrorInvalidValue;
+  GemmParams p1{};
+  p1.offsets = a.offsets;
+  p1.status = a.status;
+  p1.out = a.h;
+  p1.out_ld = a.f;
+  p1.E = a.E;
+  p1.num_kb = a.d / BK;
+  p1.n_out = a.f;
+  p1.n_blocks = (a.f + 127) / 128;
+  p1.splits = 1;
+  p1.kb_per_split = p1.num_kb;
+  cudaError_t err = launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s);
+  if (err != cudaSuccess) return err;
+  if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
+  GemmParams p2{};
+  p2.offsets = a.offsets;
+  p2.status = a.status;
+  p2.out = a.y_perm;
+  p2.out_ld = a.d;
+  p2.E = a.E;
+  p2.num_kb = a.f / BK;
+  p2.n_out = a.d;
+  p2.n_blocks = (a.d + 255) / 256;
+  p2.splits = 1;
+  p2.kb_per_split = p2.num_kb;
+  return launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s);
+}
+
+cudaError_t launch_expert_gemms(const ExpertGemmArgs& a, cudaStream_t s) {
+  if (a.variant == 1) return launch_tiled(a, s);
+  switch (a.stream_bn) {
+    case 16: return launch_stream<16>(a, s);
+    case 32: return launch_stream<32>(a, s);
+    case 64: return launch_stream<64>(a, s);
+    default: return launch_stream<128>(a, s);
+  }
+}
+
+}  // namespace moe

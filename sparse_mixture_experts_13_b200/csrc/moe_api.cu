@@ -1,0 +1,437 @@
+// C ABI of the sparse mixture-of-experts layer (declared in include/moe.h):
+// argument checks, workspace layout, choice of the expert-GEMM schedule and
+// the launch sequence.  No entry point allocates memory or synchronises
+// (except moe_read_device_status).
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "moe.h"
+#include "moe_internal.h"
+
+using namespace moe;
+
+namespace {
+
+// Split-K and workspace sizes are derived with this SM count so that the
+// workspace size is a function of the shape alone; grids use the real count.
+constexpr int kPlanSms = 148;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_shape(const moe_shape* sh) {
+  if (!sh) return MOE_ERR_INVALID_ARG;
+  if (sh->T < 0) return MOE_ERR_INVALID_ARG;
+  if (sh->E < 1 || sh->E > 32) return MOE_ERR_INVALID_ARG;
+  if (sh->k < 1 || sh->k > 4 || sh->k > sh->E) return MOE_ERR_INVALID_ARG;
+  if (sh->d_model < 64 || sh->d_model > 65536 || sh->d_model % 64) return MOE_ERR_INVALID_ARG;
+  if (sh->d_ff < 64 || sh->d_ff > 65536 || sh->d_ff % 64) return MOE_ERR_INVALID_ARG;
+  if (sh->T * (int64_t)sh->k >= ((int64_t)1 << 30)) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(sh->capacity_factor)) return MOE_ERR_INVALID_ARG;
+  if (sh->drop_policy != MOE_DROP_BY_PROB && sh->drop_policy != MOE_DROP_BY_ORDER) return MOE_ERR_INVALID_ARG;
+  if (sh->gemm_variant < MOE_VARIANT_AUTO || sh->gemm_variant > MOE_VARIANT_STREAM) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int64_t capacity_of(const moe_shape* sh) {
+  if (sh->capacity_factor <= 0.f) return -1;
+  return (int64_t)std::floor((double)sh->capacity_factor * (double)sh->T * (double)sh->k / (double)sh->E);
+}
+
+int variant_of(const moe_shape* sh) {
+  if (sh->gemm_variant != MOE_VARIANT_AUTO) return sh->gemm_variant;
+  return sh->T <= 128 ? MOE_VARIANT_STREAM : MOE_VARIANT_TILED;
+}
+
+struct Layout {
+  // control region, cleared at the start of moe_layer_forward
+  size_t status, ticket, counts, tile_state, ctrl_end;
+  size_t thresh, partials, topk_idx, topk_w, topk_p, offsets, slot_pos, perm_slot, x_perm, h, y_perm,
+      x_stage, y_stage, total;
+  int variant;
+  int32_t bn, splits;
+};
+
+Layout layout_of(const moe_shape* sh) {
+  Layout L{};
+  const int64_t T = sh->T, S = T * sh->k;
+  const int64_t d = sh->d_model, f = sh->d_ff, E = sh->E;
+  L.variant = variant_of(sh);
+  L.bn = 128;
+  L.splits = 1;
+  if (L.variant == MOE_VARIANT_STREAM) stream_params(T, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
+  size_t o = 0;
+  L.status = o;
+  L.ticket = o + 4;
+  o = align_up(o + 8);
+  L.counts = o;
+  o = align_up(o + 4 * E);
+  L.tile_state = o;
+  o = align_up(o + 4 * (size_t)permute_tiles(S) * E);
+  L.ctrl_end = o;
+  L.thresh = o;
+  o = align_up(o + 8 * E);
+  L.partials = o;
+  if (L.variant == MOE_VARIANT_STREAM) o = align_up(o + 4 * (size_t)L.splits * S * d);
+  L.topk_idx = o;
+  o = align_up(o + 4 * S);
+  L.topk_w = o;
+  o = align_up(o + 4 * S);
+  L.topk_p = o;
+  o = align_up(o + 4 * S);
+  L.offsets = o;
+  o = align_up(o + 4 * (E + 1));
+  L.slot_pos = o;
+  o = align_up(o + 4 * S);
+  L.perm_slot = o;
+  o = align_up(o + 4 * S);
+  L.x_perm = o;
+  o = align_up(o + 2 * (size_t)S * d);
+  L.h = o;
+  o = align_up(o + 2 * (size_t)S * f);
+  L.y_perm = o;
+  o = align_up(o + 2 * (size_t)S * d);
+  L.x_stage = o;
+  o = align_up(o + 2 * (size_t)T * d);
+  L.y_stage = o;
+  o = align_up(o + 2 * (size_t)T * d);
+  L.total = o;
+  return L;
+}
+
+moe_status check_ws(const moe_shape* sh, const void* ws, size_t ws_bytes) {
+  if (!ws || !aligned(ws, kAlign)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < layout_of(sh).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// Device checks, cached per device: sm_100 family and SM count.
+constexpr int kMaxDevices = 64;
+int g_dev_state[kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
+int g_dev_sms[kMaxDevices];
+
+moe_status check_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  if (g_dev_state[dev] == 0) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    g_dev_sms[dev] = sms;
+    g_dev_state[dev] = (major == 10) ? 1 : 2;
+  }
+  if (g_dev_state[dev] != 1) return MOE_ERR_UNSUPPORTED;
+  *num_sms = g_dev_sms[dev];
+  return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+#define MOE_TRY(expr)                  \
+  do {                                 \
+    moe_status _st = (expr);           \
+    if (_st != MOE_OK) return _st;     \
+  } while (0)
+
+moe_status check_bf16(const void* p) { return (p && aligned(p, 16)) ? MOE_OK : MOE_ERR_INVALID_ARG; }
+moe_status check_i32(const void* p) { return (p && aligned(p, 4)) ? MOE_OK : MOE_ERR_INVALID_ARG; }
+
+moe_status run_router(const moe_shape* sh, const moe_bf16* x, const float* Wg, float* logits, int32_t* idx, float* w,
+                      float* p, int32_t* counts, int num_sms, cudaStream_t s) {
+  RouterArgs a{x, Wg, logits, idx, w, p, counts, sh->T, sh->d_model, sh->E, sh->k};
+  return cuda_status(launch_router(a, num_sms, s));
+}
+
+moe_status run_permute(const moe_shape* sh, const Layout& L, const moe_bf16* x, const int32_t* idx, const float* p,
+                       const int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_slot,
+                       moe_bf16* x_perm, void* ws, cudaStream_t s) {
+  PermuteArgs a{};
+  a.x = x;
+  a.topk_idx = idx;
+  a.topk_p = p;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.slot_pos = slot_pos;
+  a.perm_slot = perm_slot;
+  a.x_perm = x_perm;
+  a.tile_state = at<uint32_t>(ws, L.tile_state);
+  a.ticket = at<uint32_t>(ws, L.ticket);
+  a.thresh = at<uint64_t>(ws, L.thresh);
+  a.status = at<uint32_t>(ws, L.status);
+  a.T = sh->T;
+  a.d = sh->d_model;
+  a.E = sh->E;
+  a.k = sh->k;
+  a.cap = capacity_of(sh);
+  a.policy = sh->drop_policy;
+  return cuda_status(launch_permute(a, s));
+}
+
+moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_perm, const int32_t* offsets,
+                     const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2, moe_bf16* h, moe_bf16* y_perm,
+                     void* ws, int num_sms, cudaStream_t s, cudaEvent_t between = nullptr) {
+  ExpertGemmArgs a{};
+  a.offsets = offsets;
+  a.x_perm = x_perm;
+  a.W1 = W1;
+  a.W3 = W3;
+  a.W2 = W2;
+  a.h = h;
+  a.y_perm = y_perm;
+  a.partials = at<float>(ws, L.partials);
+  a.status = at<uint32_t>(ws, L.status);
+  a.S = sh->T * sh->k;
+  a.d = sh->d_model;
+  a.f = sh->d_ff;
+  a.E = sh->E;
+  a.variant = L.variant;
+  a.stream_bn = L.bn;
+  a.splits = L.splits;
+  a.num_sms = num_sms;
+  a.between = between;
+  return cuda_status(launch_expert_gemms(a, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return layout_of(shape).total;
+}
+
+moe_status moe_router_topk(const moe_shape* sh, const moe_bf16* x, const float* Wg, float* logits,
+                           int32_t* topk_idx, float* topk_w, float* topk_p, int32_t* counts, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  MOE_TRY(check_bf16(x));
+  MOE_TRY(check_bf16(Wg));
+  MOE_TRY(check_i32(topk_idx));
+  MOE_TRY(check_i32(topk_w));
+  MOE_TRY(check_i32(topk_p));
+  MOE_TRY(check_i32(counts));
+  if (logits && !aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return run_router(sh, x, Wg, logits, topk_idx, topk_w, topk_p, counts, sms, (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const moe_shape* sh, const moe_bf16* x, const int32_t* topk_idx, const float* topk_p,
+                       const int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_slot,
+                       moe_bf16* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  MOE_TRY(check_bf16(x));
+  MOE_TRY(check_i32(topk_idx));
+  MOE_TRY(check_i32(counts));
+  MOE_TRY(check_i32(offsets));
+  MOE_TRY(check_i32(slot_pos));
+  MOE_TRY(check_i32(perm_slot));
+  MOE_TRY(check_bf16(x_perm));
+  if (sh->capacity_factor > 0.f && sh->drop_policy == MOE_DROP_BY_PROB) MOE_TRY(check_i32(topk_p));
+  MOE_TRY(check_ws(sh, ws, ws_bytes));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  const Layout L = layout_of(sh);
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 8, s)));  // status word and tile ticket
+  return run_permute(sh, L, x, topk_idx, topk_p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s);
+}
+
+moe_status moe_grouped_swiglu(const moe_shape* sh, const moe_bf16* x_perm, const int32_t* offsets,
+                              const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2, moe_bf16* h,
+                              moe_bf16* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  MOE_TRY(check_bf16(x_perm));
+  MOE_TRY(check_i32(offsets));
+  MOE_TRY(check_bf16(W1));
+  MOE_TRY(check_bf16(W3));
+  MOE_TRY(check_bf16(W2));
+  MOE_TRY(check_bf16(h));
+  MOE_TRY(check_bf16(y_perm));
+  MOE_TRY(check_ws(sh, ws, ws_bytes));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  const Layout L = layout_of(sh);
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 8, s)));
+  MOE_TRY(run_gemms(sh, L, x_perm, offsets, W1, W3, W2, h, y_perm, ws, sms, s));
+  if (L.variant == MOE_VARIANT_STREAM) {
+    const int64_t S = sh->T * sh->k;
+    const int32_t num_kb = sh->d_ff / 64;
+    const int32_t kbps = (num_kb + L.splits - 1) / L.splits;
+    const int32_t splits = (num_kb + kbps - 1) / kbps;
+    MOE_TRY(cuda_status(launch_splitk_reduce(at<float>(ws, L.partials), splits, S * (int64_t)sh->d_model, offsets,
+                                             sh->E, y_perm, S, sh->d_model, sms, s)));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_combine(const moe_shape* sh, const moe_bf16* y_perm, const int32_t* slot_pos, const float* topk_w,
+                       moe_bf16* y, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  MOE_TRY(check_bf16(y_perm));
+  MOE_TRY(check_i32(slot_pos));
+  MOE_TRY(check_i32(topk_w));
+  MOE_TRY(check_bf16(y));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  CombineArgs a{};
+  a.y_perm = y_perm;
+  a.slot_pos = slot_pos;
+  a.topk_w = topk_w;
+  a.y = y;
+  a.T = sh->T;
+  a.d = sh->d_model;
+  a.k = sh->k;
+  return cuda_status(launch_combine(a, sms, (cudaStream_t)stream));
+}
+
+static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, const float* Wg, const moe_bf16* W1,
+                                     const moe_bf16* W3, const moe_bf16* W2, moe_bf16* y, int32_t* topk_idx_out,
+                                     int32_t* counts_out, void* ws, int sms, cudaStream_t s,
+                                     cudaEvent_t const* ev = nullptr) {
+  const Layout L = layout_of(sh);
+  const int64_t S = sh->T * sh->k;
+  int32_t* idx = at<int32_t>(ws, L.topk_idx);
+  float* w = at<float>(ws, L.topk_w);
+  float* p = at<float>(ws, L.topk_p);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* slot_pos = at<int32_t>(ws, L.slot_pos);
+  int32_t* perm_slot = at<int32_t>(ws, L.perm_slot);
+  moe_bf16* x_perm = at<moe_bf16>(ws, L.x_perm);
+  moe_bf16* h = at<moe_bf16>(ws, L.h);
+  moe_bf16* y_perm = at<moe_bf16>(ws, L.y_perm);
+  auto mark = [&](int i) { return ev ? cuda_status(cudaEventRecord(ev[i], s)) : MOE_OK; };
+  MOE_TRY(mark(0));
+  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.ctrl_end, s)));
+  MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s));
+  MOE_TRY(mark(1));
+  MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s));
+  MOE_TRY(mark(2));
+  MOE_TRY(run_gemms(sh, L, x_perm, offsets, W1, W3, W2, h, y_perm, ws, sms, s, ev ? ev[3] : nullptr));
+  MOE_TRY(mark(4));
+  CombineArgs c{};
+  c.slot_pos = slot_pos;
+  c.topk_w = w;
+  c.y = y;
+  c.T = sh->T;
+  c.d = sh->d_model;
+  c.k = sh->k;
+  if (L.variant == MOE_VARIANT_STREAM) {
+    const int32_t num_kb = sh->d_ff / 64;
+    const int32_t kbps = (num_kb + L.splits - 1) / L.splits;
+    c.y_perm = nullptr;
+    c.partials = at<float>(ws, L.partials);
+    c.splits = (num_kb + kbps - 1) / kbps;
+    c.part_stride = S * (int64_t)sh->d_model;
+  } else {
+    c.y_perm = y_perm;
+  }
+  MOE_TRY(cuda_status(launch_combine(c, sms, s)));
+  MOE_TRY(mark(5));
+  if (topk_idx_out)
+    MOE_TRY(cuda_status(cudaMemcpyAsync(topk_idx_out, idx, sizeof(int32_t) * S, cudaMemcpyDeviceToDevice, s)));
+  if (counts_out)
+    MOE_TRY(cuda_status(cudaMemcpyAsync(counts_out, counts, sizeof(int32_t) * sh->E, cudaMemcpyDeviceToDevice, s)));
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_shape* sh, const moe_bf16* x, const float* Wg, const moe_bf16* W1,
+                             const moe_bf16* W3, const moe_bf16* W2, moe_bf16* y, int32_t* topk_idx_out,
+                             int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  MOE_TRY(check_bf16(x));
+  MOE_TRY(check_bf16(Wg));
+  MOE_TRY(check_bf16(W1));
+  MOE_TRY(check_bf16(W3));
+  MOE_TRY(check_bf16(W2));
+  MOE_TRY(check_bf16(y));
+  if (topk_idx_out && !aligned(topk_idx_out, 4)) return MOE_ERR_INVALID_ARG;
+  if (counts_out && !aligned(counts_out, 4)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(sh, ws, ws_bytes));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return layer_forward_impl(sh, x, Wg, W1, W3, W2, y, topk_idx_out, counts_out, ws, sms, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_forward_profiled(const moe_shape* sh, const moe_bf16* x, const float* Wg, const moe_bf16* W1,
+                                      const moe_bf16* W3, const moe_bf16* W2, moe_bf16* y, void* const* events,
+                                      void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  MOE_TRY(check_bf16(x));
+  MOE_TRY(check_bf16(Wg));
+  MOE_TRY(check_bf16(W1));
+  MOE_TRY(check_bf16(W3));
+  MOE_TRY(check_bf16(W2));
+  MOE_TRY(check_bf16(y));
+  if (!events) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(sh, ws, ws_bytes));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return layer_forward_impl(sh, x, Wg, W1, W3, W2, y, nullptr, nullptr, ws, sms, (cudaStream_t)stream,
+                            reinterpret_cast<cudaEvent_t const*>(events));
+}
+
+moe_status moe_layer_forward_host(const moe_shape* sh, const moe_bf16* x_host, const float* Wg, const moe_bf16* W1,
+                                  const moe_bf16* W3, const moe_bf16* W2, moe_bf16* y_host, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_bf16(Wg));
+  MOE_TRY(check_bf16(W1));
+  MOE_TRY(check_bf16(W3));
+  MOE_TRY(check_bf16(W2));
+  MOE_TRY(check_ws(sh, ws, ws_bytes));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  const Layout L = layout_of(sh);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t bytes = 2 * (size_t)sh->T * sh->d_model;
+  moe_bf16* xd = at<moe_bf16>(ws, L.x_stage);
+  moe_bf16* yd = at<moe_bf16>(ws, L.y_stage);
+  MOE_TRY(cuda_status(cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s)));
+  MOE_TRY(layer_forward_impl(sh, xd, Wg, W1, W3, W2, yd, nullptr, nullptr, ws, sms, s));
+  return cuda_status(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+moe_status moe_read_device_status(const void* ws, moe_stream_t stream) {
+  if (!ws || !aligned(ws, kAlign)) return MOE_ERR_WORKSPACE;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  return v == 0 ? MOE_OK : (moe_status)v;
+}
+
+const char* moe_status_string(moe_status st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported device or request";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// Internal host-side declarations shared by the kernels' launchers and the
+// C ABI (moe_api.cu).  Not part of the public interface.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+struct RouterArgs {
+  const uint16_t* x;   // [T, d] bf16
+  const float* Wg;     // [E, d]
+  float* logits;       // [T, E] or nullptr
+  int32_t* topk_idx;   // [T, k]
+  float* topk_w;       // [T, k]
+  float* topk_p;       // [T, k]
+  int32_t* counts;     // [E], zeroed by the launcher
+  int64_t T;
+  int32_t d, E, k;
+};
+cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s);
+
+struct PermuteArgs {
+  const uint16_t* x;         // [T, d]
+  const int32_t* topk_idx;   // [S]
+  const float* topk_p;       // [S] (capacity by probability only)
+  const int32_t* counts;     // [E]
+  int32_t* offsets;          // [E + 1]
+  int32_t* slot_pos;         // [S]
+  int32_t* perm_slot;        // [S]
+  uint16_t* x_perm;          // [S, d]
+  uint32_t* tile_state;      // [n_tiles * E] lookback words, zeroed by the launcher
+  uint32_t* ticket;          // tile ticket, zeroed by the launcher
+  uint64_t* thresh;          // [E] capacity thresholds
+  uint32_t* status;          // device status word
+  int64_t T;
+  int32_t d, E, k;
+  int64_t cap;               // < 0: dropless
+  int32_t policy;            // 0 by probability, 1 by token order
+};
+constexpr int kPermuteTile = 64;  // slots per permutation tile
+int64_t permute_tiles(int64_t S);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+
+// Expert GEMMs.  The tensor maps are encoded on the host per call.
+struct ExpertGemmArgs {
+  const int32_t* offsets;   // [E + 1]
+  const uint16_t* x_perm;   // [S, d]
+  const uint16_t* W1;       // [E, f, d]
+  const uint16_t* W3;       // [E, f, d]
+  const uint16_t* W2;       // [E, d, f]
+  uint16_t* h;              // [S, f]
+  uint16_t* y_perm;         // [S, d] (nullptr: leave split-K partials only)
+  float* partials;          // [splits, S, d] for the streaming variant
+  uint32_t* status;
+  int64_t S;
+  int32_t d, f, E;
+  int32_t variant;          // 1 tiled, 2 streaming
+  int32_t stream_bn;        // streaming variant: token tile (16..128)
+  int32_t splits;           // streaming variant: split-K count of the down projection
+  int num_sms;
+  cudaEvent_t between;      // recorded after the first GEMM if not null
+};
+// Streaming-variant parameters chosen from host-known sizes.
+void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,
+                   int32_t* splits);
+cudaError_t launch_expert_gemms(const ExpertGemmArgs& a, cudaStream_t s);
+
+struct CombineArgs {
+  const uint16_t* y_perm;   // [S, d] bf16, or nullptr when reading partials
+  const float* partials;    // [splits, S, d] fp32 (if y_perm == nullptr)
+  int32_t splits;
+  int64_t part_stride;      // elements between splits
+  const int32_t* slot_pos;  // [S]
+  const float* topk_w;      // [S]
+  uint16_t* y;              // [T, d]
+  int64_t T;
+  int32_t d, k;
+};
+cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
+
+// y_perm[r] = bf16(sum_s partials[s][r]) for r < offsets[E].
+cudaError_t launch_splitk_reduce(const float* partials, int32_t splits, int64_t part_stride,
+                                 const int32_t* offsets, int32_t E, uint16_t* y_perm, int64_t S,
+                                 int32_t d, int num_sms, cudaStream_t s);
+
+// Driver entry point for tensor-map encoding (resolved once through the runtime).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+}  // namespace moe

@@ -1,0 +1,235 @@
+// Capacity selection and grouping of slots by expert.
+//
+// Source: "How Mixtral 8x7B uses mixture of experts", sections "The
+// architecture in one diagram" (batch tokens by expert, run the experts,
+// scatter back) and "Routing without auxiliary loss" (capacity factor; the
+// excess slots of an expert are dropped; slots are sorted by router
+// probability per expert).
+//
+// capacity_select_kernel (capacity mode, drop by probability): one block per
+//   expert finds, by an 8-pass MSB-first radix select over 64-bit keys
+//   key = (bits of p as float) << 32 | (0xFFFFFFFF - t),
+//   the cap-th largest key of the expert's slots.  Keys are unique (a token
+//   routes to an expert at most once), so exactly cap slots satisfy
+//   key >= threshold.  Experts with at most cap slots get threshold 0.
+//
+// permute_kernel: a single-pass scan with decoupled look-back.  Each block
+//   takes a tile of kPermuteTile consecutive slots in ticket order, ranks its
+//   eligible slots per expert (warp match + popc, then across warps), publishes
+//   the tile's per-expert aggregate, and one thread per expert walks back over
+//   the predecessors' published words (flag in the top 2 bits: 1 = aggregate,
+//   2 = inclusive prefix) until it meets an inclusive prefix.  The row of a
+//   kept slot is offsets[e] + (eligible slots of e before it).  All of the
+//   block's warps then copy the kept tokens' rows of x into x_perm with
+//   16-byte vector loads and stores.
+#include <cstdint>
+
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+constexpr int kPermuteThreads = 256;
+constexpr int kPermuteWarpsSlots = kPermuteTile / 32;  // warps that rank slots
+constexpr uint32_t kFlagAgg = 1u << 30;
+constexpr uint32_t kFlagIncl = 2u << 30;
+constexpr uint32_t kValueMask = (1u << 30) - 1;
+
+int64_t permute_tiles(int64_t S) { return (S + kPermuteTile - 1) / kPermuteTile; }
+
+__device__ __forceinline__ uint64_t slot_key(float p, int64_t t) {
+  return ((uint64_t)__float_as_uint(p) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)t);
+}
+
+__global__ void __launch_bounds__(256) capacity_select_kernel(const int32_t* __restrict__ idx,
+                                                              const float* __restrict__ p,
+                                                              const int32_t* __restrict__ counts,
+                                                              uint64_t* __restrict__ thresh,
+                                                              int64_t S, int32_t k, int64_t cap) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint64_t s_prefix;
+  __shared__ int64_t s_need;
+  const int e = blockIdx.x;
+  const int64_t cnt = counts[e];
+  if (cnt <= cap) {
+    if (threadIdx.x == 0) thresh[e] = 0;  // every slot qualifies
+    return;
+  }
+  if (cap == 0) {
+    if (threadIdx.x == 0) thresh[e] = ~0ull;  // no key reaches it (keys < 2^63)
+    return;
+  }
+  if (threadIdx.x == 0) {
+    s_prefix = 0;
+    s_need = cap;
+  }
+  uint64_t mask = 0;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const uint64_t prefix = s_prefix;
+    for (int64_t s = threadIdx.x; s < S; s += blockDim.x) {
+      if (idx[s] != e) continue;
+      const uint64_t key = slot_key(p[s], s / k);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int64_t need = s_need, cum = 0;
+      int b = 255;
+      for (; b > 0; --b) {
+        if (cum + hist[b] >= need) break;
+        cum += hist[b];
+      }
+      s_need = need - cum;
+      s_prefix = prefix | ((uint64_t)b << shift);
+    }
+    mask |= 0xFFull << shift;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) thresh[e] = s_prefix;
+}
+
+__global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a) {
+  __shared__ int32_t s_off[33];
+  __shared__ int32_t s_wcnt[kPermuteWarpsSlots][32];
+  __shared__ int32_t s_wpre[kPermuteWarpsSlots][32];
+  __shared__ int32_t s_excl[32];
+  __shared__ int32_t s_tile;
+  __shared__ int32_t s_nkept;
+  __shared__ int32_t s_row[kPermuteTile];
+  __shared__ int32_t s_tok[kPermuteTile];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = a.E, k = a.k;
+  const int64_t S = a.T * k;
+  if (tid == 0) {
+    s_tile = (int32_t)atomicAdd(a.ticket, 1u);
+    s_nkept = 0;
+    int32_t acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = acc;
+      int32_t c = a.counts[e];
+      if (a.cap >= 0 && c > a.cap) c = (int32_t)a.cap;
+      acc += c;
+    }
+    s_off[E] = acc;
+  }
+  if (tid < kPermuteWarpsSlots * 32) s_wcnt[tid >> 5][tid & 31] = 0;
+  __syncthreads();
+  const int64_t tile = s_tile;
+  if (tile == 0 && tid <= E) a.offsets[tid] = s_off[tid];
+
+  // ---- rank eligible slots of this tile per expert
+  const bool ranker = tid < kPermuteTile;
+  const int64_t s = tile * kPermuteTile + tid;
+  int e = -1;
+  bool elig = false;
+  if (ranker && s < S) {
+    e = a.topk_idx[s];
+    elig = true;
+    if (a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
+  }
+  int rank_w = 0;
+  if (ranker) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, elig ? e : -1);
+    rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (elig && rank_w == 0) s_wcnt[warp][e] = __popc(peers);
+  }
+  __syncthreads();
+  if (tid < E) {
+    int32_t run = 0;
+    for (int w = 0; w < kPermuteWarpsSlots; ++w) {
+      s_wpre[w][tid] = run;
+      run += s_wcnt[w][tid];
+    }
+    // ---- decoupled look-back for expert `tid`
+    const uint32_t agg = (uint32_t)run;
+    uint32_t* words = a.tile_state;
+    int32_t excl = 0;
+    if (tile == 0) {
+      st_release_u32(&words[tid], kFlagIncl | agg);
+    } else {
+      st_release_u32(&words[tile * E + tid], kFlagAgg | agg);
+      int64_t pred = tile - 1;
+      uint64_t t0 = 0;
+      bool timed_out = false;
+      while (pred >= 0) {
+        const uint32_t v = ld_acquire_u32(&words[pred * E + tid]);
+        const uint32_t flag = v & ~kValueMask;
+        if (flag == 0) {
+          if (t0 == 0) t0 = globaltimer_ns();
+          else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            timed_out = true;
+            break;
+          }
+          continue;
+        }
+        t0 = 0;
+        excl += (int32_t)(v & kValueMask);
+        if (flag == kFlagIncl) break;
+        --pred;
+      }
+      if (timed_out) record_status(a.status, kStatusTimeout);
+      st_release_u32(&words[tile * E + tid], kFlagIncl | ((uint32_t)excl + agg));
+    }
+    s_excl[tid] = excl;
+  }
+  __syncthreads();
+
+  // ---- rows of the tile's slots
+  if (ranker && s < S) {
+    int32_t row = -1;
+    if (elig) {
+      const int32_t rank = s_excl[e] + s_wpre[warp][e] + rank_w;
+      const bool kept = !(a.cap >= 0 && a.policy == 1 && rank >= a.cap);
+      if (kept) {
+        row = s_off[e] + rank;
+        a.perm_slot[row] = (int32_t)s;
+        const int q = atomicAdd(&s_nkept, 1);
+        s_row[q] = row;
+        s_tok[q] = (int32_t)(s / k);
+      }
+    }
+    a.slot_pos[s] = row;
+  }
+  __syncthreads();
+
+  // ---- gather the kept tokens' rows (16-byte vectors, all warps)
+  const int nkept = s_nkept;
+  const int nvec = a.d >> 3;
+  const int nwarps = blockDim.x >> 5;
+  for (int i = warp; i < nkept; i += nwarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + (int64_t)s_tok[i] * a.d);
+    uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (int64_t)s_row[i] * a.d);
+    int v = lane;
+    for (; v + 224 < nvec; v += 256) {
+      uint4 r[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] = __ldg(src + v + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) dst[v + 32 * u] = r[u];
+    }
+    for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
+  const int64_t S = a.T * a.k;
+  const int64_t tiles = permute_tiles(S);
+  cudaError_t err = cudaMemsetAsync(a.tile_state, 0, sizeof(uint32_t) * tiles * a.E, s);
+  if (err != cudaSuccess) return err;
+  err = cudaMemsetAsync(a.ticket, 0, sizeof(uint32_t), s);
+  if (err != cudaSuccess) return err;
+  if (a.cap >= 0 && a.policy == 0) {
+    capacity_select_kernel<<<a.E, 256, 0, s>>>(a.topk_idx, a.topk_p, a.counts, a.thresh, S, a.k,
+                                               a.cap);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  permute_kernel<<<(unsigned)tiles, kPermuteThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,65 @@
+"""Convenience holder of one MoE layer's device weights and workspace.
+
+PyTorch provides the device memory and the stream; the computation is the
+library's ``moe_layer_forward`` (or ``moe_layer_forward_host``).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+
+class MoELayer:
+    """Weights on one CUDA device: Wg [E, d] fp32, W1/W3 [E, f, d] and
+    W2 [E, d, f] bf16 (row-major, contiguous)."""
+
+    def __init__(self, Wg: torch.Tensor, W1: torch.Tensor, W3: torch.Tensor, W2: torch.Tensor, k: int = 2,
+                 capacity_factor: float = 0.0, drop_policy: int = _lib.MOE_DROP_BY_PROB,
+                 gemm_variant: int = _lib.MOE_VARIANT_AUTO):
+        for t, dt in ((Wg, torch.float32), (W1, torch.bfloat16), (W3, torch.bfloat16), (W2, torch.bfloat16)):
+            if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+                raise ValueError("weights must be contiguous CUDA tensors (Wg fp32, W1/W3/W2 bf16)")
+        self.Wg, self.W1, self.W3, self.W2 = Wg, W1, W3, W2
+        self.E, self.f, self.d = W1.shape
+        self.k = k
+        self.capacity_factor = capacity_factor
+        self.drop_policy = drop_policy
+        self.gemm_variant = gemm_variant
+        self._ws = {}
+
+    def shape(self, T: int) -> _lib.moe_shape:
+        return _lib.make_shape(T, self.d, self.f, self.E, self.k, self.capacity_factor, self.drop_policy,
+                               self.gemm_variant)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        ws = self._ws.get(T)
+        if ws is None:
+            n = _lib.moe_workspace_size(self.shape(T))
+            if n == 0:
+                raise ValueError("invalid layer shape")
+            ws = torch.empty(n, dtype=torch.uint8, device=self.W1.device)
+            self._ws[T] = ws
+        return ws
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, topk_idx: torch.Tensor | None = None,
+                counts: torch.Tensor | None = None) -> torch.Tensor:
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.d), dtype=torch.bfloat16, device=x.device)
+        ws = self.workspace(T)
+        st = _lib.moe_layer_forward(self.shape(T), x, self.Wg, self.W1, self.W3, self.W2, y, topk_idx, counts,
+                                    ws, ws.numel())
+        _lib.check(st, "moe_layer_forward")
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
+        """x_host, y_host: page-locked CPU bf16 [T, d]; queued on the stream."""
+        T = x_host.shape[0]
+        ws = self.workspace(T)
+        st = _lib.moe_layer_forward_host(self.shape(T), x_host, self.Wg, self.W1, self.W3, self.W2, y_host, ws,
+                                         ws.numel(), stream)
+        _lib.check(st, "moe_layer_forward_host")
+
+    def device_status(self, T: int) -> int:
+        return _lib.moe_read_device_status(self.workspace(T))
