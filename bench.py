@@ -295,7 +295,11 @@ def run_ours(args):
     Wd = (None, to_dev_bf16(W1, torch), to_dev_bf16(W3, torch), to_dev_bf16(W2, torch))
 
     props = torch.cuda.get_device_properties(local)
-    sampler = ClockSampler(getattr(props, "pci_bus_id", None) if hasattr(props, "pci_bus_id") else None)
+    pci = None
+    if hasattr(props, "pci_bus_id"):
+        pci = f"{int(getattr(props, 'pci_domain_id', 0)):08x}:{int(props.pci_bus_id):02x}:" \
+              f"{int(getattr(props, 'pci_device_id', 0)):02x}.0"
+    sampler = ClockSampler(pci)
     sampler.start()
 
     out = {}

@@ -36,7 +36,7 @@
  *     time.
  *   - Arguments are checked before any work is queued; on failure the call
  *     returns the status and queues nothing.  T == 0 is a no-op (MOE_OK).
- *     Requirements: 1 <= E <= 32, 1 <= k <= min(E, 4), d_model and d_ff
+ *     Requirements: 1 <= E <= 32, 1 <= k <= min(E, 8), d_model and d_ff
  *     multiples of 64 in [64, 65536], T * k < 2^30, finite capacity_factor,
  *     bf16 / fp32 matrices 16-byte aligned, int32 arrays 4-byte aligned,
  *     workspace 256-byte aligned and at least moe_workspace_size() bytes.

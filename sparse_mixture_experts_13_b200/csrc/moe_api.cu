@@ -26,7 +26,7 @@ moe_status check_shape(const moe_shape* sh) {
   if (!sh) return MOE_ERR_INVALID_ARG;
   if (sh->T < 0) return MOE_ERR_INVALID_ARG;
   if (sh->E < 1 || sh->E > 32) return MOE_ERR_INVALID_ARG;
-  if (sh->k < 1 || sh->k > 4 || sh->k > sh->E) return MOE_ERR_INVALID_ARG;
+  if (sh->k < 1 || sh->k > 8 || sh->k > sh->E) return MOE_ERR_INVALID_ARG;
   if (sh->d_model < 64 || sh->d_model > 65536 || sh->d_model % 64) return MOE_ERR_INVALID_ARG;
   if (sh->d_ff < 64 || sh->d_ff > 65536 || sh->d_ff % 64) return MOE_ERR_INVALID_ARG;
   if (sh->T * (int64_t)sh->k >= ((int64_t)1 << 30)) return MOE_ERR_INVALID_ARG;
@@ -147,14 +147,14 @@ moe_status check_bf16(const void* p) { return (p && aligned(p, 16)) ? MOE_OK : M
 moe_status check_i32(const void* p) { return (p && aligned(p, 4)) ? MOE_OK : MOE_ERR_INVALID_ARG; }
 
 moe_status run_router(const moe_shape* sh, const moe_bf16* x, const float* Wg, float* logits, int32_t* idx, float* w,
-                      float* p, int32_t* counts, int num_sms, cudaStream_t s) {
+                      float* p, int32_t* counts, int num_sms, cudaStream_t s, bool counts_zeroed) {
   RouterArgs a{x, Wg, logits, idx, w, p, counts, sh->T, sh->d_model, sh->E, sh->k};
-  return cuda_status(launch_router(a, num_sms, s));
+  return cuda_status(launch_router(a, num_sms, s, counts_zeroed));
 }
 
 moe_status run_permute(const moe_shape* sh, const Layout& L, const moe_bf16* x, const int32_t* idx, const float* p,
                        const int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_slot,
-                       moe_bf16* x_perm, void* ws, cudaStream_t s) {
+                       moe_bf16* x_perm, void* ws, cudaStream_t s, bool state_zeroed) {
   PermuteArgs a{};
   a.x = x;
   a.topk_idx = idx;
@@ -174,7 +174,7 @@ moe_status run_permute(const moe_shape* sh, const Layout& L, const moe_bf16* x, 
   a.k = sh->k;
   a.cap = capacity_of(sh);
   a.policy = sh->drop_policy;
-  return cuda_status(launch_permute(a, s));
+  return cuda_status(launch_permute(a, s, state_zeroed));
 }
 
 moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_perm, const int32_t* offsets,
@@ -224,7 +224,7 @@ moe_status moe_router_topk(const moe_shape* sh, const moe_bf16* x, const float* 
   if (logits && !aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
   int sms = 0;
   MOE_TRY(check_device(&sms));
-  return run_router(sh, x, Wg, logits, topk_idx, topk_w, topk_p, counts, sms, (cudaStream_t)stream);
+  return run_router(sh, x, Wg, logits, topk_idx, topk_w, topk_p, counts, sms, (cudaStream_t)stream, false);
 }
 
 moe_status moe_permute(const moe_shape* sh, const moe_bf16* x, const int32_t* topk_idx, const float* topk_p,
@@ -246,7 +246,7 @@ moe_status moe_permute(const moe_shape* sh, const moe_bf16* x, const int32_t* to
   const Layout L = layout_of(sh);
   cudaStream_t s = (cudaStream_t)stream;
   MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 8, s)));  // status word and tile ticket
-  return run_permute(sh, L, x, topk_idx, topk_p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s);
+  return run_permute(sh, L, x, topk_idx, topk_p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s, false);
 }
 
 moe_status moe_grouped_swiglu(const moe_shape* sh, const moe_bf16* x_perm, const int32_t* offsets,
@@ -319,9 +319,10 @@ static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, con
   auto mark = [&](int i) { return ev ? cuda_status(cudaEventRecord(ev[i], s)) : MOE_OK; };
   MOE_TRY(mark(0));
   MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.ctrl_end, s)));
-  MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s));
+  // one clear of the control region (status, ticket, counts, look-back words)
+  MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s, true));
   MOE_TRY(mark(1));
-  MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s));
+  MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s, true));
   MOE_TRY(mark(2));
   MOE_TRY(run_gemms(sh, L, x_perm, offsets, W1, W3, W2, h, y_perm, ws, sms, s, ev ? ev[3] : nullptr));
   MOE_TRY(mark(4));

@@ -15,11 +15,11 @@ struct RouterArgs {
   int32_t* topk_idx;   // [T, k]
   float* topk_w;       // [T, k]
   float* topk_p;       // [T, k]
-  int32_t* counts;     // [E], zeroed by the launcher
+  int32_t* counts;     // [E], zeroed by the launcher unless the caller did
   int64_t T;
   int32_t d, E, k;
 };
-cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s, bool counts_zeroed);
 
 struct PermuteArgs {
   const uint16_t* x;         // [T, d]
@@ -41,7 +41,8 @@ struct PermuteArgs {
 };
 constexpr int kPermuteTile = 64;  // slots per permutation tile
 int64_t permute_tiles(int64_t S);
-cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+// state_zeroed: tile_state and ticket were cleared by the caller.
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zeroed);
 
 // Expert GEMMs.  The tensor maps are encoded on the host per call.
 struct ExpertGemmArgs {

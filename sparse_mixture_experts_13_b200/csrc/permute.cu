@@ -215,13 +215,16 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
   }
 }
 
-cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zeroed) {
   const int64_t S = a.T * a.k;
   const int64_t tiles = permute_tiles(S);
-  cudaError_t err = cudaMemsetAsync(a.tile_state, 0, sizeof(uint32_t) * tiles * a.E, s);
-  if (err != cudaSuccess) return err;
-  err = cudaMemsetAsync(a.ticket, 0, sizeof(uint32_t), s);
-  if (err != cudaSuccess) return err;
+  cudaError_t err = cudaSuccess;
+  if (!state_zeroed) {
+    err = cudaMemsetAsync(a.tile_state, 0, sizeof(uint32_t) * tiles * a.E, s);
+    if (err != cudaSuccess) return err;
+    err = cudaMemsetAsync(a.ticket, 0, sizeof(uint32_t), s);
+    if (err != cudaSuccess) return err;
+  }
   if (a.cap >= 0 && a.policy == 0) {
     capacity_select_kernel<<<a.E, 256, 0, s>>>(a.topk_idx, a.topk_p, a.counts, a.thresh, S, a.k,
                                                a.cap);

@@ -44,7 +44,7 @@ def test_status_strings(moe):
     assert moe.status_string(99) == "unknown status"
 
 
-@pytest.mark.parametrize("kw", [dict(E=0), dict(E=33), dict(k=0), dict(k=5, E=8), dict(k=3, E=2),
+@pytest.mark.parametrize("kw", [dict(E=0), dict(E=33), dict(k=0), dict(k=9, E=16), dict(k=3, E=2),
                                 dict(d_model=100), dict(d_model=0), dict(d_ff=448 + 32), dict(T=-1),
                                 dict(capacity_factor=float("nan")), dict(capacity_factor=float("inf")),
                                 dict(drop_policy=2), dict(gemm_variant=3), dict(T=1 << 29, k=2)])

@@ -233,3 +233,11 @@ def test_skew_T8192_capacity(o, policy):
 @pytest.mark.parametrize("T", [1, 8, 64, 512, 32768])
 def test_sweep(o, T):
     check_everything(o, full_workload("sweep", T=T), 0, rows=16)
+
+
+@pytest.mark.parametrize("E", [8, 16, 32])
+def test_router_many_tokens(o, E):
+    """More than 512 tokens take the shared-memory router (several tokens
+    per warp); cover it for each expert-count template."""
+    wl = synth.Workload(f"many{E}", 700, 128, 192, E=E, k=2, seed=E).generate()
+    check_everything(o, wl, 1)
