@@ -82,10 +82,12 @@ typedef enum {
 
 /* Expert-GEMM schedule.  Both compute the same function. */
 typedef enum {
-  MOE_VARIANT_AUTO = 0,   /* STREAM when T <= 128, TILED otherwise */
-  MOE_VARIANT_TILED = 1,  /* 128-token x 256-column tiles: compute-bound sizes */
-  MOE_VARIANT_STREAM = 2  /* weights as the 128-row MMA operand, tokens as N,
-                             split-K on the down projection: weight-streaming sizes */
+  MOE_VARIANT_AUTO = 0,         /* STREAM when T <= 128, TILED otherwise */
+  MOE_VARIANT_TILED = 1,        /* 256-token x 256-column tiles on CTA pairs
+                                   (one MMA over two SMs): compute-bound sizes */
+  MOE_VARIANT_STREAM = 2,       /* weights as the 128-row MMA operand, tokens as N,
+                                   split-K on the down projection: weight-streaming sizes */
+  MOE_VARIANT_TILED_SINGLE = 3  /* 128-token x 256-column tiles on single CTAs */
 } moe_gemm_variant;
 
 typedef struct {

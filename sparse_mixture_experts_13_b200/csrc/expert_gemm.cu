@@ -414,6 +414,304 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA pairs
+//
+// The token-rich schedule on CTA pairs: a cluster of two CTAs on neighbouring
+// SMs shares each tcgen05.mma (cta_group::2, M = 256 over the pair).  The
+// weights are the M operand and the tokens the N operand, so the MMA's N can
+// shrink to an expert's last, partial block of tokens (a multiple of 16)
+// instead of computing a full tile of rows that belong to the next expert.
+// A pair tile is 256 weight rows x up to 256 tokens:
+//   GEMM1: CTA r holds W1 rows n0 + 64r .. +63 over the same W3 rows (its
+//          accumulator lanes l and l + 64 are the two projections of output
+//          column n0 + 64r + l), so SiLU * mul pairs lanes inside one CTA;
+//   GEMM2: CTA r holds W2 rows n0 + 128r .. +127 (accumulator lane l is
+//          output column n0 + 128r + l).
+// The tokens are split between the CTAs: CTA r loads token rows
+// row0 + r*N/2 .. and the accumulator column n of both CTAs is token row0 + n.
+// Each CTA moves 32 KB per stage (16 KB of weights, 16 KB of tokens) for the
+// MMA work of 48 KB on a single-CTA 128 x 256 tile; six stages fit.  The
+// leader CTA (rank 0) counts both CTAs' bytes on its full barrier, issues the
+// MMAs and commits to the barriers of both CTAs; each CTA's epilogue reads its
+// own accumulator and arrives on the leader's accumulator-empty barrier.
+constexpr int kPairStages = 6;
+constexpr int kPairHalf = 128 * BK * 2;              // one 128-row operand half
+constexpr int kPairStageBytes = 2 * kPairHalf;       // A half + B half per CTA
+// Epilogue transpose buffers: two 16-token x 128-lane fp32 tiles, rows padded
+// to 132 floats.
+constexpr int kXsStride = 132;
+constexpr int kPairXbuf = 2 * 16 * kXsStride * 4;
+constexpr int kPairBarBytes = (2 * kPairStages + 5) * 8;
+constexpr int kPairSmem = 1024 + kPairStages * kPairStageBytes + kPairXbuf + kPairBarBytes;
+static_assert(kPairSmem <= 227 * 1024, "shared memory");
+
+struct PairTile {
+  int32_t e, row0, m_valid, n_mma, n0;
+};
+
+template <int EPI>
+__device__ __forceinline__ void decode_pair_tile(const GemmParams& p, const int32_t* s_off, const int32_t* s_base,
+                                                 int32_t tile, PairTile& t) {
+  int e = 0;
+  while (e < p.E - 1 && tile >= s_base[e + 1]) ++e;
+  const int32_t local = tile - s_base[e];
+  const int32_t M_e = s_off[e + 1] - s_off[e];
+  const int32_t tb_count = (M_e + 255) / 256;
+  const int32_t tb = local % tb_count, wb = local / tb_count;
+  t.e = e;
+  t.row0 = s_off[e] + tb * 256;
+  t.m_valid = min(256, M_e - tb * 256);
+  t.n_mma = (t.m_valid + 15) & ~15;
+  t.n0 = wb * (EPI == EPI_TILED_SWIGLU ? 128 : 256);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_wa,
+                            const __grid_constant__ CUtensorMap map_wb, GemmParams p) {
+  constexpr int STAGES = kPairStages;
+  constexpr int ACC_COLS = 256;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_epi_fail;
+  __shared__ int32_t s_off[33];
+  __shared__ int32_t s_base[33];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kPairHalf;
+  float* xbuf = reinterpret_cast<float*>(sB + STAGES * kPairHalf);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kPairHalf + kPairXbuf);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* tfull_bar = bars + 2 * STAGES;
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+
+  if (tid == 0) {
+    tma_prefetch_desc(&map_act);
+    tma_prefetch_desc(&map_wa);
+    if (EPI == EPI_TILED_SWIGLU) tma_prefetch_desc(&map_wb);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 8);
+    }
+    mbar_init(drain_bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&s_tmem, 512);
+    tmem_relinquish_pair();
+  }
+  if (tid == 64) {
+    s_abort = 0;
+    s_epi_fail = 0;
+    int32_t acc = 0;
+    s_base[0] = 0;
+    for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+    for (int e = 0; e < p.E; ++e) {
+      const int32_t M_e = s_off[e + 1] - s_off[e];
+      acc += (M_e > 0) ? ((M_e + 255) / 256) * p.n_blocks : 0;
+      s_base[e + 1] = acc;
+    }
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = s_tmem;
+  const int32_t total = s_base[p.E];
+  const int32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int32_t tile = pair; tile < total && ok; tile += npairs) {
+        PairTile t;
+        decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
+        const int32_t tok_row = t.row0 + (int32_t)rank * (t.n_mma >> 1);
+        for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &s_abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = map_to_rank(smem_u32(&full_bar[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kPairStageBytes);
+          uint8_t* a_dst = sA + stage * kPairHalf;
+          uint8_t* b_dst = sB + stage * kPairHalf;
+          const int32_t kx = kb * BK;
+          if (EPI == EPI_TILED_SWIGLU) {
+            const int32_t wrow = t.n0 + (int32_t)rank * 64;
+            tma_load_3d_pair(&map_wa, full_leader, a_dst, kx, wrow, t.e);
+            tma_load_3d_pair(&map_wb, full_leader, a_dst + 64 * 128, kx, wrow, t.e);
+          } else {
+            tma_load_3d_pair(&map_wa, full_leader, a_dst, kx, t.n0 + (int32_t)rank * 128, t.e);
+          }
+          tma_load_2d_pair(&map_act, full_leader, b_dst, kx, tok_row);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        s_abort = 1;
+      }
+      if (rank == 0) {
+        // The leader's full barriers count both CTAs' bytes: wait for every
+        // stage this pair filled before the pair may exit.
+        for (int s = 0; s < STAGES; ++s) {
+          if (s < issued) {
+            const int64_t uses = (issued - s + STAGES - 1) / STAGES;
+            mbar_wait(&full_bar[s], (uint32_t)((uses - 1) & 1), nullptr);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------ MMA issuer (leader only)
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t iter = 0;
+      bool ok = true;
+      for (int32_t tile = pair; tile < total && ok; tile += npairs, ++iter) {
+        PairTile t;
+        decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
+        const uint32_t idesc = make_idesc_bf16(256, t.n_mma);
+        const uint32_t acc = iter & 1, use = iter >> 1;
+        if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * kPairHalf);
+          const uint32_t b_addr = smem_u32(sB + stage * kPairHalf);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(d_tmem, make_sdesc_sw128(a_addr + kk * 32), make_sdesc_sw128(b_addr + kk * 32), idesc,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t eb = smem_u32(&empty_bar[stage]);
+          umma_commit_pair(map_to_rank(eb, 0));
+          umma_commit_pair(map_to_rank(eb, 1));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        const uint32_t fb = smem_u32(&tfull_bar[acc]);
+        umma_commit_pair(map_to_rank(fb, 0));
+        umma_commit_pair(map_to_rank(fb, 1));
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        s_abort = 1;
+      }
+      umma_commit_pair(map_to_rank(smem_u32(drain_bar), 0));
+      mbar_wait(drain_bar, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // accumulator lane
+    const int tid_epi = tid - 64;  // 0..127
+    uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
+    uint32_t iter = 0;
+    for (int32_t tile = pair; tile < total; tile += npairs, ++iter) {
+      PairTile t;
+      decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
+      const uint32_t acc = iter & 1, use = iter >> 1;
+      if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort)) s_epi_fail = 1;
+      named_bar_sync(2, 128);
+      if (s_epi_fail) {
+        record_status(p.status, kStatusTimeout);
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_acc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+      // Per chunk of 16 tokens: every thread writes its lane's 16 values into
+      // xs[token][lane], then thread i produces 8 consecutive outputs of token
+      // i / 8 and stores them as one 16-byte vector.
+      const int jt = tid_epi >> 3, g = tid_epi & 7;
+#pragma unroll 1
+      for (int c0 = 0, buf = 0; c0 < t.n_mma; c0 += 16, buf ^= 1) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(t_acc + c0, v);
+        tmem_ld_wait();
+        float* xs = xbuf + buf * 16 * kXsStride;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xs[j * kXsStride + r] = __uint_as_float(v[j]);
+        named_bar_sync(1, 128);
+        const int n = c0 + jt;
+        const float* row = xs + jt * kXsStride;
+        if (EPI == EPI_TILED_SWIGLU) {
+          // lanes 0..63: W1 projection of columns n0 + 64*rank + lane;
+          // lanes 64..127: the W3 projection of the same columns.
+          const int32_t col = t.n0 + (int32_t)rank * 64 + 8 * g;
+          if (n < t.m_valid && col < p.n_out) {
+            const float4 a0 = *reinterpret_cast<const float4*>(row + 8 * g);
+            const float4 a1 = *reinterpret_cast<const float4*>(row + 8 * g + 4);
+            const float4 b0 = *reinterpret_cast<const float4*>(row + 64 + 8 * g);
+            const float4 b1 = *reinterpret_cast<const float4*>(row + 64 + 8 * g + 4);
+            uint4 o;
+            o.x = pack_bf16x2(silu_f32(a0.x) * b0.x, silu_f32(a0.y) * b0.y);
+            o.y = pack_bf16x2(silu_f32(a0.z) * b0.z, silu_f32(a0.w) * b0.w);
+            o.z = pack_bf16x2(silu_f32(a1.x) * b1.x, silu_f32(a1.y) * b1.y);
+            o.w = pack_bf16x2(silu_f32(a1.z) * b1.z, silu_f32(a1.w) * b1.w);
+            *reinterpret_cast<uint4*>(out + (int64_t)(t.row0 + n) * p.out_ld + col) = o;
+          }
+        } else {
+          // lane l: output column n0 + 128*rank + l; thread i writes 16 columns.
+          const int32_t col = t.n0 + (int32_t)rank * 128 + 16 * g;
+          if (n < t.m_valid && col < p.n_out) {
+            const float4 q0 = *reinterpret_cast<const float4*>(row + 16 * g);
+            const float4 q1 = *reinterpret_cast<const float4*>(row + 16 * g + 4);
+            const float4 q2 = *reinterpret_cast<const float4*>(row + 16 * g + 8);
+            const float4 q3 = *reinterpret_cast<const float4*>(row + 16 * g + 12);
+            uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(t.row0 + n) * p.out_ld + col);
+            dst[0] = make_uint4(pack_bf16x2(q0.x, q0.y), pack_bf16x2(q0.z, q0.w), pack_bf16x2(q1.x, q1.y),
+                                pack_bf16x2(q1.z, q1.w));
+            dst[1] = make_uint4(pack_bf16x2(q2.x, q2.y), pack_bf16x2(q2.z, q2.w), pack_bf16x2(q3.x, q3.y),
+                                pack_bf16x2(q3.z, q3.w));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty_bar[acc]), 0));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 EncodeTiledFn get_encode_tiled() {
@@ -463,6 +761,32 @@ static cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& wa, con
   if (err != cudaSuccess) return err;
   expert_gemm_kernel<EPI, BN><<<num_sms, kGemmThreads, C::SMEM_BYTES, s>>>(act, wa, wb, p);
   return cudaGetLastError();
+}
+
+template <int EPI>
+static cudaError_t launch_pair(const CUtensorMap& act, const CUtensorMap& wa, const CUtensorMap& wb,
+                               const GemmParams& p, int num_sms, cudaStream_t s) {
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPairSmem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // As many pairs as can be resident at once (persistent kernel).
+  cfg.gridDim = dim3((unsigned)(num_sms & ~1), 1, 1);
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, expert_gemm_pair_kernel<EPI>, &cfg) == cudaSuccess && clusters > 0 &&
+      2 * clusters < (int)cfg.gridDim.x)
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+  return cudaLaunchKernelEx(&cfg, expert_gemm_pair_kernel<EPI>, act, wa, wb, p);
 }
 
 void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
@@ -532,9 +856,10 @@ static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
 
 static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   CUtensorMap mx, mw1, mw3, mh, mw2;
-  if (!encode_2d(&mx, a.x_perm, a.S, a.d, 128) || !encode_3d(&mw1, a.W1, a.E, a.f, a.d, 128) ||
-      !encode_3d(&mw3, a.W3, a.E, a.f, a.d, 128) || !encode_2d(&mh, a.h, a.S, a.f, 128) ||
-      !encode_3d(&mw2, a.W2, a.E, a.d, a.f, 256))
+  const int wbox = a.pair ? 64 : 128;
+  if (!encode_2d(&mx, a.x_perm, a.S, a.d, 128) || !encode_3d(&mw1, a.W1, a.E, a.f, a.d, wbox) ||
+      !encode_3d(&mw3, a.W3, a.E, a.f, a.d, wbox) || !encode_2d(&mh, a.h, a.S, a.f, 128) ||
+      !encode_3d(&mw2, a.W2, a.E, a.d, a.f, a.pair ? 128 : 256))
     return cudaErrorInvalidValue;
   GemmParams p1{};
   p1.offsets = a.offsets;
@@ -547,7 +872,8 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.n_blocks = (a.f + 127) / 128;
   p1.splits = 1;
   p1.kb_per_split = p1.num_kb;
-  cudaError_t err = launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s);
+  cudaError_t err = a.pair ? launch_pair<EPI_TILED_SWIGLU>(mx, mw1, mw3, p1, a.num_sms, s)
+                           : launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s);
   if (err != cudaSuccess) return err;
   if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
   GemmParams p2{};
@@ -561,7 +887,8 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p2.n_blocks = (a.d + 255) / 256;
   p2.splits = 1;
   p2.kb_per_split = p2.num_kb;
-  return launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s);
+  return a.pair ? launch_pair<EPI_TILED_STORE>(mh, mw2, mw2, p2, a.num_sms, s)
+                : launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s);
 }
 
 cudaError_t launch_expert_gemms(const ExpertGemmArgs& a, cudaStream_t s) {

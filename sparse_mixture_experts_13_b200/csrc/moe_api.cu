@@ -32,7 +32,7 @@ moe_status check_shape(const moe_shape* sh) {
   if (sh->T * (int64_t)sh->k >= ((int64_t)1 << 30)) return MOE_ERR_INVALID_ARG;
   if (!std::isfinite(sh->capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (sh->drop_policy != MOE_DROP_BY_PROB && sh->drop_policy != MOE_DROP_BY_ORDER) return MOE_ERR_INVALID_ARG;
-  if (sh->gemm_variant < MOE_VARIANT_AUTO || sh->gemm_variant > MOE_VARIANT_STREAM) return MOE_ERR_INVALID_ARG;
+  if (sh->gemm_variant < MOE_VARIANT_AUTO || sh->gemm_variant > MOE_VARIANT_TILED_SINGLE) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -194,7 +194,8 @@ moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_per
   a.d = sh->d_model;
   a.f = sh->d_ff;
   a.E = sh->E;
-  a.variant = L.variant;
+  a.variant = L.variant == MOE_VARIANT_STREAM ? 2 : 1;
+  a.pair = L.variant == MOE_VARIANT_TILED;
   a.stream_bn = L.bn;
   a.splits = L.splits;
   a.num_sms = num_sms;

@@ -62,6 +62,7 @@ struct ExpertGemmArgs {
   int32_t splits;           // streaming variant: split-K count of the down projection
   int num_sms;
   cudaEvent_t between;      // recorded after the first GEMM if not null
+  bool pair;                // tiled variant: CTA-pair (cta_group::2) kernels
 };
 // Streaming-variant parameters chosen from host-known sizes.
 void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,

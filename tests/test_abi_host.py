@@ -47,7 +47,7 @@ def test_status_strings(moe):
 @pytest.mark.parametrize("kw", [dict(E=0), dict(E=33), dict(k=0), dict(k=9, E=16), dict(k=3, E=2),
                                 dict(d_model=100), dict(d_model=0), dict(d_ff=448 + 32), dict(T=-1),
                                 dict(capacity_factor=float("nan")), dict(capacity_factor=float("inf")),
-                                dict(drop_policy=2), dict(gemm_variant=3), dict(T=1 << 29, k=2)])
+                                dict(drop_policy=2), dict(gemm_variant=4), dict(T=1 << 29, k=2)])
 def test_invalid_shapes(moe, kw):
     base = dict(T=64, d_model=128, d_ff=448, E=8, k=2)
     base.update(kw)

@@ -19,8 +19,8 @@ if torch.cuda.is_available():
 else:  # collected on CPU hosts, never run there
     moe = H = None
 
-VARIANTS = [0, 1, 2]
-VNAME = {0: "auto", 1: "tiled", 2: "stream"}
+VARIANTS = [0, 1, 2, 3]
+VNAME = {0: "auto", 1: "tiled", 2: "stream", 3: "tiled1"}
 
 
 @pytest.fixture(scope="module")
@@ -119,7 +119,7 @@ def test_tiny(o, variant):
     check_everything(o, wl, variant)
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VNAME[v])
+@pytest.mark.parametrize("variant", [1, 2, 3], ids=lambda v: VNAME[v])
 @pytest.mark.parametrize("policy", [0, 1], ids=["by_prob", "by_order"])
 @pytest.mark.parametrize("cf", [0.5, 1.0, 1.25])
 def test_tiny_capacity(o, variant, policy, cf):
@@ -128,14 +128,14 @@ def test_tiny_capacity(o, variant, policy, cf):
 
 
 @pytest.mark.parametrize("E,k", [(4, 1), (16, 2), (8, 3), (32, 4), (8, 8), (1, 1)])
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VNAME[v])
+@pytest.mark.parametrize("variant", [1, 2, 3], ids=lambda v: VNAME[v])
 def test_expert_counts(o, E, k, variant):
     wl = synth.Workload(f"E{E}k{k}", 96, 128, 256, E=E, k=k, seed=3).generate()
     check_everything(o, wl, variant)
 
 
 @pytest.mark.parametrize("T", [1, 2, 3, 17, 127, 128, 129, 300])
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VNAME[v])
+@pytest.mark.parametrize("variant", [1, 2, 3], ids=lambda v: VNAME[v])
 def test_ragged_T(o, T, variant):
     wl = synth.Workload(f"T{T}", T, 192, 320, seed=T).generate()
     check_everything(o, wl, variant)
@@ -147,7 +147,7 @@ def test_T_zero_is_noop():
     assert moe.moe_router_topk(sh, None, None, None, None, None, None, None) == moe.MOE_OK
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VNAME[v])
+@pytest.mark.parametrize("variant", [1, 2, 3], ids=lambda v: VNAME[v])
 def test_one_expert_takes_every_token(o, variant):
     """Expert 5 is every token's first choice; several experts stay empty."""
     wl = synth.Workload("hot5", 200, 128, 256, seed=5).generate()
@@ -157,7 +157,7 @@ def test_one_expert_takes_every_token(o, variant):
     check_everything(o, wl, variant)
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VNAME[v])
+@pytest.mark.parametrize("variant", [1, 2, 3], ids=lambda v: VNAME[v])
 def test_exact_logit_ties(o, variant):
     """Experts 2 and 3 have identical router rows, so their logits tie
     exactly; the smaller index must win, as in the oracle."""
@@ -179,7 +179,7 @@ def test_zero_input_ties():
     and the output is exactly zero."""
     wl = synth.Workload("zeros", 40, 128, 256).generate()
     wl.x[:] = 0
-    for variant in (1, 2):
+    for variant in (1, 2, 3):
         g = H.run_stages(H.Device(wl), variant)
         assert np.all(g["idx"].cpu().numpy().reshape(40, 2) == [0, 1])
         assert np.all(g["w"].cpu().numpy() == 0.5)
@@ -188,12 +188,12 @@ def test_zero_input_ties():
 
 def test_capacity_zero_and_huge(o):
     wl = synth.Workload("cap0", 4, 128, 256, capacity_factor=0.5).generate()   # cap = 0
-    for variant in (1, 2):
+    for variant in (1, 2, 3):
         lay = H.run_layer(H.Device(wl), variant)
         assert not lay["y"].any()
     base = synth.Workload("nocap", 100, 128, 256, seed=2).generate()
     huge = synth.Workload("hugecap", 100, 128, 256, seed=2, capacity_factor=1e9).generate()
-    for variant in (1, 2):
+    for variant in (1, 2, 3):
         a = H.run_layer(H.Device(base), variant)["y"]
         b = H.run_layer(H.Device(huge), variant)["y"]
         assert np.array_equal(a, b)
@@ -204,8 +204,9 @@ def test_variants_agree_closely():
     the order of fp32 accumulation)."""
     wl = synth.Workload("v", 100, 256, 512, seed=11).generate()
     a = H.bf16_f64(H.run_layer(H.Device(wl), 1)["y"])
-    b = H.bf16_f64(H.run_layer(H.Device(wl), 2)["y"])
-    assert H.rel_fro(a, b) < 5e-3
+    for v in (2, 3):
+        b = H.bf16_f64(H.run_layer(H.Device(wl), v)["y"])
+        assert H.rel_fro(a, b) < 5e-3
 
 
 # ------------------------------------------------------- Mixtral-shaped sizes
@@ -215,7 +216,7 @@ def test_decode_T16(o, variant):
     check_everything(o, full_workload("decode"), variant, rows=16)
 
 
-@pytest.mark.parametrize("variant", [0, 2], ids=lambda v: VNAME[v])
+@pytest.mark.parametrize("variant", [0, 2, 3], ids=lambda v: VNAME[v])
 def test_prefill_T4096(o, variant):
     check_everything(o, full_workload("prefill"), variant, rows=24)
 
