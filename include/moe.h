@@ -139,6 +139,30 @@ MOE_API moe_status moe_permute(const moe_shape *shape, const moe_bf16 *x, const 
                        int32_t *slot_pos, int32_t *perm_slot, moe_bf16 *x_perm, void *ws,
                        size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute without a workspace argument, for callers that cannot
+ * allocate device memory: for example an inference-engine plug-in whose
+ * enqueue step is handed only input/output pointers and a stream, or a
+ * latency-critical loop that must never enter the CUDA allocator (cudaMalloc
+ * can synchronise the device and take unbounded time).  The pages have no
+ * counterpart of this entry point; it exists for such callers.
+ *
+ * Same arguments (minus ws / ws_bytes), results and ordering as moe_permute.
+ * Its scratch (look-back words, tile ticket, capacity thresholds) is a fixed
+ * array of about 129 KB in the library's device memory, present on every GPU
+ * that loads the library until the process exits.  Limits: T * k <= 65536
+ * slots (E <= 32 as everywhere); larger shapes return MOE_ERR_UNSUPPORTED and
+ * queue nothing.  The first call on each device looks up the array's device
+ * address (a host-side runtime query, no allocation); make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents: each call clears what must start at zero, and calls
+ * whose work overlaps on the GPU (other streams, other host threads) race on
+ * it, so serialise them.  A device-side look-back wait that gives up is
+ * recorded only in that shared array and is not reported to the caller. */
+MOE_API moe_status moe_permute_noalloc(const moe_shape *shape, const moe_bf16 *x,
+                                       const int32_t *topk_idx, const float *topk_p,
+                                       const int32_t *counts, int32_t *offsets, int32_t *slot_pos,
+                                       int32_t *perm_slot, moe_bf16 *x_perm, moe_stream_t stream);
+
 /* Grouped SwiGLU experts on tensor cores.  Source: "Mixtral", "MoE Layer"
  * (MixtralExpert.forward) and "SwiGLU Experts".  For each expert e and row r
  * in offsets[e] .. offsets[e+1]-1:

@@ -20,7 +20,7 @@ MOE_DROP_BY_PROB, MOE_DROP_BY_ORDER = 0, 1
 MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM, MOE_VARIANT_TILED_SINGLE = 0, 1, 2, 3
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
-            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_read_device_status", "moe_status_string")
+            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc", "moe_read_device_status", "moe_status_string")
 
 
 class MoeError(RuntimeError):
@@ -56,6 +56,7 @@ def lib():
         L.moe_workspace_size.restype = sz
         L.moe_router_topk.argtypes = [S, P, P, P, P, P, P, P, P]
         L.moe_permute.argtypes = [S, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_permute_noalloc.argtypes = [S, P, P, P, P, P, P, P, P, P]
         L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.moe_combine.argtypes = [S, P, P, P, P, P]
         L.moe_layer_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, sz, P]
@@ -109,6 +110,13 @@ def moe_permute(shape, x, topk_idx, topk_p, counts, offsets, slot_pos, perm_slot
                 stream=None) -> int:
     return lib().moe_permute(ctypes.byref(shape), _p(x), _p(topk_idx), _p(topk_p), _p(counts), _p(offsets),
                              _p(slot_pos), _p(perm_slot), _p(x_perm), _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_permute_noalloc(shape, x, topk_idx, topk_p, counts, offsets, slot_pos, perm_slot, x_perm,
+                        stream=None) -> int:
+    """moe_permute with its scratch in a fixed device array (no workspace)."""
+    return lib().moe_permute_noalloc(ctypes.byref(shape), _p(x), _p(topk_idx), _p(topk_p), _p(counts), _p(offsets),
+                                     _p(slot_pos), _p(perm_slot), _p(x_perm), _stream(stream))
 
 
 def moe_grouped_swiglu(shape, x_perm, offsets, W1, W3, W2, h, y_perm, ws, ws_bytes, stream=None) -> int:

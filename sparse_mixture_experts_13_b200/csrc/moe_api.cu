@@ -205,6 +205,12 @@ moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_per
 
 }  // namespace
 
+namespace moe {
+moe_status api_check_shape(const moe_shape* sh) { return check_shape(sh); }
+moe_status api_check_device(int* num_sms) { return check_device(num_sms); }
+int64_t api_capacity(const moe_shape* sh) { return capacity_of(sh); }
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_size(const moe_shape* shape) {

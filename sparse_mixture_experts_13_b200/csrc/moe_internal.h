@@ -6,7 +6,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "moe.h"
+
 namespace moe {
+
+// Argument checks shared by the C entry points (defined in moe_api.cu).
+moe_status api_check_shape(const moe_shape* sh);
+moe_status api_check_device(int* num_sms);
+int64_t api_capacity(const moe_shape* sh);  // -1: dropless
 
 struct RouterArgs {
   const uint16_t* x;   // [T, d] bf16

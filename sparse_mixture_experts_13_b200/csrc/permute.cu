@@ -235,4 +235,75 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zero
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for moe_permute_noalloc (callers that cannot allocate device
+// memory).  Layout: [0, 256) status word and tile ticket; [256, 512) capacity
+// thresholds of up to 32 experts; then the look-back words of up to
+// kNoAllocMaxSlots / kPermuteTile tiles x 32 experts.  In host code the
+// symbol is only a stand-in, never a device address: the address is looked up
+// once per device with cudaGetSymbolAddress and passed to the kernels.
+constexpr int64_t kNoAllocMaxSlots = 65536;
+constexpr size_t kNoAllocHeader = 512;
+constexpr size_t kNoAllocBytes = kNoAllocHeader + sizeof(uint32_t) * (kNoAllocMaxSlots / kPermuteTile) * 32;
+static __device__ __align__(256) unsigned char g_permute_scratch[kNoAllocBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+void* g_scratch_addr[kNoAllocMaxDevices];  // device address per device, once looked up
+}  // namespace
+
 }  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const moe_shape* sh, const moe_bf16* x, const int32_t* topk_idx,
+                                          const float* topk_p, const int32_t* counts, int32_t* offsets,
+                                          int32_t* slot_pos, int32_t* perm_slot, moe_bf16* x_perm,
+                                          moe_stream_t stream) {
+  using namespace moe;
+  moe_status st = api_check_shape(sh);
+  if (st != MOE_OK) return st;
+  if (sh->T == 0) return MOE_OK;
+  const int64_t S = sh->T * sh->k;
+  if (S > kNoAllocMaxSlots) return MOE_ERR_UNSUPPORTED;
+  auto al = [](const void* p, uintptr_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+  if (!al(x, 16) || !al(x_perm, 16) || !al(topk_idx, 4) || !al(counts, 4) || !al(offsets, 4) || !al(slot_pos, 4) ||
+      !al(perm_slot, 4))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t cap = api_capacity(sh);
+  if (cap >= 0 && sh->drop_policy == MOE_DROP_BY_PROB && !al(topk_p, 4)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  st = api_check_device(&sms);
+  if (st != MOE_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_CUDA;
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_permute_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
+    g_scratch_addr[dev] = ptr;
+  }
+  unsigned char* base = static_cast<unsigned char*>(g_scratch_addr[dev]);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t words = (size_t)permute_tiles(S) * sh->E;
+  // status word, ticket and the look-back words this call uses start at zero
+  if (cudaMemsetAsync(base, 0, 8, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(base + kNoAllocHeader, 0, sizeof(uint32_t) * words, s) != cudaSuccess) return MOE_ERR_CUDA;
+  PermuteArgs a{};
+  a.x = x;
+  a.topk_idx = topk_idx;
+  a.topk_p = topk_p;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.slot_pos = slot_pos;
+  a.perm_slot = perm_slot;
+  a.x_perm = x_perm;
+  a.status = reinterpret_cast<uint32_t*>(base);
+  a.ticket = reinterpret_cast<uint32_t*>(base + 4);
+  a.thresh = reinterpret_cast<uint64_t*>(base + 256);
+  a.tile_state = reinterpret_cast<uint32_t*>(base + kNoAllocHeader);
+  a.T = sh->T;
+  a.d = sh->d_model;
+  a.E = sh->E;
+  a.k = sh->k;
+  a.cap = cap;
+  a.policy = sh->drop_policy;
+  return launch_permute(a, s, true) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
