@@ -62,6 +62,7 @@ struct GemmParams {
   int32_t n_blocks;     // weight blocks per expert
   int32_t splits;       // K splits (STREAM partial), else 1
   int32_t kb_per_split;
+  uint32_t* tile_counter;  // CTA-pair kernels: next tile id (zero before the launch)
 };
 
 __host__ __device__ constexpr bool epi_is_tiled(int epi) { return epi <= EPI_TILED_STORE; }
@@ -434,6 +435,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // leader CTA (rank 0) counts both CTAs' bytes on its full barrier, issues the
 // MMAs and commits to the barriers of both CTAs; each CTA's epilogue reads its
 // own accumulator and arrives on the leader's accumulator-empty barrier.
+// Tiles are handed out dynamically: the leader's producer takes the next tile
+// id from a global counter and publishes it to every role of both CTAs
+// through a small ring in shared memory.  Tile ids enumerate every full
+// 256-token block first (expert, weight block, token block), then the partial
+// last blocks (expert, weight block), so the small tiles even out the end of
+// the run.
 constexpr int kPairStages = 6;
 constexpr int kPairHalf = 128 * BK * 2;              // one 128-row operand half
 constexpr int kPairStageBytes = 2 * kPairHalf;       // A half + B half per CTA
@@ -441,7 +448,9 @@ constexpr int kPairStageBytes = 2 * kPairHalf;       // A half + B half per CTA
 // to 132 floats.
 constexpr int kXsStride = 132;
 constexpr int kPairXbuf = 2 * 16 * kXsStride * 4;
-constexpr int kPairBarBytes = (2 * kPairStages + 5) * 8;
+constexpr int kRing = 4;            // tile ids in flight
+constexpr int kRingConsumers = 10;  // leader MMA + 4 epilogue warps per CTA + peer producer
+constexpr int kPairBarBytes = (2 * kPairStages + 5 + 2 * kRing) * 8;
 constexpr int kPairSmem = 1024 + kPairStages * kPairStageBytes + kPairXbuf + kPairBarBytes;
 static_assert(kPairSmem <= 227 * 1024, "shared memory");
 
@@ -450,17 +459,28 @@ struct PairTile {
 };
 
 template <int EPI>
-__device__ __forceinline__ void decode_pair_tile(const GemmParams& p, const int32_t* s_off, const int32_t* s_base,
-                                                 int32_t tile, PairTile& t) {
+__device__ __forceinline__ void decode_pair_tile(const GemmParams& p, const int32_t* s_off, const int32_t* s_full,
+                                                 const int32_t* s_tail, int32_t tile, PairTile& t) {
+  const int32_t F = s_full[p.E];
   int e = 0;
-  while (e < p.E - 1 && tile >= s_base[e + 1]) ++e;
-  const int32_t local = tile - s_base[e];
-  const int32_t M_e = s_off[e + 1] - s_off[e];
-  const int32_t tb_count = (M_e + 255) / 256;
-  const int32_t tb = local % tb_count, wb = local / tb_count;
+  int32_t tb, wb;
+  if (tile < F) {
+    while (e < p.E - 1 && tile >= s_full[e + 1]) ++e;
+    const int32_t nfull = (s_off[e + 1] - s_off[e]) >> 8;
+    const int32_t local = tile - s_full[e];
+    tb = local % nfull;
+    wb = local / nfull;
+    t.m_valid = 256;
+  } else {
+    const int32_t j = tile - F;
+    while (e < p.E - 1 && j >= s_tail[e + 1]) ++e;
+    const int32_t M_e = s_off[e + 1] - s_off[e];
+    wb = j - s_tail[e];
+    tb = M_e >> 8;
+    t.m_valid = M_e & 255;
+  }
   t.e = e;
   t.row0 = s_off[e] + tb * 256;
-  t.m_valid = min(256, M_e - tb * 256);
   t.n_mma = (t.m_valid + 15) & ~15;
   t.n0 = wb * (EPI == EPI_TILED_SWIGLU ? 128 : 256);
 }
@@ -476,7 +496,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __shared__ int s_abort;
   __shared__ int s_epi_fail;
   __shared__ int32_t s_off[33];
-  __shared__ int32_t s_base[33];
+  __shared__ int32_t s_full[33];
+  __shared__ int32_t s_tail[33];
+  __shared__ volatile int32_t s_ring[kRing];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -488,6 +510,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull_bar = bars + 2 * STAGES;
   uint64_t* tempty_bar = bars + 2 * STAGES + 2;
   uint64_t* drain_bar = bars + 2 * STAGES + 4;
+  uint64_t* ring_full = bars + 2 * STAGES + 5;
+  uint64_t* ring_empty = ring_full + kRing;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
@@ -505,6 +529,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty_bar[a], 8);
     }
     mbar_init(drain_bar, 1);
+    for (int q = 0; q < kRing; ++q) {
+      mbar_init(&ring_full[q], 1);
+      mbar_init(&ring_empty[q], kRingConsumers);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -514,21 +542,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (tid == 64) {
     s_abort = 0;
     s_epi_fail = 0;
-    int32_t acc = 0;
-    s_base[0] = 0;
+    int32_t nf = 0, nt = 0;
+    s_full[0] = 0;
+    s_tail[0] = 0;
     for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
     for (int e = 0; e < p.E; ++e) {
       const int32_t M_e = s_off[e + 1] - s_off[e];
-      acc += (M_e > 0) ? ((M_e + 255) / 256) * p.n_blocks : 0;
-      s_base[e + 1] = acc;
+      nf += (M_e >> 8) * p.n_blocks;
+      nt += ((M_e & 255) != 0) ? p.n_blocks : 0;
+      s_full[e + 1] = nf;
+      s_tail[e + 1] = nt;
     }
   }
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = s_tmem;
-  const int32_t total = s_base[p.E];
-  const int32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int32_t total = s_full[p.E] + s_tail[p.E];
+
+  // Tile-id ring.  The leader's producer publishes; everyone else consumes
+  // and releases the slot on the leader right after reading it.
+  auto ring_get = [&](uint32_t n, int32_t& tile) -> bool {
+    const uint32_t q = n % kRing, par = (n / kRing) & 1;
+    if (!mbar_wait_cluster(&ring_full[q], par, &s_abort)) return false;
+    tile = s_ring[q];
+    mbar_arrive_cluster(map_to_rank(smem_u32(&ring_empty[q]), 0));
+    return true;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -537,12 +577,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int32_t tile = pair; tile < total && ok; tile += npairs) {
+      for (uint32_t n = 0; ok; ++n) {
+        int32_t tile;
+        if (rank == 0) {
+          const uint32_t q = n % kRing, par = (n / kRing) & 1;
+          if (!mbar_wait_cluster(&ring_empty[q], par ^ 1, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tile = (int32_t)atomicAdd(p.tile_counter, 1u);
+          if (tile >= total) tile = -1;
+          s_ring[q] = tile;
+          st_cluster_u32(map_to_rank(smem_u32((const void*)&s_ring[q]), 1), (uint32_t)tile);
+          mbar_arrive(&ring_full[q]);
+          mbar_arrive_cluster(map_to_rank(smem_u32(&ring_full[q]), 1));
+        } else if (!ring_get(n, tile)) {
+          ok = false;
+          break;
+        }
+        if (tile < 0) break;
         PairTile t;
-        decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
+        decode_pair_tile<EPI>(p, s_off, s_full, s_tail, tile, t);
         const int32_t tok_row = t.row0 + (int32_t)rank * (t.n_mma >> 1);
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &s_abort)) {
+          if (!mbar_wait_cluster(&empty_bar[stage], phase ^ 1, &s_abort)) {
             ok = false;
             break;
           }
@@ -576,7 +634,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
           if (s < issued) {
             const int64_t uses = (issued - s + STAGES - 1) / STAGES;
-            mbar_wait(&full_bar[s], (uint32_t)((uses - 1) & 1), nullptr);
+            mbar_wait_cluster(&full_bar[s], (uint32_t)((uses - 1) & 1), nullptr);
           }
         }
       }
@@ -586,21 +644,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // ------------------------------------------------ MMA issuer (leader only)
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t iter = 0;
       bool ok = true;
-      for (int32_t tile = pair; tile < total && ok; tile += npairs, ++iter) {
+      for (uint32_t n = 0; ok; ++n) {
+        int32_t tile;
+        if (!ring_get(n, tile)) {
+          ok = false;
+          break;
+        }
+        if (tile < 0) break;
         PairTile t;
-        decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
+        decode_pair_tile<EPI>(p, s_off, s_full, s_tail, tile, t);
         const uint32_t idesc = make_idesc_bf16(256, t.n_mma);
-        const uint32_t acc = iter & 1, use = iter >> 1;
-        if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) {
+        const uint32_t acc = n & 1, use = n >> 1;
+        if (!mbar_wait_cluster(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, &s_abort)) {
+          if (!mbar_wait_cluster(&full_bar[stage], phase, &s_abort)) {
             ok = false;
             break;
           }
@@ -629,7 +692,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         s_abort = 1;
       }
       umma_commit_pair(map_to_rank(smem_u32(drain_bar), 0));
-      mbar_wait(drain_bar, 0, nullptr);
+      mbar_wait_cluster(drain_bar, 0, nullptr);
     }
   } else {
     // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
@@ -637,18 +700,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = q * 32 + lane;  // accumulator lane
     const int tid_epi = tid - 64;  // 0..127
     uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
-    uint32_t iter = 0;
-    for (int32_t tile = pair; tile < total; tile += npairs, ++iter) {
-      PairTile t;
-      decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
-      const uint32_t acc = iter & 1, use = iter >> 1;
-      if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort)) s_epi_fail = 1;
+    for (uint32_t n = 0;; ++n) {
+      int32_t tile = -1;
+      if (lane == 0 && !ring_get(n, tile)) s_epi_fail = 1;
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      const uint32_t acc = n & 1, use = n >> 1;
+      // The four epilogue warps decide together whether to go on, so that a
+      // wait that gives up in one warp never leaves the others at a barrier.
+      if (tile >= 0 && !mbar_wait_cluster(&tfull_bar[acc], use & 1, &s_abort)) s_epi_fail = 1;
       named_bar_sync(2, 128);
       if (s_epi_fail) {
         record_status(p.status, kStatusTimeout);
         s_abort = 1;
         break;
       }
+      if (tile < 0) break;
+      PairTile t;
+      decode_pair_tile<EPI>(p, s_off, s_full, s_tail, tile, t);
       tc_fence_after();
       const uint32_t t_acc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
       // Per chunk of 16 tokens: every thread writes its lane's 16 values into
@@ -872,6 +940,7 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.n_blocks = (a.f + 127) / 128;
   p1.splits = 1;
   p1.kb_per_split = p1.num_kb;
+  p1.tile_counter = a.tile_counters;
   cudaError_t err = a.pair ? launch_pair<EPI_TILED_SWIGLU>(mx, mw1, mw3, p1, a.num_sms, s)
                            : launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s);
   if (err != cudaSuccess) return err;
@@ -887,6 +956,7 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p2.n_blocks = (a.d + 255) / 256;
   p2.splits = 1;
   p2.kb_per_split = p2.num_kb;
+  p2.tile_counter = a.tile_counters + 1;
   return a.pair ? launch_pair<EPI_TILED_STORE>(mh, mw2, mw2, p2, a.num_sms, s)
                 : launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s);
 }

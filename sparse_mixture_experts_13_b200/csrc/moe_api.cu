@@ -47,7 +47,8 @@ int variant_of(const moe_shape* sh) {
 }
 
 struct Layout {
-  // control region, cleared at the start of moe_layer_forward
+  // control region, cleared at the start of moe_layer_forward: status word,
+  // tile ticket, two GEMM tile counters, counts, look-back words
   size_t status, ticket, counts, tile_state, ctrl_end;
   size_t thresh, partials, topk_idx, topk_w, topk_p, offsets, slot_pos, perm_slot, x_perm, h, y_perm,
       x_stage, y_stage, total;
@@ -66,7 +67,7 @@ Layout layout_of(const moe_shape* sh) {
   size_t o = 0;
   L.status = o;
   L.ticket = o + 4;
-  o = align_up(o + 8);
+  o = align_up(o + 16);
   L.counts = o;
   o = align_up(o + 4 * E);
   L.tile_state = o;
@@ -200,6 +201,7 @@ moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_per
   a.splits = L.splits;
   a.num_sms = num_sms;
   a.between = between;
+  a.tile_counters = at<uint32_t>(ws, L.status) + 2;  // words 2 and 3 of the control header
   return cuda_status(launch_expert_gemms(a, s));
 }
 
@@ -273,7 +275,7 @@ moe_status moe_grouped_swiglu(const moe_shape* sh, const moe_bf16* x_perm, const
   MOE_TRY(check_device(&sms));
   const Layout L = layout_of(sh);
   cudaStream_t s = (cudaStream_t)stream;
-  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 8, s)));
+  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 16, s)));  // status, ticket, GEMM tile counters
   MOE_TRY(run_gemms(sh, L, x_perm, offsets, W1, W3, W2, h, y_perm, ws, sms, s));
   if (L.variant == MOE_VARIANT_STREAM) {
     const int64_t S = sh->T * sh->k;

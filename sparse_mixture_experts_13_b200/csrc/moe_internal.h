@@ -70,6 +70,7 @@ struct ExpertGemmArgs {
   int num_sms;
   cudaEvent_t between;      // recorded after the first GEMM if not null
   bool pair;                // tiled variant: CTA-pair (cta_group::2) kernels
+  uint32_t* tile_counters;  // [2] tile counters of the pair kernels, zeroed by the caller
 };
 // Streaming-variant parameters chosen from host-known sizes.
 void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,
