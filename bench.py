@@ -115,6 +115,20 @@ def to_dev_bf16(a, torch):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
+def max_over_ranks(value: float, torch, dist=None, device="cuda") -> float:
+    """The largest `value` over all ranks (every rank gets it)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch per step."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def time_steps(fn, steps, torch, dist=None):
     """K steps between a barrier + synchronize on both sides; CUDA events on
     the current stream; max over ranks."""
@@ -129,12 +143,7 @@ def time_steps(fn, steps, torch, dist=None):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(start.elapsed_time(end), torch, dist)
 
 
 class Run:
@@ -263,7 +272,7 @@ def run_reference(args):
                 warmup=args.warmup, ms_per_step=per_token * wl.T * 1e3, higher_is_better=True, scaling="weak",
                 vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
                 config=dict(workload=workload_desc(wl), T=wl.T, d_model=wl.d, d_ff=wl.f, E=wl.E, k=wl.k,
-                            l2="CPU run"),
+                            parallelism="single process on the host cores", l2="CPU run"),
                 cpu_baseline=dict(value=value, unit="tokens/s", cores=o.num_threads(), kind="oracle",
                                   sample=sample),
                 e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
@@ -330,14 +339,14 @@ def run_ours(args):
         peak_tf = peaks["bf16_sustained"] if long_run else peaks["bf16"]
         achieved_tf = g1_flops / (g1_ms * 1e-3) / 1e12
         tr = traffic_record("expert_gemm_kernel<0,256>", "prefill")
-        value = world * wl.T / (p["ms"] * 1e-3)
+        value = weak_scaling_value(world, wl.T, p["ms"])
 
         q = out["decode"]
         wq = q["wl"]
         g1_bytes_dec = q["touched"] * 2 * d * f * 2 + q["N"] * d * 2 + q["N"] * f * 2
         layer_bytes_dec = q["touched"] * expert_bytes(d, f) + wq.T * d * 2 * 2 + E * d * 4 + 2 * q["N"] * f * 2
         dec_g1_ms = q["stages"]["gemm1_swiglu"]
-        dec = dict(workload=workload_desc(wq), value=world * wq.T / (q["ms"] * 1e-3), unit="tokens/s",
+        dec = dict(workload=workload_desc(wq), value=weak_scaling_value(world, wq.T, q["ms"]), unit="tokens/s",
                    ms_per_step=q["ms"], stage_ms=q["stages"],
                    layer_gbs=layer_bytes_dec / (q["ms"] * 1e-3) / 1e9,
                    layer_frac_hbm=layer_bytes_dec / (q["ms"] * 1e-3) / 1e9 / peaks["hbm"],
@@ -346,7 +355,7 @@ def run_ours(args):
                                  frac=g1_bytes_dec / (dec_g1_ms * 1e-3) / 1e9 / peaks["hbm"],
                                  traffic=traffic_record("expert_gemm_kernel<2,16>", "decode"),
                                  peak_source=f"{peaks['source']} HBM copy bandwidth"),
-                   e2e=dict(value=world * wq.T / (q["e2e_ms"] * 1e-3), unit="tokens/s",
+                   e2e=dict(value=weak_scaling_value(world, wq.T, q["e2e_ms"]), unit="tokens/s",
                             h2d_bytes_per_step=q["h2d"], d2h_bytes_per_step=q["d2h"]),
                    experts_touched=q["touched"])
         kernels_per_step = 5 + (1 if (wl.capacity_factor > 0 and wl.drop_policy == 0) else 0)
@@ -364,7 +373,7 @@ def run_ours(args):
                           peak=peak_tf, unit="TFLOP/s", frac=achieved_tf / peak_tf, traffic=tr,
                           peak_source=f"{peaks['source']} bf16 dense "
                                       f"({'sustained' if long_run else 'burst'})"),
-            e2e=dict(value=world * wl.T / (p["e2e_ms"] * 1e-3), unit="tokens/s", h2d_bytes_per_step=p["h2d"],
+            e2e=dict(value=weak_scaling_value(world, wl.T, p["e2e_ms"]), unit="tokens/s", h2d_bytes_per_step=p["h2d"],
                      d2h_bytes_per_step=p["d2h"]),
             gpu_launches=kernels_per_step * args.steps,
             clocks=clocks,

@@ -216,6 +216,18 @@ MOE_API moe_status moe_layer_forward_host(const moe_shape *shape, const moe_bf16
                                   const moe_bf16 *W2, moe_bf16 *y_host, void *ws,
                                   size_t ws_bytes, moe_stream_t stream);
 
+/* Self-test of the failure reporting of the device-side waits (the pages
+ * have no counterpart).  Queues one small kernel that makes an mbarrier wait
+ * and a look-back wait -- the two kinds of bounded wait in the layer's
+ * kernels -- give up after `limit_us` microseconds (1 .. 10^7) on a barrier
+ * and a word that nothing completes.  Each records MOE_ERR_TIMEOUT in the
+ * status word at the start of `ws` (the first 256 bytes are used) and returns;
+ * nothing traps, and the context stays usable.  Afterwards
+ * moe_read_device_status(ws) returns MOE_ERR_TIMEOUT and the 32-bit word at
+ * byte offset 128 of `ws` holds 2 (the number of waits that gave up). */
+MOE_API moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, uint32_t limit_us,
+                                             moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the device status word of the last
  * call that used this workspace (MOE_OK or MOE_ERR_TIMEOUT), or
  * MOE_ERR_CUDA if the stream reports an error. */

@@ -20,7 +20,7 @@ MOE_DROP_BY_PROB, MOE_DROP_BY_ORDER = 0, 1
 MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM, MOE_VARIANT_TILED_SINGLE = 0, 1, 2, 3
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
-            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc", "moe_read_device_status", "moe_status_string")
+            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc", "moe_selftest_wait_timeout", "moe_read_device_status", "moe_status_string")
 
 
 class MoeError(RuntimeError):
@@ -63,6 +63,7 @@ def lib():
         L.moe_layer_forward_host.argtypes = [S, P, P, P, P, P, P, P, sz, P]
         L.moe_layer_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.moe_read_device_status.argtypes = [P, P]
+        L.moe_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_uint32, P]
         L.moe_status_string.argtypes = [st]
         L.moe_status_string.restype = ctypes.c_char_p
         for name in EXPORTED[1:-1]:
@@ -151,6 +152,10 @@ def moe_layer_forward_profiled(shape, x, Wg, W1, W3, W2, y, events, ws, ws_bytes
     arr = (ctypes.c_void_p * 6)(*handles)
     return lib().moe_layer_forward_profiled(ctypes.byref(shape), _p(x), _p(Wg), _p(W1), _p(W3), _p(W2), _p(y), arr,
                                             _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_selftest_wait_timeout(ws, ws_bytes, limit_us, stream=None) -> int:
+    return lib().moe_selftest_wait_timeout(_p(ws), int(ws_bytes), int(limit_us), _stream(stream))
 
 
 def moe_read_device_status(ws, stream=None) -> int:

@@ -433,14 +433,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // Each CTA moves 32 KB per stage (16 KB of weights, 16 KB of tokens) for the
 // MMA work of 48 KB on a single-CTA 128 x 256 tile; six stages fit.  The
 // leader CTA (rank 0) counts both CTAs' bytes on its full barrier, issues the
-// MMAs and commits to the barriers of both CTAs; each CTA's epilogue reads its
-// own accumulator and arrives on the leader's accumulator-empty barrier.
+// MMAs and commits to the barriers of both CTAs with one multicast commit;
+// each CTA's epilogue reads its own accumulator and arrives on the leader's
+// accumulator-empty barrier.
 // Tiles are handed out dynamically: the leader's producer takes the next tile
 // id from a global counter and publishes it to every role of both CTAs
-// through a small ring in shared memory.  Tile ids enumerate every full
-// 256-token block first (expert, weight block, token block), then the partial
-// last blocks (expert, weight block), so the small tiles even out the end of
-// the run.
+// through a small ring in shared memory.  Tile ids run over (expert, weight
+// block, token block), so the pairs working at the same time share each
+// weight block through L2 and it is read from HBM once.
 constexpr int kPairStages = 6;
 constexpr int kPairHalf = 128 * BK * 2;              // one 128-row operand half
 constexpr int kPairStageBytes = 2 * kPairHalf;       // A half + B half per CTA
@@ -459,28 +459,17 @@ struct PairTile {
 };
 
 template <int EPI>
-__device__ __forceinline__ void decode_pair_tile(const GemmParams& p, const int32_t* s_off, const int32_t* s_full,
-                                                 const int32_t* s_tail, int32_t tile, PairTile& t) {
-  const int32_t F = s_full[p.E];
+__device__ __forceinline__ void decode_pair_tile(const GemmParams& p, const int32_t* s_off, const int32_t* s_base,
+                                                 int32_t tile, PairTile& t) {
   int e = 0;
-  int32_t tb, wb;
-  if (tile < F) {
-    while (e < p.E - 1 && tile >= s_full[e + 1]) ++e;
-    const int32_t nfull = (s_off[e + 1] - s_off[e]) >> 8;
-    const int32_t local = tile - s_full[e];
-    tb = local % nfull;
-    wb = local / nfull;
-    t.m_valid = 256;
-  } else {
-    const int32_t j = tile - F;
-    while (e < p.E - 1 && j >= s_tail[e + 1]) ++e;
-    const int32_t M_e = s_off[e + 1] - s_off[e];
-    wb = j - s_tail[e];
-    tb = M_e >> 8;
-    t.m_valid = M_e & 255;
-  }
+  while (e < p.E - 1 && tile >= s_base[e + 1]) ++e;
+  const int32_t local = tile - s_base[e];
+  const int32_t M_e = s_off[e + 1] - s_off[e];
+  const int32_t tb_count = (M_e + 255) / 256;
+  const int32_t tb = local % tb_count, wb = local / tb_count;
   t.e = e;
   t.row0 = s_off[e] + tb * 256;
+  t.m_valid = min(256, M_e - tb * 256);
   t.n_mma = (t.m_valid + 15) & ~15;
   t.n0 = wb * (EPI == EPI_TILED_SWIGLU ? 128 : 256);
 }
@@ -496,8 +485,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __shared__ int s_abort;
   __shared__ int s_epi_fail;
   __shared__ int32_t s_off[33];
-  __shared__ int32_t s_full[33];
-  __shared__ int32_t s_tail[33];
+  __shared__ int32_t s_base[33];
   __shared__ volatile int32_t s_ring[kRing];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -542,23 +530,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (tid == 64) {
     s_abort = 0;
     s_epi_fail = 0;
-    int32_t nf = 0, nt = 0;
-    s_full[0] = 0;
-    s_tail[0] = 0;
+    int32_t acc = 0;
+    s_base[0] = 0;
     for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
     for (int e = 0; e < p.E; ++e) {
       const int32_t M_e = s_off[e + 1] - s_off[e];
-      nf += (M_e >> 8) * p.n_blocks;
-      nt += ((M_e & 255) != 0) ? p.n_blocks : 0;
-      s_full[e + 1] = nf;
-      s_tail[e + 1] = nt;
+      acc += (M_e > 0) ? ((M_e + 255) / 256) * p.n_blocks : 0;
+      s_base[e + 1] = acc;
     }
   }
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = s_tmem;
-  const int32_t total = s_full[p.E] + s_tail[p.E];
+  const int32_t total = s_base[p.E];
 
   // Tile-id ring.  The leader's producer publishes; everyone else consumes
   // and releases the slot on the leader right after reading it.
@@ -597,7 +582,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (tile < 0) break;
         PairTile t;
-        decode_pair_tile<EPI>(p, s_off, s_full, s_tail, tile, t);
+        decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
         const int32_t tok_row = t.row0 + (int32_t)rank * (t.n_mma >> 1);
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait_cluster(&empty_bar[stage], phase ^ 1, &s_abort)) {
@@ -653,7 +638,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (tile < 0) break;
         PairTile t;
-        decode_pair_tile<EPI>(p, s_off, s_full, s_tail, tile, t);
+        decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
         const uint32_t idesc = make_idesc_bf16(256, t.n_mma);
         const uint32_t acc = n & 1, use = n >> 1;
         if (!mbar_wait_cluster(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) {
@@ -674,18 +659,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16_pair(d_tmem, make_sdesc_sw128(a_addr + kk * 32), make_sdesc_sw128(b_addr + kk * 32), idesc,
                            (kb > 0 || kk > 0) ? 1u : 0u);
-          const uint32_t eb = smem_u32(&empty_bar[stage]);
-          umma_commit_pair(map_to_rank(eb, 0));
-          umma_commit_pair(map_to_rank(eb, 1));
+          umma_commit_pair_both(&empty_bar[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        const uint32_t fb = smem_u32(&tfull_bar[acc]);
-        umma_commit_pair(map_to_rank(fb, 0));
-        umma_commit_pair(map_to_rank(fb, 1));
+        umma_commit_pair_both(&tfull_bar[acc]);
       }
       if (!ok) {
         record_status(p.status, kStatusTimeout);
@@ -716,7 +697,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (tile < 0) break;
       PairTile t;
-      decode_pair_tile<EPI>(p, s_off, s_full, s_tail, tile, t);
+      decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
       tc_fence_after();
       const uint32_t t_acc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
       // Per chunk of 16 tokens: every thread writes its lane's 16 values into

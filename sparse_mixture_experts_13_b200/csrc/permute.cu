@@ -153,22 +153,15 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
     } else {
       st_release_u32(&words[tile * E + tid], kFlagAgg | agg);
       int64_t pred = tile - 1;
-      uint64_t t0 = 0;
       bool timed_out = false;
       while (pred >= 0) {
-        const uint32_t v = ld_acquire_u32(&words[pred * E + tid]);
-        const uint32_t flag = v & ~kValueMask;
-        if (flag == 0) {
-          if (t0 == 0) t0 = globaltimer_ns();
-          else if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            timed_out = true;
-            break;
-          }
-          continue;
+        uint32_t v;
+        if (!wait_published(&words[pred * E + tid], ~kValueMask, &v)) {
+          timed_out = true;
+          break;
         }
-        t0 = 0;
         excl += (int32_t)(v & kValueMask);
-        if (flag == kFlagIncl) break;
+        if ((v & ~kValueMask) == kFlagIncl) break;
         --pred;
       }
       if (timed_out) record_status(a.status, kStatusTimeout);

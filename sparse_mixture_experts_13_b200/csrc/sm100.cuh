@@ -66,7 +66,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 // Wait until the phase with the given parity has completed.  Returns false
 // if the time limit passed or *abort became non-zero first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile int* abort_flag) {
+                                          const volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -75,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (abort_flag && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -255,6 +256,27 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Spin until the global word has any of the bits in `flag_mask` set (another
+// block publishing it), returning the word in *v.  Returns false if the time
+// limit passed first.
+__device__ __forceinline__ bool wait_published(const uint32_t* word, uint32_t flag_mask, uint32_t* v,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  uint32_t x = ld_acquire_u32(word);
+  if (x & flag_mask) {
+    *v = x;
+    return true;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    x = ld_acquire_u32(word);
+    if (x & flag_mask) {
+      *v = x;
+      return true;
+    }
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 }  // namespace moe
 
 // ---------------------------------------------------------------- CTA pairs
@@ -331,6 +353,18 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive, once the pair MMAs issued so far by this thread have completed, on
+// the mbarrier at the same shared-memory offset in both CTAs of the pair
+// (one commit instruction signalling the two barriers).
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
       : "memory");
 }
 

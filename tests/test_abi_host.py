@@ -94,3 +94,12 @@ def test_valid_call_without_device_reports_cuda_error(moe):
     ok = 1 << 20
     st = moe.moe_router_topk(sh, ok, ok, None, ok, ok, ok, ok, 0)
     assert st in (moe.MOE_ERR_CUDA, moe.MOE_ERR_UNSUPPORTED)
+
+
+def test_selftest_arguments(moe):
+    ok = 1 << 20
+    assert moe.moe_selftest_wait_timeout(None, 1 << 16, 1000, 0) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_selftest_wait_timeout(ok + 16, 1 << 16, 1000, 0) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_selftest_wait_timeout(ok, 128, 1000, 0) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_selftest_wait_timeout(ok, 1 << 16, 0, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_selftest_wait_timeout(ok, 1 << 16, 20_000_000, 0) == moe.MOE_ERR_INVALID_ARG
