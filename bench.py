@@ -389,6 +389,51 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """One JSON line per workload (tiny, decode, prefill, skew, sweep T), on
+    one GPU: tokens/s, TFLOP/s, GB/s, roofline fractions, per-stage times and
+    a sampled oracle baseline.  Not the default contract line."""
+    import torch
+    import sparse_mixture_experts_13_b200 as moe
+    moe.lib()
+    peaks = load_peaks()
+    d, f, E = synth.MIXTRAL_D, synth.MIXTRAL_F, 8
+    W1 = synth.normal_bf16(0, synth.TID_W1, (E, f, d), 0.0, 1.0 / np.sqrt(d))
+    W3 = synth.normal_bf16(0, synth.TID_W3, (E, f, d), 0.0, 1.0 / np.sqrt(d))
+    W2 = synth.normal_bf16(0, synth.TID_W2, (E, d, f), 0.0, 1.0 / np.sqrt(f))
+    Wd = (None, to_dev_bf16(W1, torch), to_dev_bf16(W3, torch), to_dev_bf16(W2, torch))
+    cases = [("tiny", None), ("decode", None), ("prefill", None), ("skew", None)] + \
+            [("sweep", T) for T in synth.SWEEP_T]
+    for name, T in cases:
+        wl = synth.workload(name, T=T)
+        wl.generate(weights=(name == "tiny"))
+        if name == "tiny":
+            wd = (None, to_dev_bf16(wl.W1, torch), to_dev_bf16(wl.W3, torch), to_dev_bf16(wl.W2, torch))
+        else:
+            wd = Wd
+            wl.W1, wl.W3, wl.W2 = W1, W3, W2
+        run = Run(wl, wd, torch, moe)
+        N, touched = run.kept_and_touched()
+        for _ in range(args.warmup):
+            run.step()
+        ms = time_steps(run.step, args.steps, torch) / args.steps
+        stages = run.profiled(args.steps)
+        flops = 6.0 * N * wl.d * wl.f + 2.0 * wl.T * wl.d * wl.E
+        wbytes = touched * 3 * wl.d * wl.f * 2
+        bytes_ = wbytes + 2 * wl.T * wl.d * 2 + wl.E * wl.d * 4 + 2 * N * wl.f * 2 + 2 * N * wl.d * 2
+        tfs = flops / (ms * 1e-3) / 1e12
+        gbs = bytes_ / (ms * 1e-3) / 1e9
+        line = dict(workload=workload_desc(wl), T=wl.T, kept_slots=N, experts_touched=touched,
+                    ms_per_step=ms, tokens_per_s=wl.T / (ms * 1e-3), tflops=tfs, gbs=gbs,
+                    frac_bf16_burst=tfs / peaks["bf16"], frac_hbm=gbs / peaks["hbm"], stage_ms=stages,
+                    peaks_source=peaks["source"])
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, n_sample=min(16, wl.T))
+        print(json.dumps(line), flush=True)
+        del run
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -396,11 +441,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per workload (tiny, decode, prefill, skew, T sweep) instead of the contract line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 

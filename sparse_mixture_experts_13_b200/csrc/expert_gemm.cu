@@ -430,8 +430,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //          output column n0 + 128r + l).
 // The tokens are split between the CTAs: CTA r loads token rows
 // row0 + r*N/2 .. and the accumulator column n of both CTAs is token row0 + n.
-// Each CTA moves 32 KB per stage (16 KB of weights, 16 KB of tokens) for the
-// MMA work of 48 KB on a single-CTA 128 x 256 tile; six stages fit.  The
+// Each CTA moves 32 KB per 64-element K chunk (16 KB of weights, 16 KB of
+// tokens) for the MMA work of 48 KB on a single-CTA 128 x 256 tile; a stage
+// holds two chunks (8 MMAs per full/empty handshake) and three stages fit.  The
 // leader CTA (rank 0) counts both CTAs' bytes on its full barrier, issues the
 // MMAs and commits to the barriers of both CTAs with one multicast commit;
 // each CTA's epilogue reads its own accumulator and arrives on the leader's
@@ -441,7 +442,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // through a small ring in shared memory.  Tile ids run over (expert, weight
 // block, token block), so the pairs working at the same time share each
 // weight block through L2 and it is read from HBM once.
-constexpr int kPairStages = 6;
+constexpr int kPairStagesMax = 6;
 constexpr int kPairHalf = 128 * BK * 2;              // one 128-row operand half
 constexpr int kPairStageBytes = 2 * kPairHalf;       // A half + B half per CTA
 // Epilogue transpose buffers: two 16-token x 128-lane fp32 tiles, rows padded
@@ -450,8 +451,11 @@ constexpr int kXsStride = 132;
 constexpr int kPairXbuf = 2 * 16 * kXsStride * 4;
 constexpr int kRing = 4;            // tile ids in flight
 constexpr int kRingConsumers = 10;  // leader MMA + 4 epilogue warps per CTA + peer producer
-constexpr int kPairBarBytes = (2 * kPairStages + 5 + 2 * kRing) * 8;
-constexpr int kPairSmem = 1024 + kPairStages * kPairStageBytes + kPairXbuf + kPairBarBytes;
+constexpr int kPairBarBytes = (2 * kPairStagesMax + 5 + 2 * kRing) * 8;
+// Stage ring: 192 KB per CTA, as 6 stages of one 64-element K chunk or 3 stages
+// of two chunks (fewer full/empty handshakes per MMA).
+constexpr int kPairRingBytes = 6 * kPairStageBytes;
+constexpr int kPairSmem = 1024 + kPairRingBytes + kPairXbuf + kPairBarBytes;
 static_assert(kPairSmem <= 227 * 1024, "shared memory");
 
 struct PairTile {
@@ -474,11 +478,12 @@ __device__ __forceinline__ void decode_pair_tile(const GemmParams& p, const int3
   t.n0 = wb * (EPI == EPI_TILED_SWIGLU ? 128 : 256);
 }
 
-template <int EPI>
+template <int EPI, int CHUNKS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_wa,
                             const __grid_constant__ CUtensorMap map_wb, GemmParams p) {
-  constexpr int STAGES = kPairStages;
+  constexpr int STAGES = kPairStagesMax / CHUNKS;
+  constexpr int SHALF = CHUNKS * kPairHalf;  // bytes of one operand half per stage
   constexpr int ACC_COLS = 256;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
@@ -490,9 +495,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * kPairHalf;
-  float* xbuf = reinterpret_cast<float*>(sB + STAGES * kPairHalf);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kPairHalf + kPairXbuf);
+  uint8_t* sB = smem + STAGES * SHALF;
+  float* xbuf = reinterpret_cast<float*>(sB + STAGES * SHALF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * SHALF + kPairXbuf);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tfull_bar = bars + 2 * STAGES;
@@ -584,24 +589,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         PairTile t;
         decode_pair_tile<EPI>(p, s_off, s_base, tile, t);
         const int32_t tok_row = t.row0 + (int32_t)rank * (t.n_mma >> 1);
-        for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+        const int32_t n_steps = (p.num_kb + CHUNKS - 1) / CHUNKS;
+        for (int32_t ks = 0; ks < n_steps; ++ks) {
           if (!mbar_wait_cluster(&empty_bar[stage], phase ^ 1, &s_abort)) {
             ok = false;
             break;
           }
           const uint32_t full_leader = map_to_rank(smem_u32(&full_bar[stage]), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kPairStageBytes);
-          uint8_t* a_dst = sA + stage * kPairHalf;
-          uint8_t* b_dst = sB + stage * kPairHalf;
-          const int32_t kx = kb * BK;
-          if (EPI == EPI_TILED_SWIGLU) {
-            const int32_t wrow = t.n0 + (int32_t)rank * 64;
-            tma_load_3d_pair(&map_wa, full_leader, a_dst, kx, wrow, t.e);
-            tma_load_3d_pair(&map_wb, full_leader, a_dst + 64 * 128, kx, wrow, t.e);
-          } else {
-            tma_load_3d_pair(&map_wa, full_leader, a_dst, kx, t.n0 + (int32_t)rank * 128, t.e);
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * CHUNKS * kPairStageBytes);
+#pragma unroll
+          for (int c = 0; c < CHUNKS; ++c) {
+            // a chunk past the end of K is zero-filled by the tensor maps
+            uint8_t* a_dst = sA + stage * SHALF + c * kPairHalf;
+            uint8_t* b_dst = sB + stage * SHALF + c * kPairHalf;
+            const int32_t kx = (ks * CHUNKS + c) * BK;
+            if (EPI == EPI_TILED_SWIGLU) {
+              const int32_t wrow = t.n0 + (int32_t)rank * 64;
+              tma_load_3d_pair(&map_wa, full_leader, a_dst, kx, wrow, t.e);
+              tma_load_3d_pair(&map_wb, full_leader, a_dst + 64 * 128, kx, wrow, t.e);
+            } else {
+              tma_load_3d_pair(&map_wa, full_leader, a_dst, kx, t.n0 + (int32_t)rank * 128, t.e);
+            }
+            tma_load_2d_pair(&map_act, full_leader, b_dst, kx, tok_row);
           }
-          tma_load_2d_pair(&map_act, full_leader, b_dst, kx, tok_row);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -647,18 +657,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-        for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+        const int32_t n_steps = (p.num_kb + CHUNKS - 1) / CHUNKS;
+        for (int32_t ks = 0; ks < n_steps; ++ks) {
           if (!mbar_wait_cluster(&full_bar[stage], phase, &s_abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * kPairHalf);
-          const uint32_t b_addr = smem_u32(sB + stage * kPairHalf);
+          const uint32_t a_addr = smem_u32(sA + stage * SHALF);
+          const uint32_t b_addr = smem_u32(sB + stage * SHALF);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16_pair(d_tmem, make_sdesc_sw128(a_addr + kk * 32), make_sdesc_sw128(b_addr + kk * 32), idesc,
-                           (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int c = 0; c < CHUNKS; ++c)
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_bf16_pair(d_tmem, make_sdesc_sw128(a_addr + c * kPairHalf + kk * 32),
+                             make_sdesc_sw128(b_addr + c * kPairHalf + kk * 32), idesc,
+                             (ks > 0 || c > 0 || kk > 0) ? 1u : 0u);
           umma_commit_pair_both(&empty_bar[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -812,11 +826,11 @@ static cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& wa, con
   return cudaGetLastError();
 }
 
-template <int EPI>
+template <int EPI, int CHUNKS>
 static cudaError_t launch_pair(const CUtensorMap& act, const CUtensorMap& wa, const CUtensorMap& wb,
                                const GemmParams& p, int num_sms, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kPairSmem);
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<EPI, CHUNKS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -832,10 +846,11 @@ static cudaError_t launch_pair(const CUtensorMap& act, const CUtensorMap& wa, co
   // As many pairs as can be resident at once (persistent kernel).
   cfg.gridDim = dim3((unsigned)(num_sms & ~1), 1, 1);
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, expert_gemm_pair_kernel<EPI>, &cfg) == cudaSuccess && clusters > 0 &&
+  if (cudaOccupancyMaxActiveClusters(&clusters, expert_gemm_pair_kernel<EPI, CHUNKS>, &cfg) == cudaSuccess &&
+      clusters > 0 &&
       2 * clusters < (int)cfg.gridDim.x)
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
-  return cudaLaunchKernelEx(&cfg, expert_gemm_pair_kernel<EPI>, act, wa, wb, p);
+  return cudaLaunchKernelEx(&cfg, expert_gemm_pair_kernel<EPI, CHUNKS>, act, wa, wb, p);
 }
 
 void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
@@ -922,7 +937,8 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.splits = 1;
   p1.kb_per_split = p1.num_kb;
   p1.tile_counter = a.tile_counters;
-  cudaError_t err = a.pair ? launch_pair<EPI_TILED_SWIGLU>(mx, mw1, mw3, p1, a.num_sms, s)
+  // two 64-element K chunks per pipeline stage (3 stages): half the handshakes
+  cudaError_t err = a.pair ? launch_pair<EPI_TILED_SWIGLU, 2>(mx, mw1, mw3, p1, a.num_sms, s)
                            : launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s);
   if (err != cudaSuccess) return err;
   if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
@@ -938,7 +954,7 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p2.splits = 1;
   p2.kb_per_split = p2.num_kb;
   p2.tile_counter = a.tile_counters + 1;
-  return a.pair ? launch_pair<EPI_TILED_STORE>(mh, mw2, mw2, p2, a.num_sms, s)
+  return a.pair ? launch_pair<EPI_TILED_STORE, 2>(mh, mw2, mw2, p2, a.num_sms, s)
                 : launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s);
 }
 

@@ -6,15 +6,13 @@
 // logits, softmax over the k kept logits).
 //
 // Logits are fp32 dot products of a token's bf16 row with the E rows of W_g,
-// read as 16-byte vectors.  Many tokens: one warp per group of tokens, W_g
-// staged once per block in shared memory (E * d * 4 bytes) when it fits, each
-// W_g vector serving the whole group; a butterfly shuffle leaves every logit
-// in every lane.  Few tokens: one block per token with d split over the
-// block's threads.  The top-k (ties to the smaller expert index), the k-way
-// softmax and the full-softmax probability of each chosen expert are computed
-// redundantly per lane and lanes 0..k-1 write one slot each.  The per-expert
-// histogram is aggregated in shared memory and added to global memory once
-// per block (or added directly by the per-token blocks).
+// read as 16-byte vectors.  A block takes a group of tokens (one token when
+// there are few, so that many SMs share the work) and splits d over its warps;
+// every W_g vector a warp reads serves all tokens of the group.  The top-k
+// (ties to the smaller expert index), the k-way softmax and the full-softmax
+// probability of each chosen expert are computed redundantly per lane and
+// lanes 0..k-1 write one slot each.  The per-expert histogram is aggregated in
+// shared memory and added to global memory once per block.
 #include <cfloat>
 #include <cstdint>
 
@@ -23,9 +21,7 @@
 
 namespace moe {
 
-constexpr int kRouterThreads = 512;
 constexpr int kMaxK = 8;
-constexpr size_t kRouterMaxStage = 160 * 1024;
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -104,138 +100,101 @@ __device__ __forceinline__ float dot8(const float (&x)[8], const float4& w0, con
   return s;
 }
 
-// Many tokens: one warp per TPW tokens; each W_g vector read from shared
-// memory (when staged) serves the TPW tokens.
-template <int EMAX, int TPW, bool STAGED>
-__global__ void __launch_bounds__(kRouterThreads) router_tokens_kernel(RouterArgs a) {
-  extern __shared__ __align__(16) float s_wg[];
+// One block of 8 warps per group of G tokens.  Warp w takes the d-slice
+// [w*d/8, (w+1)*d/8): it loads the slice of all G token rows at once (16-byte
+// vectors), then streams the slice of each W_g row from L2 and applies it to
+// the G tokens held in registers.  The 8 partial sums per (token, expert) are
+// added in shared memory in warp order; warp g then finishes token g.
+constexpr int kGroupThreads = 256;
+constexpr int kGroupWarps = kGroupThreads / 32;
+
+template <int EMAX, int G>
+__global__ void __launch_bounds__(kGroupThreads) router_group_kernel(RouterArgs a) {
+  __shared__ float s_part[kGroupWarps][G][EMAX];
   __shared__ int s_count[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
   const int E = a.E, d = a.d;
+  const int64_t t0 = (int64_t)blockIdx.x * G;
   if (tid < 32) s_count[tid] = 0;
-  const float* wg = a.Wg;
-  if (STAGED) {
-    const int64_t n4 = (int64_t)E * d / 4;
-    const float4* src = reinterpret_cast<const float4*>(a.Wg);
-    float4* dst = reinterpret_cast<float4*>(s_wg);
-    for (int64_t i = tid; i < n4; i += blockDim.x) dst[i] = __ldg(src + i);
-    wg = s_wg;
+  const int nvec = d >> 3;                      // 16-byte vectors per row
+  const int per_warp = (nvec + kGroupWarps - 1) / kGroupWarps;
+  const int v0 = warp * per_warp, v1 = min(nvec, v0 + per_warp);
+  float acc[G][EMAX];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) acc[g][e] = 0.f;
+  for (int vb = v0; vb < v1; vb += 64) {
+    // this lane's (up to) two vectors of the slice chunk, for all G tokens
+    uint4 xr[G][2];
+    const int va = vb + lane, vc = vb + 32 + lane;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const uint4* row = reinterpret_cast<const uint4*>(a.x + (t0 + g) * d);
+      const bool tok = t0 + g < a.T;
+      xr[g][0] = (tok && va < v1) ? __ldg(row + va) : make_uint4(0, 0, 0, 0);
+      xr[g][1] = (tok && vc < v1) ? __ldg(row + vc) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      if (e < E) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int v = h ? vc : va;
+          if (v < v1) {
+            const float4* w = reinterpret_cast<const float4*>(a.Wg + (int64_t)e * d + (int64_t)v * 8);
+            const float4 w0 = __ldg(w), w1 = __ldg(w + 1);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              float xf[8];
+              bf16x8_to_f32(xr[g][h], xf);
+              acc[g][e] = dot8(xf, w0, w1, acc[g][e]);
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], off);
+    }
+  if (lane == 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e) s_part[warp][g][e] = acc[g][e];
   }
   __syncthreads();
-
-  const int nvec = d >> 3;
-  const int64_t groups = (a.T + TPW - 1) / TPW;
-  for (int64_t g = (int64_t)blockIdx.x * nwarps + warp; g < groups; g += (int64_t)gridDim.x * nwarps) {
-    const int64_t t0 = g * TPW;
-    float acc[TPW][EMAX];
+  if (warp < G && t0 + warp < a.T) {
+    float lg[EMAX];
 #pragma unroll
-    for (int i = 0; i < TPW; ++i)
+    for (int e = 0; e < EMAX; ++e) {
+      float v = 0.f;
 #pragma unroll
-      for (int e = 0; e < EMAX; ++e) acc[i][e] = 0.f;
-    for (int v = lane; v < nvec; v += 32) {
-      float xf[TPW][8];
-#pragma unroll
-      for (int i = 0; i < TPW; ++i) {
-        if (t0 + i < a.T) {
-          bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(a.x + (t0 + i) * d) + v), xf[i]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) xf[i][q] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-        if (e < E) {
-          const float4* w = reinterpret_cast<const float4*>(wg + (int64_t)e * d + (int64_t)v * 8);
-          const float4 w0 = w[0], w1 = w[1];
-#pragma unroll
-          for (int i = 0; i < TPW; ++i) acc[i][e] = dot8(xf[i], w0, w1, acc[i][e]);
-        }
-      }
+      for (int w = 0; w < kGroupWarps; ++w) v += s_part[w][warp][e];
+      lg[e] = v;
     }
-#pragma unroll
-    for (int i = 0; i < TPW; ++i) {
-#pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], off);
-      }
-      if (t0 + i < a.T) finish_token<EMAX>(a, t0 + i, acc[i], lane, s_count);
-    }
+    finish_token<EMAX>(a, t0 + warp, lg, lane, s_count);
   }
   __syncthreads();
   if (tid < E && s_count[tid] != 0) atomicAdd(&a.counts[tid], s_count[tid]);
 }
 
-// Few tokens: one block per token, the d dimension split over all threads,
-// W_g read straight from L2.
-constexpr int kSplitThreads = 256;
+constexpr int64_t kFewTokens = 512;
 
 template <int EMAX>
-__global__ void __launch_bounds__(kSplitThreads) router_split_kernel(RouterArgs a) {
-  __shared__ float s_part[kSplitThreads / 32][EMAX];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int E = a.E, d = a.d;
-  const int64_t t = blockIdx.x;
-  const int nvec = d >> 3;
-  float acc[EMAX];
-#pragma unroll
-  for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
-  for (int v = tid; v < nvec; v += kSplitThreads) {
-    float xf[8];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(a.x + t * d) + v), xf);
-#pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      if (e < E) {
-        const float4* w = reinterpret_cast<const float4*>(a.Wg + (int64_t)e * d + (int64_t)v * 8);
-        acc[e] = dot8(xf, __ldg(w), __ldg(w + 1), acc[e]);
-      }
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < EMAX; ++e) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int e = 0; e < EMAX; ++e) s_part[warp][e] = acc[e];
-  }
-  __syncthreads();
-  if (warp == 0) {
-#pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < kSplitThreads / 32; ++w) v += s_part[w][e];
-      acc[e] = v;
-    }
-    finish_token<EMAX>(a, t, acc, lane, a.counts);
-  }
-}
-
-constexpr int64_t kSplitMaxT = 512;
-
-template <int EMAX>
-static cudaError_t launch_router_e(const RouterArgs& a, int num_sms, cudaStream_t s) {
-  if (a.T <= kSplitMaxT) {
-    router_split_kernel<EMAX><<<(unsigned)a.T, kSplitThreads, 0, s>>>(a);
-    return cudaGetLastError();
-  }
-  constexpr int TPW = EMAX <= 8 ? 4 : 1;
-  const int warps = kRouterThreads / 32;
-  int64_t blocks = (a.T + warps * TPW - 1) / (warps * TPW);
-  if (blocks > num_sms) blocks = num_sms;
-  const size_t stage = (size_t)a.E * a.d * sizeof(float);
-  if (stage <= kRouterMaxStage) {
-    cudaError_t err = cudaFuncSetAttribute(router_tokens_kernel<EMAX, TPW, true>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRouterMaxStage);
-    if (err != cudaSuccess) return err;
-    router_tokens_kernel<EMAX, TPW, true><<<(unsigned)blocks, kRouterThreads, stage, s>>>(a);
-  } else {
-    router_tokens_kernel<EMAX, TPW, false><<<(unsigned)blocks, kRouterThreads, 0, s>>>(a);
-  }
+static cudaError_t launch_router_e(const RouterArgs& a, cudaStream_t s) {
+  constexpr int G = EMAX <= 8 ? 8 : (EMAX <= 16 ? 2 : 1);
+  const int g = a.T <= kFewTokens ? 1 : G;
+  const int64_t blocks = (a.T + g - 1) / g;
+  if (g == 1)
+    router_group_kernel<EMAX, 1><<<(unsigned)blocks, kGroupThreads, 0, s>>>(a);
+  else
+    router_group_kernel<EMAX, G><<<(unsigned)blocks, kGroupThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -244,9 +203,10 @@ cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s, bool
     cudaError_t err = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
     if (err != cudaSuccess) return err;
   }
-  if (a.E <= 8) return launch_router_e<8>(a, num_sms, s);
-  if (a.E <= 16) return launch_router_e<16>(a, num_sms, s);
-  return launch_router_e<32>(a, num_sms, s);
+  (void)num_sms;
+  if (a.E <= 8) return launch_router_e<8>(a, s);
+  if (a.E <= 16) return launch_router_e<16>(a, s);
+  return launch_router_e<32>(a, s);
 }
 
 }  // namespace moe
