@@ -853,7 +853,7 @@ static cudaError_t launch_pair(const CUtensorMap& act, const CUtensorMap& wa, co
   return cudaLaunchKernelEx(&cfg, expert_gemm_pair_kernel<EPI, CHUNKS>, act, wa, wb, p);
 }
 
-void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
+void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
   int64_t b = ((T + 15) / 16) * 16;
   if (b < 16) b = 16;
   if (b > 128) b = 128;
@@ -862,9 +862,11 @@ void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int3
   else if (b > 16) b = 32;
   *bn = (int32_t)b;
   // Split K of the down projection so that (experts x 128-row blocks x
-  // splits) tiles fill whole waves of the SMs as evenly as possible.
+  // splits) tiles fill whole waves of the SMs as evenly as possible.  At most
+  // T * k experts receive tokens, which bounds the tile count for few tokens.
   const int32_t num_kb = f / BK;
-  const int64_t base = (int64_t)E * ((d + 127) / 128);
+  const int64_t touched = T * k < E ? T * k : E;
+  const int64_t base = touched * ((d + 127) / 128);
   int32_t best = 1;
   double best_eff = 0.0;
   for (int32_t sp = 1; sp <= 16 && sp <= num_kb; ++sp) {

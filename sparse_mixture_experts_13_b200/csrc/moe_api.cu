@@ -63,7 +63,7 @@ Layout layout_of(const moe_shape* sh) {
   L.variant = variant_of(sh);
   L.bn = 128;
   L.splits = 1;
-  if (L.variant == MOE_VARIANT_STREAM) stream_params(T, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
+  if (L.variant == MOE_VARIANT_STREAM) stream_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
   size_t o = 0;
   L.status = o;
   L.ticket = o + 4;

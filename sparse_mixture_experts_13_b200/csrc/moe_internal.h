@@ -73,7 +73,7 @@ struct ExpertGemmArgs {
   uint32_t* tile_counters;  // [2] tile counters of the pair kernels, zeroed by the caller
 };
 // Streaming-variant parameters chosen from host-known sizes.
-void stream_params(int64_t T, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,
+void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,
                    int32_t* splits);
 cudaError_t launch_expert_gemms(const ExpertGemmArgs& a, cudaStream_t s);
 
