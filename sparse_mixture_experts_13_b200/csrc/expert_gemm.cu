@@ -591,7 +591,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int32_t tok_row = t.row0 + (int32_t)rank * (t.n_mma >> 1);
         const int32_t n_steps = (p.num_kb + CHUNKS - 1) / CHUNKS;
         for (int32_t ks = 0; ks < n_steps; ++ks) {
-          if (!mbar_wait_cluster(&empty_bar[stage], phase ^ 1, &s_abort)) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &s_abort)) {
             ok = false;
             break;
           }
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
         const int32_t n_steps = (p.num_kb + CHUNKS - 1) / CHUNKS;
         for (int32_t ks = 0; ks < n_steps; ++ks) {
-          if (!mbar_wait_cluster(&full_bar[stage], phase, &s_abort)) {
+          if (!mbar_wait(&full_bar[stage], phase, &s_abort)) {
             ok = false;
             break;
           }
@@ -702,7 +702,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t acc = n & 1, use = n >> 1;
       // The four epilogue warps decide together whether to go on, so that a
       // wait that gives up in one warp never leaves the others at a barrier.
-      if (tile >= 0 && !mbar_wait_cluster(&tfull_bar[acc], use & 1, &s_abort)) s_epi_fail = 1;
+      if (tile >= 0 && !mbar_wait(&tfull_bar[acc], use & 1, &s_abort)) s_epi_fail = 1;
       named_bar_sync(2, 128);
       if (s_epi_fail) {
         record_status(p.status, kStatusTimeout);
