@@ -10,7 +10,7 @@
 // where o_j is the expert output row slot_pos[t*k+j] of y_perm (bf16), or the
 // sum in split order of the fp32 split-K partials of that row.  fp32
 // accumulation in slot order, one bf16 rounding at the end; no atomics, so
-// the result is bit-reproducible.  16-byte vectors.
+// the result is bit-reproducible.
 #include <cstdint>
 
 #include "moe_internal.h"
@@ -27,24 +27,27 @@ __device__ __forceinline__ void bf16x8_unpack(const uint4& v, float (&f)[8]) {
   }
 }
 
-// One warp per (token, 256-column chunk); lane l owns columns
-// chunk*256 + 8l .. +7.  All of a lane's loads are issued before the sums.
-constexpr int kCombineCols = 256;
-
+// One warp per (token, chunk of 32 * CPL columns); lane l owns CPL
+// consecutive columns.  From bf16 rows (CPL = 16) every row load of a lane is
+// issued before the sums; from fp32 split-K partials (CPL = 8) the split loads
+// are unrolled by four.
+template <int CPL, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  constexpr int kCols = 32 * CPL;
+  constexpr int NV = CPL / 8;  // 16-byte bf16 vectors per lane
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int chunks = (a.d + kCombineCols - 1) / kCombineCols;
+  const int chunks = (a.d + kCols - 1) / kCols;
   const int64_t items = a.T * chunks;
   for (int64_t it = warp_global; it < items; it += nwarps) {
     const int64_t t = it / chunks;
-    const int col = (int)(it % chunks) * kCombineCols + lane * 8;
+    const int col = (int)(it % chunks) * kCols + lane * CPL;
     if (col >= a.d) continue;
-    int32_t pos[8];
-    float w[8];
+    int32_t pos[KMAX];
+    float w[KMAX];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
       pos[j] = -1;
       w[j] = 0.f;
       if (j < a.k) {
@@ -52,68 +55,91 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
         w[j] = __ldg(a.topk_w + t * a.k + j);
       }
     }
-    float acc[8];
+    float acc[CPL];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i = 0; i < CPL; ++i) acc[i] = 0.f;
     if (a.y_perm) {
-      uint4 raw[8];
+      uint4 raw[KMAX][NV];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (pos[j] >= 0) raw[j] = __ldg(reinterpret_cast<const uint4*>(a.y_perm + (int64_t)pos[j] * a.d + col));
+      for (int j = 0; j < KMAX; ++j)
+        if (pos[j] >= 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.y_perm + (int64_t)pos[j] * a.d + col);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+          for (int h = 0; h < NV; ++h) raw[j][h] = __ldg(src + h);
+        }
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
         if (pos[j] < 0) continue;
         float o[8];
-        bf16x8_unpack(raw[j], o);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], o[i], acc[i]);
+        for (int h = 0; h < NV; ++h) {
+          bf16x8_unpack(raw[j][h], o);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[8 * h + i] = fmaf(w[j], o[i], acc[8 * h + i]);
+        }
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < KMAX; ++j) {
         if (pos[j] < 0) continue;
         const float* base = a.partials + (int64_t)pos[j] * a.d + col;
-        float o[8];
+        float o[CPL];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = 0.f;
+        for (int i = 0; i < CPL; ++i) o[i] = 0.f;
         int sp = 0;
         for (; sp + 4 <= a.splits; sp += 4) {
-          float4 p[8];
+          float4 q[4][CPL / 4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float4* src = reinterpret_cast<const float4*>(base + (sp + u) * a.part_stride);
-            p[2 * u] = __ldg(src);
-            p[2 * u + 1] = __ldg(src + 1);
-          }
+          for (int u = 0; u < 4; ++u)
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            o[0] += p[2 * u].x; o[1] += p[2 * u].y; o[2] += p[2 * u].z; o[3] += p[2 * u].w;
-            o[4] += p[2 * u + 1].x; o[5] += p[2 * u + 1].y; o[6] += p[2 * u + 1].z; o[7] += p[2 * u + 1].w;
-          }
+            for (int c = 0; c < CPL / 4; ++c)
+              q[u][c] = __ldg(reinterpret_cast<const float4*>(base + (sp + u) * a.part_stride) + c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int c = 0; c < CPL / 4; ++c) {
+              o[4 * c] += q[u][c].x;
+              o[4 * c + 1] += q[u][c].y;
+              o[4 * c + 2] += q[u][c].z;
+              o[4 * c + 3] += q[u][c].w;
+            }
         }
         for (; sp < a.splits; ++sp) {
-          const float4* src = reinterpret_cast<const float4*>(base + sp * a.part_stride);
-          const float4 p0 = __ldg(src), p1 = __ldg(src + 1);
-          o[0] += p0.x; o[1] += p0.y; o[2] += p0.z; o[3] += p0.w;
-          o[4] += p1.x; o[5] += p1.y; o[6] += p1.z; o[7] += p1.w;
+#pragma unroll
+          for (int c = 0; c < CPL / 4; ++c) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(base + sp * a.part_stride) + c);
+            o[4 * c] += v.x;
+            o[4 * c + 1] += v.y;
+            o[4 * c + 2] += v.z;
+            o[4 * c + 3] += v.w;
+          }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], o[i], acc[i]);
+        for (int i = 0; i < CPL; ++i) acc[i] = fmaf(w[j], o[i], acc[i]);
       }
     }
-    *reinterpret_cast<uint4*>(a.y + t * a.d + col) =
-        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
+    uint4* dst = reinterpret_cast<uint4*>(a.y + t * a.d + col);
+#pragma unroll
+    for (int h = 0; h < NV; ++h)
+      dst[h] = make_uint4(pack_bf16x2(acc[8 * h], acc[8 * h + 1]), pack_bf16x2(acc[8 * h + 2], acc[8 * h + 3]),
+                          pack_bf16x2(acc[8 * h + 4], acc[8 * h + 5]), pack_bf16x2(acc[8 * h + 6], acc[8 * h + 7]));
   }
 }
 
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
-  const int64_t warps_needed = a.T * ((a.d + kCombineCols - 1) / kCombineCols);
+  const int cpl = a.y_perm ? 16 : 8;
+  const int64_t warps_needed = a.T * ((a.d + 32 * cpl - 1) / (32 * cpl));
   int64_t blocks = (warps_needed + 7) / 8;
   const int64_t cap = (int64_t)num_sms * 16;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  combine_kernel<<<(unsigned)blocks, 256, 0, s>>>(a);
+  if (a.k <= 2) {
+    if (cpl == 16) combine_kernel<16, 2><<<(unsigned)blocks, 256, 0, s>>>(a);
+    else combine_kernel<8, 2><<<(unsigned)blocks, 256, 0, s>>>(a);
+  } else {
+    if (cpl == 16) combine_kernel<16, 8><<<(unsigned)blocks, 256, 0, s>>>(a);
+    else combine_kernel<8, 8><<<(unsigned)blocks, 256, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -29,7 +29,7 @@
 
 namespace moe {
 
-constexpr int kPermuteThreads = 256;
+constexpr int kPermuteThreads = 512;
 constexpr int kPermuteWarpsSlots = kPermuteTile / 32;  // warps that rank slots
 constexpr uint32_t kFlagAgg = 1u << 30;
 constexpr uint32_t kFlagIncl = 2u << 30;
@@ -208,11 +208,88 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
   }
 }
 
+// Few slots (S <= kSmallSlots): every block ranks all slots itself in shared
+// memory -- warp 0 walks them in order, 32 at a time, keeping a running count
+// per expert -- so no look-back is needed, and the blocks then share the row
+// gather.  Block 0 writes offsets, slot_pos and perm_slot.
+constexpr int kSmallSlots = 1024;
+constexpr int kSmallBlocks = 64;
+
+__global__ void __launch_bounds__(256) permute_small_kernel(PermuteArgs a) {
+  __shared__ int32_t s_off[33];
+  __shared__ int32_t s_run[32];
+  __shared__ int32_t s_row[kSmallSlots];   // row of slot s, or -1
+  __shared__ int32_t s_list[kSmallSlots];  // kept slots in row order
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = a.E, k = a.k;
+  const int S = (int)(a.T * k);
+  if (tid == 0) {
+    int32_t acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = acc;
+      int32_t c = a.counts[e];
+      if (a.cap >= 0 && c > a.cap) c = (int32_t)a.cap;
+      acc += c;
+    }
+    s_off[E] = acc;
+  }
+  if (tid < 32) s_run[tid] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    for (int base = 0; base < S; base += 32) {
+      const int s = base + lane;
+      int e = -1;
+      bool elig = false;
+      if (s < S) {
+        e = a.topk_idx[s];
+        elig = true;
+        if (a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
+      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, elig ? e : -1);
+      const int before = __popc(peers & ((1u << lane) - 1u));
+      int32_t row = -1;
+      if (elig) {
+        const int32_t rank = s_run[e] + before;
+        if (!(a.cap >= 0 && a.policy == 1 && rank >= a.cap)) row = s_off[e] + rank;
+      }
+      __syncwarp();
+      if (elig && before == 0) s_run[e] += __popc(peers);
+      if (s < S) {
+        s_row[s] = row;
+        if (row >= 0) s_list[row] = s;
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  const int N = s_off[E];
+  if (blockIdx.x == 0) {
+    if (tid <= E) a.offsets[tid] = s_off[tid];
+    for (int s = tid; s < S; s += blockDim.x) a.slot_pos[s] = s_row[s];
+    for (int r = tid; r < N; r += blockDim.x) a.perm_slot[r] = s_list[r];
+  }
+  const int nvec = a.d >> 3;
+  const int nwarps = blockDim.x >> 5;
+  for (int r = blockIdx.x + gridDim.x * warp; r < N; r += gridDim.x * nwarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + (int64_t)(s_list[r] / k) * a.d);
+    uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (int64_t)r * a.d);
+    int v = lane;
+    for (; v + 224 < nvec; v += 256) {
+      uint4 q[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) q[u] = __ldg(src + v + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) dst[v + 32 * u] = q[u];
+    }
+    for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zeroed) {
   const int64_t S = a.T * a.k;
   const int64_t tiles = permute_tiles(S);
   cudaError_t err = cudaSuccess;
-  if (!state_zeroed) {
+  if (!state_zeroed && S > kSmallSlots) {
     err = cudaMemsetAsync(a.tile_state, 0, sizeof(uint32_t) * tiles * a.E, s);
     if (err != cudaSuccess) return err;
     err = cudaMemsetAsync(a.ticket, 0, sizeof(uint32_t), s);
@@ -224,7 +301,12 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zero
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  permute_kernel<<<(unsigned)tiles, kPermuteThreads, 0, s>>>(a);
+  if (S <= kSmallSlots) {
+    const int blocks = (int)(S < kSmallBlocks ? S : kSmallBlocks);
+    permute_small_kernel<<<blocks, 256, 0, s>>>(a);
+  } else {
+    permute_kernel<<<(unsigned)tiles, kPermuteThreads, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

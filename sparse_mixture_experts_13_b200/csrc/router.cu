@@ -100,12 +100,13 @@ __device__ __forceinline__ float dot8(const float (&x)[8], const float4& w0, con
   return s;
 }
 
-// One block of 8 warps per group of G tokens.  Warp w takes the d-slice
-// [w*d/8, (w+1)*d/8): it loads the slice of all G token rows at once (16-byte
-// vectors), then streams the slice of each W_g row from L2 and applies it to
-// the G tokens held in registers.  The 8 partial sums per (token, expert) are
-// added in shared memory in warp order; warp g then finishes token g.
-constexpr int kGroupThreads = 256;
+// One block of 16 warps per group of G tokens.  Warp w takes the d-slice
+// [w*d/16, (w+1)*d/16); each lane loads one 16-byte vector of that slice for
+// every token of the group at once, then reads the matching vectors of the E
+// rows of W_g (from L2) and applies each to the G tokens held in registers.
+// The 16 partial sums per (token, expert) are added in shared memory in warp
+// order; warp g then finishes token g.
+constexpr int kGroupThreads = 512;
 constexpr int kGroupWarps = kGroupThreads / 32;
 
 template <int EMAX, int G>
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(kGroupThreads) router_group_kernel(RouterArgs 
   const int E = a.E, d = a.d;
   const int64_t t0 = (int64_t)blockIdx.x * G;
   if (tid < 32) s_count[tid] = 0;
-  const int nvec = d >> 3;                      // 16-byte vectors per row
+  const int nvec = d >> 3;  // 16-byte vectors per row
   const int per_warp = (nvec + kGroupWarps - 1) / kGroupWarps;
   const int v0 = warp * per_warp, v1 = min(nvec, v0 + per_warp);
   float acc[G][EMAX];
@@ -124,34 +125,21 @@ __global__ void __launch_bounds__(kGroupThreads) router_group_kernel(RouterArgs 
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) acc[g][e] = 0.f;
-  for (int vb = v0; vb < v1; vb += 64) {
-    // this lane's (up to) two vectors of the slice chunk, for all G tokens
-    uint4 xr[G][2];
-    const int va = vb + lane, vc = vb + 32 + lane;
+  for (int v = v0 + lane; v < v1; v += 32) {
+    uint4 xr[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const uint4* row = reinterpret_cast<const uint4*>(a.x + (t0 + g) * d);
-      const bool tok = t0 + g < a.T;
-      xr[g][0] = (tok && va < v1) ? __ldg(row + va) : make_uint4(0, 0, 0, 0);
-      xr[g][1] = (tok && vc < v1) ? __ldg(row + vc) : make_uint4(0, 0, 0, 0);
-    }
+    for (int g = 0; g < G; ++g)
+      xr[g] = (t0 + g < a.T) ? __ldg(reinterpret_cast<const uint4*>(a.x + (t0 + g) * d) + v) : make_uint4(0, 0, 0, 0);
+    float xf[G][8];
+#pragma unroll
+    for (int g = 0; g < G; ++g) bf16x8_to_f32(xr[g], xf[g]);
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) {
       if (e < E) {
+        const float4* w = reinterpret_cast<const float4*>(a.Wg + (int64_t)e * d + (int64_t)v * 8);
+        const float4 w0 = __ldg(w), w1 = __ldg(w + 1);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int v = h ? vc : va;
-          if (v < v1) {
-            const float4* w = reinterpret_cast<const float4*>(a.Wg + (int64_t)e * d + (int64_t)v * 8);
-            const float4 w0 = __ldg(w), w1 = __ldg(w + 1);
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-              float xf[8];
-              bf16x8_to_f32(xr[g][h], xf);
-              acc[g][e] = dot8(xf, w0, w1, acc[g][e]);
-            }
-          }
-        }
+        for (int g = 0; g < G; ++g) acc[g][e] = dot8(xf[g], w0, w1, acc[g][e]);
       }
     }
   }
@@ -188,7 +176,7 @@ constexpr int64_t kFewTokens = 512;
 
 template <int EMAX>
 static cudaError_t launch_router_e(const RouterArgs& a, cudaStream_t s) {
-  constexpr int G = EMAX <= 8 ? 8 : (EMAX <= 16 ? 2 : 1);
+  constexpr int G = EMAX <= 8 ? 4 : (EMAX <= 16 ? 2 : 1);
   const int g = a.T <= kFewTokens ? 1 : G;
   const int64_t blocks = (a.T + g - 1) / g;
   if (g == 1)

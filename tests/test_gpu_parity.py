@@ -127,6 +127,15 @@ def test_tiny_capacity(o, variant, policy, cf):
     check_everything(o, wl, variant)
 
 
+@pytest.mark.parametrize("policy", [0, 1], ids=["by_prob", "by_order"])
+@pytest.mark.parametrize("cf", [0.75, 1.25])
+def test_capacity_many_slots(o, policy, cf):
+    """More than 1024 slots take the multi-block look-back grouping."""
+    wl = synth.Workload("cap_many", 1000, 128, 256, capacity_factor=cf, drop_policy=policy, skew=True,
+                        seed=9).generate()
+    check_everything(o, wl, 1)
+
+
 @pytest.mark.parametrize("E,k", [(4, 1), (16, 2), (8, 3), (32, 4), (8, 8), (1, 1)])
 @pytest.mark.parametrize("variant", [1, 2, 3], ids=lambda v: VNAME[v])
 def test_expert_counts(o, E, k, variant):
