@@ -372,7 +372,7 @@ def run_ours(args):
         long_run = args.steps * p["ms"] > 1000.0
         peak_tf = peaks["bf16_sustained"] if long_run else peaks["bf16"]
         achieved_tf = g1_flops / (g1_ms * 1e-3) / 1e12
-        tr = traffic_record("expert_gemm_pair_kernel<0>", "prefill")
+        tr = traffic_record("expert_gemm_pair_kernel<0,2>", "prefill")
         value = weak_scaling_value(world, wl.T, p["ms"])
 
         q = out["decode"]
