@@ -54,6 +54,11 @@ def _bind(path: str):
         "oracle_expert_row": [i32, i32, P, P, P, P, P, P],
         "oracle_layer_rows": [i64, i32, i32, i32, i32, P, P, P, P, P, P, P, i64, P, P, P, P],
         "oracle_num_threads": [],
+        "oracle_q4_quantize": [i32, i32, i32, P, P, P],
+        "oracle_q4_dequant": [i32, i32, i32, P, P, P],
+        "oracle_expert_row_q4": [i32, i32, P, P, P, P, P, P, P, P, P],
+        "oracle_layer_rows_q4": [i64, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P, i64, P, P, P,
+                                 P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +196,58 @@ class Oracle:
                                  self._p(w), self._p(kept), n, self._p(rows), self._p(y),
                                  self._p(h) if h is not None else None,
                                  self._p(o) if o is not None else None)
+        out = dict(y=y)
+        if want_h:
+            out["h"] = h
+        if want_o:
+            out["o"] = o
+        return out
+
+    # ------------------------------------------------------------ 4-bit experts
+    def q4_quantize(self, W: np.ndarray):
+        """W [E, R, K] bf16 bits -> (codes [E, R, K/2] uint8, scales [E, K/64, R]
+        bf16 bits): symmetric 4-bit codes with one absmax scale per 64 inputs."""
+        W = np.ascontiguousarray(W, np.uint16)
+        E, R, K = W.shape
+        assert K % 64 == 0
+        codes = np.empty((E, R, K // 2), np.uint8)
+        scales = np.empty((E, K // 64, R), np.uint16)
+        self.L.oracle_q4_quantize(E, R, K, self._p(W), self._p(codes), self._p(scales))
+        return codes, scales
+
+    def q4_dequant(self, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+        """(codes, scales) -> w_hat [E, R, K] in fp64."""
+        codes = np.ascontiguousarray(codes, np.uint8)
+        scales = np.ascontiguousarray(scales, np.uint16)
+        E, R, K2 = codes.shape
+        out = np.empty((E, R, 2 * K2), np.float64)
+        self.L.oracle_q4_dequant(E, R, 2 * K2, self._p(codes), self._p(scales), self._p(out))
+        return out
+
+    def layer_rows_q4(self, x, q1, q3, q2, route: dict, rows, want_h: bool = False,
+                      want_o: bool = False):
+        """layer_rows with 4-bit expert weights; q1, q3, q2 are the (codes,
+        scales) pairs of W1, W3 [E, f, d] and W2 [E, d, f]."""
+        T, d = x.shape
+        E, f, _ = q1[0].shape
+        idx, w, kept = route["idx"], route["w"], route["kept"]
+        k = idx.shape[1]
+        rows = np.ascontiguousarray(rows, np.int64)
+        n = rows.shape[0]
+        y = np.empty((n, d), np.float64)
+        h = np.empty((n, k, f), np.float64) if want_h else None
+        o = np.empty((n, k, d), np.float64) if want_o else None
+        x = np.ascontiguousarray(x, np.uint16)
+        ws = []
+        for c, sc in (q1, q3, q2):
+            ws += [np.ascontiguousarray(c, np.uint8), np.ascontiguousarray(sc, np.uint16)]
+        idx = np.ascontiguousarray(idx, np.int32)
+        w = np.ascontiguousarray(w, np.float64)
+        kept = np.ascontiguousarray(kept, np.uint8)
+        self.L.oracle_layer_rows_q4(T, d, f, E, k, self._p(x), *(self._p(a) for a in ws), self._p(idx),
+                                    self._p(w), self._p(kept), n, self._p(rows), self._p(y),
+                                    self._p(h) if h is not None else None,
+                                    self._p(o) if o is not None else None)
         out = dict(y=y)
         if want_h:
             out["h"] = h

@@ -261,6 +261,161 @@ void oracle_layer_rows(int64_t T, int32_t d, int32_t f, int32_t E, int32_t k, co
   }
 }
 
+/* ------------------------------------------------------------------------
+ * 4-bit expert weights.
+ *  [P1] "Deployment tradeoffs you'll actually hit", "Quantization asymmetry":
+ *       the router stays in 16-bit precision, the experts are quantised to 4
+ *       bits.
+ *  [P5] "4-bit Quantization for Single GPU" and "Memory Requirements": 4-bit
+ *       weights with block-wise absmax scales, arithmetic in bf16.
+ * Reading (the pages name formats, not their bits): symmetric 4-bit codes,
+ * one scale per 64 consecutive inputs of a weight row.  For a block b of row
+ * r of expert e:
+ *   s     = bf16(absmax_b / 7)            (fp32 division, then round to bf16)
+ *   q     = clamp(round_half_even(w / s), -8, 7)   (fp32 division; q = 0 if s = 0)
+ *   code  = q + 8                         (0 .. 15)
+ *   w_hat = (code - 8) * s
+ * Storage of W [E, R, K] (K a multiple of 64):
+ *   codes  [E, R, K/2] bytes.  The codes of inputs 8g .. 8g+7 of a row fill
+ *          one little-endian 32-bit word: nibble m (bits 4m .. 4m+3) holds
+ *          input 8g + 2m and nibble m + 4 holds input 8g + 2m + 1 (m = 0..3).
+ *   scales [E, K/64, R] bf16 bits (block-major: the scales of one block of
+ *          consecutive rows are adjacent).
+ * ------------------------------------------------------------------------ */
+
+static float q4_bf16_round(float v) {  /* fp32 -> nearest-even bf16, as fp32 */
+  uint32_t u;
+  memcpy(&u, &v, 4);
+  u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+  float r;
+  memcpy(&r, &u, 4);
+  return r;
+}
+
+/* byte offset and bit shift of input k's code inside its row */
+static void q4_locate(int64_t k, int64_t *byte, int *shift) {
+  int64_t g = k / 8;
+  int j = (int)(k % 8);
+  int nib = j / 2 + 4 * (j % 2);
+  *byte = g * 4 + nib / 2;
+  *shift = 4 * (nib % 2);
+}
+
+void oracle_q4_quantize(int32_t E, int32_t R, int32_t K, const uint16_t *W, uint8_t *codes,
+                        uint16_t *scales) {
+  int32_t nb = K / 64;
+  memset(codes, 0, (size_t)E * R * (K / 2));
+  for (int32_t e = 0; e < E; ++e)
+    for (int32_t r = 0; r < R; ++r)
+      for (int32_t b = 0; b < nb; ++b) {
+        const uint16_t *wr = W + ((int64_t)e * R + r) * K + (int64_t)b * 64;
+        float amax = 0.0f;
+        for (int i = 0; i < 64; ++i) {
+          float v = fabsf((float)bf16_to_double(wr[i]));
+          if (v > amax) amax = v;
+        }
+        float s = q4_bf16_round(amax / 7.0f);
+        uint32_t sb;
+        memcpy(&sb, &s, 4);
+        scales[((int64_t)e * nb + b) * R + r] = (uint16_t)(sb >> 16);
+        uint8_t *cr = codes + ((int64_t)e * R + r) * (K / 2);
+        for (int i = 0; i < 64; ++i) {
+          int q = 0;
+          if (s != 0.0f) {
+            float v = nearbyintf((float)bf16_to_double(wr[i]) / s);
+            q = v < -8.0f ? -8 : v > 7.0f ? 7 : (int)v;
+          }
+          int64_t byte;
+          int shift;
+          q4_locate((int64_t)b * 64 + i, &byte, &shift);
+          cr[byte] |= (uint8_t)((q + 8) << shift);
+        }
+      }
+}
+
+/* w_hat of input k of row r, expert slice (codes_e [R, K/2], scales_e [K/64, R]) */
+static double q4_weight(const uint8_t *codes_e, const uint16_t *scales_e, int32_t R, int32_t K,
+                        int64_t r, int64_t k) {
+  int64_t byte;
+  int shift;
+  q4_locate(k, &byte, &shift);
+  int code = (codes_e[r * (K / 2) + byte] >> shift) & 0xF;
+  return (double)(code - 8) * bf16_to_double(scales_e[(k / 64) * R + r]);
+}
+
+void oracle_q4_dequant(int32_t E, int32_t R, int32_t K, const uint8_t *codes,
+                       const uint16_t *scales, double *out) {
+  for (int32_t e = 0; e < E; ++e) {
+    const uint8_t *ce = codes + (int64_t)e * R * (K / 2);
+    const uint16_t *se = scales + (int64_t)e * (K / 64) * R;
+    for (int64_t r = 0; r < R; ++r)
+      for (int64_t k = 0; k < K; ++k) out[((int64_t)e * R + r) * K + k] = q4_weight(ce, se, R, K, r, k);
+  }
+}
+
+/* One expert on one token with 4-bit weights: the expert of [P3] "MoE Layer"
+ * with every weight read as w_hat.  Expert slices: W1 / W3 codes [f, d/2],
+ * scales [d/64, f]; W2 codes [d, f/2], scales [f/64, d]. */
+void oracle_expert_row_q4(int32_t d, int32_t f, const uint16_t *xrow, const uint8_t *W1c,
+                          const uint16_t *W1s, const uint8_t *W3c, const uint16_t *W3s,
+                          const uint8_t *W2c, const uint16_t *W2s, double *h, double *o) {
+  for (int32_t n = 0; n < f; ++n) {
+    double a = 0.0, b = 0.0;
+    for (int32_t i = 0; i < d; ++i) {
+      double xi = bf16_to_double(xrow[i]);
+      a += q4_weight(W1c, W1s, f, d, n, i) * xi;
+      b += q4_weight(W3c, W3s, f, d, n, i) * xi;
+    }
+    h[n] = a / (1.0 + exp(-a)) * b;
+  }
+  for (int32_t c = 0; c < d; ++c) {
+    double acc = 0.0;
+    for (int32_t n = 0; n < f; ++n) acc += q4_weight(W2c, W2s, d, f, c, n) * h[n];
+    o[c] = acc;
+  }
+}
+
+/* oracle_layer_rows with 4-bit expert weights (same combine, [P2] "How it works"). */
+void oracle_layer_rows_q4(int64_t T, int32_t d, int32_t f, int32_t E, int32_t k, const uint16_t *x,
+                          const uint8_t *W1c, const uint16_t *W1s, const uint8_t *W3c,
+                          const uint16_t *W3s, const uint8_t *W2c, const uint16_t *W2s,
+                          const int32_t *idx, const double *w, const uint8_t *kept, int64_t n_rows,
+                          const int64_t *rows, double *y, double *h_out, double *o_out) {
+  (void)T;
+  (void)E;
+#pragma omp parallel
+  {
+    double *h = (double *)malloc(sizeof(double) * (size_t)f);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t t = rows[r];
+      double *yr = y + r * d;
+      for (int32_t c = 0; c < d; ++c) yr[c] = 0.0;
+      for (int32_t j = 0; j < k; ++j) {
+        int64_t slot = t * k + j;
+        double *hs = h_out ? h_out + (r * k + j) * (int64_t)f : NULL;
+        double *os = o_out ? o_out + (r * k + j) * (int64_t)d : NULL;
+        if (!kept[slot]) {
+          if (hs) memset(hs, 0, sizeof(double) * (size_t)f);
+          if (os) memset(os, 0, sizeof(double) * (size_t)d);
+          continue;
+        }
+        int64_t e = idx[slot];
+        int64_t w13 = e * (int64_t)f * (d / 2), s13 = e * (int64_t)(d / 64) * f;
+        int64_t w2 = e * (int64_t)d * (f / 2), s2 = e * (int64_t)(f / 64) * d;
+        oracle_expert_row_q4(d, f, x + t * d, W1c + w13, W1s + s13, W3c + w13, W3s + s13, W2c + w2,
+                             W2s + s2, h, o);
+        for (int32_t c = 0; c < d; ++c) yr[c] += w[slot] * o[c];
+        if (hs) memcpy(hs, h, sizeof(double) * (size_t)f);
+        if (os) memcpy(os, o, sizeof(double) * (size_t)d);
+      }
+    }
+    free(h);
+    free(o);
+  }
+}
+
 /* Number of OpenMP threads the oracle runs with (reported with its timing). */
 int oracle_num_threads(void) {
   int n = 1;

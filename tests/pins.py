@@ -333,3 +333,90 @@ ALL_PINS = [pin_worked_example, pin_gate_forms_agree, pin_topk_ties_and_distinct
             pin_router_logits, pin_capacity_arithmetic, pin_capacity_bruteforce,
             pin_grouping_invariants, pin_silu_values, pin_expert_matmul,
             pin_dense_bruteforce, pin_special_cases, pin_dropped_slots]
+
+
+# ------------------------------------------------------- 4-bit expert weights
+
+def _exact_q4_matrix(rng, E, R, K):
+    """Random W [E, R, K] whose every 64-input block is (v * 2^j) with integer
+    v in [-7, 7], one |v| = 7 per block and a random exponent j per block:
+    exactly representable in the 4-bit format, so quantisation is lossless."""
+    nb = K // 64
+    v = rng.integers(-7, 8, size=(E, R, nb, 64))
+    pos = rng.integers(0, 64, size=(E, R, nb))
+    sign = rng.choice([-7, 7], size=(E, R, nb))
+    np.put_along_axis(v, pos[..., None], sign[..., None], axis=3)
+    j = rng.integers(-9, 2, size=(E, R, nb, 1))
+    W = (v * np.exp2(j)).reshape(E, R, K)
+    return _bf16(W), np.exp2(j[..., 0])
+
+
+def pin_q4_format_worked_example(o):
+    """Quantising the hand-worked matrix of tests/golden/q4_format.txt gives
+    the bytes and scales worked out there by hand from the format statement."""
+    g = read_golden("q4_format.txt")
+    W = np.zeros((1, 2, 128), np.float32)
+    for r, k, v in g["value"]:
+        W[0, int(r), int(k)] = float(v)
+    codes, scales = o.q4_quantize(_bf16(W))
+    want = np.full((1, 2, 64), 0x88, np.uint8)
+    for r, word, *b in g["word"]:
+        want[0, int(r), 4 * int(word):4 * int(word) + 4] = [int(x, 16) for x in b]
+    assert np.array_equal(codes, want)
+    assert [int(x, 16) for x in g["scales"]] == scales.reshape(-1).tolist()
+    assert np.array_equal(o.q4_dequant(codes, scales), W.astype(np.float64))
+
+
+def pin_q4_lossless_roundtrip(o):
+    """Weights exactly representable as 7-level multiples of a power of two
+    per block come back unchanged, with the scale equal to that power."""
+    rng = np.random.default_rng(41)
+    E, R, K = 3, 5, 192  # R != K/64, so a transposed scale index cannot pass
+    W, s = _exact_q4_matrix(rng, E, R, K)
+    codes, scales = o.q4_quantize(W)
+    assert np.array_equal(_w(scales), np.transpose(s, (0, 2, 1)))
+    assert np.array_equal(o.q4_dequant(codes, scales), _w(W))
+
+
+def pin_q4_error_bound(o):
+    """For N(0,1) weights every dequantised weight is within half a step of the
+    original (round to nearest, no clipping since |w| <= 7 s up to the bf16
+    rounding of s), and s is absmax / 7 to bf16 precision."""
+    rng = np.random.default_rng(42)
+    E, R, K = 2, 7, 256
+    W = _bf16(rng.standard_normal((E, R, K)))
+    codes, scales = o.q4_quantize(W)
+    Wd = o.q4_dequant(codes, scales)
+    s = np.repeat(np.transpose(_w(scales), (0, 2, 1)), 64, axis=2)
+    assert np.all(np.abs(Wd - _w(W)) <= 0.5 * s * (1 + 1e-12))
+    amax = np.abs(_w(W)).reshape(E, R, K // 64, 64).max(-1)
+    assert np.allclose(np.transpose(_w(scales), (0, 2, 1)), amax / 7.0, rtol=2.0 ** -8, atol=0)
+    nib = np.concatenate([codes & 0xF, codes >> 4], axis=-1)
+    assert nib.min() >= 1  # code 0 (q = -8) needs |w| > 7 s: never for these weights
+
+
+def pin_q4_layer_matches_bf16_on_exact_weights(o):
+    """With exactly representable expert weights the 4-bit layer equals the
+    (separately pinned) bf16 layer on the same weights, slot by slot, with and
+    without dropped slots."""
+    rng = np.random.default_rng(43)
+    T, d, f, E, k = 16, 64, 128, 4, 2
+    x = _bf16(rng.standard_normal((T, d)))
+    Wg = (rng.standard_normal((E, d)) / 8).astype(np.float32)
+    W1, _ = _exact_q4_matrix(rng, E, f, d)
+    W3, _ = _exact_q4_matrix(rng, E, f, d)
+    W2, _ = _exact_q4_matrix(rng, E, d, f)
+    q = [o.q4_quantize(W) for W in (W1, W3, W2)]
+    for cf in (0.0, 0.5):  # dropless, and a capacity that drops slots
+        r = o.route(x, Wg, k, cf=cf)
+        assert (r["kept"] == 0).any() == (cf > 0)
+        ref = o.layer_rows(x, W1, W3, W2, r, np.arange(T), want_h=True, want_o=True)
+        got = o.layer_rows_q4(x, *q, r, np.arange(T), want_h=True, want_o=True)
+        for key in ("y", "h", "o"):
+            assert np.allclose(got[key], ref[key], rtol=1e-12, atol=1e-12 * np.abs(ref[key]).max()), key
+
+
+Q4_PINS = [pin_q4_format_worked_example, pin_q4_lossless_roundtrip, pin_q4_error_bound,
+           pin_q4_layer_matches_bf16_on_exact_weights]
+
+ALL_PINS = ALL_PINS + Q4_PINS

@@ -26,12 +26,20 @@ def test_pin(o, pin):
     pin(o)
 
 
+# The SiLU line of the bf16 and of the 4-bit expert, each with the line before
+# it so that the anchor is unique.
+_SILU = "b += bf16_to_double(W3e[(int64_t)n * d + i]) * xi;\n    }\n    h[n] = a / (1.0 + exp(-a)) * b;"
+_SILU_Q4 = "b += q4_weight(W3c, W3s, f, d, n, i) * xi;\n    }\n    h[n] = a / (1.0 + exp(-a)) * b;"
+
 # (description, text in moe_oracle.c, replacement) -- each is a mistake that
 # a restatement of the layer could plausibly contain.
 MUTANTS = [
-    ("silu sign", "h[n] = a / (1.0 + exp(-a)) * b;", "h[n] = a / (1.0 + exp(a)) * b;"),
-    ("silu dropped", "h[n] = a / (1.0 + exp(-a)) * b;", "h[n] = a * b;"),
-    ("W1/W3 swapped in gate", "h[n] = a / (1.0 + exp(-a)) * b;", "h[n] = b / (1.0 + exp(-b)) * a;"),
+    ("silu sign", _SILU, _SILU.replace("exp(-a)", "exp(a)")),
+    ("silu dropped", _SILU, _SILU.replace("a / (1.0 + exp(-a)) * b", "a * b")),
+    ("W1/W3 swapped in gate", _SILU, _SILU.replace("a / (1.0 + exp(-a)) * b", "b / (1.0 + exp(-b)) * a")),
+    ("q4 silu sign", _SILU_Q4, _SILU_Q4.replace("exp(-a)", "exp(a)")),
+    ("q4 combine ignores gate", "yr[c] += w[slot] * o[c];", "yr[c] += o[c];"),
+    ("q4 dropped slot still added", "if (!kept[slot]) {", "if (0) {"),
     ("W2 transposed", "acc += bf16_to_double(W2e[(int64_t)c * f + n]) * h[n];",
      "acc += bf16_to_double(W2e[(int64_t)n * d + c]) * h[n];"),
     ("topk ties to larger index", "if (best < 0 || l[e] > l[best]) best = e;",
@@ -52,6 +60,17 @@ MUTANTS = [
     ("dropped slot still added", "if (!kept[s]) {", "if (0) {"),
     ("grouping in reverse token order", "for (int64_t s = 0; s < S; ++s) {\n      if (idx[s] != e) continue;",
      "for (int64_t s = S - 1; s >= 0; --s) {\n      if (idx[s] != e) continue;"),
+    ("q4 codes in plain nibble order", "int nib = j / 2 + 4 * (j % 2);", "int nib = j;"),
+    ("q4 high and low nibble swapped", "*shift = 4 * (nib % 2);", "*shift = 4 * (1 - nib % 2);"),
+    ("q4 scales read row-major", "bf16_to_double(scales_e[(k / 64) * R + r]);",
+     "bf16_to_double(scales_e[r * (K / 64) + k / 64]);"),
+    ("q4 code offset 7", "return (double)(code - 8) * bf16_to_double", "return (double)(code - 7) * bf16_to_double"),
+    ("q4 scale absmax / 8", "float s = q4_bf16_round(amax / 7.0f);", "float s = q4_bf16_round(amax / 8.0f);"),
+    ("q4 truncating round", "float v = nearbyintf((float)bf16_to_double(wr[i]) / s);",
+     "float v = truncf((float)bf16_to_double(wr[i]) / s);"),
+    ("q4 W2 read with W1 shape", "acc += q4_weight(W2c, W2s, d, f, c, n) * h[n];",
+     "acc += q4_weight(W2c, W2s, f, d, c % f, n % d) * h[n];"),
+    ("q4 W3 scales from W1", "b += q4_weight(W3c, W3s, f, d, n, i) * xi;", "b += q4_weight(W3c, W1s, f, d, n, i) * xi;"),
 ]
 
 
