@@ -29,6 +29,9 @@
  *       - "Step 2: A router picks 2 experts and mixes their outputs": the
  *         worked example (scores 2.1 0.3 1.4 -0.5 0.0 0.9 -1.2 0.2 -> weights
  *         0.6682 / 0.3318).
+ *  [P5] "Mixtral 8x7B — MoE Complete Guide" (webcoderspeed.com)
+ *       - "4-bit Quantization for Single GPU": 4-bit expert weights with
+ *         bf16 arithmetic (the 4-bit section at the end of this file).
  *
  * Readings taken where the pages are silent or disagree (each is also tested):
  *  - Gate: [P1] (softmax over all E, top-k, renormalise), [P2] (-inf mask then
