@@ -216,6 +216,66 @@ MOE_API moe_status moe_layer_forward_host(const moe_shape *shape, const moe_bf16
                                   const moe_bf16 *W2, moe_bf16 *y_host, void *ws,
                                   size_t ws_bytes, moe_stream_t stream);
 
+/* ---------------------------------------------------------------- 4-bit experts
+ * Sources: "How Mixtral 8x7B uses mixture of experts", "Deployment tradeoffs
+ * you'll actually hit" / "Quantization asymmetry" (keep the router in 16-bit
+ * precision, quantise the experts to 4 bits) and "Mixtral 8x7B — MoE
+ * Complete Guide", "4-bit Quantization for Single GPU" (4-bit weights, bf16
+ * arithmetic, block-wise absmax scales).
+ *
+ * Format of one 4-bit matrix W [E, R, K] (K a multiple of 64, R of 8):
+ *   codes  [E, R, K/2] bytes, 16-byte aligned.  The codes of inputs 8g ..
+ *          8g+7 of a row fill one little-endian 32-bit word: nibble m (bits
+ *          4m .. 4m+3) holds input 8g + 2m, nibble m + 4 input 8g + 2m + 1.
+ *   scales [E, K/64, R] bf16, 16-byte aligned: one scale per 64 consecutive
+ *          inputs of a row, stored block-major.
+ *   w = (code - 8) * scale, code in 0 .. 15.
+ * The expert matrices are W1, W3 [E, d_ff, d_model] and W2 [E, d_model, d_ff]
+ * as in the bf16 entry points; the router stays fp32.  The GPU rounds each
+ * dequantised weight to bf16 and accumulates in fp32. */
+
+/* Quantises W [E, R, K] bf16 (device) into codes and scales (device, out):
+ * per 64-input block s = bf16(absmax / 7) and code = 8 + clamp(round half to
+ * even(w / s), -8, 7), both divisions IEEE fp32; an all-zero block gets s = 0
+ * and codes 8.  Requires 1 <= E <= 32, 8 <= R <= 65536 with R % 8 == 0,
+ * 64 <= K <= 65536 with K % 64 == 0, finite weights.  Asynchronous on
+ * `stream`; allocates nothing. */
+MOE_API moe_status moe_quantize_q4(const moe_bf16 *W, int32_t E, int32_t R, int32_t K, uint8_t *codes,
+                                   moe_bf16 *scales, moe_stream_t stream);
+
+/* Workspace bytes the 4-bit entry points need for `shape` (0 if the shape is
+ * invalid).  gemm_variant is ignored: the 4-bit GEMMs have one schedule. */
+MOE_API size_t moe_workspace_size_q4(const moe_shape *shape);
+
+/* moe_grouped_swiglu with 4-bit expert weights (W1c/W1s, W3c/W3s, W2c/W2s
+ * in the format above).  h [T*k, d_ff] and y_perm [T*k, d_model] bf16 out;
+ * ws of at least moe_workspace_size_q4 bytes. */
+MOE_API moe_status moe_grouped_swiglu_q4(const moe_shape *shape, const moe_bf16 *x_perm,
+                                         const int32_t *offsets, const uint8_t *W1c,
+                                         const moe_bf16 *W1s, const uint8_t *W3c, const moe_bf16 *W3s,
+                                         const uint8_t *W2c, const moe_bf16 *W2s, moe_bf16 *h,
+                                         moe_bf16 *y_perm, void *ws, size_t ws_bytes,
+                                         moe_stream_t stream);
+
+/* moe_layer_forward with 4-bit expert weights; the router, grouping and
+ * combine are those of the bf16 layer.  ws of at least moe_workspace_size_q4
+ * bytes. */
+MOE_API moe_status moe_layer_forward_q4(const moe_shape *shape, const moe_bf16 *x, const float *Wg,
+                                        const uint8_t *W1c, const moe_bf16 *W1s, const uint8_t *W3c,
+                                        const moe_bf16 *W3s, const uint8_t *W2c, const moe_bf16 *W2s,
+                                        moe_bf16 *y, int32_t *topk_idx_out, int32_t *counts_out,
+                                        void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_layer_forward_q4 recording six CUDA events (cudaEvent_t) on `stream`
+ * between its stages, as moe_layer_forward_profiled. */
+MOE_API moe_status moe_layer_forward_q4_profiled(const moe_shape *shape, const moe_bf16 *x,
+                                                 const float *Wg, const uint8_t *W1c,
+                                                 const moe_bf16 *W1s, const uint8_t *W3c,
+                                                 const moe_bf16 *W3s, const uint8_t *W2c,
+                                                 const moe_bf16 *W2s, moe_bf16 *y,
+                                                 void *const *events, void *ws, size_t ws_bytes,
+                                                 moe_stream_t stream);
+
 /* Self-test of the failure reporting of the device-side waits (the pages
  * have no counterpart).  Queues one small kernel that makes an mbarrier wait
  * and a look-back wait -- the two kinds of bounded wait in the layer's

@@ -308,6 +308,7 @@ void oracle_q4_quantize(int32_t E, int32_t R, int32_t K, const uint16_t *W, uint
                         uint16_t *scales) {
   int32_t nb = K / 64;
   memset(codes, 0, (size_t)E * R * (K / 2));
+#pragma omp parallel for collapse(2) schedule(static)
   for (int32_t e = 0; e < E; ++e)
     for (int32_t r = 0; r < R; ++r)
       for (int32_t b = 0; b < nb; ++b) {

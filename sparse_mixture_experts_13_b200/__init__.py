@@ -10,5 +10,7 @@ from ._lib import (EXPORTED, MOE_DROP_BY_ORDER, MOE_DROP_BY_PROB, MOE_ERR_CUDA, 
                    MOE_VARIANT_STREAM, MOE_VARIANT_TILED, MOE_VARIANT_TILED_SINGLE, MoeError, check, lib, make_shape, moe_combine,
                    moe_grouped_swiglu, moe_layer_forward, moe_permute_noalloc, moe_layer_forward_host,
                    moe_layer_forward_profiled, moe_permute,
-                   moe_read_device_status, moe_router_topk, moe_selftest_wait_timeout, moe_shape, moe_workspace_size, status_string)
+                   moe_read_device_status, moe_router_topk, moe_selftest_wait_timeout, moe_shape, moe_workspace_size, status_string,
+                   moe_quantize_q4, moe_workspace_size_q4, moe_grouped_swiglu_q4, moe_layer_forward_q4,
+                   moe_layer_forward_q4_profiled)
 from .layer import MoELayer  # noqa: F401

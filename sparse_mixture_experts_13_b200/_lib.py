@@ -20,7 +20,10 @@ MOE_DROP_BY_PROB, MOE_DROP_BY_ORDER = 0, 1
 MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM, MOE_VARIANT_TILED_SINGLE = 0, 1, 2, 3
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
-            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc", "moe_selftest_wait_timeout", "moe_read_device_status", "moe_status_string")
+            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc",
+            "moe_selftest_wait_timeout", "moe_read_device_status", "moe_quantize_q4", "moe_workspace_size_q4",
+            "moe_grouped_swiglu_q4", "moe_layer_forward_q4", "moe_layer_forward_q4_profiled", "moe_status_string")
+_SIZE_RETURNING = ("moe_workspace_size", "moe_workspace_size_q4")
 
 
 class MoeError(RuntimeError):
@@ -64,10 +67,18 @@ def lib():
         L.moe_layer_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.moe_read_device_status.argtypes = [P, P]
         L.moe_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_uint32, P]
+        L.moe_quantize_q4.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P]
+        L.moe_workspace_size_q4.argtypes = [S]
+        L.moe_grouped_swiglu_q4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_layer_forward_q4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_layer_forward_q4_profiled.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_status_string.argtypes = [st]
         L.moe_status_string.restype = ctypes.c_char_p
-        for name in EXPORTED[1:-1]:
-            getattr(L, name).restype = st
+        for name in EXPORTED:
+            if name in _SIZE_RETURNING:
+                getattr(L, name).restype = sz
+            elif name != "moe_status_string":
+                getattr(L, name).restype = st
         _lib = L
     return _lib
 
@@ -141,6 +152,12 @@ def moe_layer_forward_host(shape, x_host, Wg, W1, W3, W2, y_host, ws, ws_bytes, 
 
 def moe_layer_forward_profiled(shape, x, Wg, W1, W3, W2, y, events, ws, ws_bytes, stream=None) -> int:
     """events: six torch.cuda.Event(enable_timing=True) objects (or raw handles)."""
+    arr = _event_handles(events)
+    return lib().moe_layer_forward_profiled(ctypes.byref(shape), _p(x), _p(Wg), _p(W1), _p(W3), _p(W2), _p(y), arr,
+                                            _p(ws), int(ws_bytes), _stream(stream))
+
+
+def _event_handles(events):
     handles = []
     for ev in events:
         if isinstance(ev, int):
@@ -149,9 +166,37 @@ def moe_layer_forward_profiled(shape, x, Wg, W1, W3, W2, y, events, ws, ws_bytes
             if ev.cuda_event == 0:
                 ev.record()  # creates the underlying event
             handles.append(ev.cuda_event)
-    arr = (ctypes.c_void_p * 6)(*handles)
-    return lib().moe_layer_forward_profiled(ctypes.byref(shape), _p(x), _p(Wg), _p(W1), _p(W3), _p(W2), _p(y), arr,
-                                            _p(ws), int(ws_bytes), _stream(stream))
+    return (ctypes.c_void_p * 6)(*handles)
+
+
+# ------------------------------------------------------------ 4-bit experts
+# A 4-bit matrix is passed as a (codes, scales) pair: codes [E, R, K/2] uint8,
+# scales [E, K/64, R] bf16 bits.
+
+def moe_quantize_q4(W, E, R, K, codes, scales, stream=None) -> int:
+    return lib().moe_quantize_q4(_p(W), int(E), int(R), int(K), _p(codes), _p(scales), _stream(stream))
+
+
+def moe_workspace_size_q4(shape: moe_shape) -> int:
+    return int(lib().moe_workspace_size_q4(ctypes.byref(shape)))
+
+
+def moe_grouped_swiglu_q4(shape, x_perm, offsets, q1, q3, q2, h, y_perm, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_grouped_swiglu_q4(ctypes.byref(shape), _p(x_perm), _p(offsets), _p(q1[0]), _p(q1[1]),
+                                       _p(q3[0]), _p(q3[1]), _p(q2[0]), _p(q2[1]), _p(h), _p(y_perm), _p(ws),
+                                       int(ws_bytes), _stream(stream))
+
+
+def moe_layer_forward_q4(shape, x, Wg, q1, q3, q2, y, topk_idx_out, counts_out, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_layer_forward_q4(ctypes.byref(shape), _p(x), _p(Wg), _p(q1[0]), _p(q1[1]), _p(q3[0]),
+                                      _p(q3[1]), _p(q2[0]), _p(q2[1]), _p(y), _p(topk_idx_out), _p(counts_out),
+                                      _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_layer_forward_q4_profiled(shape, x, Wg, q1, q3, q2, y, events, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_layer_forward_q4_profiled(ctypes.byref(shape), _p(x), _p(Wg), _p(q1[0]), _p(q1[1]),
+                                               _p(q3[0]), _p(q3[1]), _p(q2[0]), _p(q2[1]), _p(y),
+                                               _event_handles(events), _p(ws), int(ws_bytes), _stream(stream))
 
 
 def moe_selftest_wait_timeout(ws, ws_bytes, limit_us, stream=None) -> int:

@@ -53,17 +53,30 @@ struct Layout {
   size_t thresh, partials, topk_idx, topk_w, topk_p, offsets, slot_pos, perm_slot, x_perm, h, y_perm,
       x_stage, y_stage, total;
   int variant;
-  int32_t bn, splits;
+  bool q4;                 // 4-bit expert weights (always the streaming schedule)
+  int32_t bn, splits;      // streaming schedule: token tile, requested split-K count
+  int32_t eff_splits;      // split-K partial buffers the down projection writes
 };
 
-Layout layout_of(const moe_shape* sh) {
+// q4: layout of the 4-bit entry points (split-K partials always present).
+Layout layout_of(const moe_shape* sh, bool q4 = false) {
   Layout L{};
   const int64_t T = sh->T, S = T * sh->k;
   const int64_t d = sh->d_model, f = sh->d_ff, E = sh->E;
-  L.variant = variant_of(sh);
+  L.variant = q4 ? MOE_VARIANT_STREAM : variant_of(sh);
+  L.q4 = q4;
   L.bn = 128;
   L.splits = 1;
-  if (L.variant == MOE_VARIANT_STREAM) stream_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
+  L.eff_splits = 1;
+  if (q4) {
+    q4_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
+    L.eff_splits = q4_effective_splits(sh->d_ff, L.splits);
+  } else if (L.variant == MOE_VARIANT_STREAM) {
+    stream_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
+    const int32_t num_kb = sh->d_ff / 64;
+    const int32_t kbps = (num_kb + L.splits - 1) / L.splits;
+    L.eff_splits = (num_kb + kbps - 1) / kbps;
+  }
   size_t o = 0;
   L.status = o;
   L.ticket = o + 4;
@@ -76,7 +89,7 @@ Layout layout_of(const moe_shape* sh) {
   L.thresh = o;
   o = align_up(o + 8 * E);
   L.partials = o;
-  if (L.variant == MOE_VARIANT_STREAM) o = align_up(o + 4 * (size_t)L.splits * S * d);
+  if (L.variant == MOE_VARIANT_STREAM) o = align_up(o + 4 * (size_t)L.eff_splits * S * d);
   L.topk_idx = o;
   o = align_up(o + 4 * S);
   L.topk_w = o;
@@ -103,9 +116,9 @@ Layout layout_of(const moe_shape* sh) {
   return L;
 }
 
-moe_status check_ws(const moe_shape* sh, const void* ws, size_t ws_bytes) {
+moe_status check_ws(const moe_shape* sh, const void* ws, size_t ws_bytes, bool q4 = false) {
   if (!ws || !aligned(ws, kAlign)) return MOE_ERR_WORKSPACE;
-  if (ws_bytes < layout_of(sh).total) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < layout_of(sh, q4).total) return MOE_ERR_WORKSPACE;
   return MOE_OK;
 }
 
@@ -205,6 +218,46 @@ moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_per
   return cuda_status(launch_expert_gemms(a, s));
 }
 
+// Expert weights of one call: bf16 matrices, or 4-bit codes and scales.
+struct ExpertWeights {
+  const moe_bf16 *W1, *W3, *W2;
+  const uint8_t *W1c, *W3c, *W2c;
+  const moe_bf16 *W1s, *W3s, *W2s;
+};
+
+moe_status run_gemms_q4(const moe_shape* sh, const Layout& L, const moe_bf16* x_perm, const int32_t* offsets,
+                        const ExpertWeights& W, moe_bf16* h, void* ws, int num_sms, cudaStream_t s,
+                        cudaEvent_t between = nullptr) {
+  ExpertGemmQ4Args a{};
+  a.offsets = offsets;
+  a.x_perm = x_perm;
+  a.W1c = W.W1c;
+  a.W1s = W.W1s;
+  a.W3c = W.W3c;
+  a.W3s = W.W3s;
+  a.W2c = W.W2c;
+  a.W2s = W.W2s;
+  a.h = h;
+  a.partials = at<float>(ws, L.partials);
+  a.status = at<uint32_t>(ws, L.status);
+  a.S = sh->T * sh->k;
+  a.d = sh->d_model;
+  a.f = sh->d_ff;
+  a.E = sh->E;
+  a.bn = L.bn;
+  a.splits = L.splits;
+  a.num_sms = num_sms;
+  a.between = between;
+  return cuda_status(launch_expert_gemms_q4(a, s));
+}
+
+moe_status check_q4_weights(const ExpertWeights& W) {
+  const void* ps[6] = {W.W1c, W.W3c, W.W2c, W.W1s, W.W3s, W.W2s};
+  for (const void* p : ps)
+    if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
 }  // namespace
 
 namespace moe {
@@ -279,11 +332,8 @@ moe_status moe_grouped_swiglu(const moe_shape* sh, const moe_bf16* x_perm, const
   MOE_TRY(run_gemms(sh, L, x_perm, offsets, W1, W3, W2, h, y_perm, ws, sms, s));
   if (L.variant == MOE_VARIANT_STREAM) {
     const int64_t S = sh->T * sh->k;
-    const int32_t num_kb = sh->d_ff / 64;
-    const int32_t kbps = (num_kb + L.splits - 1) / L.splits;
-    const int32_t splits = (num_kb + kbps - 1) / kbps;
-    MOE_TRY(cuda_status(launch_splitk_reduce(at<float>(ws, L.partials), splits, S * (int64_t)sh->d_model, offsets,
-                                             sh->E, y_perm, S, sh->d_model, sms, s)));
+    MOE_TRY(cuda_status(launch_splitk_reduce(at<float>(ws, L.partials), L.eff_splits, S * (int64_t)sh->d_model,
+                                             offsets, sh->E, y_perm, S, sh->d_model, sms, s)));
   }
   return MOE_OK;
 }
@@ -309,11 +359,10 @@ moe_status moe_combine(const moe_shape* sh, const moe_bf16* y_perm, const int32_
   return cuda_status(launch_combine(a, sms, (cudaStream_t)stream));
 }
 
-static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, const float* Wg, const moe_bf16* W1,
-                                     const moe_bf16* W3, const moe_bf16* W2, moe_bf16* y, int32_t* topk_idx_out,
-                                     int32_t* counts_out, void* ws, int sms, cudaStream_t s,
-                                     cudaEvent_t const* ev = nullptr) {
-  const Layout L = layout_of(sh);
+static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, const float* Wg, const ExpertWeights& W,
+                                     bool q4, moe_bf16* y, int32_t* topk_idx_out, int32_t* counts_out, void* ws,
+                                     int sms, cudaStream_t s, cudaEvent_t const* ev = nullptr) {
+  const Layout L = layout_of(sh, q4);
   const int64_t S = sh->T * sh->k;
   int32_t* idx = at<int32_t>(ws, L.topk_idx);
   float* w = at<float>(ws, L.topk_w);
@@ -333,7 +382,10 @@ static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, con
   MOE_TRY(mark(1));
   MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s, true));
   MOE_TRY(mark(2));
-  MOE_TRY(run_gemms(sh, L, x_perm, offsets, W1, W3, W2, h, y_perm, ws, sms, s, ev ? ev[3] : nullptr));
+  if (q4)
+    MOE_TRY(run_gemms_q4(sh, L, x_perm, offsets, W, h, ws, sms, s, ev ? ev[3] : nullptr));
+  else
+    MOE_TRY(run_gemms(sh, L, x_perm, offsets, W.W1, W.W3, W.W2, h, y_perm, ws, sms, s, ev ? ev[3] : nullptr));
   MOE_TRY(mark(4));
   CombineArgs c{};
   c.slot_pos = slot_pos;
@@ -343,11 +395,9 @@ static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, con
   c.d = sh->d_model;
   c.k = sh->k;
   if (L.variant == MOE_VARIANT_STREAM) {
-    const int32_t num_kb = sh->d_ff / 64;
-    const int32_t kbps = (num_kb + L.splits - 1) / L.splits;
     c.y_perm = nullptr;
     c.partials = at<float>(ws, L.partials);
-    c.splits = (num_kb + kbps - 1) / kbps;
+    c.splits = L.eff_splits;
     c.part_stride = S * (int64_t)sh->d_model;
   } else {
     c.y_perm = y_perm;
@@ -377,7 +427,8 @@ moe_status moe_layer_forward(const moe_shape* sh, const moe_bf16* x, const float
   MOE_TRY(check_ws(sh, ws, ws_bytes));
   int sms = 0;
   MOE_TRY(check_device(&sms));
-  return layer_forward_impl(sh, x, Wg, W1, W3, W2, y, topk_idx_out, counts_out, ws, sms, (cudaStream_t)stream);
+  const ExpertWeights Wt{W1, W3, W2, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  return layer_forward_impl(sh, x, Wg, Wt, false, y, topk_idx_out, counts_out, ws, sms, (cudaStream_t)stream);
 }
 
 moe_status moe_layer_forward_profiled(const moe_shape* sh, const moe_bf16* x, const float* Wg, const moe_bf16* W1,
@@ -397,7 +448,8 @@ moe_status moe_layer_forward_profiled(const moe_shape* sh, const moe_bf16* x, co
   MOE_TRY(check_ws(sh, ws, ws_bytes));
   int sms = 0;
   MOE_TRY(check_device(&sms));
-  return layer_forward_impl(sh, x, Wg, W1, W3, W2, y, nullptr, nullptr, ws, sms, (cudaStream_t)stream,
+  const ExpertWeights Wt{W1, W3, W2, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  return layer_forward_impl(sh, x, Wg, Wt, false, y, nullptr, nullptr, ws, sms, (cudaStream_t)stream,
                             reinterpret_cast<cudaEvent_t const*>(events));
 }
 
@@ -420,8 +472,89 @@ moe_status moe_layer_forward_host(const moe_shape* sh, const moe_bf16* x_host, c
   moe_bf16* xd = at<moe_bf16>(ws, L.x_stage);
   moe_bf16* yd = at<moe_bf16>(ws, L.y_stage);
   MOE_TRY(cuda_status(cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s)));
-  MOE_TRY(layer_forward_impl(sh, xd, Wg, W1, W3, W2, yd, nullptr, nullptr, ws, sms, s));
+  const ExpertWeights Wt{W1, W3, W2, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  MOE_TRY(layer_forward_impl(sh, xd, Wg, Wt, false, yd, nullptr, nullptr, ws, sms, s));
   return cuda_status(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+moe_status moe_quantize_q4(const moe_bf16* W, int32_t E, int32_t R, int32_t K, uint8_t* codes, moe_bf16* scales,
+                           moe_stream_t stream) {
+  if (E < 1 || E > 32 || R < 8 || R > 65536 || R % 8 || K < 64 || K > 65536 || K % 64) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_bf16(W));
+  MOE_TRY(check_bf16(codes));
+  MOE_TRY(check_bf16(scales));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return cuda_status(launch_quantize_q4(W, E, R, K, codes, scales, (cudaStream_t)stream));
+}
+
+size_t moe_workspace_size_q4(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return layout_of(shape, true).total;
+}
+
+moe_status moe_grouped_swiglu_q4(const moe_shape* sh, const moe_bf16* x_perm, const int32_t* offsets,
+                                 const uint8_t* W1c, const moe_bf16* W1s, const uint8_t* W3c, const moe_bf16* W3s,
+                                 const uint8_t* W2c, const moe_bf16* W2s, moe_bf16* h, moe_bf16* y_perm, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  const ExpertWeights Wt{nullptr, nullptr, nullptr, W1c, W3c, W2c, W1s, W3s, W2s};
+  MOE_TRY(check_bf16(x_perm));
+  MOE_TRY(check_i32(offsets));
+  MOE_TRY(check_q4_weights(Wt));
+  MOE_TRY(check_bf16(h));
+  MOE_TRY(check_bf16(y_perm));
+  MOE_TRY(check_ws(sh, ws, ws_bytes, true));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  const Layout L = layout_of(sh, true);
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 16, s)));
+  MOE_TRY(run_gemms_q4(sh, L, x_perm, offsets, Wt, h, ws, sms, s));
+  const int64_t S = sh->T * sh->k;
+  return cuda_status(launch_splitk_reduce(at<float>(ws, L.partials), L.eff_splits, S * (int64_t)sh->d_model, offsets,
+                                          sh->E, y_perm, S, sh->d_model, sms, s));
+}
+
+static moe_status check_layer_q4(const moe_shape* sh, const moe_bf16* x, const float* Wg, const ExpertWeights& W,
+                                 const moe_bf16* y, const void* ws, size_t ws_bytes, int* sms) {
+  MOE_TRY(check_bf16(x));
+  MOE_TRY(check_bf16(Wg));
+  MOE_TRY(check_q4_weights(W));
+  MOE_TRY(check_bf16(y));
+  MOE_TRY(check_ws(sh, ws, ws_bytes, true));
+  return check_device(sms);
+}
+
+moe_status moe_layer_forward_q4(const moe_shape* sh, const moe_bf16* x, const float* Wg, const uint8_t* W1c,
+                                const moe_bf16* W1s, const uint8_t* W3c, const moe_bf16* W3s, const uint8_t* W2c,
+                                const moe_bf16* W2s, moe_bf16* y, int32_t* topk_idx_out, int32_t* counts_out,
+                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  const ExpertWeights Wt{nullptr, nullptr, nullptr, W1c, W3c, W2c, W1s, W3s, W2s};
+  if (topk_idx_out && !aligned(topk_idx_out, 4)) return MOE_ERR_INVALID_ARG;
+  if (counts_out && !aligned(counts_out, 4)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  MOE_TRY(check_layer_q4(sh, x, Wg, Wt, y, ws, ws_bytes, &sms));
+  return layer_forward_impl(sh, x, Wg, Wt, true, y, topk_idx_out, counts_out, ws, sms, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_forward_q4_profiled(const moe_shape* sh, const moe_bf16* x, const float* Wg, const uint8_t* W1c,
+                                         const moe_bf16* W1s, const uint8_t* W3c, const moe_bf16* W3s,
+                                         const uint8_t* W2c, const moe_bf16* W2s, moe_bf16* y, void* const* events,
+                                         void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  const ExpertWeights Wt{nullptr, nullptr, nullptr, W1c, W3c, W2c, W1s, W3s, W2s};
+  if (!events) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  MOE_TRY(check_layer_q4(sh, x, Wg, Wt, y, ws, ws_bytes, &sms));
+  return layer_forward_impl(sh, x, Wg, Wt, true, y, nullptr, nullptr, ws, sms, (cudaStream_t)stream,
+                            reinterpret_cast<cudaEvent_t const*>(events));
 }
 
 moe_status moe_read_device_status(const void* ws, moe_stream_t stream) {

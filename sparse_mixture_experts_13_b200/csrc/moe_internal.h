@@ -77,6 +77,36 @@ void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int nu
                    int32_t* splits);
 cudaError_t launch_expert_gemms(const ExpertGemmArgs& a, cudaStream_t s);
 
+// Expert GEMMs with 4-bit weights (codes [E, R, K/2], scales [E, K/64, R]
+// bf16; w = (code - 8) * scale).  One schedule: the streaming one, with the
+// down projection's K split into fp32 partials summed by the combine.
+struct ExpertGemmQ4Args {
+  const int32_t* offsets;   // [E + 1]
+  const uint16_t* x_perm;   // [S, d]
+  const uint8_t* W1c;       // [E, f, d/2]
+  const uint16_t* W1s;      // [E, d/64, f]
+  const uint8_t* W3c;
+  const uint16_t* W3s;
+  const uint8_t* W2c;       // [E, d, f/2]
+  const uint16_t* W2s;      // [E, f/64, d]
+  uint16_t* h;              // [S, f]
+  float* partials;          // [splits, S, d]
+  uint32_t* status;
+  int64_t S;
+  int32_t d, f, E;
+  int32_t bn;               // token tile (16..128)
+  int32_t splits;           // requested split-K count of the down projection
+  int num_sms;
+  cudaEvent_t between;      // recorded after the first GEMM if not null
+};
+void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits);
+// number of K splits the down projection really uses for a requested count
+int32_t q4_effective_splits(int32_t f, int32_t splits);
+cudaError_t launch_expert_gemms_q4(const ExpertGemmQ4Args& a, cudaStream_t s);
+// W [E, R, K] bf16 -> codes and scales (K a multiple of 64, R a multiple of 8)
+cudaError_t launch_quantize_q4(const uint16_t* W, int32_t E, int32_t R, int32_t K, uint8_t* codes,
+                               uint16_t* scales, cudaStream_t s);
+
 struct CombineArgs {
   const uint16_t* y_perm;   // [S, d] bf16, or nullptr when reading partials
   const float* partials;    // [splits, S, d] fp32 (if y_perm == nullptr)

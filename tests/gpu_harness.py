@@ -217,3 +217,59 @@ def sample_tokens(wl: synth.Workload, r: dict, n: int, seed: int = 1) -> np.ndar
         pick.add(int(t))
     pick.update({0, T - 1})
     return np.array(sorted(pick), np.int64)
+
+
+# ------------------------------------------------------------ 4-bit experts
+
+class QDevice(Device):
+    """A workload's inputs on the GPU with the expert weights in the 4-bit
+    format, quantised by the oracle (the GPU consumes the oracle's bytes)."""
+
+    def __init__(self, wl: synth.Workload, o: oracle.Oracle, q=None):
+        self.wl = wl
+        self.x = to_dev_bf16(wl.x)
+        self.Wg = torch.from_numpy(wl.Wg).cuda()
+        self.q_host = q if q is not None else tuple(o.q4_quantize(W) for W in (wl.W1, wl.W3, wl.W2))
+        self.q = tuple((torch.from_numpy(c).cuda(), to_dev_bf16(s)) for c, s in self.q_host)
+
+
+def run_layer_q4(dev: QDevice, reps: int = 1) -> dict:
+    wl = dev.wl
+    sh = dev.shape(0)
+    nws = moe.moe_workspace_size_q4(sh)
+    ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+    y = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(wl.T * wl.k, dtype=torch.int32, device="cuda")
+    counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    ys = []
+    for _ in range(reps):
+        moe.check(moe.moe_layer_forward_q4(sh, dev.x, dev.Wg, *dev.q, y, idx, counts, ws, nws), "layer_forward_q4")
+        st = moe.moe_read_device_status(ws)
+        assert st == moe.MOE_OK, moe.status_string(st)
+        ys.append(bf16_host(y).copy())
+    return dict(y=ys[0], ys=ys, idx=idx.cpu().numpy(), counts=counts.cpu().numpy())
+
+
+def run_stages_q4(dev: QDevice) -> dict:
+    """Router -> permute -> 4-bit grouped SwiGLU -> combine through the stage entry points."""
+    wl = dev.wl
+    T, d, f, E, k = wl.T, wl.d, wl.f, wl.E, wl.k
+    S = T * k
+    sh = dev.shape(0)
+    cu = lambda *shape, dt: torch.empty(*shape, dtype=dt, device="cuda")
+    o = dict(idx=cu(S, dt=torch.int32), w=cu(S, dt=torch.float32), p=cu(S, dt=torch.float32),
+             counts=cu(E, dt=torch.int32), offsets=cu(E + 1, dt=torch.int32), slot_pos=cu(S, dt=torch.int32),
+             perm_slot=cu(S, dt=torch.int32), x_perm=cu(S, d, dt=torch.bfloat16), h=cu(S, f, dt=torch.bfloat16),
+             y_perm=cu(S, d, dt=torch.bfloat16), y=cu(T, d, dt=torch.bfloat16))
+    nws = max(moe.moe_workspace_size_q4(sh), moe.moe_workspace_size(sh))
+    ws = cu(nws, dt=torch.uint8)
+    moe.check(moe.moe_router_topk(sh, dev.x, dev.Wg, None, o["idx"], o["w"], o["p"], o["counts"]), "router")
+    moe.check(moe.moe_permute(sh, dev.x, o["idx"], o["p"], o["counts"], o["offsets"], o["slot_pos"],
+                              o["perm_slot"], o["x_perm"], ws, nws), "permute")
+    moe.check(moe.moe_grouped_swiglu_q4(sh, o["x_perm"], o["offsets"], *dev.q, o["h"], o["y_perm"], ws, nws),
+              "grouped_swiglu_q4")
+    moe.check(moe.moe_combine(sh, o["y_perm"], o["slot_pos"], o["w"], o["y"]), "combine")
+    st = moe.moe_read_device_status(ws)
+    assert st == moe.MOE_OK, moe.status_string(st)
+    torch.cuda.synchronize()
+    return o

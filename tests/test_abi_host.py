@@ -103,3 +103,30 @@ def test_selftest_arguments(moe):
     assert moe.moe_selftest_wait_timeout(ok, 128, 1000, 0) == moe.MOE_ERR_WORKSPACE
     assert moe.moe_selftest_wait_timeout(ok, 1 << 16, 0, 0) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_selftest_wait_timeout(ok, 1 << 16, 20_000_000, 0) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_q4_arguments_rejected_before_device(moe):
+    sh = moe.make_shape(64, 128, 448)
+    assert moe.moe_workspace_size_q4(moe.make_shape(64, 100, 448)) == 0
+    n = moe.moe_workspace_size_q4(sh)
+    assert n > 0
+    ok = 1 << 20
+    q = (ok, ok)
+    E, W = moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_WORKSPACE
+    assert moe.moe_layer_forward_q4(sh, ok, ok, (None, ok), q, q, ok, None, None, ok, n, 0) == E
+    assert moe.moe_layer_forward_q4(sh, ok, ok, q, (ok, ok + 2), q, ok, None, None, ok, n, 0) == E
+    assert moe.moe_layer_forward_q4(sh, ok, ok, q, q, q, ok, None, None, ok, n - 1, 0) == W
+    assert moe.moe_grouped_swiglu_q4(sh, ok, ok, q, q, (ok + 8, ok), ok, ok, ok, n, 0) == E
+    assert moe.moe_layer_forward_q4_profiled(sh, ok, ok, q, q, q, ok, [ok] * 6, None, n, 0) == W
+    for bad in ((0, 64, 128), (2, 60, 128), (2, 64, 96), (33, 64, 128), (2, 64, 65600)):
+        assert moe.moe_quantize_q4(ok, *bad, ok, ok, 0) == E
+    assert moe.moe_quantize_q4(ok, 2, 64, 128, ok + 4, ok, 0) == E
+    # T == 0 is a no-op
+    assert moe.moe_layer_forward_q4(moe.make_shape(0, 128, 448), None, None, (None, None), (None, None),
+                                    (None, None), None, None, None, None, 0, 0) == moe.MOE_OK
+
+
+def test_q4_workspace_holds_partials(moe):
+    for T in (1, 16, 129, 4096):
+        sh = moe.make_shape(T, 4096, 14336)
+        assert moe.moe_workspace_size_q4(sh) >= T * 2 * 4096 * 4  # at least one fp32 partial buffer
