@@ -229,8 +229,90 @@ class Run:
         return ms, nbytes, nbytes
 
 
+class RunQ4(Run):
+    """The decode workload with 4-bit expert weights (quantised on the device
+    by moe_quantize_q4 from the same bf16 weights)."""
+
+    def __init__(self, wl, weights_dev, torch, moe):
+        self.wl, self.torch, self.moe = wl, torch, moe
+        _, W1, W3, W2 = weights_dev
+        self.layer = moe.MoELayerQ4.from_bf16(torch.from_numpy(wl.Wg).cuda(), W1, W3, W2, k=wl.k,
+                                              capacity_factor=wl.capacity_factor, drop_policy=wl.drop_policy)
+        self.x = to_dev_bf16(wl.x, torch)
+        self.y = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+        self.counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+
+    def profiled(self, steps):
+        torch, moe = self.torch, self.moe
+        L = self.layer
+        sums = np.zeros(5)
+        sh, ws = L.shape(self.wl.T), L.workspace(self.wl.T)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            moe.check(moe.moe_layer_forward_q4_profiled(sh, self.x, L.Wg, L.q1, L.q3, L.q2, self.y, evs[i], ws,
+                                                        ws.numel()), "moe_layer_forward_q4_profiled")
+        torch.cuda.synchronize()
+        for i in range(steps):
+            sums += [evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
+        return dict(zip(["router", "capacity_and_permute", "gemm1_swiglu", "gemm2", "combine"],
+                        (sums / steps).tolist()))
+
+    def e2e(self, steps, dist):
+        """As Run.e2e, with the host copies queued by torch around
+        moe_layer_forward_q4 on each of the two streams."""
+        torch, moe = self.torch, self.moe
+        wl, L = self.wl, self.layer
+        layers = [L, moe.MoELayerQ4(L.Wg, L.q1, L.q3, L.q2, k=wl.k, capacity_factor=wl.capacity_factor,
+                                    drop_policy=wl.drop_policy)]
+        streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+        xh = [torch.from_numpy(np.ascontiguousarray(wl.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+              for _ in range(2)]
+        yh = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        xd = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        yd = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+
+        def one(j):
+            with torch.cuda.stream(streams[j]):
+                xd[j].copy_(xh[j], non_blocking=True)
+                layers[j].forward(xd[j], yd[j], stream=streams[j])
+                yh[j].copy_(yd[j], non_blocking=True)
+
+        for j in range(2):
+            one(j)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        cur = torch.cuda.current_stream()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(cur)
+        for s_ in streams:
+            s_.wait_event(start)
+        for i in range(steps):
+            one(i & 1)
+        for s_ in streams:
+            ev = torch.cuda.Event()
+            ev.record(s_)
+            cur.wait_event(ev)
+        end.record(cur)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        ms = max_over_ranks(start.elapsed_time(end), torch, dist)
+        for j in range(2):
+            if layers[j].device_status(wl.T) != moe.MOE_OK:
+                raise RuntimeError("device status after the end-to-end run")
+        nbytes = wl.T * wl.d * 2
+        return ms, nbytes, nbytes
+
+
 def expert_bytes(d, f):
     return 3 * d * f * 2
+
+
+def expert_bytes_q4(d, f):
+    """codes (half a byte per weight) + one bf16 scale per 64 weights"""
+    return 3 * (d * f // 2 + (d * f // 64) * 2)
 
 
 def cpu_baseline(wl, n_sample=48):
@@ -345,10 +427,10 @@ def run_ours(args):
     out = {}
     # decode first: the light, bandwidth-bound workload is measured before the
     # power-capped prefill phase heats the GPU; a short pause separates them
-    for name in ("decode", "prefill"):
+    for name in ("decode", "decode_q4", "prefill"):
         time.sleep(1.0)
-        wl = make_workload(name, rank)
-        run = Run(wl, Wd, torch, moe)
+        wl = make_workload("decode" if name == "decode_q4" else name, rank)
+        run = (RunQ4 if name == "decode_q4" else Run)(wl, Wd, torch, moe)
         N, touched = run.kept_and_touched()
         for _ in range(args.warmup):
             run.step()
@@ -392,6 +474,22 @@ def run_ours(args):
                    e2e=dict(value=weak_scaling_value(world, wq.T, q["e2e_ms"]), unit="tokens/s",
                             h2d_bytes_per_step=q["h2d"], d2h_bytes_per_step=q["d2h"]),
                    experts_touched=q["touched"])
+        q4 = out["decode_q4"]
+        g1_bytes_q4 = q4["touched"] * 2 * expert_bytes_q4(d, f) // 3 + q4["N"] * d * 2 + q4["N"] * f * 2
+        layer_bytes_q4 = q4["touched"] * expert_bytes_q4(d, f) + wq.T * d * 2 * 2 + E * d * 4 + 2 * q4["N"] * f * 2
+        q4_g1_ms = q4["stages"]["gemm1_swiglu"]
+        dec_q4 = dict(workload=workload_desc(wq) + ", 4-bit expert weights (one bf16 scale per 64)",
+                      value=weak_scaling_value(world, wq.T, q4["ms"]), unit="tokens/s", ms_per_step=q4["ms"],
+                      stage_ms=q4["stages"], layer_gbs=layer_bytes_q4 / (q4["ms"] * 1e-3) / 1e9,
+                      layer_frac_hbm=layer_bytes_q4 / (q4["ms"] * 1e-3) / 1e9 / peaks["hbm"],
+                      roofline=dict(bound="hbm", kernel="4-bit gate/up-projection GEMM (SwiGLU fused)",
+                                    achieved=g1_bytes_q4 / (q4_g1_ms * 1e-3) / 1e9, peak=peaks["hbm"], unit="GB/s",
+                                    frac=g1_bytes_q4 / (q4_g1_ms * 1e-3) / 1e9 / peaks["hbm"],
+                                    traffic=traffic_record("expert_gemm_q4_kernel<0,16>", "decode_q4"),
+                                    peak_source=f"{peaks['source']} HBM copy bandwidth"),
+                      e2e=dict(value=weak_scaling_value(world, wq.T, q4["e2e_ms"]), unit="tokens/s",
+                               h2d_bytes_per_step=q4["h2d"], d2h_bytes_per_step=q4["d2h"]),
+                      experts_touched=q4["touched"])
         kernels_per_step = 5 + (1 if (wl.capacity_factor > 0 and wl.drop_policy == 0) else 0)
         line = dict(
             metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
@@ -412,6 +510,7 @@ def run_ours(args):
             gpu_launches=kernels_per_step * args.steps,
             clocks=clocks,
             decode=dec,
+            decode_q4=dec_q4,
         )
         if world == 1 and not args.no_cpu_baseline:
             wl.W1, wl.W3, wl.W2 = W1, W3, W2

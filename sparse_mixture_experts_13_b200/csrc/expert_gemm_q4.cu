@@ -26,15 +26,20 @@
 //   warp 1      allocates tensor memory; one thread issues tcgen05.mma
 //               kind::f16 with A read from tensor memory, B from shared memory;
 //   warps 2-5   epilogue (SiLU * mul, or fp32 split-K partials);
-//   warps 6-13  dequantise: thread i of warp w owns weight row 32 (w % 4) + i
-//               (its tensor-memory lane) and one 64-input half of the stage;
-//               it converts 64 codes to bf16, multiplies by the block scale and
-//               writes 32 columns of the A buffer with tcgen05.st.
-// Four A buffers of 64 columns sit behind the two accumulators.  Reading the
+//   warps 6-21  dequantise: thread i of warp w owns weight row 32 (w % 4) + i
+//               (its tensor-memory lane) and a quarter (32 inputs) of the
+//               stage; it turns 32 codes into bf16, multiplies by the block
+//               scale and writes 16 columns of the A buffer with tcgen05.st.
+// Four A buffers of 64 columns sit behind the two accumulators.  An A buffer
+// is reused once the MMAs of the stage that last read it have completed,
+// which the one commit per stage that frees the stage's shared memory also
+// reports (a commit costs about as much to issue as an MMA).  Reading the
 // 4-bit codes moves a quarter of the bf16 bytes from HBM; the bf16 weights
 // never pass through shared memory.
 #include <cstdint>
 #include <cstdio>
+
+#include <cuda_bf16.h>
 
 #include "moe_internal.h"
 #include "sm100.cuh"
@@ -44,9 +49,9 @@ namespace moe {
 namespace {
 
 constexpr int KQ = 128;                  // inputs per stage (two scale blocks)
-constexpr int kQ4Threads = 14 * 32;
 constexpr int kDeqWarp0 = 6;             // first dequantising warp
-constexpr int kDeqWarps = 8;
+constexpr int kDeqWarps = 16;
+constexpr int kQ4Threads = (kDeqWarp0 + kDeqWarps) * 32;
 constexpr int kCodeBytes = 128 * KQ / 2;  // 128 rows x 64 bytes
 constexpr int kScaleBytes = 1024;         // 2 blocks x 128 rows x bf16 = 512, padded
 constexpr int kABufs = 4;
@@ -60,14 +65,15 @@ template <int EPI, int BN>
 struct Q4Cfg {
   static constexpr int B_BYTES = BN * KQ * 2;  // two 64-input chunks of BN token rows
   static constexpr int STAGE_BYTES = B_BYTES + kCodeBytes + kScaleBytes;
-  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 12 ? 12 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = (212 * 1024) / STAGE_BYTES > 12 ? 12 : (212 * 1024) / STAGE_BYTES;
   static constexpr int XBUF_BYTES = (EPI == Q4_SWIGLU) ? 64 * 16 * 4 : 0;
-  static constexpr int BAR_BYTES = (2 * STAGES + 2 * kABufs + 5) * 8;
+  static constexpr int BAR_BYTES = (2 * STAGES + kABufs + 5) * 8;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + XBUF_BYTES + BAR_BYTES;
   static constexpr uint32_t IDESC = make_idesc_bf16(128, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "MMA N");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(2 * BN <= kACol0, "accumulators overlap the A buffers");
+  static_assert(STAGES > kABufs, "A-buffer reuse is read from the stage barriers");
   static_assert(STAGES >= 3 && SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -120,32 +126,27 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
-// 32 lanes x 32 consecutive columns from registers: thread i writes lane
+// 32 lanes x 16 consecutive columns from registers: thread i writes lane
 // (base lane + i).
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
+// (code - 8) * s for the two codes in bits 0..3 and 16..19 of `bits`.
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t bits, __nv_bfloat162 s2) {
+  const uint32_t b = (bits & 0x000F000Fu) | 0x43004300u;  // 128 + code, exact
+  const uint32_t k136 = 0x43084308u;                       // 136 in both halves
+  const __nv_bfloat162 w = __hmul2(__hsub2(*reinterpret_cast<const __nv_bfloat162*>(&b),
+                                           *reinterpret_cast<const __nv_bfloat162*>(&k136)),
+                                   s2);
+  return *reinterpret_cast<const uint32_t*>(&w);
 }
 
 template <int EPI, int BN>
@@ -172,8 +173,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* afull_bar = bars + 2 * STAGES;
-  uint64_t* aempty_bar = bars + 2 * STAGES + kABufs;
-  uint64_t* tfull_bar = bars + 2 * STAGES + 2 * kABufs;
+  uint64_t* tfull_bar = bars + 2 * STAGES + kABufs;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* drain_bar = tfull_bar + 4;
 
@@ -191,10 +191,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int a = 0; a < kABufs; ++a) {
-      mbar_init(&afull_bar[a], kDeqWarps);
-      mbar_init(&aempty_bar[a], 1);
-    }
+    for (int a = 0; a < kABufs; ++a) mbar_init(&afull_bar[a], kDeqWarps);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
       mbar_init(&tempty_bar[a], 4);
@@ -304,8 +301,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
             umma_bf16_ts(d_tmem, a_tmem + kk * 8, make_sdesc_sw128(b_addr + (kk >> 2) * (BN * 128) + (kk & 3) * 32),
                          C::IDESC, (kq > t.kq0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&empty_bar[stage]);
-          umma_commit(&aempty_bar[abuf]);
+          umma_commit(&empty_bar[stage]);  // frees the stage and its A buffer
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -326,46 +322,48 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
       mbar_wait(drain_bar, 0, nullptr);
     }
   } else if (warp >= kDeqWarp0) {
-    // ------------------------------------------------ dequantise (warps 6..13)
-    const int q = warp & 3;                   // TMEM lane quarter
-    const int half = (warp - kDeqWarp0) >> 2;  // inputs 64*half .. +63 of the stage
-    const int r = q * 32 + lane;               // weight row of the A tile
-    // scale of this row's block in the stage's scale tile
-    const int s_idx = (EPI == Q4_SWIGLU) ? ((r >> 6) * 128 + half * 64 + (r & 63)) : (half * 128 + r);
+    // ------------------------------------------------ dequantise (warps 6..21)
+    const int q = warp & 3;                      // TMEM lane quarter
+    const int part = (warp - kDeqWarp0) >> 2;    // inputs 32*part .. +31 of the stage
+    const int r = q * 32 + lane;                 // weight row of the A tile
+    const int s_idx = (EPI == Q4_SWIGLU) ? ((r >> 6) * 128 + (part >> 1) * 64 + (r & 63)) : ((part >> 1) * 128 + r);
     // codes: row r is 64 bytes; 16-byte chunk c sits at chunk c ^ ((r >> 1) & 3) (64-byte swizzle)
-    const uint32_t sw = (uint32_t)((r >> 1) & 3);
-    const uint32_t c_off0 = (uint32_t)r * 64 + (((uint32_t)(2 * half) ^ sw) << 4);
-    const uint32_t c_off1 = (uint32_t)r * 64 + (((uint32_t)(2 * half + 1) ^ sw) << 4);
-    const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + kACol0 + half * 32;
+    const uint32_t c_off = (uint32_t)r * 64 + (((uint32_t)part ^ (uint32_t)((r >> 1) & 3)) << 4);
+    const uint32_t t_col = tmem_base + ((uint32_t)(q * 32) << 16) + kACol0 + part * 16;
     int stage = 0, abuf = 0;
-    uint32_t phase = 0, aphase = 0;
+    uint32_t phase = 0;
+    int64_t i = 0;  // stages dequantised so far
     bool ok = true;
     for (int32_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       Q4Tile t;
       q4_decode_tile<EPI, BN>(p, s_off, s_base, tile, t);
-      for (int32_t kq = t.kq0; kq < t.kq1; ++kq) {
-        if (!mbar_wait(&full_bar[stage], phase, &s_abort) ||
-            !mbar_wait(&aempty_bar[abuf], aphase ^ 1, &s_abort)) {
+      for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i) {
+        bool w_ok = mbar_wait(&full_bar[stage], phase, &s_abort);
+        if (w_ok && i >= kABufs) {
+          // the A buffer was last read by the MMAs of stage i - kABufs; the
+          // barrier cannot have moved on further, since that needs stage
+          // i - kABufs + STAGES, which this warp has not dequantised yet
+          const int64_t j = i - kABufs;
+          w_ok = mbar_wait(&empty_bar[j % STAGES], (uint32_t)((j / STAGES) & 1), &s_abort);
+        }
+        if (!w_ok) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint8_t* st = smem + stage * C::STAGE_BYTES + C::B_BYTES;
-        const uint4 w0 = *reinterpret_cast<const uint4*>(st + c_off0);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(st + c_off1);
-        const uint32_t sb = *reinterpret_cast<const uint16_t*>(st + kCodeBytes + 2 * s_idx);
-        const uint32_t s2 = sb | (sb << 16);
-        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint32_t v[32];
+        const uint4 w4 = *reinterpret_cast<const uint4*>(st + c_off);
+        const uint16_t sb = *reinterpret_cast<const uint16_t*>(st + kCodeBytes + 2 * s_idx);
+        const uint32_t s2u = uint32_t(sb) | (uint32_t(sb) << 16);
+        const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
+        const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
+        uint32_t v[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int k = 0; k < 4; ++k) {
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint32_t b = ((words[i] >> (4 * m)) & 0x000F000Fu) | 0x43004300u;  // 128 + code
-            v[4 * i + m] = bf16x2_mul(bf16x2_sub(b, 0x43084308u), s2);              // (code - 8) * s
-          }
+          for (int m = 0; m < 4; ++m) v[4 * k + m] = dequant_pair(words[k] >> (4 * m), s2);
         }
-        tmem_st_32x32b_x32(t_row + abuf * kACols, v);
+        tmem_st_32x32b_x16(t_col + abuf * kACols, v);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -374,10 +372,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
           stage = 0;
           phase ^= 1;
         }
-        if (++abuf == kABufs) {
-          abuf = 0;
-          aphase ^= 1;
-        }
+        if (++abuf == kABufs) abuf = 0;
       }
     }
     if (!ok) {

@@ -63,3 +63,67 @@ class MoELayer:
 
     def device_status(self, T: int) -> int:
         return _lib.moe_read_device_status(self.workspace(T))
+
+
+class MoELayerQ4:
+    """One MoE layer with 4-bit expert weights on one CUDA device: Wg [E, d]
+    fp32 and, per expert matrix, a (codes, scales) pair -- codes [E, R, K/2]
+    uint8, scales [E, K/64, R] bf16 (W1, W3: R = d_ff, K = d_model; W2: R =
+    d_model, K = d_ff).  The computation is ``moe_layer_forward_q4``."""
+
+    def __init__(self, Wg: torch.Tensor, q1, q3, q2, k: int = 2, capacity_factor: float = 0.0,
+                 drop_policy: int = _lib.MOE_DROP_BY_PROB):
+        for c, s in (q1, q3, q2):
+            if c.dtype != torch.uint8 or s.dtype != torch.bfloat16 or not (c.is_cuda and s.is_cuda) or \
+                    not (c.is_contiguous() and s.is_contiguous()):
+                raise ValueError("4-bit weights must be contiguous CUDA (uint8 codes, bf16 scales) pairs")
+        if Wg.dtype != torch.float32 or not Wg.is_cuda or not Wg.is_contiguous():
+            raise ValueError("Wg must be a contiguous CUDA fp32 tensor")
+        self.Wg, self.q1, self.q3, self.q2 = Wg, q1, q3, q2
+        self.E, self.f, half_d = q1[0].shape
+        self.d = 2 * half_d
+        self.k = k
+        self.capacity_factor = capacity_factor
+        self.drop_policy = drop_policy
+        self._ws = {}
+
+    @staticmethod
+    def quantize_matrix(W: torch.Tensor, stream=None):
+        """bf16 [E, R, K] on the device -> (codes, scales) with moe_quantize_q4."""
+        E, R, K = W.shape
+        codes = torch.empty(E, R, K // 2, dtype=torch.uint8, device=W.device)
+        scales = torch.empty(E, K // 64, R, dtype=torch.bfloat16, device=W.device)
+        _lib.check(_lib.moe_quantize_q4(W, E, R, K, codes, scales, stream), "moe_quantize_q4")
+        return codes, scales
+
+    @classmethod
+    def from_bf16(cls, Wg, W1, W3, W2, **kw) -> "MoELayerQ4":
+        q = [cls.quantize_matrix(W) for W in (W1, W3, W2)]
+        return cls(Wg, *q, **kw)
+
+    def shape(self, T: int) -> _lib.moe_shape:
+        return _lib.make_shape(T, self.d, self.f, self.E, self.k, self.capacity_factor, self.drop_policy)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        ws = self._ws.get(T)
+        if ws is None:
+            n = _lib.moe_workspace_size_q4(self.shape(T))
+            if n == 0:
+                raise ValueError("invalid layer shape")
+            ws = torch.empty(n, dtype=torch.uint8, device=self.Wg.device)
+            self._ws[T] = ws
+        return ws
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, topk_idx: torch.Tensor | None = None,
+                counts: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.d), dtype=torch.bfloat16, device=x.device)
+        ws = self.workspace(T)
+        st = _lib.moe_layer_forward_q4(self.shape(T), x, self.Wg, self.q1, self.q3, self.q2, y, topk_idx, counts,
+                                       ws, ws.numel(), stream)
+        _lib.check(st, "moe_layer_forward_q4")
+        return y
+
+    def device_status(self, T: int) -> int:
+        return _lib.moe_read_device_status(self.workspace(T))

@@ -22,7 +22,7 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 from . import _lib  # noqa: E402
-from .layer import MoELayer  # noqa: E402
+from .layer import MoELayer, MoELayerQ4  # noqa: E402
 
 
 def main(argv=None):
@@ -36,14 +36,19 @@ def main(argv=None):
     ap.add_argument("--policy", type=int, default=0)
     ap.add_argument("--variant", type=int, default=0)
     ap.add_argument("--skew", action="store_true")
+    ap.add_argument("--q4", action="store_true", help="4-bit expert weights (quantised on the device)")
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=1)
     a = ap.parse_args(argv)
     wl = synth.Workload("case", a.T, a.d, a.f, E=a.E, k=a.k, capacity_factor=a.cf, drop_policy=a.policy,
                         skew=a.skew).generate()
     dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).cuda()
-    layer = MoELayer(torch.from_numpy(wl.Wg).cuda(), dev(wl.W1), dev(wl.W3), dev(wl.W2), k=a.k,
-                     capacity_factor=a.cf, drop_policy=a.policy, gemm_variant=a.variant)
+    if a.q4:
+        layer = MoELayerQ4.from_bf16(torch.from_numpy(wl.Wg).cuda(), dev(wl.W1), dev(wl.W3), dev(wl.W2), k=a.k,
+                                     capacity_factor=a.cf, drop_policy=a.policy)
+    else:
+        layer = MoELayer(torch.from_numpy(wl.Wg).cuda(), dev(wl.W1), dev(wl.W3), dev(wl.W2), k=a.k,
+                         capacity_factor=a.cf, drop_policy=a.policy, gemm_variant=a.variant)
     x = dev(wl.x)
     y = torch.empty(a.T, a.d, dtype=torch.bfloat16, device="cuda")
     for _ in range(a.warmup):
@@ -59,7 +64,7 @@ def main(argv=None):
     _lib.check(st, "device status")
     ms = s.elapsed_time(e) / max(1, a.iters)
     flops = 6.0 * a.T * a.k * a.d * a.f + 2.0 * a.T * a.d * a.E
-    print(f"T={a.T} d={a.d} f={a.f} E={a.E} k={a.k} cf={a.cf} variant={a.variant}: {ms:.4f} ms/step, "
+    print(f"T={a.T} d={a.d} f={a.f} E={a.E} k={a.k} cf={a.cf} variant={a.variant} q4={a.q4}: {ms:.4f} ms/step, "
           f"{a.T / ms * 1e3:.1f} tokens/s, {flops / ms / 1e9:.1f} TFLOP/s (dropless count)")
 
 
