@@ -54,6 +54,7 @@ def _bind(path: str):
         "oracle_expert_row": [i32, i32, P, P, P, P, P, P],
         "oracle_layer_rows": [i64, i32, i32, i32, i32, P, P, P, P, P, P, P, i64, P, P, P, P],
         "oracle_num_threads": [],
+        "oracle_router_stats": [i64, i32, i32, P, P, P],
         "oracle_q4_quantize": [i32, i32, i32, P, P, P],
         "oracle_q4_dequant": [i32, i32, i32, P, P, P],
         "oracle_expert_row_q4": [i32, i32, P, P, P, P, P, P, P, P, P],
@@ -202,6 +203,16 @@ class Oracle:
         if want_o:
             out["o"] = o
         return out
+
+    def router_stats(self, idx: np.ndarray, E: int):
+        """Per-slot expert histograms [k, E] and first-two-choice pair counts
+        [E, E] of top-k indices idx [T, k]."""
+        idx = np.ascontiguousarray(idx, np.int32)
+        T, k = idx.shape
+        slot = np.empty((k, E), np.int32)
+        pair = np.empty((E, E), np.int32)
+        self.L.oracle_router_stats(T, E, k, self._p(idx), self._p(slot), self._p(pair))
+        return slot, pair
 
     # ------------------------------------------------------------ 4-bit experts
     def q4_quantize(self, W: np.ndarray):

@@ -264,6 +264,24 @@ void oracle_layer_rows(int64_t T, int32_t d, int32_t f, int32_t E, int32_t k, co
   }
 }
 
+/* Router statistics [P1] "Expert specialization" (get_expert_activations:
+ * per layer, the bincount of the top-2 expert indices over all tokens) and
+ * [P5] "Inspecting Expert Routing" (the most common expert in each top-k
+ * position).  slot_counts[j * E + e] = number of tokens whose j-th choice is
+ * e; pair_counts[a * E + b] = number of tokens whose first two choices are
+ * (a, b) (k >= 2; may be NULL).  Summing slot_counts over j gives the
+ * bincount of the flattened top-k indices. */
+void oracle_router_stats(int64_t T, int32_t E, int32_t k, const int32_t *idx, int32_t *slot_counts,
+                         int32_t *pair_counts) {
+  for (int64_t i = 0; i < (int64_t)k * E; ++i) slot_counts[i] = 0;
+  if (pair_counts)
+    for (int64_t i = 0; i < (int64_t)E * E; ++i) pair_counts[i] = 0;
+  for (int64_t t = 0; t < T; ++t) {
+    for (int32_t j = 0; j < k; ++j) slot_counts[j * E + idx[t * k + j]] += 1;
+    if (pair_counts && k >= 2) pair_counts[idx[t * k] * E + idx[t * k + 1]] += 1;
+  }
+}
+
 /* ------------------------------------------------------------------------
  * 4-bit expert weights.
  *  [P1] "Deployment tradeoffs you'll actually hit", "Quantization asymmetry":

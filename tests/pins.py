@@ -420,3 +420,35 @@ Q4_PINS = [pin_q4_format_worked_example, pin_q4_lossless_roundtrip, pin_q4_error
            pin_q4_layer_matches_bf16_on_exact_weights]
 
 ALL_PINS = ALL_PINS + Q4_PINS
+
+
+# ------------------------------------------------------------ router statistics
+
+def pin_router_stats(o):
+    """The worked example's token picks experts 0 then 2; per-slot histograms
+    sum to T per slot and, over the slots, to the bincount of the flattened
+    top-k indices (numpy); the pair counts' margins are the first two slots'
+    histograms and their diagonal is empty (the k experts are distinct)."""
+    g = read_golden("worked_routing_example.txt")
+    scores = np.array([float(v) for v in g["scores"]], np.float64)[None, :]
+    slot, pair = o.router_stats(o.topk(scores, 2), 8)
+    want = np.zeros((2, 8), np.int32)
+    want[0, 0] = want[1, 2] = 1
+    assert np.array_equal(slot, want) and pair[0, 2] == 1 and pair.sum() == 1
+    for E, k in ((8, 2), (16, 4), (4, 1)):
+        x, Wg, *_ = tiny_problem(T=50, d=32, f=32, E=E, seed=E * k)
+        idx = o.topk(o.router_logits(x, Wg), k)
+        slot, pair = o.router_stats(idx, E)
+        assert np.all(slot.sum(1) == 50)
+        assert np.array_equal(slot.sum(0), np.bincount(idx.ravel(), minlength=E))
+        for j in range(k):
+            assert np.array_equal(slot[j], np.bincount(idx[:, j], minlength=E))
+        if k >= 2:
+            assert np.array_equal(pair.sum(1), slot[0]) and np.array_equal(pair.sum(0), slot[1])
+            assert np.trace(pair) == 0
+            brute = np.zeros((E, E), np.int64)
+            np.add.at(brute, (idx[:, 0], idx[:, 1]), 1)
+            assert np.array_equal(pair, brute)
+
+
+ALL_PINS = ALL_PINS + [pin_router_stats]

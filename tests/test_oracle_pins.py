@@ -60,6 +60,9 @@ MUTANTS = [
     ("dropped slot still added", "if (!kept[s]) {", "if (0) {"),
     ("grouping in reverse token order", "for (int64_t s = 0; s < S; ++s) {\n      if (idx[s] != e) continue;",
      "for (int64_t s = S - 1; s >= 0; --s) {\n      if (idx[s] != e) continue;"),
+    ("stats slot index swapped", "slot_counts[j * E + idx[t * k + j]] += 1;", "slot_counts[(k - 1 - j) * E + idx[t * k + j]] += 1;"),
+    ("stats pair transposed", "pair_counts[idx[t * k] * E + idx[t * k + 1]] += 1;",
+     "pair_counts[idx[t * k + 1] * E + idx[t * k]] += 1;"),
     ("q4 codes in plain nibble order", "int nib = j / 2 + 4 * (j % 2);", "int nib = j;"),
     ("q4 high and low nibble swapped", "*shift = 4 * (nib % 2);", "*shift = 4 * (1 - nib % 2);"),
     ("q4 scales read row-major", "bf16_to_double(scales_e[(k / 64) * R + r]);",
