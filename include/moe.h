@@ -216,6 +216,24 @@ MOE_API moe_status moe_layer_forward_host(const moe_shape *shape, const moe_bf16
                                   const moe_bf16 *W2, moe_bf16 *y_host, void *ws,
                                   size_t ws_bytes, moe_stream_t stream);
 
+/* Router statistics of one layer's top-k indices (device topk_idx [T, k], as
+ * written by moe_router_topk or returned by moe_layer_forward):
+ *   slot_counts [k, E] int32 (out): slot_counts[j][e] = number of tokens whose
+ *       j-th choice (j = 0 the largest logit) is expert e.  The sum over j is
+ *       the bincount of the flattened top-k indices, i.e. the layer's counts.
+ *   pair_counts [E, E] int32 (out, nullable, needs k >= 2): pair_counts[a][b] =
+ *       number of tokens whose first two choices are (a, b).
+ * accumulate = 0 overwrites the outputs, 1 adds to them (e.g. over batches,
+ * or into row `layer` of a [layers, ...] table).  The most common expert of
+ * position j is the argmax of slot_counts[j].  Sources: "How Mixtral 8x7B
+ * uses mixture of experts", "Expert specialization" (per-layer bincount of the
+ * top-2 indices) and "Mixtral 8x7B — MoE Complete Guide", "Inspecting Expert
+ * Routing" (most common expert per top-k position).  Indices outside [0, E)
+ * are not counted.  Asynchronous on `stream`; allocates nothing.  T == 0
+ * only clears the outputs (accumulate = 0). */
+MOE_API moe_status moe_router_stats(const moe_shape *shape, const int32_t *topk_idx, int32_t *slot_counts,
+                                    int32_t *pair_counts, int32_t accumulate, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- 4-bit experts
  * Sources: "How Mixtral 8x7B uses mixture of experts", "Deployment tradeoffs
  * you'll actually hit" / "Quantization asymmetry" (keep the router in 16-bit

@@ -21,7 +21,7 @@ MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM, MOE_VARIANT_TILED_SINGL
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc",
-            "moe_selftest_wait_timeout", "moe_read_device_status", "moe_quantize_q4", "moe_workspace_size_q4",
+            "moe_selftest_wait_timeout", "moe_read_device_status", "moe_router_stats", "moe_quantize_q4", "moe_workspace_size_q4",
             "moe_grouped_swiglu_q4", "moe_layer_forward_q4", "moe_layer_forward_q4_profiled", "moe_status_string")
 _SIZE_RETURNING = ("moe_workspace_size", "moe_workspace_size_q4")
 
@@ -67,6 +67,7 @@ def lib():
         L.moe_layer_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.moe_read_device_status.argtypes = [P, P]
         L.moe_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_uint32, P]
+        L.moe_router_stats.argtypes = [S, P, P, P, ctypes.c_int32, P]
         L.moe_quantize_q4.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P]
         L.moe_workspace_size_q4.argtypes = [S]
         L.moe_grouped_swiglu_q4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, sz, P]
@@ -167,6 +168,12 @@ def _event_handles(events):
                 ev.record()  # creates the underlying event
             handles.append(ev.cuda_event)
     return (ctypes.c_void_p * 6)(*handles)
+
+
+def moe_router_stats(shape, topk_idx, slot_counts, pair_counts=None, accumulate=0, stream=None) -> int:
+    """Per-slot expert histograms [k, E] and first-two-choice pair counts [E, E]."""
+    return lib().moe_router_stats(ctypes.byref(shape), _p(topk_idx), _p(slot_counts), _p(pair_counts),
+                                  int(accumulate), _stream(stream))
 
 
 # ------------------------------------------------------------ 4-bit experts

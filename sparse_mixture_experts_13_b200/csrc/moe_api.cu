@@ -477,6 +477,19 @@ moe_status moe_layer_forward_host(const moe_shape* sh, const moe_bf16* x_host, c
   return cuda_status(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s));
 }
 
+moe_status moe_router_stats(const moe_shape* sh, const int32_t* topk_idx, int32_t* slot_counts, int32_t* pair_counts,
+                            int32_t accumulate, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  MOE_TRY(check_i32(slot_counts));
+  if (pair_counts && (sh->k < 2 || !aligned(pair_counts, 4))) return MOE_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return MOE_ERR_INVALID_ARG;
+  if (sh->T > 0) MOE_TRY(check_i32(topk_idx));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return cuda_status(launch_router_stats(topk_idx, sh->T, sh->E, sh->k, slot_counts, pair_counts, accumulate != 0,
+                                         sms, (cudaStream_t)stream));
+}
+
 moe_status moe_quantize_q4(const moe_bf16* W, int32_t E, int32_t R, int32_t K, uint8_t* codes, moe_bf16* scales,
                            moe_stream_t stream) {
   if (E < 1 || E > 32 || R < 8 || R > 65536 || R % 8 || K < 64 || K > 65536 || K % 64) return MOE_ERR_INVALID_ARG;

@@ -107,6 +107,11 @@ cudaError_t launch_expert_gemms_q4(const ExpertGemmQ4Args& a, cudaStream_t s);
 cudaError_t launch_quantize_q4(const uint16_t* W, int32_t E, int32_t R, int32_t K, uint8_t* codes,
                                uint16_t* scales, cudaStream_t s);
 
+// Per-slot expert histograms [k, E] and first-two-choice pair counts [E, E]
+// (nullable; k >= 2) of topk_idx [T, k]; zeroed first unless `accumulate`.
+cudaError_t launch_router_stats(const int32_t* idx, int64_t T, int32_t E, int32_t k, int32_t* slot_counts,
+                                int32_t* pair_counts, bool accumulate, int num_sms, cudaStream_t s);
+
 struct CombineArgs {
   const uint16_t* y_perm;   // [S, d] bf16, or nullptr when reading partials
   const float* partials;    // [splits, S, d] fp32 (if y_perm == nullptr)

@@ -130,3 +130,15 @@ def test_q4_workspace_holds_partials(moe):
     for T in (1, 16, 129, 4096):
         sh = moe.make_shape(T, 4096, 14336)
         assert moe.moe_workspace_size_q4(sh) >= T * 2 * 4096 * 4  # at least one fp32 partial buffer
+
+
+def test_router_stats_arguments(moe):
+    sh = moe.make_shape(64, 128, 448)
+    ok = 1 << 20
+    E = moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_router_stats(sh, ok, None, None, 0, 0) == E          # slot_counts missing
+    assert moe.moe_router_stats(sh, None, ok, None, 0, 0) == E          # topk_idx missing
+    assert moe.moe_router_stats(sh, ok, ok + 2, None, 0, 0) == E        # misaligned
+    assert moe.moe_router_stats(sh, ok, ok, ok, 2, 0) == E              # accumulate flag
+    assert moe.moe_router_stats(moe.make_shape(64, 128, 448, E=8, k=1), ok, ok, ok, 0, 0) == E  # pairs need k >= 2
+    assert moe.moe_router_stats(moe.make_shape(64, 100, 448), ok, ok, None, 0, 0) == E
