@@ -29,6 +29,8 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 DROP_BY_PROB, DROP_BY_ORDER = 0, 1
+# the same policies, with a dropped slot moving to the token's next-best expert
+DROP_BY_PROB_NEXT_BEST, DROP_BY_ORDER_NEXT_BEST = 2, 3
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB, defines=()) -> str:
@@ -55,6 +57,7 @@ def _bind(path: str):
         "oracle_layer_rows": [i64, i32, i32, i32, i32, P, P, P, P, P, P, P, i64, P, P, P, P],
         "oracle_num_threads": [],
         "oracle_router_stats": [i64, i32, i32, P, P, P],
+        "oracle_capacity_fallback": [i64, i32, i32, dbl, i32, P, P, P, P, P],
         "oracle_q4_quantize": [i32, i32, i32, P, P, P],
         "oracle_q4_dequant": [i32, i32, i32, P, P, P],
         "oracle_expert_row_q4": [i32, i32, P, P, P, P, P, P, P, P, P],
@@ -66,6 +69,7 @@ def _bind(path: str):
         fn.argtypes = args
         fn.restype = None
     lib.oracle_capacity.restype = ctypes.c_int64
+    lib.oracle_capacity_fallback.restype = ctypes.c_int64
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
@@ -127,6 +131,20 @@ class Oracle:
                                      self._p(kept))
         return kept, (None if cap < 0 else int(cap))
 
+    def capacity_fallback(self, logits: np.ndarray, idx: np.ndarray, p: np.ndarray, E: int, cf: float,
+                          policy: int):
+        """Capacity with the next-best-expert fallback (policy 0 / 1 as in
+        capacity()).  Returns (expert per slot, kept, cap)."""
+        logits = np.ascontiguousarray(logits, np.float64)
+        idx = np.ascontiguousarray(idx, np.int32)
+        p = np.ascontiguousarray(p, np.float64)
+        T, k = idx.shape
+        expert = np.empty(T * k, np.int32)
+        kept = np.empty(T * k, np.uint8)
+        cap = self.L.oracle_capacity_fallback(T, E, k, float(cf), int(policy), self._p(logits), self._p(idx),
+                                              self._p(p), self._p(expert), self._p(kept))
+        return expert, kept, (None if cap < 0 else int(cap))
+
     def permute(self, idx: np.ndarray, kept: np.ndarray, E: int):
         idx = np.ascontiguousarray(idx, np.int32)
         kept = np.ascontiguousarray(kept, np.uint8)
@@ -169,20 +187,28 @@ class Oracle:
             idx = idx.copy()
             idx[rows] = idx_override[rows]
         w, p = self.gates(logits, idx)
+        if policy >= DROP_BY_PROB_NEXT_BEST:
+            assert kept_override is None
+            expert, kept, cap = self.capacity_fallback(logits, idx, p, E, cf, policy - 2)
+            perm = self.permute(expert.reshape(idx.shape), kept, E)
+            # counts stay the router's histogram; the grouping follows `expert`
+            perm["counts"] = np.bincount(idx.ravel(), minlength=E).astype(np.int32)
+            return dict(logits=logits, idx=idx, w=w, p=p, kept=kept, cap=cap, expert=expert.reshape(idx.shape),
+                        **perm)
         kept, cap = self.capacity(idx, p, E, cf, policy)
         if kept_override is not None:
             sel = kept_override >= 0
             kept = kept.copy()
             kept[sel] = kept_override[sel].astype(np.uint8)
         perm = self.permute(idx, kept, E)
-        return dict(logits=logits, idx=idx, w=w, p=p, kept=kept, cap=cap, **perm)
+        return dict(logits=logits, idx=idx, w=w, p=p, kept=kept, cap=cap, expert=idx, **perm)
 
     def layer_rows(self, x, W1, W3, W2, route: dict, rows, want_h: bool = False,
                    want_o: bool = False):
         """y (fp64) for the token indices in ``rows``; optionally per-slot h and o."""
         T, d = x.shape
         E, f, _ = W1.shape
-        idx, w, kept = route["idx"], route["w"], route["kept"]
+        idx, w, kept = route.get("expert", route["idx"]), route["w"], route["kept"]
         k = idx.shape[1]
         rows = np.ascontiguousarray(rows, np.int64)
         n = rows.shape[0]
@@ -241,7 +267,7 @@ class Oracle:
         scales) pairs of W1, W3 [E, f, d] and W2 [E, d, f]."""
         T, d = x.shape
         E, f, _ = q1[0].shape
-        idx, w, kept = route["idx"], route["w"], route["kept"]
+        idx, w, kept = route.get("expert", route["idx"]), route["w"], route["kept"]
         k = idx.shape[1]
         rows = np.ascontiguousarray(rows, np.int64)
         n = rows.shape[0]

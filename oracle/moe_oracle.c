@@ -170,6 +170,84 @@ int64_t oracle_capacity(int64_t T, int32_t E, int32_t k, double cf, int32_t poli
   return cap;
 }
 
+/* Next-best-expert fallback [P1] "Routing without auxiliary loss": the excess
+ * slots of a full expert are processed by a fallback, "typically the
+ * next-best expert".  Reading: after the capacity pass of oracle_capacity,
+ * the dropped slots of token t, in slot order, move to t's next experts in
+ * the router order (logit descending, index ascending) past its top k: the
+ * first dropped slot to rank k, the second to rank k + 1, and so on (none
+ * past rank E - 1).  At each expert the moved slots compete for the capacity
+ * the first pass left (cap minus its kept slots) under the same policy:
+ * policy 0 by the full router probability of the new expert (ties: smaller
+ * token first), policy 1 in token order.  A moved slot keeps its gate weight;
+ * one that does not fit is dropped.  expert[s] = the expert that processes
+ * slot s (its top-k choice, or the fallback it moved to), kept[s] = 1 / 0.
+ * Returns cap, or -1 when dropless. */
+int64_t oracle_capacity_fallback(int64_t T, int32_t E, int32_t k, double cf, int32_t policy,
+                                 const double *logits, const int32_t *idx, const double *p,
+                                 int32_t *expert, uint8_t *kept) {
+  int64_t S = T * k;
+  int64_t cap = oracle_capacity(T, E, k, cf, policy, idx, p, kept);
+  for (int64_t s = 0; s < S; ++s) expert[s] = idx[s];
+  if (cap < 0) return cap;
+  int64_t *used = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+  for (int64_t s = 0; s < S; ++s)
+    if (kept[s]) used[idx[s]] += 1;
+  /* candidates: moved slot s goes to cand_e[s] with probability cand_p[s] */
+  int32_t *cand_e = (int32_t *)malloc(sizeof(int32_t) * (size_t)(S > 0 ? S : 1));
+  double *cand_p = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+  int32_t *order = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+  for (int64_t t = 0; t < T; ++t) {
+    const double *l = logits + t * E;
+    /* router order of all E experts: logit descending, index ascending */
+    for (int32_t e = 0; e < E; ++e) order[e] = e;
+    for (int32_t a = 1; a < E; ++a) {
+      int32_t v = order[a], b = a - 1;
+      while (b >= 0 && (l[order[b]] < l[v] || (l[order[b]] == l[v] && order[b] > v))) {
+        order[b + 1] = order[b];
+        --b;
+      }
+      order[b + 1] = v;
+    }
+    double M = l[order[0]], zE = 0.0;
+    for (int32_t e = 0; e < E; ++e) zE += exp(l[e] - M);
+    int32_t moved = 0;
+    for (int32_t j = 0; j < k; ++j) {
+      int64_t s = t * k + j;
+      cand_e[s] = -1;
+      if (kept[s]) continue;
+      int32_t r = k + moved;
+      ++moved;
+      if (r >= E) continue;
+      cand_e[s] = order[r];
+      cand_p[s] = exp(l[order[r]] - M) / zE;
+    }
+  }
+  prio_t *list = (prio_t *)malloc(sizeof(prio_t) * (size_t)(S > 0 ? S : 1));
+  for (int32_t e = 0; e < E; ++e) {
+    int64_t n = 0;
+    for (int64_t s = 0; s < S; ++s)
+      if (cand_e[s] == e) {
+        list[n].p = cand_p[s];
+        list[n].t = s / k;
+        list[n].s = s;
+        ++n;
+      }
+    if (policy == 0) qsort(list, (size_t)n, sizeof(prio_t), prio_cmp);
+    int64_t room = cap - used[e];
+    for (int64_t r = 0; r < n && r < room; ++r) {
+      kept[list[r].s] = 1;
+      expert[list[r].s] = e;
+    }
+  }
+  free(list);
+  free(order);
+  free(cand_p);
+  free(cand_e);
+  free(used);
+  return cap;
+}
+
 /* Grouping of slots by expert [P1] "The architecture in one diagram" (batch
  * tokens by expert, run the experts, scatter back): for e = 0..E-1, the kept
  * slots routed to e in ascending token order form rows offsets[e] ..

@@ -452,3 +452,114 @@ def pin_router_stats(o):
 
 
 ALL_PINS = ALL_PINS + [pin_router_stats]
+
+
+# --------------------------------------------------- next-best-expert fallback
+
+def skewed_tiny(T=64, E=8, seed=4):
+    """Tiny problem with two hot experts (a constant feature biases the router)."""
+    x, Wg, W1, W3, W2 = tiny_problem(T=T, d=32, f=40, E=E, seed=seed)
+    x = x.copy()
+    Wg = Wg.copy()
+    x[:, 0] = _bf16(np.ones(T))
+    Wg[0, 0] += 1.5
+    Wg[3 % E, 0] += 1.0
+    return x, Wg, W1, W3, W2
+
+
+def _brute_fallback(L, k, cf, policy):
+    """Restatement of the fallback reading with numpy sorts: pass 1 as the
+    capacity brute force, then each token's dropped slots (in slot order)
+    move to its experts at router ranks k, k+1, ...; per expert the moved
+    slots fill what pass 1 left, by full-softmax probability (ties: smaller
+    token) or in token order."""
+    T, E = L.shape
+    order = np.array([sorted(range(E), key=lambda e: (-L[t, e], e)) for t in range(T)])
+    idx = order[:, :k]
+    P = np.exp(L - L.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    cap = int(np.floor(cf * T * k / E))
+    S = T * k
+    kept = _brute_capacity(idx.astype(np.int32), P[np.arange(T)[:, None], idx], E, cap, policy)
+    expert = idx.ravel().copy()
+    room = np.array([cap - sum(1 for s in range(S) if kept[s] and expert[s] == e) for e in range(E)])
+    cands = {e: [] for e in range(E)}
+    for t in range(T):
+        m = 0
+        for j in range(k):
+            s = t * k + j
+            if kept[s]:
+                continue
+            r = k + m
+            m += 1
+            if r < E:
+                cands[order[t, r]].append((s, t, P[t, order[t, r]]))
+    for e, lst in cands.items():
+        if policy == 0:
+            lst = sorted(lst, key=lambda c: (-c[2], c[1]))
+        for s, t, _ in lst[:max(room[e], 0)]:
+            kept[s] = 1
+            expert[s] = e
+    return expert, kept, cap
+
+
+def pin_fallback_bruteforce(o):
+    """The oracle's fallback equals the brute-force restatement; pass 1 is
+    the plain capacity policy; a moved slot lands outside its token's top-k,
+    on ranks k, k+1, ... in slot order; no expert exceeds its capacity; with
+    a huge capacity nothing moves, with capacity 0 nothing is kept."""
+    for (T, E, k, cf) in ((64, 8, 2, 1.0), (48, 8, 3, 0.75), (40, 4, 2, 1.25), (30, 16, 4, 1.0)):
+        x, Wg, *_ = skewed_tiny(T=T, E=E, seed=T + E)
+        L = o.router_logits(x, Wg)
+        for base in (0, 1):
+            r = o.route(x, Wg, k, cf=cf, policy=2 + base)
+            expert, kept, cap = _brute_fallback(L, k, cf, base)
+            assert r["cap"] == cap
+            assert np.array_equal(r["kept"], kept) and np.array_equal(r["expert"].ravel(), expert), (T, E, k, base)
+            plain = o.route(x, Wg, k, cf=cf, policy=base)
+            stayed = r["expert"].ravel() == r["idx"].ravel()
+            assert np.array_equal(plain["kept"].astype(bool), r["kept"].astype(bool) & stayed)
+            moved = np.nonzero(~stayed & (r["kept"] == 1))[0]
+            assert moved.size > 0
+            for s in moved:
+                assert r["expert"].ravel()[s] not in r["idx"][s // k]
+            per = np.bincount(r["expert"].ravel()[r["kept"] == 1], minlength=E)
+            assert per.max() <= cap
+            assert np.array_equal(np.diff(r["offsets"]), per)
+    # experts 4 and 5 with identical router rows: their logits tie exactly, and
+    # a moved slot that reaches the pair takes the smaller index
+    x, Wg, *_ = skewed_tiny(T=96, seed=12)
+    Wg[5] = Wg[4]
+    L = o.router_logits(x, Wg)
+    for base in (0, 1):
+        r = o.route(x, Wg, 2, cf=1.0, policy=2 + base)
+        expert, kept, _ = _brute_fallback(L, 2, 1.0, base)
+        assert np.array_equal(r["expert"].ravel(), expert) and np.array_equal(r["kept"], kept)
+        landed = r["expert"].ravel()[(r["kept"] == 1) & (r["expert"].ravel() != r["idx"].ravel())]
+        assert (landed == 4).any()
+    x, Wg, *_ = skewed_tiny()
+    assert not (o.route(x, Wg, 2, cf=1e9, policy=2)["expert"] != o.route(x, Wg, 2)["idx"]).any()
+    assert not o.route(x, Wg, 2, cf=0.01, policy=3)["kept"].any()
+
+
+def pin_fallback_layer(o):
+    """With the fallback, y(t) = sum over kept slots of w_j * Expert_e(x_t),
+    e the expert the slot landed on (numpy experts), the gate weight being
+    the slot's own top-k weight."""
+    x, Wg, W1, W3, W2 = skewed_tiny()
+    r = o.route(x, Wg, 2, cf=1.0, policy=2)
+    y = o.layer_rows(x, W1, W3, W2, r, np.arange(64))["y"]
+    moved = 0
+    for t in range(64):
+        ref = np.zeros(32)
+        for j in range(2):
+            s = 2 * t + j
+            if r["kept"][s]:
+                e = r["expert"][t, j]
+                moved += e != r["idx"][t, j]
+                ref += r["w"][t, j] * _np_expert(_w(x[t]), W1[e], W3[e], W2[e])[1]
+        assert np.allclose(y[t], ref, rtol=1e-12, atol=1e-13)
+    assert moved > 0
+
+
+ALL_PINS = ALL_PINS + [pin_fallback_bruteforce, pin_fallback_layer]

@@ -63,6 +63,13 @@ MUTANTS = [
     ("stats slot index swapped", "slot_counts[j * E + idx[t * k + j]] += 1;", "slot_counts[(k - 1 - j) * E + idx[t * k + j]] += 1;"),
     ("stats pair transposed", "pair_counts[idx[t * k] * E + idx[t * k + 1]] += 1;",
      "pair_counts[idx[t * k + 1] * E + idx[t * k]] += 1;"),
+    ("fallback always to rank k", "int32_t r = k + moved;", "int32_t r = k;"),
+    ("fallback ignores pass-1 load", "int64_t room = cap - used[e];", "int64_t room = cap;"),
+    ("fallback by order under policy 0", "    if (policy == 0) qsort(list, (size_t)n, sizeof(prio_t), prio_cmp);\n    int64_t room",
+     "    int64_t room"),
+    ("fallback tie to larger logit index",
+     "while (b >= 0 && (l[order[b]] < l[v] || (l[order[b]] == l[v] && order[b] > v))) {",
+     "while (b >= 0 && (l[order[b]] < l[v] || (l[order[b]] == l[v] && order[b] < v))) {"),
     ("q4 codes in plain nibble order", "int nib = j / 2 + 4 * (j % 2);", "int nib = j;"),
     ("q4 high and low nibble swapped", "*shift = 4 * (nib % 2);", "*shift = 4 * (1 - nib % 2);"),
     ("q4 scales read row-major", "bf16_to_double(scales_e[(k / 64) * R + r]);",
