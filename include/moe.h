@@ -77,7 +77,18 @@ typedef enum {
 typedef enum {
   MOE_DROP_BY_PROB = 0, /* keep the cap slots of highest router probability
                            (full softmax over E), ties to the smaller token */
-  MOE_DROP_BY_ORDER = 1 /* keep the first cap slots in token order */
+  MOE_DROP_BY_ORDER = 1, /* keep the first cap slots in token order */
+  /* The same two policies with a next-best-expert fallback ("How Mixtral 8x7B
+   * uses mixture of experts", "Routing without auxiliary loss": the excess is
+   * processed by "typically the next-best expert").  After the capacity pass,
+   * the dropped slots of a token, in slot order, move to its experts at
+   * router ranks k, k+1, ... (logit descending, index ascending); at each
+   * expert they compete under the same policy (probability of that expert,
+   * or token order) for the capacity the first pass left; a moved slot keeps
+   * its gate weight; one that does not fit is dropped.  Whole-layer entry
+   * points only (moe_permute returns MOE_ERR_UNSUPPORTED). */
+  MOE_DROP_BY_PROB_NEXT_BEST = 2,
+  MOE_DROP_BY_ORDER_NEXT_BEST = 3
 } moe_drop_policy;
 
 /* Expert-GEMM schedule.  Both compute the same function. */

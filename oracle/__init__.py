@@ -57,7 +57,7 @@ def _bind(path: str):
         "oracle_layer_rows": [i64, i32, i32, i32, i32, P, P, P, P, P, P, P, i64, P, P, P, P],
         "oracle_num_threads": [],
         "oracle_router_stats": [i64, i32, i32, P, P, P],
-        "oracle_capacity_fallback": [i64, i32, i32, dbl, i32, P, P, P, P, P],
+        "oracle_capacity_fallback": [i64, i32, i32, dbl, i32, P, P, P, P, P, P],
         "oracle_q4_quantize": [i32, i32, i32, P, P, P],
         "oracle_q4_dequant": [i32, i32, i32, P, P, P],
         "oracle_expert_row_q4": [i32, i32, P, P, P, P, P, P, P, P, P],
@@ -132,17 +132,21 @@ class Oracle:
         return kept, (None if cap < 0 else int(cap))
 
     def capacity_fallback(self, logits: np.ndarray, idx: np.ndarray, p: np.ndarray, E: int, cf: float,
-                          policy: int):
+                          policy: int, order_override=None):
         """Capacity with the next-best-expert fallback (policy 0 / 1 as in
-        capacity()).  Returns (expert per slot, kept, cap)."""
+        capacity()).  order_override: (T, E) int array or None; a row whose
+        first entry is >= 0 replaces that token's router order.  Returns
+        (expert per slot, kept, cap)."""
         logits = np.ascontiguousarray(logits, np.float64)
         idx = np.ascontiguousarray(idx, np.int32)
         p = np.ascontiguousarray(p, np.float64)
         T, k = idx.shape
         expert = np.empty(T * k, np.int32)
         kept = np.empty(T * k, np.uint8)
+        ov = None if order_override is None else np.ascontiguousarray(order_override, np.int32)
         cap = self.L.oracle_capacity_fallback(T, E, k, float(cf), int(policy), self._p(logits), self._p(idx),
-                                              self._p(p), self._p(expert), self._p(kept))
+                                              self._p(p), self._p(ov) if ov is not None else None,
+                                              self._p(expert), self._p(kept))
         return expert, kept, (None if cap < 0 else int(cap))
 
     def permute(self, idx: np.ndarray, kept: np.ndarray, E: int):
@@ -173,7 +177,7 @@ class Oracle:
         return h, o
 
     def route(self, x, Wg, k: int, cf: float = 0.0, policy: int = DROP_BY_PROB,
-              idx_override=None, kept_override=None, logits=None) -> dict:
+              idx_override=None, kept_override=None, logits=None, order_override=None) -> dict:
         """Steps logits .. grouping.  ``idx_override``: (T, k) array or None;
         entries >= 0 replace the oracle's top-k choice for that token (all k
         of a row are replaced together).  ``kept_override``: (S,) int array or
@@ -189,7 +193,7 @@ class Oracle:
         w, p = self.gates(logits, idx)
         if policy >= DROP_BY_PROB_NEXT_BEST:
             assert kept_override is None
-            expert, kept, cap = self.capacity_fallback(logits, idx, p, E, cf, policy - 2)
+            expert, kept, cap = self.capacity_fallback(logits, idx, p, E, cf, policy - 2, order_override)
             perm = self.permute(expert.reshape(idx.shape), kept, E)
             # counts stay the router's histogram; the grouping follows `expert`
             perm["counts"] = np.bincount(idx.ravel(), minlength=E).astype(np.int32)

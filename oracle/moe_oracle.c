@@ -182,10 +182,12 @@ int64_t oracle_capacity(int64_t T, int32_t E, int32_t k, double cf, int32_t poli
  * token first), policy 1 in token order.  A moved slot keeps its gate weight;
  * one that does not fit is dropped.  expert[s] = the expert that processes
  * slot s (its top-k choice, or the fallback it moved to), kept[s] = 1 / 0.
- * Returns cap, or -1 when dropless. */
+ * order_override (may be NULL) [T, E]: a row whose first entry is >= 0
+ * replaces that token's router order (the comparison rule for tokens with
+ * near-tied logits).  Returns cap, or -1 when dropless. */
 int64_t oracle_capacity_fallback(int64_t T, int32_t E, int32_t k, double cf, int32_t policy,
                                  const double *logits, const int32_t *idx, const double *p,
-                                 int32_t *expert, uint8_t *kept) {
+                                 const int32_t *order_override, int32_t *expert, uint8_t *kept) {
   int64_t S = T * k;
   int64_t cap = oracle_capacity(T, E, k, cf, policy, idx, p, kept);
   for (int64_t s = 0; s < S; ++s) expert[s] = idx[s];
@@ -200,16 +202,22 @@ int64_t oracle_capacity_fallback(int64_t T, int32_t E, int32_t k, double cf, int
   for (int64_t t = 0; t < T; ++t) {
     const double *l = logits + t * E;
     /* router order of all E experts: logit descending, index ascending */
-    for (int32_t e = 0; e < E; ++e) order[e] = e;
-    for (int32_t a = 1; a < E; ++a) {
-      int32_t v = order[a], b = a - 1;
-      while (b >= 0 && (l[order[b]] < l[v] || (l[order[b]] == l[v] && order[b] > v))) {
-        order[b + 1] = order[b];
-        --b;
+    if (order_override && order_override[t * E] >= 0) {
+      for (int32_t e = 0; e < E; ++e) order[e] = order_override[t * E + e];
+    } else {
+      for (int32_t e = 0; e < E; ++e) order[e] = e;
+      for (int32_t a = 1; a < E; ++a) {
+        int32_t v = order[a], b = a - 1;
+        while (b >= 0 && (l[order[b]] < l[v] || (l[order[b]] == l[v] && order[b] > v))) {
+          order[b + 1] = order[b];
+          --b;
+        }
+        order[b + 1] = v;
       }
-      order[b + 1] = v;
     }
-    double M = l[order[0]], zE = 0.0;
+    double M = l[0], zE = 0.0;
+    for (int32_t e = 1; e < E; ++e)
+      if (l[e] > M) M = l[e];
     for (int32_t e = 0; e < E; ++e) zE += exp(l[e] - M);
     int32_t moved = 0;
     for (int32_t j = 0; j < k; ++j) {

@@ -31,7 +31,7 @@ moe_status check_shape(const moe_shape* sh) {
   if (sh->d_ff < 64 || sh->d_ff > 65536 || sh->d_ff % 64) return MOE_ERR_INVALID_ARG;
   if (sh->T * (int64_t)sh->k >= ((int64_t)1 << 30)) return MOE_ERR_INVALID_ARG;
   if (!std::isfinite(sh->capacity_factor)) return MOE_ERR_INVALID_ARG;
-  if (sh->drop_policy != MOE_DROP_BY_PROB && sh->drop_policy != MOE_DROP_BY_ORDER) return MOE_ERR_INVALID_ARG;
+  if (sh->drop_policy < MOE_DROP_BY_PROB || sh->drop_policy > MOE_DROP_BY_ORDER_NEXT_BEST) return MOE_ERR_INVALID_ARG;
   if (sh->gemm_variant < MOE_VARIANT_AUTO || sh->gemm_variant > MOE_VARIANT_TILED_SINGLE) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
@@ -39,6 +39,11 @@ moe_status check_shape(const moe_shape* sh) {
 int64_t capacity_of(const moe_shape* sh) {
   if (sh->capacity_factor <= 0.f) return -1;
   return (int64_t)std::floor((double)sh->capacity_factor * (double)sh->T * (double)sh->k / (double)sh->E);
+}
+
+// Capacity mode with the next-best-expert fallback.
+bool fallback_of(const moe_shape* sh) {
+  return sh->capacity_factor > 0.f && sh->drop_policy >= MOE_DROP_BY_PROB_NEXT_BEST;
 }
 
 int variant_of(const moe_shape* sh) {
@@ -52,6 +57,10 @@ struct Layout {
   size_t status, ticket, counts, tile_state, ctrl_end;
   size_t thresh, partials, topk_idx, topk_w, topk_p, offsets, slot_pos, perm_slot, x_perm, h, y_perm,
       x_stage, y_stage, total;
+  // next-best-expert fallback only (0 otherwise); fb_counts sits in the
+  // control region: kept1_count, cand_count, counts_eff [3 E]
+  size_t fb_counts, next_idx, next_p, keys1, keys2, cand, eff, thresh2;
+  bool fallback;
   int variant;
   bool q4;                 // 4-bit expert weights (always the streaming schedule)
   int32_t bn, splits;      // streaming schedule: token tile, requested split-K count
@@ -83,6 +92,11 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
   o = align_up(o + 16);
   L.counts = o;
   o = align_up(o + 4 * E);
+  L.fallback = fallback_of(sh);
+  if (L.fallback) {
+    L.fb_counts = o;
+    o = align_up(o + 3 * 4 * E);
+  }
   L.tile_state = o;
   o = align_up(o + 4 * (size_t)permute_tiles(S) * E);
   L.ctrl_end = o;
@@ -112,6 +126,22 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
   o = align_up(o + 2 * (size_t)T * d);
   L.y_stage = o;
   o = align_up(o + 2 * (size_t)T * d);
+  if (L.fallback) {
+    L.next_idx = o;
+    o = align_up(o + 4 * S);
+    L.next_p = o;
+    o = align_up(o + 4 * S);
+    L.keys1 = o;
+    o = align_up(o + 8 * S);
+    L.keys2 = o;
+    o = align_up(o + 8 * S);
+    L.cand = o;
+    o = align_up(o + 4 * S);
+    L.eff = o;
+    o = align_up(o + 4 * S);
+    L.thresh2 = o;
+    o = align_up(o + 8 * E);
+  }
   L.total = o;
   return L;
 }
@@ -161,8 +191,9 @@ moe_status check_bf16(const void* p) { return (p && aligned(p, 16)) ? MOE_OK : M
 moe_status check_i32(const void* p) { return (p && aligned(p, 4)) ? MOE_OK : MOE_ERR_INVALID_ARG; }
 
 moe_status run_router(const moe_shape* sh, const moe_bf16* x, const float* Wg, float* logits, int32_t* idx, float* w,
-                      float* p, int32_t* counts, int num_sms, cudaStream_t s, bool counts_zeroed) {
-  RouterArgs a{x, Wg, logits, idx, w, p, counts, sh->T, sh->d_model, sh->E, sh->k};
+                      float* p, int32_t* counts, int num_sms, cudaStream_t s, bool counts_zeroed,
+                      int32_t* next_idx = nullptr, float* next_p = nullptr) {
+  RouterArgs a{x, Wg, logits, idx, w, p, counts, next_idx, next_p, sh->T, sh->d_model, sh->E, sh->k};
   return cuda_status(launch_router(a, num_sms, s, counts_zeroed));
 }
 
@@ -302,6 +333,9 @@ moe_status moe_permute(const moe_shape* sh, const moe_bf16* x, const int32_t* to
   MOE_TRY(check_i32(perm_slot));
   MOE_TRY(check_bf16(x_perm));
   if (sh->capacity_factor > 0.f && sh->drop_policy == MOE_DROP_BY_PROB) MOE_TRY(check_i32(topk_p));
+  // the fallback needs the router's ranks past the top k, which only the
+  // whole-layer entry points compute
+  if (fallback_of(sh)) return MOE_ERR_UNSUPPORTED;
   MOE_TRY(check_ws(sh, ws, ws_bytes));
   int sms = 0;
   MOE_TRY(check_device(&sms));
@@ -378,9 +412,42 @@ static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, con
   MOE_TRY(mark(0));
   MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.ctrl_end, s)));
   // one clear of the control region (status, ticket, counts, look-back words)
-  MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s, true));
-  MOE_TRY(mark(1));
-  MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s, true));
+  if (L.fallback) {
+    MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s, true, at<int32_t>(ws, L.next_idx),
+                       at<float>(ws, L.next_p)));
+    MOE_TRY(mark(1));
+    FallbackArgs fa{};
+    fa.topk_idx = idx;
+    fa.topk_p = p;
+    fa.counts = counts;
+    fa.next_idx = at<int32_t>(ws, L.next_idx);
+    fa.next_p = at<float>(ws, L.next_p);
+    fa.keys1 = at<uint64_t>(ws, L.keys1);
+    fa.keys2 = at<uint64_t>(ws, L.keys2);
+    fa.cand = at<int32_t>(ws, L.cand);
+    fa.eff = at<int32_t>(ws, L.eff);
+    fa.thresh1 = at<uint64_t>(ws, L.thresh);
+    fa.thresh2 = at<uint64_t>(ws, L.thresh2);
+    fa.kept1_count = at<int32_t>(ws, L.fb_counts);
+    fa.cand_count = fa.kept1_count + sh->E;
+    fa.counts_eff = fa.kept1_count + 2 * sh->E;
+    fa.T = sh->T;
+    fa.E = sh->E;
+    fa.k = sh->k;
+    fa.cap = capacity_of(sh);
+    fa.policy = sh->drop_policy - MOE_DROP_BY_PROB_NEXT_BEST;
+    MOE_TRY(cuda_status(launch_fallback(fa, sms, s)));
+    // group by the expert each slot landed on; dropped slots carry -1
+    moe_shape dropless = *sh;
+    dropless.capacity_factor = 0.f;
+    dropless.drop_policy = MOE_DROP_BY_PROB;
+    MOE_TRY(run_permute(&dropless, L, x, fa.eff, p, fa.counts_eff, offsets, slot_pos, perm_slot, x_perm, ws, s,
+                        true));
+  } else {
+    MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s, true));
+    MOE_TRY(mark(1));
+    MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s, true));
+  }
   MOE_TRY(mark(2));
   if (q4)
     MOE_TRY(run_gemms_q4(sh, L, x_perm, offsets, W, h, ws, sms, s, ev ? ev[3] : nullptr));

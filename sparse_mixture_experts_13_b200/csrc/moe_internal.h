@@ -23,6 +23,8 @@ struct RouterArgs {
   float* topk_w;       // [T, k]
   float* topk_p;       // [T, k]
   int32_t* counts;     // [E], zeroed by the launcher unless the caller did
+  int32_t* next_idx;   // [T, k] router ranks k .. 2k-1 (-1 past E - 1), or nullptr
+  float* next_p;       // [T, k] their full-softmax probabilities
   int64_t T;
   int32_t d, E, k;
 };
@@ -111,6 +113,31 @@ cudaError_t launch_quantize_q4(const uint16_t* W, int32_t E, int32_t R, int32_t 
 // (nullable; k >= 2) of topk_idx [T, k]; zeroed first unless `accumulate`.
 cudaError_t launch_router_stats(const int32_t* idx, int64_t T, int32_t E, int32_t k, int32_t* slot_counts,
                                 int32_t* pair_counts, bool accumulate, int num_sms, cudaStream_t s);
+
+// Next-best-expert fallback (capacity mode): decides the expert of every
+// slot (eff, -1 = dropped) and its histogram counts_eff; kept1_count,
+// cand_count and counts_eff must be zero before the launch.
+struct FallbackArgs {
+  const int32_t* topk_idx;   // [S]
+  const float* topk_p;       // [S]
+  const int32_t* counts;     // [E] router histogram
+  const int32_t* next_idx;   // [T, k] router ranks k ..
+  const float* next_p;       // [T, k]
+  uint64_t* keys1;           // [S]
+  uint64_t* keys2;           // [S]
+  int32_t* cand;             // [S]
+  int32_t* eff;              // [S] out
+  uint64_t* thresh1;         // [E]
+  uint64_t* thresh2;         // [E]
+  int32_t* kept1_count;      // [E]
+  int32_t* cand_count;       // [E]
+  int32_t* counts_eff;       // [E] out
+  int64_t T;
+  int32_t E, k;
+  int64_t cap;
+  int32_t policy;            // 0 by probability, 1 by token order
+};
+cudaError_t launch_fallback(const FallbackArgs& a, int num_sms, cudaStream_t s);
 
 struct CombineArgs {
   const uint16_t* y_perm;   // [S, d] bf16, or nullptr when reading partials

@@ -12,6 +12,8 @@
 //   the cap-th largest key of the expert's slots.  Keys are unique (a token
 //   routes to an expert at most once), so exactly cap slots satisfy
 //   key >= threshold.  Experts with at most cap slots get threshold 0.
+//   A slot whose expert is negative was dropped before grouping (the
+//   next-best-expert fallback marks slots so) and is skipped.
 //
 // permute_kernel: a single-pass scan with decoupled look-back.  Each block
 //   takes a tile of kPermuteTile consecutive slots in ticket order, ranks its
@@ -128,8 +130,8 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
   bool elig = false;
   if (ranker && s < S) {
     e = a.topk_idx[s];
-    elig = true;
-    if (a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
+    elig = e >= 0;  // a negative expert marks a slot dropped before grouping
+    if (elig && a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
   }
   int rank_w = 0;
   if (ranker) {
@@ -242,8 +244,8 @@ __global__ void __launch_bounds__(256) permute_small_kernel(PermuteArgs a) {
       bool elig = false;
       if (s < S) {
         e = a.topk_idx[s];
-        elig = true;
-        if (a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
+        elig = e >= 0;  // a negative expert marks a slot dropped before grouping
+        if (elig && a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
       }
       const uint32_t peers = __match_any_sync(0xffffffffu, elig ? e : -1);
       const int before = __popc(peers & ((1u << lane) - 1u));
@@ -345,6 +347,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* sh, const moe_bf16* x
     return MOE_ERR_INVALID_ARG;
   const int64_t cap = api_capacity(sh);
   if (cap >= 0 && sh->drop_policy == MOE_DROP_BY_PROB && !al(topk_p, 4)) return MOE_ERR_INVALID_ARG;
+  if (cap >= 0 && sh->drop_policy >= MOE_DROP_BY_PROB_NEXT_BEST) return MOE_ERR_UNSUPPORTED;
   int sms = 0;
   st = api_check_device(&sms);
   if (st != MOE_OK) return st;

@@ -86,6 +86,28 @@ __device__ __forceinline__ void finish_token(const RouterArgs& a, int64_t t, con
     for (int e = 0; e < EMAX; ++e)
       if (e < E && lane == e) a.logits[t * E + e] = acc[e];
   }
+  if (a.next_idx) {
+    // ranks k .. 2k-1 (capacity fallback): continue the same arg-max order
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        int best = -1;
+        float bl = -FLT_MAX;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+          if (e < E && !((chosen >> e) & 1u) && (best < 0 || acc[e] > bl)) {
+            best = e;
+            bl = acc[e];
+          }
+        }
+        if (best >= 0) chosen |= 1u << best;
+        if (lane == j) {
+          a.next_idx[t * k + j] = best;
+          a.next_p[t * k + j] = best >= 0 ? expf(bl - m) / zE : 0.f;
+        }
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ float dot8(const float (&x)[8], const float4& w0, const float4& w1, float s) {

@@ -273,3 +273,49 @@ def run_stages_q4(dev: QDevice) -> dict:
     assert st == moe.MOE_OK, moe.status_string(st)
     torch.cuda.synchronize()
     return o
+
+
+# ------------------------------------------------- next-best-expert fallback
+
+def gpu_logits(dev: Device) -> np.ndarray:
+    """The router's fp32 logits (moe_router_topk with its logits output)."""
+    wl = dev.wl
+    sh = dev.shape(0)
+    S, E = wl.T * wl.k, wl.E
+    cu = lambda *shape, dt: torch.empty(*shape, dtype=dt, device="cuda")
+    lg = cu(wl.T, E, dt=torch.float32)
+    moe.check(moe.moe_router_topk(moe.make_shape(wl.T, wl.d, wl.f, E, wl.k), dev.x, dev.Wg, lg, cu(S, dt=torch.int32),
+                                  cu(S, dt=torch.float32), cu(S, dt=torch.float32), cu(E, dt=torch.int32)), "router")
+    torch.cuda.synchronize()
+    return lg.cpu().numpy().astype(np.float64)
+
+
+def fallback_route(o: oracle.Oracle, wl: synth.Workload, gpu_idx: np.ndarray, gl: np.ndarray,
+                   stats: dict | None = None) -> dict:
+    """Oracle routing with the fallback.  A token whose oracle logits have two
+    of the 2k+1 largest within 1e-3 is ambiguous: the GPU's router order
+    (from its fp32 logits, ties to the smaller index) must order the
+    oracle's values within 1e-3, and the oracle then takes that order for the
+    token (its top-k and the ranks the fallback reads)."""
+    T, k, E = wl.T, wl.k, wl.E
+    L = o.router_logits(wl.x, wl.Wg)
+    m = min(2 * k + 1, E)
+    order = np.argsort(-L, axis=1, kind="stable")
+    srt = np.take_along_axis(L, order, 1)
+    amb = (srt[:, :m - 1] - srt[:, 1:m] <= AMBIG_LOGIT).any(axis=1) if m > 1 else np.zeros(T, bool)
+    gorder = np.argsort(-gl, axis=1, kind="stable")
+    gi = gpu_idx.reshape(T, k)
+    bad = np.nonzero((~amb) & (gorder[:, :m] != order[:, :m]).any(1))[0]
+    assert bad.size == 0, f"router order differs on unambiguous tokens {bad[:10]}"
+    assert np.array_equal(gi, gorder[:, :k]), "GPU top-k is not the order of its own logits"
+    idx_ov = np.full((T, k), -1, np.int32)
+    ord_ov = np.full((T, E), -1, np.int32)
+    for t in np.nonzero(amb)[0]:
+        vals = L[t, gorder[t, :m]]
+        assert (vals >= srt[t, :m] - AMBIG_LOGIT).all() and (np.diff(vals) <= AMBIG_LOGIT).all(), (t, L[t], gorder[t])
+        idx_ov[t] = gorder[t, :k]
+        ord_ov[t] = gorder[t]
+    if stats is not None:
+        stats.update(ambiguous_tokens=int(amb.sum()))
+    return o.route(wl.x, wl.Wg, k, wl.capacity_factor, wl.drop_policy, idx_override=idx_ov, logits=L,
+                   order_override=ord_ov)

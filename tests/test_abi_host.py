@@ -47,7 +47,7 @@ def test_status_strings(moe):
 @pytest.mark.parametrize("kw", [dict(E=0), dict(E=33), dict(k=0), dict(k=9, E=16), dict(k=3, E=2),
                                 dict(d_model=100), dict(d_model=0), dict(d_ff=448 + 32), dict(T=-1),
                                 dict(capacity_factor=float("nan")), dict(capacity_factor=float("inf")),
-                                dict(drop_policy=2), dict(gemm_variant=4), dict(T=1 << 29, k=2)])
+                                dict(drop_policy=4), dict(drop_policy=-1), dict(gemm_variant=4), dict(T=1 << 29, k=2)])
 def test_invalid_shapes(moe, kw):
     base = dict(T=64, d_model=128, d_ff=448, E=8, k=2)
     base.update(kw)
@@ -142,3 +142,16 @@ def test_router_stats_arguments(moe):
     assert moe.moe_router_stats(sh, ok, ok, ok, 2, 0) == E              # accumulate flag
     assert moe.moe_router_stats(moe.make_shape(64, 128, 448, E=8, k=1), ok, ok, ok, 0, 0) == E  # pairs need k >= 2
     assert moe.moe_router_stats(moe.make_shape(64, 100, 448), ok, ok, None, 0, 0) == E
+
+
+def test_fallback_policies_accepted(moe):
+    """Policies 2 and 3 (next-best-expert fallback) are valid shapes; the
+    whole layer takes them, and their workspace holds the fallback's arrays."""
+    plain = moe.moe_workspace_size(moe.make_shape(256, 128, 448, capacity_factor=1.0, drop_policy=0))
+    for pol in (2, 3):
+        sh = moe.make_shape(256, 128, 448, capacity_factor=1.0, drop_policy=pol)
+        assert moe.moe_workspace_size(sh) > plain
+        assert moe.moe_workspace_size_q4(sh) > 0
+    # dropless ignores the policy
+    assert moe.moe_workspace_size(moe.make_shape(256, 128, 448, drop_policy=2)) == \
+        moe.moe_workspace_size(moe.make_shape(256, 128, 448))
