@@ -20,6 +20,7 @@
 #include <cstdint>
 
 #include "moe_internal.h"
+#include "select.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -43,14 +44,11 @@ __global__ void __launch_bounds__(kFbThreads) fb_keys_kernel(const float* __rest
 // One block per expert: thresh[e] = the r-th largest key among the slots with
 // expert[s] == e, r = cap - (used ? used[e] : 0).  0 when every such slot
 // fits, ~0 when none does.
-__global__ void __launch_bounds__(kFbThreads) fb_select_kernel(const int32_t* __restrict__ expert,
-                                                               const uint64_t* __restrict__ keys,
-                                                               const int32_t* __restrict__ counts,
-                                                               const int32_t* __restrict__ used, int64_t cap,
-                                                               uint64_t* __restrict__ thresh, int64_t S) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint64_t s_prefix;
-  __shared__ int64_t s_need;
+__global__ void __launch_bounds__(kSelectThreads) fb_select_kernel(const int32_t* __restrict__ expert,
+                                                                   const uint64_t* __restrict__ keys,
+                                                                   const int32_t* __restrict__ counts,
+                                                                   const int32_t* __restrict__ used, int64_t cap,
+                                                                   uint64_t* __restrict__ thresh, int64_t S) {
   const int e = blockIdx.x;
   const int64_t cnt = counts[e];
   const int64_t room = cap - (used ? (int64_t)used[e] : 0);
@@ -62,36 +60,14 @@ __global__ void __launch_bounds__(kFbThreads) fb_select_kernel(const int32_t* __
     if (threadIdx.x == 0) thresh[e] = ~0ull;
     return;
   }
-  if (threadIdx.x == 0) {
-    s_prefix = 0;
-    s_need = room;
-  }
-  uint64_t mask = 0;
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = 56 - 8 * pass;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    const uint64_t prefix = s_prefix;
-    for (int64_t s = threadIdx.x; s < S; s += blockDim.x) {
-      if (expert[s] != e) continue;
-      const uint64_t key = keys[s];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1u);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int64_t need = s_need, cum = 0;
-      int b = 255;
-      for (; b > 0; --b) {
-        if (cum + hist[b] >= need) break;
-        cum += hist[b];
-      }
-      s_need = need - cum;
-      s_prefix = prefix | ((uint64_t)b << shift);
-    }
-    mask |= 0xFFull << shift;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) thresh[e] = s_prefix;
+  const uint64_t t = block_radix_select(
+      [&](int64_t s, uint64_t& key) {
+        if (expert[s] != e) return false;
+        key = keys[s];
+        return true;
+      },
+      S, cnt, room);
+  if (threadIdx.x == 0) thresh[e] = t;
 }
 
 // One thread per token: keep or move each slot.  A kept slot keeps its
@@ -176,11 +152,15 @@ cudaError_t launch_fallback(const FallbackArgs& a, int num_sms, cudaStream_t s) 
   const int64_t S = a.T * a.k;
   const int32_t by_prob = a.policy == 0 ? 1 : 0;
   fb_keys_kernel<<<grid_for(S, num_sms), kFbThreads, 0, s>>>(a.topk_p, a.keys1, S, a.k, by_prob);
-  fb_select_kernel<<<a.E, kFbThreads, 0, s>>>(a.topk_idx, a.keys1, a.counts, nullptr, a.cap, a.thresh1, S);
+  cudaError_t err = cudaFuncSetAttribute(fb_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
+  if (err != cudaSuccess) return err;
+  fb_select_kernel<<<a.E, kSelectThreads, kSelectSmem, s>>>(a.topk_idx, a.keys1, a.counts, nullptr, a.cap,
+                                                            a.thresh1, S);
   fb_classify_kernel<<<grid_for(a.T, num_sms), kFbThreads, 0, s>>>(a.topk_idx, a.keys1, a.thresh1, a.next_idx,
                                                                     a.next_p, a.eff, a.cand, a.keys2, a.kept1_count,
                                                                     a.cand_count, a.T, a.k, a.E, by_prob);
-  fb_select_kernel<<<a.E, kFbThreads, 0, s>>>(a.cand, a.keys2, a.cand_count, a.kept1_count, a.cap, a.thresh2, S);
+  fb_select_kernel<<<a.E, kSelectThreads, kSelectSmem, s>>>(a.cand, a.keys2, a.cand_count, a.kept1_count, a.cap,
+                                                            a.thresh2, S);
   fb_finalize_kernel<<<grid_for(S, num_sms), kFbThreads, 0, s>>>(a.cand, a.keys2, a.thresh2, a.eff, a.counts_eff, S,
                                                                   a.E);
   return cudaGetLastError();

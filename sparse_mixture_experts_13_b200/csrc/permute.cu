@@ -7,7 +7,7 @@
 // probability per expert).
 //
 // capacity_select_kernel (capacity mode, drop by probability): one block per
-//   expert finds, by an 8-pass MSB-first radix select over 64-bit keys
+//   expert finds, by an 8-pass MSB-first radix select (select.cuh) over 64-bit keys
 //   key = (bits of p as float) << 32 | (0xFFFFFFFF - t),
 //   the cap-th largest key of the expert's slots.  Keys are unique (a token
 //   routes to an expert at most once), so exactly cap slots satisfy
@@ -27,6 +27,7 @@
 #include <cstdint>
 
 #include "moe_internal.h"
+#include "select.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -43,14 +44,11 @@ __device__ __forceinline__ uint64_t slot_key(float p, int64_t t) {
   return ((uint64_t)__float_as_uint(p) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)t);
 }
 
-__global__ void __launch_bounds__(256) capacity_select_kernel(const int32_t* __restrict__ idx,
-                                                              const float* __restrict__ p,
-                                                              const int32_t* __restrict__ counts,
-                                                              uint64_t* __restrict__ thresh,
-                                                              int64_t S, int32_t k, int64_t cap) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint64_t s_prefix;
-  __shared__ int64_t s_need;
+__global__ void __launch_bounds__(kSelectThreads) capacity_select_kernel(const int32_t* __restrict__ idx,
+                                                                         const float* __restrict__ p,
+                                                                         const int32_t* __restrict__ counts,
+                                                                         uint64_t* __restrict__ thresh,
+                                                                         int64_t S, int32_t k, int64_t cap) {
   const int e = blockIdx.x;
   const int64_t cnt = counts[e];
   if (cnt <= cap) {
@@ -61,36 +59,14 @@ __global__ void __launch_bounds__(256) capacity_select_kernel(const int32_t* __r
     if (threadIdx.x == 0) thresh[e] = ~0ull;  // no key reaches it (keys < 2^63)
     return;
   }
-  if (threadIdx.x == 0) {
-    s_prefix = 0;
-    s_need = cap;
-  }
-  uint64_t mask = 0;
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = 56 - 8 * pass;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    const uint64_t prefix = s_prefix;
-    for (int64_t s = threadIdx.x; s < S; s += blockDim.x) {
-      if (idx[s] != e) continue;
-      const uint64_t key = slot_key(p[s], s / k);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1u);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int64_t need = s_need, cum = 0;
-      int b = 255;
-      for (; b > 0; --b) {
-        if (cum + hist[b] >= need) break;
-        cum += hist[b];
-      }
-      s_need = need - cum;
-      s_prefix = prefix | ((uint64_t)b << shift);
-    }
-    mask |= 0xFFull << shift;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) thresh[e] = s_prefix;
+  const uint64_t t = block_radix_select(
+      [&](int64_t s, uint64_t& key) {
+        if (idx[s] != e) return false;
+        key = slot_key(p[s], s / k);
+        return true;
+      },
+      S, cnt, cap);
+  if (threadIdx.x == 0) thresh[e] = t;
 }
 
 __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a) {
@@ -298,8 +274,10 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zero
     if (err != cudaSuccess) return err;
   }
   if (a.cap >= 0 && a.policy == 0) {
-    capacity_select_kernel<<<a.E, 256, 0, s>>>(a.topk_idx, a.topk_p, a.counts, a.thresh, S, a.k,
-                                               a.cap);
+    err = cudaFuncSetAttribute(capacity_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
+    if (err != cudaSuccess) return err;
+    capacity_select_kernel<<<a.E, kSelectThreads, kSelectSmem, s>>>(a.topk_idx, a.topk_p, a.counts, a.thresh, S,
+                                                                    a.k, a.cap);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
