@@ -245,6 +245,54 @@ MOE_API moe_status moe_layer_forward_host(const moe_shape *shape, const moe_bf16
 MOE_API moe_status moe_router_stats(const moe_shape *shape, const int32_t *topk_idx, int32_t *slot_counts,
                                     int32_t *pair_counts, int32_t accumulate, moe_stream_t stream);
 
+/* ------------------------------------------------------ expert parallelism
+ * Sources: "How Mixtral 8x7B uses mixture of experts", "Tensor parallelism vs
+ * expert parallelism" (each GPU holds a subset of the experts; an all-to-all
+ * sends every token to the ranks owning its experts and a second one brings
+ * the results back; expert_parallel_forward: router, dispatch, local
+ * experts, combine).
+ *
+ * `world` ranks, one per GPU; rank o owns experts o*epr .. o*epr+epr-1 with
+ * epr = E / world (E % world == 0, world <= 32).  Dropless only.  One layer
+ * step on rank r (the caller provides the collectives and barriers):
+ *   1. moe_router_topk on its own tokens -> topk_idx, topk_w, counts [E];
+ *   2. all-gather the counts of every rank into counts_all [world, E];
+ *   3. moe_ep_plan -> recv_off [E] and owner_off [epr + 1];
+ *   4. moe_ep_dispatch: stores each slot's token row into its owner's
+ *      receive buffer x_recv (peer memory) and records the row in ret_row;
+ *   5. barrier; moe_grouped_swiglu on this rank's x_recv with owner_off, its
+ *      local experts' weights, a shape with E = epr, k = 1 and T = the
+ *      receive buffer's rows, writing y_recv;
+ *   6. barrier; moe_ep_combine: y[t] = sum_j w[t, j] * y_recv of the owner at
+ *      ret_row (peer memory), fp32 in slot order, one bf16 rounding.
+ * An owner's receive buffer holds its experts' rows expert by expert, the
+ * source ranks in rank order within an expert, each in token order; it needs
+ * room for every slot that can reach it (at most the sum over ranks of T*k).
+ * The dispatch and combine kernels never wait on another rank. */
+
+/* counts_all [world, E] int32 (device) -> recv_off [E]: start row of this
+ * rank's slots of expert e in the receive buffer of e's owner; owner_off
+ * [epr + 1]: row ranges of this rank's local experts in its own receive
+ * buffer. */
+MOE_API moe_status moe_ep_plan(const int32_t *counts_all, int32_t E, int32_t rank, int32_t world,
+                               int32_t *recv_off, int32_t *owner_off, moe_stream_t stream);
+
+/* shape: this rank's T, the global E, k (capacity_factor must be <= 0).
+ * x [T, d], topk_idx [T, k], counts [E] from moe_router_topk; recv_off from
+ * moe_ep_plan; peer_x: DEVICE array of `world` device pointers, entry o the
+ * receive buffer [rows, d] bf16 of rank o (this rank's own included).
+ * ret_row [T, k] int32 (out).  ws: at least moe_workspace_size(shape). */
+MOE_API moe_status moe_ep_dispatch(const moe_shape *shape, int32_t world, const moe_bf16 *x,
+                                   const int32_t *topk_idx, const int32_t *counts, const int32_t *recv_off,
+                                   moe_bf16 *const *peer_x, int32_t *ret_row, void *ws, size_t ws_bytes,
+                                   moe_stream_t stream);
+
+/* peer_y: DEVICE array of `world` device pointers, entry o the expert output
+ * buffer y_recv [rows, d] bf16 of rank o.  y [T, d] bf16 (out). */
+MOE_API moe_status moe_ep_combine(const moe_shape *shape, int32_t world, const int32_t *topk_idx,
+                                  const float *topk_w, const int32_t *ret_row, const moe_bf16 *const *peer_y,
+                                  moe_bf16 *y, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- 4-bit experts
  * Sources: "How Mixtral 8x7B uses mixture of experts", "Deployment tradeoffs
  * you'll actually hit" / "Quantization asymmetry" (keep the router in 16-bit

@@ -12,5 +12,5 @@ from ._lib import (EXPORTED, MOE_DROP_BY_ORDER, MOE_DROP_BY_PROB, MOE_ERR_CUDA, 
                    moe_layer_forward_profiled, moe_permute,
                    moe_read_device_status, moe_router_topk, moe_selftest_wait_timeout, moe_shape, moe_workspace_size, status_string,
                    moe_quantize_q4, moe_workspace_size_q4, moe_grouped_swiglu_q4, moe_layer_forward_q4,
-                   moe_layer_forward_q4_profiled, moe_router_stats)
+                   moe_layer_forward_q4_profiled, moe_router_stats, moe_ep_plan, moe_ep_dispatch, moe_ep_combine)
 from .layer import MoELayer, MoELayerQ4  # noqa: F401

@@ -21,7 +21,8 @@ MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM, MOE_VARIANT_TILED_SINGL
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc",
-            "moe_selftest_wait_timeout", "moe_read_device_status", "moe_router_stats", "moe_quantize_q4", "moe_workspace_size_q4",
+            "moe_selftest_wait_timeout", "moe_read_device_status", "moe_router_stats", "moe_ep_plan", "moe_ep_dispatch",
+            "moe_ep_combine", "moe_quantize_q4", "moe_workspace_size_q4",
             "moe_grouped_swiglu_q4", "moe_layer_forward_q4", "moe_layer_forward_q4_profiled", "moe_status_string")
 _SIZE_RETURNING = ("moe_workspace_size", "moe_workspace_size_q4")
 
@@ -68,6 +69,10 @@ def lib():
         L.moe_read_device_status.argtypes = [P, P]
         L.moe_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_uint32, P]
         L.moe_router_stats.argtypes = [S, P, P, P, ctypes.c_int32, P]
+        i32 = ctypes.c_int32
+        L.moe_ep_plan.argtypes = [P, i32, i32, i32, P, P, P]
+        L.moe_ep_dispatch.argtypes = [S, i32, P, P, P, P, P, P, P, sz, P]
+        L.moe_ep_combine.argtypes = [S, i32, P, P, P, P, P, P]
         L.moe_quantize_q4.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P]
         L.moe_workspace_size_q4.argtypes = [S]
         L.moe_grouped_swiglu_q4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, sz, P]
@@ -174,6 +179,24 @@ def moe_router_stats(shape, topk_idx, slot_counts, pair_counts=None, accumulate=
     """Per-slot expert histograms [k, E] and first-two-choice pair counts [E, E]."""
     return lib().moe_router_stats(ctypes.byref(shape), _p(topk_idx), _p(slot_counts), _p(pair_counts),
                                   int(accumulate), _stream(stream))
+
+
+# ------------------------------------------------------ expert parallelism
+# peer_x / peer_y: int64 CUDA tensors holding one device pointer per rank.
+
+def moe_ep_plan(counts_all, E, rank, world, recv_off, owner_off, stream=None) -> int:
+    return lib().moe_ep_plan(_p(counts_all), int(E), int(rank), int(world), _p(recv_off), _p(owner_off),
+                             _stream(stream))
+
+
+def moe_ep_dispatch(shape, world, x, topk_idx, counts, recv_off, peer_x, ret_row, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_ep_dispatch(ctypes.byref(shape), int(world), _p(x), _p(topk_idx), _p(counts), _p(recv_off),
+                                 _p(peer_x), _p(ret_row), _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_ep_combine(shape, world, topk_idx, topk_w, ret_row, peer_y, y, stream=None) -> int:
+    return lib().moe_ep_combine(ctypes.byref(shape), int(world), _p(topk_idx), _p(topk_w), _p(ret_row), _p(peer_y),
+                                _p(y), _stream(stream))
 
 
 # ------------------------------------------------------------ 4-bit experts

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["router.cu", "permute.cu", "expert_gemm.cu", "expert_gemm_q4.cu", "router_stats.cu", "fallback.cu", "combine.cu", "moe_api.cu", "selftest.cu"]
+SOURCES = ["router.cu", "permute.cu", "expert_gemm.cu", "expert_gemm_q4.cu", "router_stats.cu", "fallback.cu", "ep.cu", "combine.cu", "moe_api.cu", "selftest.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -544,6 +544,63 @@ moe_status moe_layer_forward_host(const moe_shape* sh, const moe_bf16* x_host, c
   return cuda_status(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s));
 }
 
+moe_status moe_ep_plan(const int32_t* counts_all, int32_t E, int32_t rank, int32_t world, int32_t* recv_off,
+                       int32_t* owner_off, moe_stream_t stream) {
+  if (E < 1 || E > 32 || world < 1 || world > 32 || E % world || rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_i32(counts_all));
+  MOE_TRY(check_i32(recv_off));
+  MOE_TRY(check_i32(owner_off));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return cuda_status(launch_ep_plan(counts_all, E, rank, world, recv_off, owner_off, (cudaStream_t)stream));
+}
+
+moe_status moe_ep_dispatch(const moe_shape* sh, int32_t world, const moe_bf16* x, const int32_t* topk_idx,
+                           const int32_t* counts, const int32_t* recv_off, moe_bf16* const* peer_x, int32_t* ret_row,
+                           void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (world < 1 || world > 32 || sh->E % world) return MOE_ERR_INVALID_ARG;
+  if (sh->T == 0) return MOE_OK;
+  if (sh->capacity_factor > 0.f) return MOE_ERR_UNSUPPORTED;  // the expert-parallel layer is dropless
+  MOE_TRY(check_bf16(x));
+  MOE_TRY(check_i32(topk_idx));
+  MOE_TRY(check_i32(counts));
+  MOE_TRY(check_i32(recv_off));
+  MOE_TRY(check_bf16(peer_x));
+  MOE_TRY(check_i32(ret_row));
+  MOE_TRY(check_ws(sh, ws, ws_bytes));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  const Layout L = layout_of(sh);
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 8, s)));  // status word and tile ticket
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* slot_pos = at<int32_t>(ws, L.slot_pos);
+  // this rank's slots ranked per expert in token order (no local copy of x)
+  MOE_TRY(run_permute(sh, L, x, topk_idx, nullptr, counts, offsets, slot_pos, at<int32_t>(ws, L.perm_slot), nullptr,
+                      ws, s, false));
+  return cuda_status(launch_ep_dispatch(x, topk_idx, offsets, slot_pos, recv_off,
+                                        reinterpret_cast<uint16_t* const*>(peer_x), ret_row, sh->T * sh->k, sh->k,
+                                        sh->d_model, sh->E / world, sms, s));
+}
+
+moe_status moe_ep_combine(const moe_shape* sh, int32_t world, const int32_t* topk_idx, const float* topk_w,
+                          const int32_t* ret_row, const moe_bf16* const* peer_y, moe_bf16* y, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (world < 1 || world > 32 || sh->E % world) return MOE_ERR_INVALID_ARG;
+  if (sh->T == 0) return MOE_OK;
+  if (sh->capacity_factor > 0.f) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(check_i32(topk_idx));
+  MOE_TRY(check_i32(topk_w));
+  MOE_TRY(check_i32(ret_row));
+  MOE_TRY(check_bf16(peer_y));
+  MOE_TRY(check_bf16(y));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return cuda_status(launch_ep_combine(topk_idx, topk_w, ret_row, reinterpret_cast<const uint16_t* const*>(peer_y),
+                                       y, sh->T, sh->k, sh->d_model, sh->E / world, sms, (cudaStream_t)stream));
+}
+
 moe_status moe_router_stats(const moe_shape* sh, const int32_t* topk_idx, int32_t* slot_counts, int32_t* pair_counts,
                             int32_t accumulate, moe_stream_t stream) {
   MOE_TRY(check_shape(sh));

@@ -139,6 +139,17 @@ struct FallbackArgs {
 };
 cudaError_t launch_fallback(const FallbackArgs& a, int num_sms, cudaStream_t s);
 
+// Expert parallelism (csrc/ep.cu).
+cudaError_t launch_ep_plan(const int32_t* counts_all, int32_t E, int32_t rank, int32_t world, int32_t* recv_off,
+                           int32_t* owner_off, cudaStream_t s);
+cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, const int32_t* offsets,
+                               const int32_t* slot_pos, const int32_t* recv_off, uint16_t* const* peer_x,
+                               int32_t* ret_row, int64_t S, int32_t k, int32_t d, int32_t epr, int num_sms,
+                               cudaStream_t s);
+cudaError_t launch_ep_combine(const int32_t* topk_idx, const float* topk_w, const int32_t* ret_row,
+                              const uint16_t* const* peer_y, uint16_t* y, int64_t T, int32_t k, int32_t d, int32_t epr,
+                              int num_sms, cudaStream_t s);
+
 struct CombineArgs {
   const uint16_t* y_perm;   // [S, d] bf16, or nullptr when reading partials
   const float* partials;    // [splits, S, d] fp32 (if y_perm == nullptr)

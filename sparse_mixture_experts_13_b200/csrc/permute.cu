@@ -167,8 +167,9 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
   }
   __syncthreads();
 
-  // ---- gather the kept tokens' rows (16-byte vectors, all warps)
-  const int nkept = s_nkept;
+  // ---- gather the kept tokens' rows (16-byte vectors, all warps); skipped
+  // when only the grouping is wanted (x_perm == nullptr)
+  const int nkept = a.x_perm ? s_nkept : 0;
   const int nvec = a.d >> 3;
   const int nwarps = blockDim.x >> 5;
   for (int i = warp; i < nkept; i += nwarps) {
@@ -248,7 +249,8 @@ __global__ void __launch_bounds__(256) permute_small_kernel(PermuteArgs a) {
   }
   const int nvec = a.d >> 3;
   const int nwarps = blockDim.x >> 5;
-  for (int r = blockIdx.x + gridDim.x * warp; r < N; r += gridDim.x * nwarps) {
+  const int n_gather = a.x_perm ? N : 0;  // grouping only when x_perm == nullptr
+  for (int r = blockIdx.x + gridDim.x * warp; r < n_gather; r += gridDim.x * nwarps) {
     const uint4* src = reinterpret_cast<const uint4*>(a.x + (int64_t)(s_list[r] / k) * a.d);
     uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (int64_t)r * a.d);
     int v = lane;

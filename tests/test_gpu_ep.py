@@ -1,0 +1,89 @@
+"""Expert parallelism emulated on one GPU: `world` ranks' buffers on one
+device, their steps run phase by phase in stream order.  Each rank's output
+is compared with the oracle's layer on that rank's tokens; the top-k and
+counts bit for bit, y within the layer tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import sparse_mixture_experts_13_b200 as moe
+    from sparse_mixture_experts_13_b200 import ep
+    import gpu_harness as H
+else:  # collected on CPU hosts, never run there
+    moe = ep = H = None
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.Oracle()
+
+
+def run_ep(o, world, Ts, d, f, E=8, k=2, rows=None, weights=None):
+    base = synth.Workload("ep", max(Ts), d, f, E=E, k=k, seed=world)
+    if weights is None:
+        base.generate()
+        weights = (base.W1, base.W3, base.W2)
+    else:
+        base.generate(weights=False)
+    W1, W3, W2 = weights
+    xs_host = [synth.normal_bf16(100 + r, synth.TID_X, (T, d)) for r, T in enumerate(Ts)]
+    dev_w = [H.to_dev_bf16(W) for W in (W1, W3, W2)]
+    Wg = torch.from_numpy(base.Wg).cuda()
+    xs = [H.to_dev_bf16(x) for x in xs_host]
+    ys, idx, counts = ep.ep_forward_emulated(xs, Wg, *dev_w, world=world, k=k)
+    torch.cuda.synchronize()
+    for r, T in enumerate(Ts):
+        wl = synth.Workload(f"ep{r}", T, d, f, E=E, k=k)
+        wl.x, wl.Wg, wl.W1, wl.W3, wl.W2 = xs_host[r], base.Wg, W1, W3, W2
+        rt = H.conditional_route(o, wl, idx[r].cpu().numpy(), None, None)
+        assert np.array_equal(idx[r].cpu().numpy().reshape(T, k), rt["idx"])
+        assert np.array_equal(counts[r].cpu().numpy(), rt["counts"])
+        toks = np.arange(T) if rows is None else H.sample_tokens(wl, rt, rows)
+        ref = o.layer_rows(wl.x, W1, W3, W2, rt, toks)
+        H.assert_close(H.bf16_f64(H.bf16_host(ys[r]))[toks], ref["y"], f"y (rank {r} of {world})")
+    return ys
+
+
+@pytest.mark.parametrize("world", [1, 2, 4, 8])
+def test_ep_small(o, world):
+    run_ep(o, world, [97 + 13 * r for r in range(world)], 128, 256)
+
+
+def test_ep_uneven_and_empty_rank(o):
+    """A rank with a single token and expert counts of 16 over 4 ranks."""
+    run_ep(o, 4, [1, 300, 64, 129], 128, 192, E=16, k=2)
+
+
+def test_ep_matches_single_gpu_layer(o):
+    """The expert-parallel layer and the single-GPU layer on the same tokens
+    agree to bf16 rounding (same routing, same expert arithmetic)."""
+    wl = synth.Workload("epsg", 200, 128, 256, seed=4).generate()
+    dev = H.Device(wl)
+    single = H.bf16_f64(H.run_layer(dev, 1)["y"])
+    ys, _, _ = ep.ep_forward_emulated([dev.x[:100], dev.x[100:]], dev.Wg, dev.W1, dev.W3, dev.W2, world=2)
+    both = np.concatenate([H.bf16_f64(H.bf16_host(y)) for y in ys])
+    assert H.rel_fro(both, single) < 2e-3
+
+
+def test_ep_mixtral_eight_ranks(o):
+    """Mixtral shapes, one expert per rank, 512 tokens per rank (sampled rows)."""
+    wl = synth.workload("decode")
+    wl.generate()
+    run_ep(o, 8, [512] * 8, synth.MIXTRAL_D, synth.MIXTRAL_F, rows=12, weights=(wl.W1, wl.W3, wl.W2))
+
+
+def test_ep_rejects_capacity_and_bad_world():
+    sh = moe.make_shape(16, 128, 256, E=8, k=2, capacity_factor=1.0)
+    z = torch.zeros(64, dtype=torch.int32, device="cuda")
+    x = torch.zeros(16, 128, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    assert moe.moe_ep_dispatch(sh, 2, x, z, z, z, z, z, ws, ws.numel()) == moe.MOE_ERR_UNSUPPORTED
+    sh2 = moe.make_shape(16, 128, 256, E=8, k=2)
+    assert moe.moe_ep_dispatch(sh2, 3, x, z, z, z, z, z, ws, ws.numel()) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_ep_plan(z, 8, 2, 2, z, z) == moe.MOE_ERR_INVALID_ARG

@@ -59,3 +59,59 @@ def test_weak_scaling_value_single_rank():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.weak_scaling_value(1, 16, 0.5) == pytest.approx(32000.0)
+
+
+def _ep_plan_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_13_b200.ep import ep_plan_host
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        E = 8
+        g = torch.Generator().manual_seed(rank)
+        counts = torch.randint(0, 50, (E,), generator=g, dtype=torch.int32)
+        gathered = [torch.empty(E, dtype=torch.int32) for _ in range(world)]
+        dist.all_gather(gathered, counts)
+        counts_all = [c.tolist() for c in gathered]
+        recv_off, owner_off = ep_plan_host(counts_all, rank, world)
+        # share every rank's plan so each owner can check its receive layout
+        plans = [None] * world
+        dist.all_gather_object(plans, (recv_off, owner_off))
+        q.put((rank, counts_all, plans))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_plan_two_ranks_gloo():
+    """Expert-parallel plan across 2 gloo ranks: the counts are all-gathered,
+    every rank derives the same layout, and in each owner's receive buffer
+    the sources' row ranges tile the owner's expert ranges without gap or
+    overlap."""
+    import multiprocessing as mp
+    import socket
+    ctx = mp.get_context("spawn")
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    q = ctx.Queue()
+    world = 2
+    ps = [ctx.Process(target=_ep_plan_worker, args=(r, world, port, q)) for r in range(world)]
+    for p_ in ps:
+        p_.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p_ in ps:
+        p_.join(timeout=60)
+        assert p_.exitcode == 0
+    res.sort()
+    counts_all = res[0][1]
+    assert all(r[1] == counts_all for r in res)
+    plans = res[0][2]
+    E, epr = 8, 8 // world
+    for o in range(world):
+        owner_off = plans[o][1]
+        for l in range(epr):
+            e = o * epr + l
+            spans = sorted((plans[r][0][e], plans[r][0][e] + counts_all[r][e]) for r in range(world))
+            assert spans[0][0] == owner_off[l] and spans[-1][1] == owner_off[l + 1]
+            for a, b in zip(spans, spans[1:]):
+                assert a[1] == b[0]
