@@ -26,10 +26,15 @@
 //   warp 1      allocates tensor memory; one thread issues tcgen05.mma
 //               kind::f16 with A read from tensor memory, B from shared memory;
 //   warps 2-5   epilogue (SiLU * mul, or fp32 split-K partials);
-//   warps 6-21  dequantise: thread i of warp w owns weight row 32 (w % 4) + i
-//               (its tensor-memory lane) and a quarter (32 inputs) of the
-//               stage; it turns 32 codes into bf16, multiplies by the block
-//               scale and writes 16 columns of the A buffer with tcgen05.st.
+//   warps 6-9   dequantise: thread i of warp w owns weight row 32 (w % 4) + i
+//               (its tensor-memory lane) and the stage's 128 inputs of it; it
+//               turns the codes into bf16, multiplies by the block scales and
+//               writes 64 columns of the A buffer with tcgen05.st.
+// The MMA-issuing thread shares its scheduler with one epilogue and one
+// dequantising warp (TMEM lane quarters fix which warps run where); small-N
+// MMAs are bound by how fast that thread issues, so the dequantisation uses
+// as few warps as keep up (4; 8 and 16 measured slower) and the issue loop
+// is kept short.
 // Four A buffers of 64 columns sit behind the two accumulators.  An A buffer
 // is reused once the MMAs of the stage that last read it have completed,
 // which the one commit per stage that frees the stage's shared memory also
@@ -50,7 +55,9 @@ namespace {
 
 constexpr int KQ = 128;                  // inputs per stage (two scale blocks)
 constexpr int kDeqWarp0 = 6;             // first dequantising warp
-constexpr int kDeqWarps = 16;
+constexpr int kDeqWarps = 4;
+constexpr int kDeqParts = kDeqWarps / 4;    // warps per TMEM lane quarter
+constexpr int kDeqChunks = 4 / kDeqParts;   // 16-byte code chunks (32 inputs) per thread and stage
 constexpr int kQ4Threads = (kDeqWarp0 + kDeqWarps) * 32;
 constexpr int kCodeBytes = 128 * KQ / 2;  // 128 rows x 64 bytes
 constexpr int kScaleBytes = 1024;         // 2 blocks x 128 rows x bf16 = 512, padded
@@ -294,13 +301,17 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t b_addr = smem_u32(smem + stage * C::STAGE_BYTES);
+          // The issuing thread shares its scheduler with dequantising warps
+          // (TMEM lane quarters fix which warps run where), so its stream is
+          // kept short: the B descriptor is built once per stage and moved by
+          // constant offsets (the start-address field counts 16 bytes).
+          const uint64_t b_desc = make_sdesc_sw128(smem_u32(smem + stage * C::STAGE_BYTES));
           const uint32_t a_tmem = tmem_base + kACol0 + abuf * kACols;
+          umma_bf16_ts(d_tmem, a_tmem, b_desc, C::IDESC, kq > t.kq0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < KQ / 16; ++kk) {
-            umma_bf16_ts(d_tmem, a_tmem + kk * 8, make_sdesc_sw128(b_addr + (kk >> 2) * (BN * 128) + (kk & 3) * 32),
-                         C::IDESC, (kq > t.kq0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 1; kk < KQ / 16; ++kk)
+            umma_bf16_ts(d_tmem, a_tmem + kk * 8, b_desc + (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4),
+                         C::IDESC, 1u);
           umma_commit(&empty_bar[stage]);  // frees the stage and its A buffer
           if (++stage == STAGES) {
             stage = 0;
@@ -322,14 +333,21 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
       mbar_wait(drain_bar, 0, nullptr);
     }
   } else if (warp >= kDeqWarp0) {
-    // ------------------------------------------------ dequantise (warps 6..21)
+    // ------------------------------------------------ dequantise (warps 6..)
     const int q = warp & 3;                      // TMEM lane quarter
-    const int part = (warp - kDeqWarp0) >> 2;    // inputs 32*part .. +31 of the stage
+    const int part = (warp - kDeqWarp0) >> 2;    // chunks kDeqChunks*part .. of the stage
     const int r = q * 32 + lane;                 // weight row of the A tile
-    const int s_idx = (EPI == Q4_SWIGLU) ? ((r >> 6) * 128 + (part >> 1) * 64 + (r & 63)) : ((part >> 1) * 128 + r);
-    // codes: row r is 64 bytes; 16-byte chunk c sits at chunk c ^ ((r >> 1) & 3) (64-byte swizzle)
-    const uint32_t c_off = (uint32_t)r * 64 + (((uint32_t)part ^ (uint32_t)((r >> 1) & 3)) << 4);
-    const uint32_t t_col = tmem_base + ((uint32_t)(q * 32) << 16) + kACol0 + part * 16;
+    // codes: row r is 64 bytes; 16-byte chunk c (inputs 32c .. 32c+31) sits at
+    // chunk c ^ ((r >> 1) & 3) (64-byte swizzle); its scale is block c / 2
+    uint32_t c_off[kDeqChunks], s_off_b[kDeqChunks];
+#pragma unroll
+    for (int c = 0; c < kDeqChunks; ++c) {
+      const int chunk = part * kDeqChunks + c;
+      const int blk = chunk >> 1;
+      c_off[c] = (uint32_t)r * 64 + (((uint32_t)chunk ^ (uint32_t)((r >> 1) & 3)) << 4);
+      s_off_b[c] = kCodeBytes + 2 * ((EPI == Q4_SWIGLU) ? ((r >> 6) * 128 + blk * 64 + (r & 63)) : (blk * 128 + r));
+    }
+    const uint32_t t_col = tmem_base + ((uint32_t)(q * 32) << 16) + kACol0 + part * kDeqChunks * 16;
     int stage = 0, abuf = 0;
     uint32_t phase = 0;
     int64_t i = 0;  // stages dequantised so far
@@ -352,18 +370,21 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
         }
         tc_fence_after();
         const uint8_t* st = smem + stage * C::STAGE_BYTES + C::B_BYTES;
-        const uint4 w4 = *reinterpret_cast<const uint4*>(st + c_off);
-        const uint16_t sb = *reinterpret_cast<const uint16_t*>(st + kCodeBytes + 2 * s_idx);
-        const uint32_t s2u = uint32_t(sb) | (uint32_t(sb) << 16);
-        const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
-        const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
-        uint32_t v[16];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int c = 0; c < kDeqChunks; ++c) {
+          const uint4 w4 = *reinterpret_cast<const uint4*>(st + c_off[c]);
+          const uint16_t sb = *reinterpret_cast<const uint16_t*>(st + s_off_b[c]);
+          const uint32_t s2u = uint32_t(sb) | (uint32_t(sb) << 16);
+          const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
+          const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
+          uint32_t v[16];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) v[4 * k + m] = dequant_pair(words[k] >> (4 * m), s2);
+          for (int k = 0; k < 4; ++k) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) v[4 * k + m] = dequant_pair(words[k] >> (4 * m), s2);
+          }
+          tmem_st_32x32b_x16(t_col + abuf * kACols + c * 16, v);
         }
-        tmem_st_32x32b_x16(t_col + abuf * kACols, v);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
