@@ -120,10 +120,16 @@ class EPLayer:
         self.rows = max_tokens * k * self.world
         self.x_recv = symm_mem.empty(self.rows, self.d, dtype=torch.bfloat16, device=dev)
         self.y_recv = symm_mem.empty(self.rows, self.d, dtype=torch.bfloat16, device=dev)
-        hx = symm_mem.rendezvous(self.x_recv, group=group or dist.group.WORLD)
-        hy = symm_mem.rendezvous(self.y_recv, group=group or dist.group.WORLD)
-        self.peer_x = torch.tensor(list(hx.buffer_ptrs), dtype=torch.int64, device=dev)
-        self.peer_y = torch.tensor(list(hy.buffer_ptrs), dtype=torch.int64, device=dev)
+        g = group or dist.group.WORLD
+        hx = symm_mem.rendezvous(self.x_recv, group=g)
+        hy = symm_mem.rendezvous(self.y_recv, group=g)
+        # the tensor may sit at an offset inside its symmetric buffer; every
+        # rank's copy sits at the same offset
+        ox = self.x_recv.data_ptr() - hx.buffer_ptrs[self.rank]
+        oy = self.y_recv.data_ptr() - hy.buffer_ptrs[self.rank]
+        self.peer_x = torch.tensor([p_ + ox for p_ in hx.buffer_ptrs], dtype=torch.int64, device=dev)
+        self.peer_y = torch.tensor([p_ + oy for p_ in hy.buffer_ptrs], dtype=torch.int64, device=dev)
+        self._handles = (hx, hy)
         self.h_recv = torch.empty(self.rows, self.f, dtype=torch.bfloat16, device=dev)
         self.owner_shape = _lib.make_shape(self.rows, self.d, self.f, self.epr, 1)
         self.owner_ws = torch.empty(_lib.moe_workspace_size(self.owner_shape), dtype=torch.uint8, device=dev)

@@ -87,3 +87,28 @@ def test_ep_rejects_capacity_and_bad_world():
     sh2 = moe.make_shape(16, 128, 256, E=8, k=2)
     assert moe.moe_ep_dispatch(sh2, 3, x, z, z, z, z, z, ws, ws.numel()) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_ep_plan(z, 8, 2, 2, z, z) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_ep_layer_one_process_group_of_one(o):
+    """The one-process-per-GPU driver (NCCL counts all-gather, receive buffers
+    in symmetric memory, barriers) in a group of one rank: its plumbing runs
+    end to end on one GPU and matches the oracle."""
+    import socket
+    import torch.distributed as dist
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        wl = synth.Workload("eplayer", 96, 128, 256, seed=6).generate()
+        dev = H.Device(wl)
+        layer = ep.EPLayer(dev.Wg, dev.W1, dev.W3, dev.W2, E=wl.E, k=wl.k, max_tokens=wl.T)
+        y = layer.forward(dev.x)
+        torch.cuda.synchronize()
+        r = H.conditional_route(o, wl, H.run_layer(dev, 1)["idx"], None, None)
+        ref = o.layer_rows(wl.x, wl.W1, wl.W3, wl.W2, r, np.arange(wl.T))
+        H.assert_close(H.bf16_f64(H.bf16_host(y)), ref["y"], "y (EPLayer, one rank)")
+        del layer
+    finally:
+        dist.destroy_process_group()
