@@ -155,3 +155,18 @@ def test_fallback_policies_accepted(moe):
     # dropless ignores the policy
     assert moe.moe_workspace_size(moe.make_shape(256, 128, 448, drop_policy=2)) == \
         moe.moe_workspace_size(moe.make_shape(256, 128, 448))
+
+
+def test_fallback_rejected_by_stage_permute(moe):
+    """The next-best fallback needs the router's ranks past the top k, which
+    only the whole-layer entry points compute: the stage grouping entry points
+    refuse those policies before touching a device."""
+    ok = 1 << 20
+    for pol in (2, 3):
+        sh = moe.make_shape(64, 128, 448, capacity_factor=1.0, drop_policy=pol)
+        n = moe.moe_workspace_size(sh)
+        assert moe.moe_permute(sh, ok, ok, ok, ok, ok, ok, ok, ok, ok, n, 0) == moe.MOE_ERR_UNSUPPORTED
+        assert moe.moe_permute_noalloc(sh, ok, ok, ok, ok, ok, ok, ok, ok, 0) == moe.MOE_ERR_UNSUPPORTED
+    # dropless with the same policy value is an ordinary grouping (no fallback to take)
+    sh0 = moe.make_shape(64, 128, 448, drop_policy=2)
+    assert moe.moe_permute(sh0, ok, ok, ok, ok, ok, ok, ok, ok, None, 0, 0) == moe.MOE_ERR_WORKSPACE
