@@ -67,7 +67,7 @@ typedef uint16_t moe_bf16;                /* raw bfloat16 bits */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or enum */
-  MOE_ERR_UNSUPPORTED = 2, /* valid request this build does not handle (e.g. not sm_100) */
+  MOE_ERR_UNSUPPORTED = 2, /* valid request the library does not handle (e.g. not sm_100) */
   MOE_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
   MOE_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
   MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up */
