@@ -5,7 +5,8 @@ PyTorch serves only for device memory and streams; every step of the layer
 (router, top-k gate, capacity, grouping, grouped SwiGLU GEMMs, combine) runs
 in the library's kernels.
 """
-from ._lib import (EXPORTED, MOE_DROP_BY_ORDER, MOE_DROP_BY_PROB, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG,  # noqa: F401
+from ._lib import (EXPORTED, MOE_DROP_BY_ORDER, MOE_DROP_BY_ORDER_NEXT_BEST, MOE_DROP_BY_PROB,
+                   MOE_DROP_BY_PROB_NEXT_BEST, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG,  # noqa: F401
                    MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_OK, MOE_VARIANT_AUTO,
                    MOE_VARIANT_STREAM, MOE_VARIANT_TILED, MOE_VARIANT_TILED_SINGLE, MoeError, check, lib, make_shape, moe_combine,
                    moe_grouped_swiglu, moe_layer_forward, moe_permute_noalloc, moe_layer_forward_host,

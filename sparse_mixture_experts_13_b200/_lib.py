@@ -16,7 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
-MOE_DROP_BY_PROB, MOE_DROP_BY_ORDER = 0, 1
+MOE_DROP_BY_PROB, MOE_DROP_BY_ORDER, MOE_DROP_BY_PROB_NEXT_BEST, MOE_DROP_BY_ORDER_NEXT_BEST = 0, 1, 2, 3
 MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM, MOE_VARIANT_TILED_SINGLE = 0, 1, 2, 3
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",

@@ -33,6 +33,15 @@ def test_exports_match_header(moe):
     assert sorted(moe.EXPORTED) == names
 
 
+def test_binding_constants_match_header(moe):
+    """Every enum value include/moe.h declares has the same value in the binding."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    vals = re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(\d+)", src)
+    assert len(vals) >= 14, vals
+    for name, v in vals:
+        assert getattr(moe, name) == int(v), name
+
+
 def test_shape_struct_layout(moe):
     assert ctypes.sizeof(moe.moe_shape) == 40
     assert moe.moe_shape.capacity_factor.offset == 24
