@@ -50,6 +50,16 @@
  *  - A dropped slot contributes zero (the token passes on the residual path,
  *    [P3] MixtralBlock); the remaining gate weights are not renormalised.
  *
+ * Parity unpinned (readings the pages leave open; each function is pinned
+ * only against its own stated rule, by brute force and invariants, not
+ * against anything the pages fix):
+ *  - which slots overflow: policy 0 (router probability) against policy 1
+ *    (token order); only [P1]'s comment supports policy 0;
+ *  - the next-best fallback's rule (one move per dropped slot to the token's
+ *    next router ranks, competing for the capacity left), which [P1] names
+ *    without stating;
+ *  - the bits of the 4-bit format, which [P1] and [P5] name but do not give.
+ *
  * Layouts (row-major): x [T, d] bf16 bits; Wg [E, d] fp32 (logit = x . Wg[e]);
  * W1, W3 [E, f, d] bf16 bits; W2 [E, d, f] bf16 bits.  Slot s = t * k + j.
  */
