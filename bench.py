@@ -47,23 +47,55 @@ def load_peaks():
                     source="fallback")
 
 
+def strip_c_comments(text: str) -> str:
+    """C/C++/CUDA source without its comments, whitespace runs collapsed to
+    one space: what the compiler sees, so that editing a comment does not
+    count as changing a kernel."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_source_sha(root: str = None) -> str:
+    """Hash of the CUDA sources (comments and layout ignored)."""
+    import hashlib
+    src = os.path.join(root or ROOT, "sparse_mixture_experts_13_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(src, name), encoding="utf-8") as fh:
+                h.update(strip_c_comments(fh.read()).encode())
+    return h.hexdigest()[:16]
+
+
 def traffic_record(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, only while the
-    kernel's source is unchanged since the capture (else None)."""
-    import hashlib
+    kernel sources are unchanged (up to comments) since the capture (else
+    None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as fh:
             recs = json.load(fh)
     except (OSError, ValueError):
         return None
-    src = os.path.join(ROOT, "sparse_mixture_experts_13_b200", "csrc")
-    h = hashlib.sha256()
-    for name in sorted(os.listdir(src)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(src, name), "rb") as fh:
-                h.update(fh.read())
-    sha = h.hexdigest()[:16]
+    sha = kernel_source_sha(ROOT)
     for r in recs:
         if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
             return r.get("dram_bytes_per_launch")

@@ -1,7 +1,6 @@
 """Host logic of bench.py that needs no GPU: the clock samples taken during
 the timed region, the DRAM-traffic record that is reported only while the
 kernel sources are unchanged since the capture, and the warm-up floor."""
-import hashlib
 import json
 import os
 import subprocess
@@ -65,17 +64,28 @@ def _fake_tree(tmp, src_text):
     csrc.mkdir(parents=True)
     (csrc / "k.cu").write_text(src_text)
     (tmp / "profiles").mkdir()
-    return hashlib.sha256(src_text.encode()).hexdigest()[:16]
+    return bench.kernel_source_sha(str(tmp))
 
 
-def test_traffic_record_only_for_unchanged_sources(tmp_path, monkeypatch):
-    sha = _fake_tree(tmp_path, "__global__ void k() {}\n")
+def test_strip_c_comments():
+    src = ('#include "a.h"  // the header\n/* block\n comment */ int f(char c) {\n'
+           '  const char* s = "not // a comment /* either */";\n  return c == \'"\' ? 1 : \'/\';  // done\n}\n')
+    assert bench.strip_c_comments(src) == ('#include "a.h" int f(char c) { const char* s = '
+                                           '"not // a comment /* either */"; return c == \'"\' ? 1 : \'/\'; }')
+
+
+def test_traffic_record_only_for_unchanged_kernels(tmp_path, monkeypatch):
+    code = "// kernel k\n__global__ void k(int* p) { p[0] = 1; }\n"
+    sha = _fake_tree(tmp_path, code)
     rec = [dict(kernel="k", workload="w", source_sha=sha, dram_bytes_per_launch=1234)]
     (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    cu = tmp_path / "sparse_mixture_experts_13_b200" / "csrc" / "k.cu"
     assert bench.traffic_record("k", "w") == 1234
     assert bench.traffic_record("k", "other") is None
-    (tmp_path / "sparse_mixture_experts_13_b200" / "csrc" / "k.cu").write_text("__global__ void k() { }\n")
+    cu.write_text("/* kernel k, reworded\n   over two lines */\n__global__ void k(int* p) {\n  p[0] = 1;\n}\n")
+    assert bench.traffic_record("k", "w") == 1234   # comments and layout only
+    cu.write_text(code.replace("p[0] = 1", "p[0] = 2"))
     assert bench.traffic_record("k", "w") is None   # the kernel changed since the capture
 
 
