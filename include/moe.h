@@ -79,8 +79,9 @@ typedef enum {
                            (full softmax over E), ties to the smaller token */
   MOE_DROP_BY_ORDER = 1, /* keep the first cap slots in token order */
   /* The same two policies with a next-best-expert fallback ("How Mixtral 8x7B
-   * uses mixture of experts", "Routing without auxiliary loss": the excess is
-   * processed by "typically the next-best expert").  After the capacity pass,
+   * uses mixture of experts", "Routing without auxiliary loss": slots beyond
+   * a full expert's capacity go to a fallback, usually the token's next-best
+   * expert).  After the capacity pass,
    * the dropped slots of a token, in slot order, move to its experts at
    * router ranks k, k+1, ... (logit descending, index ascending); at each
    * expert they compete under the same policy (probability of that expert,
@@ -247,7 +248,7 @@ MOE_API moe_status moe_router_stats(const moe_shape *shape, const int32_t *topk_
 
 /* ------------------------------------------------------ expert parallelism
  * Sources: "How Mixtral 8x7B uses mixture of experts", "Tensor parallelism vs
- * expert parallelism" (each GPU holds a subset of the experts; an all-to-all
+ * expert parallelism" (the experts are divided among the GPUs; an all-to-all
  * sends every token to the ranks owning its experts and a second one brings
  * the results back; expert_parallel_forward: router, dispatch, local
  * experts, combine).

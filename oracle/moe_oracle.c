@@ -14,8 +14,8 @@
  *       - "The architecture in one diagram": router logits -> softmax -> top-2
  *         -> renormalise; outputs weighted and summed.
  *       - "Routing without auxiliary loss": capacity factor; excess tokens are
- *         dropped; "sort tokens by router probability for each expert, keep ...
- *         up to capacity".
+ *         dropped; each expert keeps its slots in order of router probability
+ *         until it is full.
  *  [P2] "Mixtral and Mixture-of-Experts, Explained" (automatone.win)
  *       - "How it works": G(x) = Softmax(TopK(x . W_g)), logits outside the
  *         top-k set to -inf; y = sum_i G(x)_i . Expert_i(x).
@@ -39,13 +39,14 @@
  *    except under exact ties; this file computes the [P3] form.
  *  - Top-k order and ties: slot j = 0 holds the largest logit; equal logits
  *    are ordered by the smaller expert index.
- *  - Experts are numbered from 0 ([P4]'s "expert 1 and 3" are indices 0, 2).
+ *  - Experts are numbered from 0 ([P4] calls the first and third scores
+ *    experts 1 and 3; here they are indices 0 and 2).
  *  - SiLU(a) = a * sigmoid(a) = a / (1 + exp(-a)).
  *  - Capacity per expert = floor(cf * T * k / E) (the pages' cf * T / E per
  *    slot of top-k); cf <= 0 means no capacity limit (dropless).
  *  - Which slots overflow: policy 0 keeps, per expert, the `cap` slots with
- *    the largest full-softmax router probability ([P1] "sort tokens by router
- *    probability"), ties to the smaller token index; policy 1 keeps the first
+ *    the largest full-softmax router probability ([P1]'s sketch orders each
+ *    expert's tokens by it), ties to the smaller token index; policy 1 keeps the first
  *    `cap` slots in token order.
  *  - A dropped slot contributes zero (the token passes on the residual path,
  *    [P3] MixtralBlock); the remaining gate weights are not renormalised.
@@ -180,9 +181,9 @@ int64_t oracle_capacity(int64_t T, int32_t E, int32_t k, double cf, int32_t poli
   return cap;
 }
 
-/* Next-best-expert fallback [P1] "Routing without auxiliary loss": the excess
- * slots of a full expert are processed by a fallback, "typically the
- * next-best expert".  Reading: after the capacity pass of oracle_capacity,
+/* Next-best-expert fallback [P1] "Routing without auxiliary loss": slots
+ * beyond a full expert's capacity go to a fallback, usually the token's
+ * next-best expert.  Reading: after the capacity pass of oracle_capacity,
  * the dropped slots of token t, in slot order, move to t's next experts in
  * the router order (logit descending, index ascending) past its top k: the
  * first dropped slot to rank k, the second to rank k + 1, and so on (none

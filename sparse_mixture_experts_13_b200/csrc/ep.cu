@@ -2,11 +2,11 @@
 // (one process per GPU), rank o owning experts o*epr .. o*epr + epr - 1.
 //
 // Source: "How Mixtral 8x7B uses mixture of experts", sections "Tensor
-// parallelism vs expert parallelism" (each GPU holds a subset of the experts;
+// parallelism vs expert parallelism" (the experts are divided among the GPUs;
 // an all-to-all at the MoE layer sends the tokens to the ranks that own
 // their experts, a second one sends the results back; expert_parallel_forward:
 // router, dispatch, local experts, combine) and "Capacity factor tuning"
-// (load imbalance across GPUs in expert-parallel setups).
+// (with expert parallelism, uneven routing loads some GPUs more than others).
 //
 // The two all-to-all steps are fused into the kernels on either side of
 // them, over peer memory:

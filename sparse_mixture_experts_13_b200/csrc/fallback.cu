@@ -1,8 +1,8 @@
 // Next-best-expert fallback for slots that overflow an expert's capacity.
 //
 // Source: "How Mixtral 8x7B uses mixture of experts", section "Routing
-// without auxiliary loss": the excess slots of a full expert are processed
-// by a fallback, typically the next-best expert.  Reading taken: after the
+// without auxiliary loss": slots beyond a full expert's capacity go to a
+// fallback, usually the token's next-best expert.  Reading taken: after the
 // capacity pass, the dropped slots of token t, in slot order, move to t's
 // experts at router ranks k, k+1, ... (logit descending, index ascending; the
 // router writes those ranks and their full-softmax probabilities).  At each

@@ -1,10 +1,10 @@
 // Capacity selection and grouping of slots by expert.
 //
 // Source: "How Mixtral 8x7B uses mixture of experts", sections "The
-// architecture in one diagram" (batch tokens by expert, run the experts,
-// scatter back) and "Routing without auxiliary loss" (capacity factor; the
-// excess slots of an expert are dropped; slots are sorted by router
-// probability per expert).
+// architecture in one diagram" (group the tokens by expert, run each expert
+// on its group, return the results to the tokens) and "Routing without
+// auxiliary loss" (capacity factor; the excess slots of an expert are
+// dropped; each expert's slots are ordered by router probability).
 //
 // capacity_select_kernel (capacity mode, drop by probability): one block per
 //   expert finds, by an 8-pass MSB-first radix select (select.cuh) over 64-bit keys
