@@ -181,7 +181,10 @@ MOE_API moe_status moe_permute_noalloc(const moe_shape *shape, const moe_bf16 *x
  *   h[r]      = SiLU(x_perm[r] . W1[e]^T) * (x_perm[r] . W3[e]^T)   [f] bf16
  *   y_perm[r] = h[r] . W2[e]^T                                        [d] bf16
  * bf16 operands, fp32 accumulation, results rounded to bf16 (nearest even).
- * Rows r >= offsets[E] of h and y_perm are left untouched. */
+ * Rows r >= offsets[E] of h and y_perm are left untouched.
+ * Precondition (not checked: offsets live on the device): offsets[0] = 0,
+ * offsets non-decreasing and offsets[E] <= T * k, as moe_permute writes
+ * them.  Other offsets make the kernels read and write outside the buffers. */
 MOE_API moe_status moe_grouped_swiglu(const moe_shape *shape, const moe_bf16 *x_perm,
                               const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
                               const moe_bf16 *W2, moe_bf16 *h, moe_bf16 *y_perm, void *ws,
@@ -192,7 +195,9 @@ MOE_API moe_status moe_grouped_swiglu(const moe_shape *shape, const moe_bf16 *x_
  *   y[t] = sum over j with slot_pos[t*k+j] >= 0 of
  *          topk_w[t, j] * y_perm[slot_pos[t*k+j]]
  * accumulated in fp32 in slot order, stored bf16; y[t] = 0 when every slot
- * of t was dropped.  The remaining weights are not renormalised. */
+ * of t was dropped.  The remaining weights are not renormalised.
+ * Precondition (not checked): every slot_pos entry is -1 or a row < T * k of
+ * y_perm, as moe_permute writes them. */
 MOE_API moe_status moe_combine(const moe_shape *shape, const moe_bf16 *y_perm, const int32_t *slot_pos,
                        const float *topk_w, moe_bf16 *y, moe_stream_t stream);
 
@@ -282,7 +287,10 @@ MOE_API moe_status moe_ep_plan(const int32_t *counts_all, int32_t E, int32_t ran
  * x [T, d], topk_idx [T, k], counts [E] from moe_router_topk; recv_off from
  * moe_ep_plan; peer_x: DEVICE array of `world` device pointers, entry o the
  * receive buffer [rows, d] bf16 of rank o (this rank's own included).
- * ret_row [T, k] int32 (out).  ws: at least moe_workspace_size(shape). */
+ * ret_row [T, k] int32 (out).  ws: at least moe_workspace_size(shape).
+ * Precondition (not checked): counts and recv_off come from this step's
+ * moe_router_topk and moe_ep_plan, and every owner's buffer has room for the
+ * rows the plan gives it. */
 MOE_API moe_status moe_ep_dispatch(const moe_shape *shape, int32_t world, const moe_bf16 *x,
                                    const int32_t *topk_idx, const int32_t *counts, const int32_t *recv_off,
                                    moe_bf16 *const *peer_x, int32_t *ret_row, void *ws, size_t ws_bytes,
@@ -327,7 +335,8 @@ MOE_API size_t moe_workspace_size_q4(const moe_shape *shape);
 
 /* moe_grouped_swiglu with 4-bit expert weights (W1c/W1s, W3c/W3s, W2c/W2s
  * in the format above).  h [T*k, d_ff] and y_perm [T*k, d_model] bf16 out;
- * ws of at least moe_workspace_size_q4 bytes. */
+ * ws of at least moe_workspace_size_q4 bytes.  Same precondition on offsets
+ * as moe_grouped_swiglu. */
 MOE_API moe_status moe_grouped_swiglu_q4(const moe_shape *shape, const moe_bf16 *x_perm,
                                          const int32_t *offsets, const uint8_t *W1c,
                                          const moe_bf16 *W1s, const uint8_t *W3c, const moe_bf16 *W3s,
