@@ -81,6 +81,32 @@ MUTANTS = [
     ("q4 W2 read with W1 shape", "acc += q4_weight(W2c, W2s, d, f, c, n) * h[n];",
      "acc += q4_weight(W2c, W2s, f, d, c % f, n % d) * h[n];"),
     ("q4 W3 scales from W1", "b += q4_weight(W3c, W3s, f, d, n, i) * xi;", "b += q4_weight(W3c, W1s, f, d, n, i) * xi;"),
+    ("capacity rounded up", "cap = (int64_t)floor(cf * (double)T * (double)k / (double)E);",
+     "cap = (int64_t)ceil(cf * (double)T * (double)k / (double)E);"),
+    ("topk picks the smallest logit", "if (best < 0 || l[e] > l[best]) best = e;",
+     "if (best < 0 || l[e] < l[best]) best = e;"),
+    ("topk may repeat an expert", "taken |= (idx[t * k + q] == e);", "taken |= 0;"),
+    ("probability normalised over the top k", "p[t * k + j] = exp(l[idx[t * k + j]] - M) / zE;",
+     "p[t * k + j] = exp(l[idx[t * k + j]] - m) / zk;"),
+    ("router reads Wg transposed", "(double)Wg[(int64_t)e * d + i]", "(double)Wg[(int64_t)i * E + e]"),
+    ("router writes logits to the next expert", "logits[t * E + e] = acc;", "logits[t * E + (e + 1) % E] = acc;"),
+    ("swiglu sum instead of product", _SILU, _SILU.replace("a / (1.0 + exp(-a)) * b", "a / (1.0 + exp(-a)) + b")),
+    ("up projection from W1", "b += bf16_to_double(W3e[(int64_t)n * d + i]) * xi;",
+     "b += bf16_to_double(W1e[(int64_t)n * d + i]) * xi;"),
+    ("layer runs every slot on the first choice's expert", "int64_t e = idx[s];", "int64_t e = idx[t * k];"),
+    ("capacity keeps the end of the priority list", "for (int64_t r = 0; r < n && r < cap; ++r) kept[list[r].s] = 1;",
+     "for (int64_t r = 0; r < n && r < cap; ++r) kept[list[n - 1 - r].s] = 1;"),
+    ("capacity keeps one slot fewer", "for (int64_t r = 0; r < n && r < cap; ++r) kept[list[r].s] = 1;",
+     "for (int64_t r = 0; r < n && r < cap - 1; ++r) kept[list[r].s] = 1;"),
+    ("capacity lists other experts' slots", "if (idx[s] == e) {\n        list[n].p = p[s];",
+     "if (idx[s] != e) {\n        list[n].p = p[s];"),
+    ("offsets hold starts, not ends", "offsets[e + 1] = (int32_t)row;", "offsets[e + 1] = (int32_t)row - kept_counts[e];"),
+    ("dropped slot gets row 0", "slot_pos[s] = -1;", "slot_pos[s] = 0;"),
+    ("fallback keeps the old expert's probability", "cand_p[s] = exp(l[order[r]] - M) / zE;", "cand_p[s] = p[s];"),
+    ("fallback skips rank k", "int32_t r = k + moved;", "int32_t r = k + 1 + moved;"),
+    ("fallback moves kept slots too", "if (kept[s]) continue;", "if (0) continue;"),
+    ("fallback ignores the capacity", "int64_t room = cap - used[e];", "int64_t room = n;"),
+    ("fallback router order ascending", "while (b >= 0 && (l[order[b]] < l[v] ||", "while (b >= 0 && (l[order[b]] > l[v] ||"),
 ]
 
 
