@@ -107,7 +107,24 @@ MUTANTS = [
     ("fallback moves kept slots too", "if (kept[s]) continue;", "if (0) continue;"),
     ("fallback ignores the capacity", "int64_t room = cap - used[e];", "int64_t room = n;"),
     ("fallback router order ascending", "while (b >= 0 && (l[order[b]] < l[v] ||", "while (b >= 0 && (l[order[b]] > l[v] ||"),
+    ("q4 scale not rounded to bf16", "float s = q4_bf16_round(amax / 7.0f);", "float s = amax / 7.0f;"),
+    ("q4 bf16 rounding truncates", "u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;", "u = u & 0xFFFF0000u;"),
+    ("q4 absmax without magnitude", "float v = fabsf((float)bf16_to_double(wr[i]));",
+     "float v = (float)bf16_to_double(wr[i]);"),
+    ("q4 absmax over half the block", "for (int i = 0; i < 64; ++i) {\n          float v = fabsf",
+     "for (int i = 0; i < 32; ++i) {\n          float v = fabsf"),
+    ("q4 wrong byte within the word", "*byte = g * 4 + nib / 2;", "*byte = g * 4 + nib % 4;"),
+    ("q4 scale stored for the next row", "scales[((int64_t)e * nb + b) * R + r] = (uint16_t)(sb >> 16);",
+     "scales[((int64_t)e * nb + b) * R + (r + 1) % R] = (uint16_t)(sb >> 16);"),
+    ("q4 dequantiser ignores the expert's scale offset", "const uint16_t *se = scales + (int64_t)e * (K / 64) * R;",
+     "const uint16_t *se = scales;"),
 ]
+# Not listed because they cannot change any output for bf16 weights:
+# * rounding the scale's ties upward instead of to even: absmax / 7 with an
+#   8-bit absmax mantissa is never a bf16 tie (past its 8th bit the quotient
+#   repeats the bits of 1/7, never exactly 1000...0);
+# * clamping codes at -7 instead of -8: |w / s| <= 7 (1 + 2^-8) < 7.5, so the
+#   lower clamp is never reached.
 
 
 @pytest.mark.parametrize("desc,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
