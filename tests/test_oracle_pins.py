@@ -119,10 +119,11 @@ MUTANTS = [
     ("q4 dequantiser ignores the expert's scale offset", "const uint16_t *se = scales + (int64_t)e * (K / 64) * R;",
      "const uint16_t *se = scales;"),
 ]
-# Not listed because they cannot change any output for bf16 weights:
+# Not listed because they cannot change any output for bf16 weights (the
+# first while absmax / 7 is a normal fp32 number):
 # * rounding the scale's ties upward instead of to even: absmax / 7 with an
 #   8-bit absmax mantissa is never a bf16 tie (past its 8th bit the quotient
-#   repeats the bits of 1/7, never exactly 1000...0);
+#   repeats the bits of a multiple of 1/7, never exactly 1000...0);
 # * clamping codes at -7 instead of -8: |w / s| <= 7 (1 + 2^-8) < 7.5, so the
 #   lower clamp is never reached.
 
