@@ -1,8 +1,12 @@
-"""The multi-rank host path of bench.py on CPU: world size 2 over gloo.
+"""Multi-rank host paths on CPU over gloo.
 
-Each rank processes its own batch (weak scaling, no data-path collective);
-the step time reported is the maximum over ranks and the whole-job value
-counts every rank's tokens.  The reference arm runs on rank 0 only.
+bench.py (world size 2): each rank processes its own batch (weak scaling, no
+data-path collective); the step time reported is the maximum over ranks and
+the whole-job value counts every rank's tokens.  The reference arm runs on
+rank 0 only.
+
+Expert parallelism (world sizes 2 and 4): the plan every rank derives from
+the all-gathered counts lays out each owner's receive buffer consistently.
 """
 import json
 import os
@@ -61,15 +65,16 @@ def test_weak_scaling_value_single_rank():
     assert bench.weak_scaling_value(1, 16, 0.5) == pytest.approx(32000.0)
 
 
-def _ep_plan_worker(rank, world, port, q):
+def _ep_plan_worker(rank, world, port, q, E=8):
     import torch
     import torch.distributed as dist
     from sparse_mixture_experts_13_b200.ep import ep_plan_host
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
-        E = 8
         g = torch.Generator().manual_seed(rank)
         counts = torch.randint(0, 50, (E,), generator=g, dtype=torch.int32)
+        if rank == world - 1:
+            counts[0] = 0                      # a source with no slots for expert 0
         gathered = [torch.empty(E, dtype=torch.int32) for _ in range(world)]
         dist.all_gather(gathered, counts)
         counts_all = [c.tolist() for c in gathered]
@@ -82,11 +87,12 @@ def _ep_plan_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_ep_plan_two_ranks_gloo():
-    """Expert-parallel plan across 2 gloo ranks: the counts are all-gathered,
+@pytest.mark.parametrize("world,E", [(2, 8), (4, 8), (4, 16)])
+def test_ep_plan_gloo(world, E):
+    """Expert-parallel plan across gloo ranks: the counts are all-gathered,
     every rank derives the same layout, and in each owner's receive buffer
     the sources' row ranges tile the owner's expert ranges without gap or
-    overlap."""
+    overlap, experts in order and sources in rank order within an expert."""
     import multiprocessing as mp
     import socket
     ctx = mp.get_context("spawn")
@@ -94,24 +100,27 @@ def test_ep_plan_two_ranks_gloo():
         s_.bind(("127.0.0.1", 0))
         port = s_.getsockname()[1]
     q = ctx.Queue()
-    world = 2
-    ps = [ctx.Process(target=_ep_plan_worker, args=(r, world, port, q)) for r in range(world)]
+    ps = [ctx.Process(target=_ep_plan_worker, args=(r, world, port, q, E)) for r in range(world)]
     for p_ in ps:
         p_.start()
     res = [q.get(timeout=120) for _ in range(world)]
     for p_ in ps:
         p_.join(timeout=60)
         assert p_.exitcode == 0
-    res.sort()
+    res.sort(key=lambda r: r[0])
     counts_all = res[0][1]
     assert all(r[1] == counts_all for r in res)
     plans = res[0][2]
-    E, epr = 8, 8 // world
+    assert all(r[2] == plans for r in res)
+    epr = E // world
     for o in range(world):
         owner_off = plans[o][1]
+        assert owner_off[0] == 0
+        assert owner_off[epr] == sum(counts_all[r][e] for r in range(world) for e in range(o * epr, (o + 1) * epr))
         for l in range(epr):
             e = o * epr + l
-            spans = sorted((plans[r][0][e], plans[r][0][e] + counts_all[r][e]) for r in range(world))
-            assert spans[0][0] == owner_off[l] and spans[-1][1] == owner_off[l + 1]
-            for a, b in zip(spans, spans[1:]):
-                assert a[1] == b[0]
+            starts = [plans[r][0][e] for r in range(world)]
+            assert starts[0] == owner_off[l]
+            for r in range(world - 1):
+                assert starts[r + 1] == starts[r] + counts_all[r][e]
+            assert starts[-1] + counts_all[world - 1][e] == owner_off[l + 1]
