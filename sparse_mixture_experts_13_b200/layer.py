@@ -10,6 +10,28 @@ import torch
 from . import _lib
 
 
+def check_activation(t: torch.Tensor, T: int, d: int, device, name: str) -> None:
+    """Raise ValueError unless `t` is a contiguous bf16 [T, d] tensor on
+    `device`.  The kernels read and write exactly T * d elements through the
+    raw pointer, so a smaller or differently placed tensor must be refused
+    before anything is queued."""
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.dim() != 2 or \
+            tuple(t.shape) != (T, d) or not t.is_contiguous() or t.device != device:
+        got = (f"{tuple(t.shape)} {t.dtype} on {t.device}, contiguous={t.is_contiguous()}"
+               if isinstance(t, torch.Tensor) else type(t).__name__)
+        raise ValueError(f"{name} must be a contiguous bf16 [{T}, {d}] tensor on {device}; got {got}")
+
+
+def check_index_out(t, n: int, device, name: str) -> None:
+    """Raise ValueError unless `t` (optional) is a contiguous int32 tensor of
+    at least n elements on `device`."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.int32 or not t.is_contiguous() or \
+            t.numel() < n or t.device != device:
+        raise ValueError(f"{name} must be a contiguous int32 tensor of at least {n} elements on {device}")
+
+
 class MoELayer:
     """Weights on one CUDA device: Wg [E, d] fp32, W1/W3 [E, f, d] and
     W2 [E, d, f] bf16 (row-major, contiguous)."""
@@ -45,8 +67,13 @@ class MoELayer:
     def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, topk_idx: torch.Tensor | None = None,
                 counts: torch.Tensor | None = None) -> torch.Tensor:
         T = x.shape[0]
+        dev = self.W1.device
+        check_activation(x, T, self.d, dev, "x")
         if y is None:
             y = torch.empty((T, self.d), dtype=torch.bfloat16, device=x.device)
+        check_activation(y, T, self.d, dev, "y")
+        check_index_out(topk_idx, T * self.k, dev, "topk_idx")
+        check_index_out(counts, self.E, dev, "counts")
         ws = self.workspace(T)
         st = _lib.moe_layer_forward(self.shape(T), x, self.Wg, self.W1, self.W3, self.W2, y, topk_idx, counts,
                                     ws, ws.numel())
@@ -56,6 +83,9 @@ class MoELayer:
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
         """x_host, y_host: page-locked CPU bf16 [T, d]; queued on the stream."""
         T = x_host.shape[0]
+        cpu = torch.device("cpu")
+        check_activation(x_host, T, self.d, cpu, "x_host")
+        check_activation(y_host, T, self.d, cpu, "y_host")
         ws = self.workspace(T)
         st = _lib.moe_layer_forward_host(self.shape(T), x_host, self.Wg, self.W1, self.W3, self.W2, y_host, ws,
                                          ws.numel(), stream)
@@ -117,8 +147,13 @@ class MoELayerQ4:
     def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, topk_idx: torch.Tensor | None = None,
                 counts: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         T = x.shape[0]
+        dev = self.Wg.device
+        check_activation(x, T, self.d, dev, "x")
         if y is None:
             y = torch.empty((T, self.d), dtype=torch.bfloat16, device=x.device)
+        check_activation(y, T, self.d, dev, "y")
+        check_index_out(topk_idx, T * self.k, dev, "topk_idx")
+        check_index_out(counts, self.E, dev, "counts")
         ws = self.workspace(T)
         st = _lib.moe_layer_forward_q4(self.shape(T), x, self.Wg, self.q1, self.q3, self.q2, y, topk_idx, counts,
                                        ws, ws.numel(), stream)
