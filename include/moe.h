@@ -34,6 +34,12 @@
  *   - Calls are asynchronous on `stream`; none synchronises except
  *     moe_read_device_status.  A workspace may serve one call in flight at a
  *     time.
+ *   - Host threads: the first call on each device fills a small per-device
+ *     cache (compute capability and SM count; for moe_permute_noalloc also
+ *     its scratch address).  Make one call on each device from a single
+ *     thread before calling from several threads at once; afterwards calls
+ *     from different threads are independent if their buffers, workspaces
+ *     and streams are.
  *   - Arguments are checked before any work is queued; on failure the call
  *     returns the status and queues nothing.  T == 0 is a no-op (MOE_OK).
  *     Requirements: 1 <= E <= 32, 1 <= k <= min(E, 8), d_model and d_ff
