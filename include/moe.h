@@ -39,7 +39,8 @@
  *     its scratch address).  Make one call on each device from a single
  *     thread before calling from several threads at once; afterwards calls
  *     from different threads are independent if their buffers, workspaces
- *     and streams are.
+ *     and streams are (not moe_permute_noalloc: all its calls share one
+ *     scratch array).
  *   - Arguments are checked before any work is queued; on failure the call
  *     returns the status and queues nothing.  T == 0 is a no-op (MOE_OK).
  *     Requirements: 1 <= E <= 32, 1 <= k <= min(E, 8), d_model and d_ff
