@@ -21,6 +21,13 @@ import torch.multiprocessing as mp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        return s_.getsockname()[1]
+
+
 def _worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
@@ -38,7 +45,7 @@ def _worker(rank, world, port, out):
 def test_max_over_ranks_and_weak_scaling_gloo():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29500 + (os.getpid() % 1000)
+    port = _free_port()
     procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
@@ -93,12 +100,8 @@ def test_ep_plan_gloo(world, E):
     every rank derives the same layout, and in each owner's receive buffer
     the sources' row ranges tile the owner's expert ranges without gap or
     overlap, experts in order and sources in rank order within an expert."""
-    import multiprocessing as mp
-    import socket
     ctx = mp.get_context("spawn")
-    with socket.socket() as s_:
-        s_.bind(("127.0.0.1", 0))
-        port = s_.getsockname()[1]
+    port = _free_port()
     q = ctx.Queue()
     ps = [ctx.Process(target=_ep_plan_worker, args=(r, world, port, q, E)) for r in range(world)]
     for p_ in ps:
