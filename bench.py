@@ -9,20 +9,29 @@ reported beside it on the HBM roofline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU runs (torchrun, one rank per GPU) shard the tokens: each rank runs
-the same layer on its own batch with no data-path collective (weak scaling);
-the step time is the max over ranks.  ``--impl reference`` times the CPU
-oracle on the host cores on a bounded sample of the same workload.
+Multi-GPU runs (one rank per GPU) shard the tokens: each rank runs the same
+layer on its own batch with no data-path collective (weak scaling); the step
+time is the max over ranks.  Under torchrun the ranks come from the
+environment; ``--gpus N`` with N > 1 and no WORLD_SIZE relaunches this script
+under torchrun with N ranks.  ``--impl reference`` times the CPU oracle on the
+host cores on a bounded sample of the same workload.  ``--dry-run`` checks the
+launcher and the rank plumbing without a GPU (gloo, a fixed step time per
+rank).
+
+Clocks are sampled in-process through NVML (read-only queries) every 5 ms
+while a timed loop runs, per workload.
 """
 from __future__ import annotations
 
 import argparse
+import contextlib
 import json
 import os
 import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -141,6 +150,110 @@ class ClockSampler:
                     power_w_max=max(power) if power else None, reasons=reasons, samples=len(sm))
 
 
+class NvmlSampler:
+    """This GPU's SM clock, power draw and clock-event reasons, queried
+    in-process through NVML (read-only) every `period_s` while a timed region
+    is open.  Samples are tagged with the region's name; nothing is sampled
+    outside regions, so every sample is "under load"."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, pci_bus_id: str | None, period_s: float = 0.005, nvml=None):
+        if nvml is None:
+            import pynvml as nvml
+        self.nvml = nvml
+        nvml.nvmlInit()
+        self.handle = self._find(pci_bus_id)
+        self.max_mhz = float(nvml.nvmlDeviceGetMaxClockInfo(self.handle, nvml.NVML_CLOCK_SM))
+        self.masks = [(name, int(getattr(nvml, attr, 0))) for name, attr in self.REASONS]
+        self.period = period_s
+        self.samples = []          # (tag, sm_mhz, power_w, reason mask)
+        self._tag = None
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _find(self, pci):
+        nv = self.nvml
+        n = nv.nvmlDeviceGetCount()
+        want = (pci or "").lower()[-12:]
+        for i in range(n):
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            bus = nv.nvmlDeviceGetPciInfo(h).busId
+            bus = bus.decode() if isinstance(bus, bytes) else str(bus)
+            if want and bus.lower().endswith(want):
+                return h
+        if n == 1 or not want:
+            return nv.nvmlDeviceGetHandleByIndex(0)
+        raise RuntimeError(f"no NVML device with PCI bus id {pci}")
+
+    def _reasons(self):
+        nv = self.nvml
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(fn(self.handle))
+
+    def sample(self, tag):
+        nv = self.nvml
+        sm = float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+        pw = float(nv.nvmlDeviceGetPowerUsage(self.handle)) / 1000.0
+        self.samples.append((tag, sm, pw, self._reasons()))
+
+    def _run(self):
+        while not self._stop.is_set():
+            tag = self._tag
+            if tag is not None:
+                try:
+                    self.sample(tag)
+                except Exception:  # a failed query leaves no sample
+                    pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        self._thread.start()
+
+    @contextlib.contextmanager
+    def region(self, tag: str):
+        self._tag = tag
+        try:
+            yield
+        finally:
+            self._tag = None
+
+    def _summary(self, rows) -> dict:
+        sm = [r[1] for r in rows]
+        reasons = sorted({n for r in rows for n, m in self.masks if m and (r[3] & m)})
+        return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=self.max_mhz,
+                    power_w_max=max((r[2] for r in rows), default=None), reasons=reasons, samples=len(rows))
+
+    def stop(self) -> dict:
+        self._stop.set()
+        if self._thread.is_alive():
+            self._thread.join(timeout=1.0)
+        out = self._summary(self.samples)
+        out["source"] = f"NVML, every {self.period * 1e3:.0f} ms inside the timed loops"
+        tags = []
+        for r in self.samples:
+            if r[0] not in tags:
+                tags.append(r[0])
+        out["by_region"] = {t: self._summary([r for r in self.samples if r[0] == t]) for t in tags}
+        return out
+
+
+def make_clock_sampler(pci):
+    """NVML in-process sampler, else nvidia-smi polling."""
+    try:
+        return NvmlSampler(pci)
+    except Exception:
+        return ClockSampler(pci)
+
+
+def sampler_region(sampler, tag):
+    return sampler.region(tag) if hasattr(sampler, "region") else contextlib.nullcontext()
+
+
 # ---------------------------------------------------------------- helpers
 
 def to_dev_bf16(a, torch):
@@ -176,6 +289,23 @@ def time_steps(fn, steps, torch, dist=None):
     if dist is not None:
         dist.barrier()
     return max_over_ranks(start.elapsed_time(end), torch, dist)
+
+
+def flushed_median_ms(fn, iters, torch, flush, dist=None):
+    """Median of per-iteration CUDA-event times, L2 flushed before every
+    iteration by writing `flush` (a buffer over twice the L2 size); max over
+    ranks of each rank's median."""
+    times = []
+    torch.cuda.synchronize()
+    for i in range(iters):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return max_over_ranks(statistics.median(times), torch, dist)
 
 
 class Run:
@@ -218,16 +348,49 @@ class Run:
         return dict(zip(["router", "capacity_and_permute", "gemm1_swiglu", "gemm2", "combine"],
                         (sums / steps).tolist()))
 
+    def twin(self):
+        """A second layer on the same weights with its own workspace."""
+        wl, L = self.wl, self.layer
+        return self.moe.MoELayer(L.Wg, L.W1, L.W3, L.W2, k=wl.k, capacity_factor=wl.capacity_factor,
+                                 drop_policy=wl.drop_policy)
+
     def e2e(self, steps, dist):
-        """Tokens/s through moe_layer_forward_host with page-locked host x and
-        y.  Every step copies its own x in and its y out; consecutive steps
-        alternate between two streams (each with its own workspace and host
-        buffers), so one step's copies overlap another step's kernels."""
+        """Tokens/s through the host-buffer entry point (moe_layer_forward_host
+        here) with page-locked host x and y, one call after another on one
+        stream: every step copies its x in, runs the layer and copies its y out
+        before the next step starts."""
+        torch, moe = self.torch, self.moe
+        wl, L = self.wl, self.layer
+        s_ = torch.cuda.Stream()
+        xh = torch.from_numpy(np.ascontiguousarray(wl.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+        yh = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+        for _ in range(2):
+            L.forward_host(xh, yh, s_)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(s_)
+        for _ in range(steps):
+            L.forward_host(xh, yh, s_)
+        end.record(s_)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        ms = max_over_ranks(start.elapsed_time(end), torch, dist)
+        if L.device_status(wl.T) != moe.MOE_OK:
+            raise RuntimeError("device status after the end-to-end run")
+        nbytes = wl.T * wl.d * 2
+        return ms, nbytes, nbytes
+
+    def e2e_pipelined(self, steps, dist):
+        """As e2e, but consecutive steps alternate between two streams (each
+        with its own workspace and host buffers), so one step's copies overlap
+        another step's kernels: a throughput, not a per-call time."""
         torch, moe = self.torch, self.moe
         wl = self.wl
         L = self.layer
-        layers = [L, moe.MoELayer(L.Wg, L.W1, L.W3, L.W2, k=wl.k, capacity_factor=wl.capacity_factor,
-                                  drop_policy=wl.drop_policy)]
+        layers = [L, self.twin()]
         streams = [torch.cuda.Stream(), torch.cuda.Stream()]
         xh = [torch.from_numpy(np.ascontiguousarray(wl.x).view(np.int16)).view(torch.bfloat16).pin_memory()
               for _ in range(2)]
@@ -290,52 +453,10 @@ class RunQ4(Run):
         return dict(zip(["router", "capacity_and_permute", "gemm1_swiglu", "gemm2", "combine"],
                         (sums / steps).tolist()))
 
-    def e2e(self, steps, dist):
-        """As Run.e2e, with the host copies queued by torch around
-        moe_layer_forward_q4 on each of the two streams."""
-        torch, moe = self.torch, self.moe
+    def twin(self):
         wl, L = self.wl, self.layer
-        layers = [L, moe.MoELayerQ4(L.Wg, L.q1, L.q3, L.q2, k=wl.k, capacity_factor=wl.capacity_factor,
-                                    drop_policy=wl.drop_policy)]
-        streams = [torch.cuda.Stream(), torch.cuda.Stream()]
-        xh = [torch.from_numpy(np.ascontiguousarray(wl.x).view(np.int16)).view(torch.bfloat16).pin_memory()
-              for _ in range(2)]
-        yh = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-        xd = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-        yd = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-
-        def one(j):
-            with torch.cuda.stream(streams[j]):
-                xd[j].copy_(xh[j], non_blocking=True)
-                layers[j].forward(xd[j], yd[j], stream=streams[j])
-                yh[j].copy_(yd[j], non_blocking=True)
-
-        for j in range(2):
-            one(j)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        cur = torch.cuda.current_stream()
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        start.record(cur)
-        for s_ in streams:
-            s_.wait_event(start)
-        for i in range(steps):
-            one(i & 1)
-        for s_ in streams:
-            ev = torch.cuda.Event()
-            ev.record(s_)
-            cur.wait_event(ev)
-        end.record(cur)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        ms = max_over_ranks(start.elapsed_time(end), torch, dist)
-        for j in range(2):
-            if layers[j].device_status(wl.T) != moe.MOE_OK:
-                raise RuntimeError("device status after the end-to-end run")
-        nbytes = wl.T * wl.d * 2
-        return ms, nbytes, nbytes
+        return self.moe.MoELayerQ4(L.Wg, L.q1, L.q3, L.q2, k=wl.k, capacity_factor=wl.capacity_factor,
+                                   drop_policy=wl.drop_policy)
 
 
 def expert_bytes(d, f):
@@ -347,11 +468,13 @@ def expert_bytes_q4(d, f):
     return 3 * (d * f // 2 + (d * f // 64) * 2)
 
 
-def cpu_baseline(wl, n_sample=48):
+def cpu_baseline(wl, n_sample=None):
     """The oracle on the host cores: routing of every token plus the expert
-    FFN of a seeded sample of tokens; tokens/s scaled to the whole batch."""
+    FFN of a seeded sample of tokens (two per oracle thread unless given, so
+    that no thread idles); tokens/s scaled to the whole batch."""
     import oracle
     o = oracle.Oracle()
+    n_sample = n_sample or 2 * o.num_threads()
     t0 = time.perf_counter()
     r = o.route(wl.x, wl.Wg, wl.k, wl.capacity_factor, wl.drop_policy)
     t_route = time.perf_counter() - t0
@@ -381,6 +504,14 @@ def workload_desc(wl):
     return f"{wl.name}: T={wl.T} d_model={wl.d} d_ff={wl.f} E={wl.E} top-{wl.k} {cap}"
 
 
+def bench_config(wl, world: int) -> dict:
+    """The `config` of both arms' lines (identical for the same workload and N)."""
+    return dict(workload=workload_desc(wl), T=wl.T, d_model=wl.d, d_ff=wl.f, E=wl.E, k=wl.k,
+                parallelism=f"dp{world} (token shards, weights replicated)" if world > 1 else "single GPU",
+                l2="inputs larger than L2: 2.82 GB of expert weights streamed every step; "
+                   "ms_per_step_median_l2_flushed: median of per-step events with L2 flushed before each step")
+
+
 # ---------------------------------------------------------------- arms
 
 def run_reference(args):
@@ -388,15 +519,20 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if "WORLD_SIZE" in os.environ and os.environ.get("OMP_NUM_THREADS") == "1":
+        # torchrun's one-thread default: the other ranks exit at once, so
+        # rank 0 may use every host core
+        os.environ["OMP_NUM_THREADS"] = str(os.cpu_count() or 1)
     wl = synth.workload("prefill")
     wl.generate(weights=True)
     import oracle
     o = oracle.Oracle()
-    n_sample = 8
+    n_sample = 2 * o.num_threads()
     rng = np.random.default_rng(7)
 
     def one_step():
-        """Seconds per token of the oracle on this step's sample."""
+        """(seconds of the step, seconds per token) of the oracle on this
+        step's sample: routing of every token + the FFN of n_sample tokens."""
         t0 = time.perf_counter()
         r = o.route(wl.x, wl.Wg, wl.k, wl.capacity_factor, wl.drop_policy)
         t_route = time.perf_counter() - t0
@@ -404,24 +540,74 @@ def run_reference(args):
         t0 = time.perf_counter()
         o.layer_rows(wl.x, wl.W1, wl.W3, wl.W2, r, rows)
         t_ffn = time.perf_counter() - t0
-        return t_ffn / n_sample + t_route / wl.T
+        return t_route + t_ffn, t_ffn / n_sample + t_route / wl.T
 
     for _ in range(args.warmup):
         one_step()
-    t_steps = [one_step() for _ in range(args.steps)]
-    per_token = float(np.mean(t_steps))
+    res = [one_step() for _ in range(args.steps)]
+    step_s = float(np.mean([a for a, _ in res]))
+    per_token = float(np.mean([b for _, b in res]))
     value = 1.0 / per_token
-    sample = (f"per step: routing of all {wl.T} tokens + expert FFN of {n_sample} seeded tokens (fp64 oracle); "
-              f"tokens/s = 1 / (t_ffn/{n_sample} + t_route/{wl.T})")
+    sample = (f"per step: routing of all {wl.T} tokens + expert FFN of {n_sample} seeded tokens "
+              f"(2 per oracle thread), fp64 oracle; tokens/s = 1 / (t_ffn/{n_sample} + t_route/{wl.T})")
     line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=args.gpus, steps=args.steps,
-                warmup=args.warmup, ms_per_step=per_token * wl.T * 1e3, higher_is_better=True, scaling="weak",
+                warmup=args.warmup, ms_per_step=step_s * 1e3, higher_is_better=True, scaling="weak",
                 vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
-                config=dict(workload=workload_desc(wl), T=wl.T, d_model=wl.d, d_ff=wl.f, E=wl.E, k=wl.k,
-                            parallelism="single process on the host cores", l2="CPU run"),
+                config=bench_config(wl, args.gpus),
+                ms_per_step_note=f"measured time of one step's sample ({n_sample} tokens' FFN + routing of all "
+                                 f"{wl.T}); the whole batch would take ms_full_batch_estimate",
+                ms_full_batch_estimate=per_token * wl.T * 1e3,
                 cpu_baseline=dict(value=value, unit="tokens/s", cores=o.num_threads(), kind="oracle",
                                   sample=sample),
                 e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
+
+
+def run_dry(args):
+    """Launcher and rank plumbing without a GPU: every rank joins a gloo
+    group and reports a fixed step time (1 ms + rank); rank 0 prints the max
+    over ranks and the whole-job value."""
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        dist = tdist
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks")
+    ms = max_over_ranks(1.0 + rank, torch, dist, device="cpu")
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(dict(dry_run=True, n_gpus=world, ranks_seen=world, ms_per_step=ms,
+                              value=weak_scaling_value(world, 4096, ms))), flush=True)
+
+
+def stage_report(wl, q, world, peaks, kernel, traffic_kernel, workload_key, q4=False):
+    """The decode-shaped sub-line (HBM roofline of the gate/up GEMM)."""
+    d, f, E = wl.d, wl.f, wl.E
+    ebytes = expert_bytes_q4(d, f) if q4 else expert_bytes(d, f)
+    g1_bytes = q["touched"] * 2 * ebytes // 3 + q["N"] * d * 2 + q["N"] * f * 2
+    layer_bytes = q["touched"] * ebytes + wl.T * d * 2 * 2 + E * d * 4 + 2 * q["N"] * f * 2
+    g1_ms = q["stages"]["gemm1_swiglu"]
+    return dict(workload=workload_desc(wl) + (", 4-bit expert weights (one bf16 scale per 64)" if q4 else ""),
+                value=weak_scaling_value(world, wl.T, q["ms"]), unit="tokens/s", ms_per_step=q["ms"],
+                ms_per_step_median_l2_flushed=q["ms_flushed"], stage_ms=q["stages"],
+                layer_gbs=layer_bytes / (q["ms"] * 1e-3) / 1e9,
+                layer_frac_hbm=layer_bytes / (q["ms"] * 1e-3) / 1e9 / peaks["hbm"],
+                roofline=dict(bound="hbm", kernel=kernel, achieved=g1_bytes / (g1_ms * 1e-3) / 1e9,
+                              peak=peaks["hbm"], unit="GB/s", frac=g1_bytes / (g1_ms * 1e-3) / 1e9 / peaks["hbm"],
+                              traffic=traffic_record(traffic_kernel, workload_key),
+                              peak_source=f"{peaks['source']} HBM copy bandwidth"),
+                e2e=dict(value=weak_scaling_value(world, wl.T, q["e2e_ms"]), unit="tokens/s",
+                         h2d_bytes_per_step=q["h2d"], d2h_bytes_per_step=q["d2h"],
+                         entry_point=q["entry"]),
+                e2e_pipelined=dict(value=weak_scaling_value(world, wl.T, q["e2e_pipe_ms"]), unit="tokens/s",
+                                   note="two streams, consecutive steps overlap"),
+                experts_touched=q["touched"])
 
 
 def run_ours(args):
@@ -429,6 +615,8 @@ def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks (launch with torchrun or without WORLD_SIZE)")
     dist = None
     torch.cuda.set_device(local)
     if world > 1:
@@ -453,8 +641,10 @@ def run_ours(args):
     if hasattr(props, "pci_bus_id"):
         pci = f"{int(getattr(props, 'pci_domain_id', 0)):08x}:{int(props.pci_bus_id):02x}:" \
               f"{int(getattr(props, 'pci_device_id', 0)):02x}.0"
-    sampler = ClockSampler(pci)
+    sampler = make_clock_sampler(pci)
     sampler.start()
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
 
     out = {}
     # decode first: the light, bandwidth-bound workload is measured before the
@@ -466,14 +656,19 @@ def run_ours(args):
         N, touched = run.kept_and_touched()
         for _ in range(args.warmup):
             run.step()
-        ms = time_steps(run.step, args.steps, torch, dist) / args.steps
-        stages = run.profiled(args.steps)
-        e2e_ms, h2d, d2h = run.e2e(args.steps, dist)
+        with sampler_region(sampler, name):
+            ms = time_steps(run.step, args.steps, torch, dist) / args.steps
+            stages = run.profiled(args.steps)
+            e2e_ms, h2d, d2h = run.e2e(args.steps, dist)
+            e2e_pipe_ms, _, _ = run.e2e_pipelined(args.steps, dist)
+        ms_flushed = flushed_median_ms(run.step, max(args.steps, 20), torch, flush, dist)
         out[name] = dict(wl=wl, ms=ms, stages=stages, N=N, touched=touched, e2e_ms=e2e_ms / args.steps,
-                         h2d=h2d, d2h=d2h)
+                         e2e_pipe_ms=e2e_pipe_ms / args.steps, h2d=h2d, d2h=d2h, ms_flushed=ms_flushed,
+                         entry="moe_layer_forward_q4_host" if name == "decode_q4" else "moe_layer_forward_host")
         del run
         torch.cuda.empty_cache()
     clocks = sampler.stop()
+    del flush
 
     line = None
     if rank == 0:
@@ -488,57 +683,34 @@ def run_ours(args):
         achieved_tf = g1_flops / (g1_ms * 1e-3) / 1e12
         tr = traffic_record("expert_gemm_pair_kernel<0,2>", "prefill")
         value = weak_scaling_value(world, wl.T, p["ms"])
-
-        q = out["decode"]
-        wq = q["wl"]
-        g1_bytes_dec = q["touched"] * 2 * d * f * 2 + q["N"] * d * 2 + q["N"] * f * 2
-        layer_bytes_dec = q["touched"] * expert_bytes(d, f) + wq.T * d * 2 * 2 + E * d * 4 + 2 * q["N"] * f * 2
-        dec_g1_ms = q["stages"]["gemm1_swiglu"]
-        dec = dict(workload=workload_desc(wq), value=weak_scaling_value(world, wq.T, q["ms"]), unit="tokens/s",
-                   ms_per_step=q["ms"], stage_ms=q["stages"],
-                   layer_gbs=layer_bytes_dec / (q["ms"] * 1e-3) / 1e9,
-                   layer_frac_hbm=layer_bytes_dec / (q["ms"] * 1e-3) / 1e9 / peaks["hbm"],
-                   roofline=dict(bound="hbm", kernel="gate/up-projection GEMM (SwiGLU fused)",
-                                 achieved=g1_bytes_dec / (dec_g1_ms * 1e-3) / 1e9, peak=peaks["hbm"], unit="GB/s",
-                                 frac=g1_bytes_dec / (dec_g1_ms * 1e-3) / 1e9 / peaks["hbm"],
-                                 traffic=traffic_record("expert_gemm_kernel<2,16>", "decode"),
-                                 peak_source=f"{peaks['source']} HBM copy bandwidth"),
-                   e2e=dict(value=weak_scaling_value(world, wq.T, q["e2e_ms"]), unit="tokens/s",
-                            h2d_bytes_per_step=q["h2d"], d2h_bytes_per_step=q["d2h"]),
-                   experts_touched=q["touched"])
-        q4 = out["decode_q4"]
-        g1_bytes_q4 = q4["touched"] * 2 * expert_bytes_q4(d, f) // 3 + q4["N"] * d * 2 + q4["N"] * f * 2
-        layer_bytes_q4 = q4["touched"] * expert_bytes_q4(d, f) + wq.T * d * 2 * 2 + E * d * 4 + 2 * q4["N"] * f * 2
-        q4_g1_ms = q4["stages"]["gemm1_swiglu"]
-        dec_q4 = dict(workload=workload_desc(wq) + ", 4-bit expert weights (one bf16 scale per 64)",
-                      value=weak_scaling_value(world, wq.T, q4["ms"]), unit="tokens/s", ms_per_step=q4["ms"],
-                      stage_ms=q4["stages"], layer_gbs=layer_bytes_q4 / (q4["ms"] * 1e-3) / 1e9,
-                      layer_frac_hbm=layer_bytes_q4 / (q4["ms"] * 1e-3) / 1e9 / peaks["hbm"],
-                      roofline=dict(bound="hbm", kernel="4-bit gate/up-projection GEMM (SwiGLU fused)",
-                                    achieved=g1_bytes_q4 / (q4_g1_ms * 1e-3) / 1e9, peak=peaks["hbm"], unit="GB/s",
-                                    frac=g1_bytes_q4 / (q4_g1_ms * 1e-3) / 1e9 / peaks["hbm"],
-                                    traffic=traffic_record("expert_gemm_q4_kernel<0,16>", "decode_q4"),
-                                    peak_source=f"{peaks['source']} HBM copy bandwidth"),
-                      e2e=dict(value=weak_scaling_value(world, wq.T, q4["e2e_ms"]), unit="tokens/s",
-                               h2d_bytes_per_step=q4["h2d"], d2h_bytes_per_step=q4["d2h"]),
-                      experts_touched=q4["touched"])
+        tflops = flops_layer / (p["ms"] * 1e-3) / 1e12
+        pre_clk = (clocks.get("by_region") or {}).get("prefill", {}).get("sm_mhz")
+        dec = stage_report(out["decode"]["wl"], out["decode"], world, peaks,
+                           "gate/up-projection GEMM (SwiGLU fused)", "expert_gemm_kernel<2,16>", "decode")
+        dec_q4 = stage_report(out["decode_q4"]["wl"], out["decode_q4"], world, peaks,
+                              "4-bit gate/up-projection GEMM (SwiGLU fused)", "expert_gemm_q4_kernel<0,16>",
+                              "decode_q4", q4=True)
         kernels_per_step = 5 + (1 if (wl.capacity_factor > 0 and wl.drop_policy == 0) else 0)
         line = dict(
             metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
-            ms_per_step=p["ms"], higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+            ms_per_step=p["ms"], ms_per_step_median_l2_flushed=p["ms_flushed"], higher_is_better=True,
+            scaling="weak", vs_baseline=None, dtype="bf16",
             data="synthetic (seeded counter-based N(0,1) tokens, random-init Mixtral-shaped expert weights)",
-            config=dict(workload=workload_desc(wl), T=wl.T, d_model=d, d_ff=f, E=E, k=wl.k,
-                        parallelism=f"dp{world} (token shards, weights replicated)" if world > 1 else "single GPU",
-                        l2="inputs larger than L2: 2.82 GB of expert weights streamed every step"),
-            tflops=flops_layer / (p["ms"] * 1e-3) / 1e12,
-            frac_layer_of_peak=flops_layer / (p["ms"] * 1e-3) / 1e12 / peak_tf,
+            config=bench_config(wl, world),
+            tflops=tflops,
+            tflops_per_ghz=tflops / (pre_clk / 1000.0) if pre_clk else None,
+            frac_layer_of_peak=tflops / peak_tf,
             stage_ms=p["stages"],
             roofline=dict(bound="tensor", kernel="gate/up-projection GEMM (SwiGLU fused)", achieved=achieved_tf,
                           peak=peak_tf, unit="TFLOP/s", frac=achieved_tf / peak_tf, traffic=tr,
+                          achieved_per_ghz=achieved_tf / (pre_clk / 1000.0) if pre_clk else None,
                           peak_source=f"{peaks['source']} bf16 dense "
                                       f"({'sustained' if long_run else 'burst'})"),
             e2e=dict(value=weak_scaling_value(world, wl.T, p["e2e_ms"]), unit="tokens/s", h2d_bytes_per_step=p["h2d"],
-                     d2h_bytes_per_step=p["d2h"]),
+                     d2h_bytes_per_step=p["d2h"], entry_point=p["entry"],
+                     note="one stream; each step copies x in and y out around the layer"),
+            e2e_pipelined=dict(value=weak_scaling_value(world, wl.T, p["e2e_pipe_ms"]), unit="tokens/s",
+                               note="two streams, consecutive steps overlap"),
             gpu_launches=kernels_per_step * args.steps,
             clocks=clocks,
             decode=dec,
@@ -556,8 +728,9 @@ def run_ours(args):
 
 def run_sweep(args):
     """One JSON line per workload (tiny, decode, prefill, skew, sweep T), on
-    one GPU: tokens/s, TFLOP/s, GB/s, roofline fractions, per-stage times and
-    a sampled oracle baseline.  Not the default contract line."""
+    one GPU: tokens/s, TFLOP/s, GB/s, roofline fractions, per-stage times,
+    the SM clock during the timed loop and a sampled oracle baseline.  Not the
+    driver's contract line."""
     import torch
     import sparse_mixture_experts_13_b200 as moe
     moe.lib()
@@ -567,6 +740,8 @@ def run_sweep(args):
     W3 = synth.normal_bf16(0, synth.TID_W3, (E, f, d), 0.0, 1.0 / np.sqrt(d))
     W2 = synth.normal_bf16(0, synth.TID_W2, (E, d, f), 0.0, 1.0 / np.sqrt(f))
     Wd = (None, to_dev_bf16(W1, torch), to_dev_bf16(W3, torch), to_dev_bf16(W2, torch))
+    sampler = make_clock_sampler(None)
+    sampler.start()
     cases = [("tiny", None), ("decode", None), ("prefill", None), ("skew", None)] + \
             [("sweep", T) for T in synth.SWEEP_T]
     for name, T in cases:
@@ -581,7 +756,9 @@ def run_sweep(args):
         N, touched = run.kept_and_touched()
         for _ in range(args.warmup):
             run.step()
-        ms = time_steps(run.step, args.steps, torch) / args.steps
+        tag = f"{name}{'' if T is None else T}"
+        with sampler_region(sampler, tag):
+            ms = time_steps(run.step, args.steps, torch) / args.steps
         stages = run.profiled(args.steps)
         flops = 6.0 * N * wl.d * wl.f + 2.0 * wl.T * wl.d * wl.E
         wbytes = touched * 3 * wl.d * wl.f * 2
@@ -592,11 +769,29 @@ def run_sweep(args):
                     ms_per_step=ms, tokens_per_s=wl.T / (ms * 1e-3), tflops=tfs, gbs=gbs,
                     frac_bf16_burst=tfs / peaks["bf16"], frac_hbm=gbs / peaks["hbm"], stage_ms=stages,
                     peaks_source=peaks["source"])
+        if hasattr(sampler, "samples"):
+            rows = [r for r in sampler.samples if r[0] == tag]
+            line["clocks"] = sampler._summary(rows)
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, n_sample=min(16, wl.T))
         print(json.dumps(line), flush=True)
         del run
         torch.cuda.empty_cache()
+    sampler.stop()
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        return s_.getsockname()[1]
+
+
+def launch_ranks(args) -> int:
+    """Relaunch this script under torchrun with --gpus ranks on this node."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -608,10 +803,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload (tiny, decode, prefill, skew, T sweep) instead of the contract line")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="check the rank launcher and plumbing on CPU (gloo): no GPU work")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args))
+    if args.dry_run:
+        run_dry(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.sweep:
         run_sweep(args)

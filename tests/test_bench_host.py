@@ -106,3 +106,106 @@ def test_expert_bytes(d, f):
     assert bench.expert_bytes(d, f) == 3 * d * f * 2
     # 4 bits a weight plus one bf16 scale per 64 weights
     assert bench.expert_bytes_q4(d, f) * 64 == 3 * d * f * (32 + 2)
+
+
+class _FakeNvml:
+    """Just the NVML calls NvmlSampler makes, over a scripted clock trace."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonHwPowerBrakeSlowdown = 0x80
+
+    class _Pci:
+        def __init__(self, bus):
+            self.busId = bus
+
+    def __init__(self, buses, trace):
+        self.buses, self.trace, self.i = buses, trace, 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetCount(self):
+        return len(self.buses)
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+    def nvmlDeviceGetPciInfo(self, h):
+        return self._Pci(self.buses[h].encode())
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        assert h == 1, "sampled the wrong GPU"
+        return self.trace[min(self.i, len(self.trace) - 1)][0]
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return self.trace[min(self.i, len(self.trace) - 1)][1] * 1000
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        r = self.trace[min(self.i, len(self.trace) - 1)][2]
+        self.i += 1
+        return r
+
+
+def test_nvml_sampler_regions_and_reasons():
+    fake = _FakeNvml(["00000000:1A:00.0", "00000000:1B:00.0"],
+                     [(1965, 300, 0), (1900, 500, 0), (1500, 990, 0x4), (1300, 1000, 0x4 | 0x20)])
+    s = bench.NvmlSampler("00000000:1b:00.0", nvml=fake)   # picks device 1 by PCI bus id
+    assert s.max_mhz == 1965
+    s.sample("decode")
+    s.sample("decode")
+    s.sample("prefill")
+    s.sample("prefill")
+    c = s.stop()
+    assert c["samples"] == 4 and c["sm_max_mhz"] == 1965
+    assert c["by_region"]["decode"]["sm_mhz"] == 1932.5 and c["by_region"]["decode"]["reasons"] == []
+    assert c["by_region"]["prefill"]["sm_mhz"] == 1400 and c["by_region"]["prefill"]["power_w_max"] == 1000
+    assert c["by_region"]["prefill"]["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    assert c["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+
+
+def test_nvml_sampler_samples_only_inside_regions():
+    import time as _t
+    fake = _FakeNvml(["00000000:1A:00.0", "00000000:1B:00.0"], [(1965, 300, 0)])
+    s = bench.NvmlSampler("00000000:1B:00.0", period_s=0.001, nvml=fake)
+    s.start()
+    _t.sleep(0.02)
+    assert s.samples == []
+    with s.region("prefill"):
+        _t.sleep(0.05)
+    n = len(s.samples)
+    _t.sleep(0.02)
+    c = s.stop()
+    assert n > 0 and len(s.samples) <= n + 1
+    assert set(c["by_region"]) == {"prefill"}
+
+
+def test_dry_run_launches_ranks():
+    """--gpus 2 without torchrun relaunches itself with two ranks; the slower
+    rank's step time (2 ms) is reported and the value counts both ranks."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run", "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["n_gpus"] == 2 and line["ranks_seen"] == 2
+    assert line["ms_per_step"] == 2.0 and line["value"] == 2 * 4096 / 2e-3
+
+
+def test_world_size_must_match_gpus():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0 and "--gpus 2 but 1 ranks" in r.stderr
+
+
+def test_both_arms_share_the_config():
+    import synth
+    wl = synth.workload("prefill")
+    assert bench.bench_config(wl, 1) == bench.bench_config(synth.workload("prefill"), 1)
+    assert bench.bench_config(wl, 8)["parallelism"].startswith("dp8")
