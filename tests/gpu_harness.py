@@ -59,6 +59,27 @@ class Device:
                               wl.drop_policy, variant)
 
 
+class guarded:
+    """With the debug library loaded, arm the workspace guards before the
+    calls inside the block and check them (and the device status) after;
+    with the release library, nothing."""
+
+    def __init__(self, sh, ws, nws, q4=False):
+        self.sh, self.ws, self.nws, self.q4 = sh, ws, nws, q4
+        self.on = moe.moe_debug_build() == 1
+
+    def __enter__(self):
+        if self.on:
+            moe.check(moe.moe_debug_workspace_arm(self.sh, self.ws, self.nws, self.q4), "debug_workspace_arm")
+        return self
+
+    def __exit__(self, exc_type, exc, tb):
+        if self.on and exc_type is None:
+            st = moe.moe_debug_workspace_check(self.sh, self.ws, self.nws, self.q4)
+            assert st == moe.MOE_OK, f"workspace guard overwritten: {moe.status_string(st)}"
+        return False
+
+
 def run_stages(dev: Device, variant: int = 0) -> dict:
     """Router -> permute -> grouped SwiGLU -> combine through the stage entry points."""
     wl = dev.wl
@@ -74,12 +95,14 @@ def run_stages(dev: Device, variant: int = 0) -> dict:
     nws = moe.moe_workspace_size(sh)
     ws = cu(nws, dt=torch.uint8)
     o = out
-    moe.check(moe.moe_router_topk(sh, dev.x, dev.Wg, o["logits"], o["idx"], o["w"], o["p"], o["counts"]), "router")
-    moe.check(moe.moe_permute(sh, dev.x, o["idx"], o["p"], o["counts"], o["offsets"], o["slot_pos"],
-                              o["perm_slot"], o["x_perm"], ws, nws), "permute")
-    moe.check(moe.moe_grouped_swiglu(sh, o["x_perm"], o["offsets"], dev.W1, dev.W3, dev.W2, o["h"], o["y_perm"],
-                                     ws, nws), "grouped_swiglu")
-    moe.check(moe.moe_combine(sh, o["y_perm"], o["slot_pos"], o["w"], o["y"]), "combine")
+    with guarded(sh, ws, nws):
+        moe.check(moe.moe_router_topk(sh, dev.x, dev.Wg, o["logits"], o["idx"], o["w"], o["p"], o["counts"]),
+                  "router")
+        moe.check(moe.moe_permute(sh, dev.x, o["idx"], o["p"], o["counts"], o["offsets"], o["slot_pos"],
+                                  o["perm_slot"], o["x_perm"], ws, nws), "permute")
+        moe.check(moe.moe_grouped_swiglu(sh, o["x_perm"], o["offsets"], dev.W1, dev.W3, dev.W2, o["h"],
+                                         o["y_perm"], ws, nws), "grouped_swiglu")
+        moe.check(moe.moe_combine(sh, o["y_perm"], o["slot_pos"], o["w"], o["y"]), "combine")
     st = moe.moe_read_device_status(ws)
     assert st == moe.MOE_OK, moe.status_string(st)
     torch.cuda.synchronize()
@@ -96,8 +119,9 @@ def run_layer(dev: Device, variant: int = 0, reps: int = 1) -> dict:
     counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
     ys = []
     for _ in range(reps):
-        moe.check(moe.moe_layer_forward(sh, dev.x, dev.Wg, dev.W1, dev.W3, dev.W2, y, idx, counts, ws, nws),
-                  "layer_forward")
+        with guarded(sh, ws, nws):
+            moe.check(moe.moe_layer_forward(sh, dev.x, dev.Wg, dev.W1, dev.W3, dev.W2, y, idx, counts, ws, nws),
+                      "layer_forward")
         st = moe.moe_read_device_status(ws)
         assert st == moe.MOE_OK, moe.status_string(st)
         ys.append(bf16_host(y).copy())
@@ -205,18 +229,42 @@ def compare_routing(gpu: dict, r: dict, wl: synth.Workload):
     return N
 
 
-def sample_tokens(wl: synth.Workload, r: dict, n: int, seed: int = 1) -> np.ndarray:
-    """n token indices, always including dropped ones when there are any."""
-    T = wl.T
+def sample_tokens(wl: synth.Workload, r: dict, n: int, seed: int = 1, block_rows: int | None = None) -> np.ndarray:
+    """n random token indices, plus: dropped tokens when there are any, the
+    first and last token, and -- with block_rows, the token-block height of
+    the GEMM schedule in use -- the token of one random row in every
+    (expert, token block) tile and of the last row of every expert, so that
+    every tile of both GEMMs (a full row of h or y_perm spans all weight
+    blocks) and every partial last block is checked."""
+    T, k = wl.T, wl.k
     if T <= n:
         return np.arange(T)
     rng = np.random.default_rng(seed)
     pick = set(rng.choice(T, size=n, replace=False).tolist())
-    dropped = np.nonzero((r["slot_pos"].reshape(T, wl.k) < 0).any(1))[0]
+    dropped = np.nonzero((r["slot_pos"].reshape(T, k) < 0).any(1))[0]
     for t in dropped[: max(1, n // 4)]:
         pick.add(int(t))
     pick.update({0, T - 1})
+    if block_rows:
+        off, perm = r["offsets"], r["perm_slot"]
+        for e in range(len(off) - 1):
+            lo, hi = int(off[e]), int(off[e + 1])
+            for b0 in range(lo, hi, block_rows):
+                row = int(rng.integers(b0, min(hi, b0 + block_rows)))
+                pick.add(int(perm[row]) // k)
+            if hi > lo:
+                pick.add(int(perm[hi - 1]) // k)
     return np.array(sorted(pick), np.int64)
+
+
+def schedule_block_rows(T: int, variant: int) -> int:
+    """Token rows per tile of the expert GEMMs: the streaming schedule's
+    token tile (T <= 128 under AUTO), 256 for CTA pairs, 128 for single-CTA
+    tiles."""
+    if variant == 2 or (variant == 0 and T <= 128):
+        b = max(16, ((T + 15) // 16) * 16)
+        return 16 if b <= 16 else 32 if b <= 32 else 64 if b <= 64 else 128
+    return 128 if variant == 3 else 256
 
 
 # ------------------------------------------------------------ 4-bit experts
@@ -243,7 +291,9 @@ def run_layer_q4(dev: QDevice, reps: int = 1) -> dict:
     counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
     ys = []
     for _ in range(reps):
-        moe.check(moe.moe_layer_forward_q4(sh, dev.x, dev.Wg, *dev.q, y, idx, counts, ws, nws), "layer_forward_q4")
+        with guarded(sh, ws, nws, q4=True):
+            moe.check(moe.moe_layer_forward_q4(sh, dev.x, dev.Wg, *dev.q, y, idx, counts, ws, nws),
+                      "layer_forward_q4")
         st = moe.moe_read_device_status(ws)
         assert st == moe.MOE_OK, moe.status_string(st)
         ys.append(bf16_host(y).copy())

@@ -112,3 +112,24 @@ def test_ep_layer_one_process_group_of_one(o):
         del layer
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,E", [(1, 8), (2, 8), (4, 8), (8, 8), (4, 16), (8, 32)])
+def test_ep_plan_kernel_equals_host_plan(world, E):
+    """moe_ep_plan (the device plan the layer uses) equals ep_plan_host (the
+    host restatement the multi-rank CPU tests check), for every rank, on
+    random counts with empty sources and empty experts."""
+    from sparse_mixture_experts_13_b200.ep import ep_plan_host
+    g = torch.Generator().manual_seed(world * 100 + E)
+    counts_all = torch.randint(0, 300, (world, E), generator=g, dtype=torch.int32)
+    counts_all[0, 0] = 0
+    counts_all[:, E - 1] = 0
+    dev_counts = counts_all.cuda().contiguous()
+    epr = E // world
+    for rank in range(world):
+        recv_off = torch.full((E,), -1, dtype=torch.int32, device="cuda")
+        owner_off = torch.full((epr + 1,), -1, dtype=torch.int32, device="cuda")
+        moe.check(moe.moe_ep_plan(dev_counts, E, rank, world, recv_off, owner_off), "moe_ep_plan")
+        want_recv, want_owner = ep_plan_host(counts_all.tolist(), rank, world)
+        assert recv_off.cpu().tolist() == want_recv, rank
+        assert owner_off.cpu().tolist() == want_owner, rank

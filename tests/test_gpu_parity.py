@@ -82,7 +82,8 @@ def check_everything(o, wl, variant, rows=None, stages=True):
         assert r is not None
     assert np.array_equal(lay["idx"].reshape(wl.T, wl.k), r["idx"]), "layer topk_idx"
     assert np.array_equal(lay["counts"], r["counts"]), "layer counts"
-    toks = np.arange(wl.T) if rows is None else H.sample_tokens(wl, r, rows)
+    toks = np.arange(wl.T) if rows is None else \
+        H.sample_tokens(wl, r, rows, block_rows=H.schedule_block_rows(wl.T, variant))
     ref = o.layer_rows(wl.x, wl.W1, wl.W3, wl.W2, r, toks, want_h=stages, want_o=stages)
     y_gpu = H.bf16_f64(lay["y"])[toks]
     H.assert_close(y_gpu, ref["y"], f"y (layer, {VNAME[variant]})")
@@ -227,14 +228,14 @@ def test_decode_T16(o, variant):
 
 @pytest.mark.parametrize("variant", [0, 2, 3], ids=lambda v: VNAME[v])
 def test_prefill_T4096(o, variant):
-    check_everything(o, full_workload("prefill"), variant, rows=24)
+    check_everything(o, full_workload("prefill"), variant, rows=64)
 
 
 @pytest.mark.parametrize("policy", [0, 1], ids=["by_prob", "by_order"])
 def test_skew_T8192_capacity(o, policy):
     wl = full_workload("skew")
     wl.drop_policy = policy
-    stats = check_everything(o, wl, 0, rows=24)
+    stats = check_everything(o, wl, 0, rows=64)
     share = float((H.run_layer(device_inputs(wl), 0)["counts"][0])) / (wl.T * wl.k)
     assert 0.37 < share < 0.43, share
     wl.drop_policy = 0
@@ -242,7 +243,7 @@ def test_skew_T8192_capacity(o, policy):
 
 @pytest.mark.parametrize("T", [1, 8, 64, 512, 32768])
 def test_sweep(o, T):
-    check_everything(o, full_workload("sweep", T=T), 0, rows=16)
+    check_everything(o, full_workload("sweep", T=T), 0, rows=64 if T >= 4096 else 16)
 
 
 @pytest.mark.parametrize("E", [8, 16, 32])
