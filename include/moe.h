@@ -77,7 +77,8 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2, /* valid request the library does not handle (e.g. not sm_100) */
   MOE_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
   MOE_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
-  MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up */
+  MOE_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+  MOE_ERR_BOUNDS = 6       /* a device-side bounds check failed (debug build only) */
 } moe_status;
 
 /* Which slots an overfull expert drops (capacity mode only). */
@@ -176,11 +177,24 @@ MOE_API moe_status moe_permute(const moe_shape *shape, const moe_bf16 *x, const 
  * last call's contents: each call clears what must start at zero, and calls
  * whose work overlaps on the GPU (other streams, other host threads) race on
  * it, so serialise them.  A device-side look-back wait that gives up is
- * recorded only in that shared array and is not reported to the caller. */
+ * recorded in that shared array; moe_permute_noalloc_status reads it.  The
+ * looked-up address belongs to the device's context as it was at that first
+ * call: after cudaDeviceReset (or any other teardown of the device's primary
+ * context) in the same process, the address is stale and this entry point
+ * must not be called on that device again. */
 MOE_API moe_status moe_permute_noalloc(const moe_shape *shape, const moe_bf16 *x,
                                        const int32_t *topk_idx, const float *topk_p,
                                        const int32_t *counts, int32_t *offsets, int32_t *slot_pos,
                                        int32_t *perm_slot, moe_bf16 *x_perm, moe_stream_t stream);
+
+/* Device status of the last moe_permute_noalloc call on the current device
+ * (the pages have no counterpart): synchronises `stream`, then reads the
+ * status word of the shared scratch array.  MOE_OK, or MOE_ERR_TIMEOUT if a
+ * look-back wait of that call gave up (its outputs are then invalid), or
+ * MOE_ERR_CUDA if the stream reports an error.  Each moe_permute_noalloc
+ * call clears the word first, so only the most recent call is reported;
+ * before any call on the device it returns MOE_OK.  Allocates nothing. */
+MOE_API moe_status moe_permute_noalloc_status(moe_stream_t stream);
 
 /* Grouped SwiGLU experts on tensor cores.  Source: "Mixtral", "MoE Layer"
  * (MixtralExpert.forward) and "SwiGLU Experts".  For each expert e and row r
@@ -360,6 +374,17 @@ MOE_API moe_status moe_layer_forward_q4(const moe_shape *shape, const moe_bf16 *
                                         moe_bf16 *y, int32_t *topk_idx_out, int32_t *counts_out,
                                         void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_layer_forward_q4 with the activations in HOST memory, as
+ * moe_layer_forward_host: copies x_host [T, d] into the workspace, runs the
+ * 4-bit layer and copies y back to y_host [T, d], all queued on `stream`.
+ * The workspace is the one of moe_workspace_size_q4.  Use page-locked host
+ * buffers; y_host is valid once the stream has been synchronised. */
+MOE_API moe_status moe_layer_forward_q4_host(const moe_shape *shape, const moe_bf16 *x_host,
+                                             const float *Wg, const uint8_t *W1c, const moe_bf16 *W1s,
+                                             const uint8_t *W3c, const moe_bf16 *W3s, const uint8_t *W2c,
+                                             const moe_bf16 *W2s, moe_bf16 *y_host, void *ws,
+                                             size_t ws_bytes, moe_stream_t stream);
+
 /* moe_layer_forward_q4 recording six CUDA events (cudaEvent_t) on `stream`
  * between its stages, as moe_layer_forward_profiled. */
 MOE_API moe_status moe_layer_forward_q4_profiled(const moe_shape *shape, const moe_bf16 *x,
@@ -386,6 +411,35 @@ MOE_API moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, uint32_t
  * call that used this workspace (MOE_OK or MOE_ERR_TIMEOUT), or
  * MOE_ERR_CUDA if the stream reports an error. */
 MOE_API moe_status moe_read_device_status(const void *ws, moe_stream_t stream);
+
+/* ------------------------------------------------------------ debug build
+ * The pages have no counterpart of this section.  The library also builds as
+ * libmoe_debug.so (compiled with MOE_DEBUG): the same entry points, plus
+ *   - in-kernel bounds checks on the indices the kernels derive on the device
+ *     (grouped rows below offsets[e+1] and below T * k, slot rows read by the
+ *     combine below T * k, token indices below T).  A failed check skips the
+ *     access and records MOE_ERR_BOUNDS in the status word; nothing traps;
+ *   - a 256-byte guard after each workspace region past the control region
+ *     (the debug build's moe_workspace_size includes them);
+ *   - a host-side stage-failure hook: with the environment variable
+ *     MOE_DEBUG_FAIL_STAGE=n (1 router, 2 capacity / grouping, 3 expert
+ *     GEMMs, 4 combine, 5 output copies), the whole-layer entry points return
+ *     MOE_ERR_CUDA just before queuing stage n, so nothing from stage n on is
+ *     queued.
+ * The release library returns 0 from moe_debug_build and MOE_ERR_UNSUPPORTED
+ * from the two guard calls. */
+MOE_API int32_t moe_debug_build(void);
+
+/* Debug build: fill the guards of a workspace laid out for `shape` (q4 != 0:
+ * the layout of moe_workspace_size_q4) with a fixed byte pattern, queued on
+ * `stream`. */
+MOE_API moe_status moe_debug_workspace_arm(const moe_shape *shape, void *ws, size_t ws_bytes,
+                                           int32_t q4, moe_stream_t stream);
+
+/* Debug build: synchronise `stream` and check that every guard still holds
+ * the pattern: MOE_OK, or MOE_ERR_WORKSPACE if any byte changed. */
+MOE_API moe_status moe_debug_workspace_check(const moe_shape *shape, const void *ws, size_t ws_bytes,
+                                             int32_t q4, moe_stream_t stream);
 
 /* Static English text of a status code. */
 MOE_API const char *moe_status_string(moe_status status);

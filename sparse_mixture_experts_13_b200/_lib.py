@@ -13,17 +13,22 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe.so")
+# MOE_LIB=debug selects the debug build (device-side bounds checks, workspace
+# guards, stage-failure hook); the default is the release library.
+LIB_PATH = os.path.join(_PKG, "libmoe_debug.so" if os.environ.get("MOE_LIB") == "debug" else "libmoe.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
+    MOE_ERR_BOUNDS = range(7)
 MOE_DROP_BY_PROB, MOE_DROP_BY_ORDER, MOE_DROP_BY_PROB_NEXT_BEST, MOE_DROP_BY_ORDER_NEXT_BEST = 0, 1, 2, 3
 MOE_VARIANT_AUTO, MOE_VARIANT_TILED, MOE_VARIANT_STREAM, MOE_VARIANT_TILED_SINGLE = 0, 1, 2, 3
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc",
+            "moe_permute_noalloc_status",
             "moe_selftest_wait_timeout", "moe_read_device_status", "moe_router_stats", "moe_ep_plan", "moe_ep_dispatch",
             "moe_ep_combine", "moe_quantize_q4", "moe_workspace_size_q4",
-            "moe_grouped_swiglu_q4", "moe_layer_forward_q4", "moe_layer_forward_q4_profiled", "moe_status_string")
+            "moe_grouped_swiglu_q4", "moe_layer_forward_q4", "moe_layer_forward_q4_profiled", "moe_layer_forward_q4_host",
+            "moe_debug_build", "moe_debug_workspace_arm", "moe_debug_workspace_check", "moe_status_string")
 _SIZE_RETURNING = ("moe_workspace_size", "moe_workspace_size_q4")
 
 
@@ -61,6 +66,7 @@ def lib():
         L.moe_router_topk.argtypes = [S, P, P, P, P, P, P, P, P]
         L.moe_permute.argtypes = [S, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_permute_noalloc.argtypes = [S, P, P, P, P, P, P, P, P, P]
+        L.moe_permute_noalloc_status.argtypes = [P]
         L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.moe_combine.argtypes = [S, P, P, P, P, P]
         L.moe_layer_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, sz, P]
@@ -78,6 +84,10 @@ def lib():
         L.moe_grouped_swiglu_q4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_layer_forward_q4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_layer_forward_q4_profiled.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_layer_forward_q4_host.argtypes = [S, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_debug_build.argtypes = []
+        L.moe_debug_workspace_arm.argtypes = [S, P, sz, ctypes.c_int32, P]
+        L.moe_debug_workspace_check.argtypes = [S, P, sz, ctypes.c_int32, P]
         L.moe_status_string.argtypes = [st]
         L.moe_status_string.restype = ctypes.c_char_p
         for name in EXPORTED:
@@ -135,6 +145,11 @@ def moe_permute_noalloc(shape, x, topk_idx, topk_p, counts, offsets, slot_pos, p
     """moe_permute with its scratch in a fixed device array (no workspace)."""
     return lib().moe_permute_noalloc(ctypes.byref(shape), _p(x), _p(topk_idx), _p(topk_p), _p(counts), _p(offsets),
                                      _p(slot_pos), _p(perm_slot), _p(x_perm), _stream(stream))
+
+
+def moe_permute_noalloc_status(stream=None) -> int:
+    """Status of the last moe_permute_noalloc call on the current device."""
+    return lib().moe_permute_noalloc_status(_stream(stream))
 
 
 def moe_grouped_swiglu(shape, x_perm, offsets, W1, W3, W2, h, y_perm, ws, ws_bytes, stream=None) -> int:
@@ -223,6 +238,12 @@ def moe_layer_forward_q4(shape, x, Wg, q1, q3, q2, y, topk_idx_out, counts_out, 
                                       _p(ws), int(ws_bytes), _stream(stream))
 
 
+def moe_layer_forward_q4_host(shape, x_host, Wg, q1, q3, q2, y_host, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_layer_forward_q4_host(ctypes.byref(shape), _p(x_host), _p(Wg), _p(q1[0]), _p(q1[1]),
+                                           _p(q3[0]), _p(q3[1]), _p(q2[0]), _p(q2[1]), _p(y_host), _p(ws),
+                                           int(ws_bytes), _stream(stream))
+
+
 def moe_layer_forward_q4_profiled(shape, x, Wg, q1, q3, q2, y, events, ws, ws_bytes, stream=None) -> int:
     return lib().moe_layer_forward_q4_profiled(ctypes.byref(shape), _p(x), _p(Wg), _p(q1[0]), _p(q1[1]),
                                                _p(q3[0]), _p(q3[1]), _p(q2[0]), _p(q2[1]), _p(y),
@@ -235,3 +256,18 @@ def moe_selftest_wait_timeout(ws, ws_bytes, limit_us, stream=None) -> int:
 
 def moe_read_device_status(ws, stream=None) -> int:
     return lib().moe_read_device_status(_p(ws), _stream(stream))
+
+
+# ------------------------------------------------------------ debug build
+
+def moe_debug_build() -> int:
+    return int(lib().moe_debug_build())
+
+
+def moe_debug_workspace_arm(shape, ws, ws_bytes, q4=False, stream=None) -> int:
+    return lib().moe_debug_workspace_arm(ctypes.byref(shape), _p(ws), int(ws_bytes), int(bool(q4)), _stream(stream))
+
+
+def moe_debug_workspace_check(shape, ws, ws_bytes, q4=False, stream=None) -> int:
+    return lib().moe_debug_workspace_check(ctypes.byref(shape), _p(ws), int(ws_bytes), int(bool(q4)),
+                                           _stream(stream))

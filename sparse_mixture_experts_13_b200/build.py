@@ -16,6 +16,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
+# debug build: -DMOE_DEBUG (device-side bounds checks, workspace guards,
+# stage-failure hook), objects in _build/debug
+LIB_DEBUG = os.path.join(PKG, "libmoe_debug.so")
 SOURCES = ["router.cu", "permute.cu", "expert_gemm.cu", "expert_gemm_q4.cu", "router_stats.cu", "fallback.cu", "ep.cu", "combine.cu", "moe_api.cu", "selftest.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,30 +38,32 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, extra):
-    obj = os.path.join(BUILD, os.path.basename(src).replace(".cu", ".o"))
+def _compile(src, extra, outdir=BUILD):
+    obj = os.path.join(outdir, os.path.basename(src).replace(".cu", ".o"))
     if _stale(obj, [src] + _headers()):
         cmd = [NVCC] + FLAGS + list(extra) + ["-c", src, "-o", obj]
         subprocess.run(cmd, check=True)
     return obj
 
 
-def build(force: bool = False, extra_flags=(), verbose_ptxas: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
-    extra = list(extra_flags) + (["-Xptxas", "-v"] if verbose_ptxas else [])
+def build(force: bool = False, extra_flags=(), verbose_ptxas: bool = False, debug: bool = False) -> str:
+    outdir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = LIB_DEBUG if debug else LIB
+    os.makedirs(outdir, exist_ok=True)
+    extra = list(extra_flags) + (["-Xptxas", "-v"] if verbose_ptxas else []) + (["-DMOE_DEBUG"] if debug else [])
     if force:
-        for o in glob.glob(os.path.join(BUILD, "*.o")):
+        for o in glob.glob(os.path.join(outdir, "*.o")):
             os.remove(o)
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
     with cf.ThreadPoolExecutor(max_workers=len(srcs)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra), srcs))
-    if force or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, extra, outdir), srcs))
+    if force or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.run([NVCC] + ARCH + ["-shared", "-o", tmp] + objs, check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     import sys
-    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv, debug="--debug" in sys.argv))

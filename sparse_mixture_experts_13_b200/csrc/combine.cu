@@ -35,6 +35,8 @@ template <int CPL, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   constexpr int kCols = 32 * CPL;
   constexpr int NV = CPL / 8;  // 16-byte bf16 vectors per lane
+  pdl_wait();  // the expert GEMMs' outputs (and, through them, the router's)
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -51,8 +53,9 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
       pos[j] = -1;
       w[j] = 0.f;
       if (j < a.k) {
-        pos[j] = __ldg(a.slot_pos + t * a.k + j);
-        w[j] = __ldg(a.topk_w + t * a.k + j);
+        pos[j] = a.slot_pos[t * a.k + j];
+        w[j] = a.topk_w[t * a.k + j];
+        if (pos[j] >= 0 && !MOE_DCHECK(a.status, pos[j] < a.T * a.k)) pos[j] = -1;
       }
     }
     float acc[CPL];
@@ -65,7 +68,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
         if (pos[j] >= 0) {
           const uint4* src = reinterpret_cast<const uint4*>(a.y_perm + (int64_t)pos[j] * a.d + col);
 #pragma unroll
-          for (int h = 0; h < NV; ++h) raw[j][h] = __ldg(src + h);
+          for (int h = 0; h < NV; ++h) raw[j][h] = src[h];
         }
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
@@ -93,7 +96,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
           for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int c = 0; c < CPL / 4; ++c)
-              q[u][c] = __ldg(reinterpret_cast<const float4*>(base + (sp + u) * a.part_stride) + c);
+              q[u][c] = reinterpret_cast<const float4*>(base + (sp + u) * a.part_stride)[c];
 #pragma unroll
           for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
         for (; sp < a.splits; ++sp) {
 #pragma unroll
           for (int c = 0; c < CPL / 4; ++c) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(base + sp * a.part_stride) + c);
+            const float4 v = reinterpret_cast<const float4*>(base + sp * a.part_stride)[c];
             o[4 * c] += v.x;
             o[4 * c + 1] += v.y;
             o[4 * c + 2] += v.z;
@@ -133,21 +136,22 @@ cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
   const int64_t cap = (int64_t)num_sms * 16;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
+  const dim3 g((unsigned)blocks), b(256);
   if (a.k <= 2) {
-    if (cpl == 16) combine_kernel<16, 2><<<(unsigned)blocks, 256, 0, s>>>(a);
-    else combine_kernel<8, 2><<<(unsigned)blocks, 256, 0, s>>>(a);
-  } else {
-    if (cpl == 16) combine_kernel<16, 8><<<(unsigned)blocks, 256, 0, s>>>(a);
-    else combine_kernel<8, 8><<<(unsigned)blocks, 256, 0, s>>>(a);
+    if (cpl == 16) return launch_k(combine_kernel<16, 2>, g, b, 0, s, a.pdl, a);
+    return launch_k(combine_kernel<8, 2>, g, b, 0, s, a.pdl, a);
   }
-  return cudaGetLastError();
+  if (cpl == 16) return launch_k(combine_kernel<16, 8>, g, b, 0, s, a.pdl, a);
+  return launch_k(combine_kernel<8, 8>, g, b, 0, s, a.pdl, a);
 }
 
 // y_perm[r] = bf16(sum over splits of partials[sp][r]) for rows r < offsets[E].
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partials, int32_t splits,
                                                             int64_t part_stride, const int32_t* __restrict__ offsets,
-                                                            int32_t E, uint16_t* __restrict__ y_perm, int32_t d) {
-  const int64_t rows = offsets[E];
+                                                            int32_t E, uint16_t* __restrict__ y_perm, int32_t d,
+                                                            int64_t S, uint32_t* status) {
+  int64_t rows = offsets[E];
+  if (!MOE_DCHECK(status, rows >= 0 && rows <= S)) rows = 0;
   const int nvec = d >> 3;
   const int64_t total = rows * nvec;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
@@ -168,12 +172,14 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
 }
 
 cudaError_t launch_splitk_reduce(const float* partials, int32_t splits, int64_t part_stride, const int32_t* offsets,
-                                 int32_t E, uint16_t* y_perm, int64_t S, int32_t d, int num_sms, cudaStream_t s) {
+                                 int32_t E, uint16_t* y_perm, int64_t S, int32_t d, int num_sms, cudaStream_t s,
+                                 uint32_t* status) {
   int64_t blocks = (S * (d / 8) + 255) / 256;
   const int64_t cap = (int64_t)num_sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(partials, splits, part_stride, offsets, E, y_perm, d);
+  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(partials, splits, part_stride, offsets, E, y_perm, d, S,
+                                                         status);
   return cudaGetLastError();
 }
 

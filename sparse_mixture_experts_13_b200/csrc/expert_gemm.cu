@@ -63,6 +63,9 @@ struct GemmParams {
   int32_t splits;       // K splits (STREAM partial), else 1
   int32_t kb_per_split;
   uint32_t* tile_counter;  // CTA-pair kernels: next tile id (zero before the launch)
+  int64_t S;               // rows of the activation and output buffers (T * k)
+  int32_t prefetch_kb;     // streaming kernels launched as dependents: K chunks of the
+                           // first tile's weights to prefetch into L2 before waiting (0: none)
 };
 
 __host__ __device__ constexpr bool epi_is_tiled(int epi) { return epi <= EPI_TILED_STORE; }
@@ -170,12 +173,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(&s_tmem, C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (!C::kTiled && tid == 0 && p.prefetch_kb > 0) {
+    // While the router and the grouping still run, start pulling into L2 the
+    // weights of this CTA's first tile as it would be if every expert had one
+    // block of tokens (the usual decode case).  A wrong guess costs only L2
+    // traffic: nothing is written to shared memory and nothing waits.
+    const int32_t per_e = p.n_blocks * p.splits;
+    const int32_t e = (int32_t)blockIdx.x / per_e;
+    if (e < p.E) {
+      const int32_t rest = (int32_t)blockIdx.x % per_e;
+      const int32_t kb0 = (rest % p.splits) * p.kb_per_split;
+      const int32_t n0 = (rest / p.splits) * C::W_ROWS;
+      const int32_t kb1 = min(p.num_kb, kb0 + min(p.kb_per_split, p.prefetch_kb));
+      for (int32_t kb = kb0; kb < kb1; ++kb) {
+        tma_prefetch_l2_3d(&map_wa, kb * BK, n0, e);
+        if (EPI == EPI_STREAM_SWIGLU) tma_prefetch_l2_3d(&map_wb, kb * BK, n0, e);
+      }
+    }
+  }
+  pdl_wait();     // offsets and activations of the kernels before this one
+  pdl_trigger();  // the next kernel may start its own set-up
   if (tid == 64) {
     s_abort = 0;
     s_epi_fail = 0;
     int32_t acc = 0;
     s_base[0] = 0;
     for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+#ifdef MOE_DEBUG
+    {  // offsets must start at 0, not decrease and stay within the S rows
+      bool bad = s_off[0] != 0 || (int64_t)s_off[p.E] > p.S;
+      for (int e = 0; e < p.E; ++e) bad = bad || s_off[e + 1] < s_off[e];
+      if (bad) {
+        record_status(p.status, kStatusBounds);
+        for (int e = 0; e <= p.E; ++e) s_off[e] = 0;
+      }
+    }
+#endif
     for (int e = 0; e < p.E; ++e) {
       const int32_t M_e = s_off[e + 1] - s_off[e];
       int32_t n = 0;
@@ -323,7 +356,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_32x32b_x32(t_acc + c0, va);
           tmem_ld_32x32b_x32(t_acc + 128 + c0, vb);
           tmem_ld_wait();
-          if (row_ok && t.n0 + c0 < p.n_out) {
+          if (row_ok && t.n0 + c0 < p.n_out && MOE_DCHECK(p.status, t.row0 + r < p.S)) {
             uint32_t packed[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -345,7 +378,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t v[32];
           tmem_ld_32x32b_x32(t_acc + c0, v);
           tmem_ld_wait();
-          if (row_ok && t.n0 + c0 < p.n_out) {
+          if (row_ok && t.n0 + c0 < p.n_out && MOE_DCHECK(p.status, t.row0 + r < p.S)) {
             uint32_t packed[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -374,7 +407,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int tok = c0 + j;
-              if (tok < t.m_valid) {
+              if (tok < t.m_valid && MOE_DCHECK(p.status, t.row0 + tok < p.S)) {
                 const float hv = silu_f32(__uint_as_float(v[j])) * xbuf[j * 64 + r];
                 out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] =
                     (uint16_t)(pack_bf16x2(hv, 0.f) & 0xFFFFu);
@@ -396,7 +429,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int tok = c0 + j;
-              if (tok < t.m_valid) out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] = __uint_as_float(v[j]);
+              if (tok < t.m_valid && MOE_DCHECK(p.status, t.row0 + tok < p.S))
+                out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] = __uint_as_float(v[j]);
             }
           }
         }
@@ -532,12 +566,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc_pair(&s_tmem, 512);
     tmem_relinquish_pair();
   }
+  pdl_wait();     // offsets and activations of the kernels before this one
+  pdl_trigger();  // the next kernel may start its own set-up
   if (tid == 64) {
     s_abort = 0;
     s_epi_fail = 0;
     int32_t acc = 0;
     s_base[0] = 0;
     for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+#ifdef MOE_DEBUG
+    {  // offsets must start at 0, not decrease and stay within the S rows
+      bool bad = s_off[0] != 0 || (int64_t)s_off[p.E] > p.S;
+      for (int e = 0; e < p.E; ++e) bad = bad || s_off[e + 1] < s_off[e];
+      if (bad) {
+        record_status(p.status, kStatusBounds);
+        for (int e = 0; e <= p.E; ++e) s_off[e] = 0;
+      }
+    }
+#endif
     for (int e = 0; e < p.E; ++e) {
       const int32_t M_e = s_off[e + 1] - s_off[e];
       acc += (M_e > 0) ? ((M_e + 255) / 256) * p.n_blocks : 0;
@@ -733,7 +779,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // lanes 0..63: W1 projection of columns n0 + 64*rank + lane;
           // lanes 64..127: the W3 projection of the same columns.
           const int32_t col = t.n0 + (int32_t)rank * 64 + 8 * g;
-          if (n < t.m_valid && col < p.n_out) {
+          if (n < t.m_valid && col < p.n_out && MOE_DCHECK(p.status, t.row0 + n < p.S)) {
             const float4 a0 = *reinterpret_cast<const float4*>(row + 8 * g);
             const float4 a1 = *reinterpret_cast<const float4*>(row + 8 * g + 4);
             const float4 b0 = *reinterpret_cast<const float4*>(row + 64 + 8 * g);
@@ -748,7 +794,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
           // lane l: output column n0 + 128*rank + l; thread i writes 16 columns.
           const int32_t col = t.n0 + (int32_t)rank * 128 + 16 * g;
-          if (n < t.m_valid && col < p.n_out) {
+          if (n < t.m_valid && col < p.n_out && MOE_DCHECK(p.status, t.row0 + n < p.S)) {
             const float4 q0 = *reinterpret_cast<const float4*>(row + 16 * g);
             const float4 q1 = *reinterpret_cast<const float4*>(row + 16 * g + 4);
             const float4 q2 = *reinterpret_cast<const float4*>(row + 16 * g + 8);
@@ -817,40 +863,53 @@ static bool encode_3d(CUtensorMap* m, const void* base, int64_t E, int64_t rows,
 
 template <int EPI, int BN>
 static cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& wa, const CUtensorMap& wb,
-                              const GemmParams& p, int num_sms, cudaStream_t s) {
+                              const GemmParams& p, int num_sms, cudaStream_t s, bool pdl) {
   using C = GemmCfg<EPI, BN>;
   cudaError_t err = cudaFuncSetAttribute(expert_gemm_kernel<EPI, BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  expert_gemm_kernel<EPI, BN><<<num_sms, kGemmThreads, C::SMEM_BYTES, s>>>(act, wa, wb, p);
-  return cudaGetLastError();
+  return launch_k(expert_gemm_kernel<EPI, BN>, dim3(num_sms), dim3(kGemmThreads), C::SMEM_BYTES, s, pdl, act, wa,
+                  wb, p);
 }
 
 template <int EPI, int CHUNKS>
 static cudaError_t launch_pair(const CUtensorMap& act, const CUtensorMap& wa, const CUtensorMap& wb,
-                               const GemmParams& p, int num_sms, cudaStream_t s) {
+                               const GemmParams& p, int num_sms, cudaStream_t s, bool pdl) {
   cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<EPI, CHUNKS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = kPairSmem;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   // As many pairs as can be resident at once (persistent kernel).
   cfg.gridDim = dim3((unsigned)(num_sms & ~1), 1, 1);
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, expert_gemm_pair_kernel<EPI, CHUNKS>, &cfg) == cudaSuccess &&
+  cudaLaunchConfig_t occ = cfg;
+  occ.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&clusters, expert_gemm_pair_kernel<EPI, CHUNKS>, &occ) == cudaSuccess &&
       clusters > 0 &&
       2 * clusters < (int)cfg.gridDim.x)
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
   return cudaLaunchKernelEx(&cfg, expert_gemm_pair_kernel<EPI, CHUNKS>, act, wa, wb, p);
+}
+
+// K chunks (16 KB of weights each) of its first tile that a streaming CTA
+// prefetches into L2 while the kernels before it finish: about 64 MB over all
+// CTAs, half of L2.
+static int32_t prefetch_chunks(int num_sms) {
+  const int64_t budget = 64ll << 20, chunk = 16 << 10;
+  const int64_t n = budget / ((int64_t)(num_sms > 0 ? num_sms : 1) * chunk);
+  return (int32_t)(n < 1 ? 1 : n);
 }
 
 void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
@@ -893,6 +952,7 @@ static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
   GemmParams p1{};
   p1.offsets = a.offsets;
   p1.status = a.status;
+  p1.S = a.S;
   p1.out = a.h;
   p1.out_ld = a.f;
   p1.part_stride = 0;
@@ -902,12 +962,14 @@ static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.n_blocks = a.f / 64;
   p1.splits = 1;
   p1.kb_per_split = p1.num_kb;
-  cudaError_t err = launch_one<EPI_STREAM_SWIGLU, BN>(mx, mw1, mw3, p1, a.num_sms, s);
+  p1.prefetch_kb = a.pdl ? prefetch_chunks(a.num_sms) : 0;
+  cudaError_t err = launch_one<EPI_STREAM_SWIGLU, BN>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl);
   if (err != cudaSuccess) return err;
   if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
   GemmParams p2{};
   p2.offsets = a.offsets;
   p2.status = a.status;
+  p2.S = a.S;
   p2.out = a.partials;
   p2.out_ld = a.d;
   p2.part_stride = a.S * (int64_t)a.d;
@@ -917,7 +979,9 @@ static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
   p2.n_blocks = (a.d + 127) / 128;
   p2.kb_per_split = (p2.num_kb + a.splits - 1) / a.splits;
   p2.splits = (p2.num_kb + p2.kb_per_split - 1) / p2.kb_per_split;
-  return launch_one<EPI_STREAM_PARTIAL, BN>(mh, mw2, mw2, p2, a.num_sms, s);
+  const bool pdl2 = a.pdl && !a.between;
+  p2.prefetch_kb = pdl2 ? prefetch_chunks(a.num_sms) : 0;
+  return launch_one<EPI_STREAM_PARTIAL, BN>(mh, mw2, mw2, p2, a.num_sms, s, pdl2);
 }
 
 static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
@@ -930,6 +994,7 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   GemmParams p1{};
   p1.offsets = a.offsets;
   p1.status = a.status;
+  p1.S = a.S;
   p1.out = a.h;
   p1.out_ld = a.f;
   p1.E = a.E;
@@ -940,13 +1005,14 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.kb_per_split = p1.num_kb;
   p1.tile_counter = a.tile_counters;
   // two 64-element K chunks per pipeline stage (3 stages): half the handshakes
-  cudaError_t err = a.pair ? launch_pair<EPI_TILED_SWIGLU, 2>(mx, mw1, mw3, p1, a.num_sms, s)
-                           : launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s);
+  cudaError_t err = a.pair ? launch_pair<EPI_TILED_SWIGLU, 2>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl)
+                           : launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl);
   if (err != cudaSuccess) return err;
   if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
   GemmParams p2{};
   p2.offsets = a.offsets;
   p2.status = a.status;
+  p2.S = a.S;
   p2.out = a.y_perm;
   p2.out_ld = a.d;
   p2.E = a.E;
@@ -956,8 +1022,9 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p2.splits = 1;
   p2.kb_per_split = p2.num_kb;
   p2.tile_counter = a.tile_counters + 1;
-  return a.pair ? launch_pair<EPI_TILED_STORE, 2>(mh, mw2, mw2, p2, a.num_sms, s)
-                : launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s);
+  const bool pdl2 = a.pdl && !a.between;
+  return a.pair ? launch_pair<EPI_TILED_STORE, 2>(mh, mw2, mw2, p2, a.num_sms, s, pdl2)
+                : launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s, pdl2);
 }
 
 cudaError_t launch_expert_gemms(const ExpertGemmArgs& a, cudaStream_t s) {

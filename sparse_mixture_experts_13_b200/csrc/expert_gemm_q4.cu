@@ -96,6 +96,7 @@ struct Q4Params {
   int32_t n_blocks;     // weight blocks per expert (64 rows of W1 and W3, or 128 of W2)
   int32_t splits;
   int32_t kq_per_split;
+  int64_t S;            // rows of the activation and output buffers (T * k)
 };
 
 struct Q4Tile {
@@ -210,12 +211,24 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
     tmem_alloc(&s_tmem, kTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();     // offsets and activations of the kernels before this one
+  pdl_trigger();  // the next kernel may start its own set-up
   if (tid == 64) {
     s_abort = 0;
     s_epi_fail = 0;
     int32_t acc = 0;
     s_base[0] = 0;
     for (int e = 0; e <= p.E; ++e) s_off[e] = p.offsets[e];
+#ifdef MOE_DEBUG
+    {  // offsets must start at 0, not decrease and stay within the S rows
+      bool bad = s_off[0] != 0 || (int64_t)s_off[p.E] > p.S;
+      for (int e = 0; e < p.E; ++e) bad = bad || s_off[e + 1] < s_off[e];
+      if (bad) {
+        record_status(p.status, kStatusBounds);
+        for (int e = 0; e <= p.E; ++e) s_off[e] = 0;
+      }
+    }
+#endif
     for (int e = 0; e < p.E; ++e) {
       const int32_t M_e = s_off[e + 1] - s_off[e];
       acc += M_e > 0 ? ((M_e + BN - 1) / BN) * p.n_blocks * p.splits : 0;
@@ -435,7 +448,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int tok = c0 + j;
-              if (tok < t.m_valid) {
+              if (tok < t.m_valid && MOE_DCHECK(p.status, t.row0 + tok < p.S)) {
                 const float hv = silu_f32(__uint_as_float(v[j])) * xbuf[j * 64 + r];
                 out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] = (uint16_t)(pack_bf16x2(hv, 0.f) & 0xFFFFu);
               }
@@ -455,7 +468,8 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int tok = c0 + j;
-              if (tok < t.m_valid) out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] = __uint_as_float(v[j]);
+              if (tok < t.m_valid && MOE_DCHECK(p.status, t.row0 + tok < p.S))
+                out[(int64_t)(t.row0 + tok) * p.out_ld + t.n0 + r] = __uint_as_float(v[j]);
             }
           }
         }
@@ -561,13 +575,13 @@ bool encode_tokens(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
 template <int EPI, int BN>
 cudaError_t launch_q4_one(const CUtensorMap& act, const CUtensorMap& ca, const CUtensorMap& cb,
                           const CUtensorMap& sa, const CUtensorMap& sb, const Q4Params& p, int num_sms,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool pdl) {
   using C = Q4Cfg<EPI, BN>;
   cudaError_t err =
       cudaFuncSetAttribute(expert_gemm_q4_kernel<EPI, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  expert_gemm_q4_kernel<EPI, BN><<<num_sms, kQ4Threads, C::SMEM_BYTES, s>>>(act, ca, cb, sa, sb, p);
-  return cudaGetLastError();
+  return launch_k(expert_gemm_q4_kernel<EPI, BN>, dim3(num_sms), dim3(kQ4Threads), C::SMEM_BYTES, s, pdl, act, ca,
+                  cb, sa, sb, p);
 }
 
 template <int BN>
@@ -581,6 +595,7 @@ cudaError_t launch_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
   Q4Params p1{};
   p1.offsets = a.offsets;
   p1.status = a.status;
+  p1.S = a.S;
   p1.out = a.h;
   p1.out_ld = a.f;
   p1.E = a.E;
@@ -589,12 +604,13 @@ cudaError_t launch_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
   p1.n_blocks = a.f / 64;
   p1.splits = 1;
   p1.kq_per_split = p1.num_kq;
-  cudaError_t err = launch_q4_one<Q4_SWIGLU, BN>(mx, mc1, mc3, ms1, ms3, p1, a.num_sms, s);
+  cudaError_t err = launch_q4_one<Q4_SWIGLU, BN>(mx, mc1, mc3, ms1, ms3, p1, a.num_sms, s, a.pdl);
   if (err != cudaSuccess) return err;
   if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
   Q4Params p2{};
   p2.offsets = a.offsets;
   p2.status = a.status;
+  p2.S = a.S;
   p2.out = a.partials;
   p2.out_ld = a.d;
   p2.part_stride = a.S * (int64_t)a.d;
@@ -604,7 +620,7 @@ cudaError_t launch_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
   p2.n_blocks = (a.d + 127) / 128;
   p2.kq_per_split = (p2.num_kq + a.splits - 1) / a.splits;
   p2.splits = (p2.num_kq + p2.kq_per_split - 1) / p2.kq_per_split;
-  return launch_q4_one<Q4_PARTIAL, BN>(mh, mc2, mc2, ms2, ms2, p2, a.num_sms, s);
+  return launch_q4_one<Q4_PARTIAL, BN>(mh, mc2, mc2, ms2, ms2, p2, a.num_sms, s, a.pdl && !a.between);
 }
 
 }  // namespace

@@ -4,6 +4,7 @@
 // (except moe_read_device_status).
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "moe.h"
@@ -17,6 +18,16 @@ namespace {
 // workspace size is a function of the shape alone; grids use the real count.
 constexpr int kPlanSms = 148;
 constexpr size_t kAlign = 256;
+#ifdef MOE_DEBUG
+constexpr bool kDebugBuild = true;
+#else
+constexpr bool kDebugBuild = false;
+#endif
+constexpr size_t kGuard = 256;        // debug build: guard bytes after each region past the control region
+constexpr int kMaxGuards = 32;
+#ifdef MOE_DEBUG
+constexpr unsigned char kGuardByte = 0xA5;
+#endif
 
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
@@ -65,7 +76,20 @@ struct Layout {
   bool q4;                 // 4-bit expert weights (always the streaming schedule)
   int32_t bn, splits;      // streaming schedule: token tile, requested split-K count
   int32_t eff_splits;      // split-K partial buffers the down projection writes
+  size_t guards[kMaxGuards];  // debug build: offsets of the guards
+  int nguards;
 };
+
+// End of a region that ends at `end`: the next 256-byte boundary, followed
+// in debug builds by a guard.
+size_t next_region(Layout& L, size_t end) {
+  size_t o = align_up(end);
+  if (kDebugBuild && L.nguards < kMaxGuards) {
+    L.guards[L.nguards++] = o;
+    o += kGuard;
+  }
+  return o;
+}
 
 // q4: layout of the 4-bit entry points (split-K partials always present).
 Layout layout_of(const moe_shape* sh, bool q4 = false) {
@@ -101,46 +125,46 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
   o = align_up(o + 4 * (size_t)permute_tiles(S) * E);
   L.ctrl_end = o;
   L.thresh = o;
-  o = align_up(o + 8 * E);
+  o = next_region(L, o + 8 * E);
   L.partials = o;
-  if (L.variant == MOE_VARIANT_STREAM) o = align_up(o + 4 * (size_t)L.eff_splits * S * d);
+  if (L.variant == MOE_VARIANT_STREAM) o = next_region(L, o + 4 * (size_t)L.eff_splits * S * d);
   L.topk_idx = o;
-  o = align_up(o + 4 * S);
+  o = next_region(L, o + 4 * S);
   L.topk_w = o;
-  o = align_up(o + 4 * S);
+  o = next_region(L, o + 4 * S);
   L.topk_p = o;
-  o = align_up(o + 4 * S);
+  o = next_region(L, o + 4 * S);
   L.offsets = o;
-  o = align_up(o + 4 * (E + 1));
+  o = next_region(L, o + 4 * (E + 1));
   L.slot_pos = o;
-  o = align_up(o + 4 * S);
+  o = next_region(L, o + 4 * S);
   L.perm_slot = o;
-  o = align_up(o + 4 * S);
+  o = next_region(L, o + 4 * S);
   L.x_perm = o;
-  o = align_up(o + 2 * (size_t)S * d);
+  o = next_region(L, o + 2 * (size_t)S * d);
   L.h = o;
-  o = align_up(o + 2 * (size_t)S * f);
+  o = next_region(L, o + 2 * (size_t)S * f);
   L.y_perm = o;
-  o = align_up(o + 2 * (size_t)S * d);
+  o = next_region(L, o + 2 * (size_t)S * d);
   L.x_stage = o;
-  o = align_up(o + 2 * (size_t)T * d);
+  o = next_region(L, o + 2 * (size_t)T * d);
   L.y_stage = o;
-  o = align_up(o + 2 * (size_t)T * d);
+  o = next_region(L, o + 2 * (size_t)T * d);
   if (L.fallback) {
     L.next_idx = o;
-    o = align_up(o + 4 * S);
+    o = next_region(L, o + 4 * S);
     L.next_p = o;
-    o = align_up(o + 4 * S);
+    o = next_region(L, o + 4 * S);
     L.keys1 = o;
-    o = align_up(o + 8 * S);
+    o = next_region(L, o + 8 * S);
     L.keys2 = o;
-    o = align_up(o + 8 * S);
+    o = next_region(L, o + 8 * S);
     L.cand = o;
-    o = align_up(o + 4 * S);
+    o = next_region(L, o + 4 * S);
     L.eff = o;
-    o = align_up(o + 4 * S);
+    o = next_region(L, o + 4 * S);
     L.thresh2 = o;
-    o = align_up(o + 8 * E);
+    o = next_region(L, o + 8 * E);
   }
   L.total = o;
   return L;
@@ -153,7 +177,6 @@ moe_status check_ws(const moe_shape* sh, const void* ws, size_t ws_bytes, bool q
 }
 
 // Device checks, cached per device: sm_100 family and SM count.
-constexpr int kMaxDevices = 64;
 int g_dev_state[kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
 int g_dev_sms[kMaxDevices];
 
@@ -192,15 +215,16 @@ moe_status check_i32(const void* p) { return (p && aligned(p, 4)) ? MOE_OK : MOE
 
 moe_status run_router(const moe_shape* sh, const moe_bf16* x, const float* Wg, float* logits, int32_t* idx, float* w,
                       float* p, int32_t* counts, int num_sms, cudaStream_t s, bool counts_zeroed,
-                      int32_t* next_idx = nullptr, float* next_p = nullptr) {
-  RouterArgs a{x, Wg, logits, idx, w, p, counts, next_idx, next_p, sh->T, sh->d_model, sh->E, sh->k};
+                      int32_t* next_idx = nullptr, float* next_p = nullptr, uint32_t* status = nullptr) {
+  RouterArgs a{x, Wg, logits, idx, w, p, counts, next_idx, next_p, sh->T, sh->d_model, sh->E, sh->k, status};
   return cuda_status(launch_router(a, num_sms, s, counts_zeroed));
 }
 
 moe_status run_permute(const moe_shape* sh, const Layout& L, const moe_bf16* x, const int32_t* idx, const float* p,
                        const int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_slot,
-                       moe_bf16* x_perm, void* ws, cudaStream_t s, bool state_zeroed) {
+                       moe_bf16* x_perm, void* ws, cudaStream_t s, bool state_zeroed, bool pdl = false) {
   PermuteArgs a{};
+  a.pdl = pdl;
   a.x = x;
   a.topk_idx = idx;
   a.topk_p = p;
@@ -224,8 +248,9 @@ moe_status run_permute(const moe_shape* sh, const Layout& L, const moe_bf16* x, 
 
 moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_perm, const int32_t* offsets,
                      const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2, moe_bf16* h, moe_bf16* y_perm,
-                     void* ws, int num_sms, cudaStream_t s, cudaEvent_t between = nullptr) {
+                     void* ws, int num_sms, cudaStream_t s, cudaEvent_t between = nullptr, bool pdl = false) {
   ExpertGemmArgs a{};
+  a.pdl = pdl;
   a.offsets = offsets;
   a.x_perm = x_perm;
   a.W1 = W1;
@@ -258,8 +283,9 @@ struct ExpertWeights {
 
 moe_status run_gemms_q4(const moe_shape* sh, const Layout& L, const moe_bf16* x_perm, const int32_t* offsets,
                         const ExpertWeights& W, moe_bf16* h, void* ws, int num_sms, cudaStream_t s,
-                        cudaEvent_t between = nullptr) {
+                        cudaEvent_t between = nullptr, bool pdl = false) {
   ExpertGemmQ4Args a{};
+  a.pdl = pdl;
   a.offsets = offsets;
   a.x_perm = x_perm;
   a.W1c = W.W1c;
@@ -367,7 +393,8 @@ moe_status moe_grouped_swiglu(const moe_shape* sh, const moe_bf16* x_perm, const
   if (L.variant == MOE_VARIANT_STREAM) {
     const int64_t S = sh->T * sh->k;
     MOE_TRY(cuda_status(launch_splitk_reduce(at<float>(ws, L.partials), L.eff_splits, S * (int64_t)sh->d_model,
-                                             offsets, sh->E, y_perm, S, sh->d_model, sms, s)));
+                                             offsets, sh->E, y_perm, S, sh->d_model, sms, s,
+                                             at<uint32_t>(ws, L.status))));
   }
   return MOE_OK;
 }
@@ -393,6 +420,19 @@ moe_status moe_combine(const moe_shape* sh, const moe_bf16* y_perm, const int32_
   return cuda_status(launch_combine(a, sms, (cudaStream_t)stream));
 }
 
+// Debug build: MOE_DEBUG_FAIL_STAGE=n makes the layer entry points fail with
+// MOE_ERR_CUDA just before queuing stage n (1 router, 2 capacity / grouping,
+// 3 expert GEMMs, 4 combine, 5 output copies).
+static int debug_fail_stage() {
+  if (!kDebugBuild) return 0;
+  const char* v = std::getenv("MOE_DEBUG_FAIL_STAGE");
+  return v ? std::atoi(v) : 0;
+}
+#define MOE_STAGE(n)                                     \
+  do {                                                   \
+    if (fail_at == (n)) return MOE_ERR_CUDA;             \
+  } while (0)
+
 static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, const float* Wg, const ExpertWeights& W,
                                      bool q4, moe_bf16* y, int32_t* topk_idx_out, int32_t* counts_out, void* ws,
                                      int sms, cudaStream_t s, cudaEvent_t const* ev = nullptr) {
@@ -409,13 +449,20 @@ static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, con
   moe_bf16* h = at<moe_bf16>(ws, L.h);
   moe_bf16* y_perm = at<moe_bf16>(ws, L.y_perm);
   auto mark = [&](int i) { return ev ? cuda_status(cudaEventRecord(ev[i], s)) : MOE_OK; };
+  // Without events between them, each kernel after the router is launched
+  // as a programmatic dependent of the one before (its set-up overlaps that
+  // kernel; it waits for it before reading its output).
+  const bool pdl = ev == nullptr;
+  const int fail_at = debug_fail_stage();
   MOE_TRY(mark(0));
   MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.ctrl_end, s)));
   // one clear of the control region (status, ticket, counts, look-back words)
+  MOE_STAGE(1);
   if (L.fallback) {
     MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s, true, at<int32_t>(ws, L.next_idx),
-                       at<float>(ws, L.next_p)));
+                       at<float>(ws, L.next_p), at<uint32_t>(ws, L.status)));
     MOE_TRY(mark(1));
+    MOE_STAGE(2);
     FallbackArgs fa{};
     fa.topk_idx = idx;
     fa.topk_p = p;
@@ -442,19 +489,25 @@ static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, con
     dropless.capacity_factor = 0.f;
     dropless.drop_policy = MOE_DROP_BY_PROB;
     MOE_TRY(run_permute(&dropless, L, x, fa.eff, p, fa.counts_eff, offsets, slot_pos, perm_slot, x_perm, ws, s,
-                        true));
+                        true, pdl));
   } else {
-    MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s, true));
+    MOE_TRY(run_router(sh, x, Wg, nullptr, idx, w, p, counts, sms, s, true, nullptr, nullptr,
+                       at<uint32_t>(ws, L.status)));
     MOE_TRY(mark(1));
-    MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s, true));
+    MOE_STAGE(2);
+    MOE_TRY(run_permute(sh, L, x, idx, p, counts, offsets, slot_pos, perm_slot, x_perm, ws, s, true, pdl));
   }
   MOE_TRY(mark(2));
+  MOE_STAGE(3);
   if (q4)
-    MOE_TRY(run_gemms_q4(sh, L, x_perm, offsets, W, h, ws, sms, s, ev ? ev[3] : nullptr));
+    MOE_TRY(run_gemms_q4(sh, L, x_perm, offsets, W, h, ws, sms, s, ev ? ev[3] : nullptr, pdl));
   else
-    MOE_TRY(run_gemms(sh, L, x_perm, offsets, W.W1, W.W3, W.W2, h, y_perm, ws, sms, s, ev ? ev[3] : nullptr));
+    MOE_TRY(run_gemms(sh, L, x_perm, offsets, W.W1, W.W3, W.W2, h, y_perm, ws, sms, s, ev ? ev[3] : nullptr, pdl));
   MOE_TRY(mark(4));
+  MOE_STAGE(4);
   CombineArgs c{};
+  c.pdl = pdl;
+  c.status = at<uint32_t>(ws, L.status);
   c.slot_pos = slot_pos;
   c.topk_w = w;
   c.y = y;
@@ -471,6 +524,7 @@ static moe_status layer_forward_impl(const moe_shape* sh, const moe_bf16* x, con
   }
   MOE_TRY(cuda_status(launch_combine(c, sms, s)));
   MOE_TRY(mark(5));
+  MOE_STAGE(5);
   if (topk_idx_out)
     MOE_TRY(cuda_status(cudaMemcpyAsync(topk_idx_out, idx, sizeof(int32_t) * S, cudaMemcpyDeviceToDevice, s)));
   if (counts_out)
@@ -651,7 +705,7 @@ moe_status moe_grouped_swiglu_q4(const moe_shape* sh, const moe_bf16* x_perm, co
   MOE_TRY(run_gemms_q4(sh, L, x_perm, offsets, Wt, h, ws, sms, s));
   const int64_t S = sh->T * sh->k;
   return cuda_status(launch_splitk_reduce(at<float>(ws, L.partials), L.eff_splits, S * (int64_t)sh->d_model, offsets,
-                                          sh->E, y_perm, S, sh->d_model, sms, s));
+                                          sh->E, y_perm, S, sh->d_model, sms, s, at<uint32_t>(ws, L.status)));
 }
 
 static moe_status check_layer_q4(const moe_shape* sh, const moe_bf16* x, const float* Wg, const ExpertWeights& W,
@@ -678,6 +732,29 @@ moe_status moe_layer_forward_q4(const moe_shape* sh, const moe_bf16* x, const fl
   return layer_forward_impl(sh, x, Wg, Wt, true, y, topk_idx_out, counts_out, ws, sms, (cudaStream_t)stream);
 }
 
+moe_status moe_layer_forward_q4_host(const moe_shape* sh, const moe_bf16* x_host, const float* Wg, const uint8_t* W1c,
+                                     const moe_bf16* W1s, const uint8_t* W3c, const moe_bf16* W3s, const uint8_t* W2c,
+                                     const moe_bf16* W2s, moe_bf16* y_host, void* ws, size_t ws_bytes,
+                                     moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (sh->T == 0) return MOE_OK;
+  if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  const ExpertWeights Wt{nullptr, nullptr, nullptr, W1c, W3c, W2c, W1s, W3s, W2s};
+  MOE_TRY(check_bf16(Wg));
+  MOE_TRY(check_q4_weights(Wt));
+  MOE_TRY(check_ws(sh, ws, ws_bytes, true));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  const Layout L = layout_of(sh, true);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t bytes = 2 * (size_t)sh->T * sh->d_model;
+  moe_bf16* xd = at<moe_bf16>(ws, L.x_stage);
+  moe_bf16* yd = at<moe_bf16>(ws, L.y_stage);
+  MOE_TRY(cuda_status(cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s)));
+  MOE_TRY(layer_forward_impl(sh, xd, Wg, Wt, true, yd, nullptr, nullptr, ws, sms, s));
+  return cuda_status(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s));
+}
+
 moe_status moe_layer_forward_q4_profiled(const moe_shape* sh, const moe_bf16* x, const float* Wg, const uint8_t* W1c,
                                          const moe_bf16* W1s, const uint8_t* W3c, const moe_bf16* W3s,
                                          const uint8_t* W2c, const moe_bf16* W2s, moe_bf16* y, void* const* events,
@@ -702,6 +779,43 @@ moe_status moe_read_device_status(const void* ws, moe_stream_t stream) {
   return v == 0 ? MOE_OK : (moe_status)v;
 }
 
+int32_t moe_debug_build(void) { return kDebugBuild ? 1 : 0; }
+
+moe_status moe_debug_workspace_arm(const moe_shape* sh, void* ws, size_t ws_bytes, int32_t q4, moe_stream_t stream) {
+#ifndef MOE_DEBUG
+  (void)sh, (void)ws, (void)ws_bytes, (void)q4, (void)stream;
+  return MOE_ERR_UNSUPPORTED;
+#else
+  MOE_TRY(check_shape(sh));
+  MOE_TRY(check_ws(sh, ws, ws_bytes, q4 != 0));
+  const Layout L = layout_of(sh, q4 != 0);
+  for (int i = 0; i < L.nguards; ++i)
+    MOE_TRY(cuda_status(cudaMemsetAsync(at<uint8_t>(ws, L.guards[i]), kGuardByte, kGuard, (cudaStream_t)stream)));
+  return MOE_OK;
+#endif
+}
+
+moe_status moe_debug_workspace_check(const moe_shape* sh, const void* ws, size_t ws_bytes, int32_t q4,
+                                     moe_stream_t stream) {
+#ifndef MOE_DEBUG
+  (void)sh, (void)ws, (void)ws_bytes, (void)q4, (void)stream;
+  return MOE_ERR_UNSUPPORTED;
+#else
+  MOE_TRY(check_shape(sh));
+  MOE_TRY(check_ws(sh, ws, ws_bytes, q4 != 0));
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const Layout L = layout_of(sh, q4 != 0);
+  unsigned char buf[kGuard];
+  for (int i = 0; i < L.nguards; ++i) {
+    if (cudaMemcpy(buf, static_cast<const uint8_t*>(ws) + L.guards[i], kGuard, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    for (size_t j = 0; j < kGuard; ++j)
+      if (buf[j] != kGuardByte) return MOE_ERR_WORKSPACE;
+  }
+  return MOE_OK;
+#endif
+}
+
 const char* moe_status_string(moe_status st) {
   switch (st) {
     case MOE_OK: return "ok";
@@ -710,6 +824,7 @@ const char* moe_status_string(moe_status st) {
     case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_BOUNDS: return "device-side bounds check failed (debug build)";
   }
   return "unknown status";
 }

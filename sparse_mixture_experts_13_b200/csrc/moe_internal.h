@@ -10,6 +10,33 @@
 
 namespace moe {
 
+// Launch `kernel` on `s`; with pdl, as a programmatic dependent of the kernel
+// queued before it (it may start while that kernel runs and must call
+// griddepcontrol.wait before reading that kernel's output).  Only used when
+// the previous operation in the stream is one of this library's kernels.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                     Args&&... args) {
+  if (!pdl) {
+    kernel<<<grid, block, smem, s>>>(static_cast<KArgs>(args)...);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Devices with a per-device cache entry (device checks, scratch addresses).
+constexpr int kMaxDevices = 64;
+
 // Argument checks shared by the C entry points (defined in moe_api.cu).
 moe_status api_check_shape(const moe_shape* sh);
 moe_status api_check_device(int* num_sms);
@@ -27,6 +54,7 @@ struct RouterArgs {
   float* next_p;       // [T, k] their full-softmax probabilities
   int64_t T;
   int32_t d, E, k;
+  uint32_t* status;    // device status word (a wait that gives up), or nullptr
 };
 cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s, bool counts_zeroed);
 
@@ -47,6 +75,7 @@ struct PermuteArgs {
   int32_t d, E, k;
   int64_t cap;               // < 0: dropless
   int32_t policy;            // 0 by probability, 1 by token order
+  bool pdl;                  // launched as dependents of the router's kernel
 };
 constexpr int kPermuteTile = 64;  // slots per permutation tile
 int64_t permute_tiles(int64_t S);
@@ -73,6 +102,7 @@ struct ExpertGemmArgs {
   cudaEvent_t between;      // recorded after the first GEMM if not null
   bool pair;                // tiled variant: CTA-pair (cta_group::2) kernels
   uint32_t* tile_counters;  // [2] tile counters of the pair kernels, zeroed by the caller
+  bool pdl;                 // launched as dependents of the grouping kernel (no event in between)
 };
 // Streaming-variant parameters chosen from host-known sizes.
 void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,
@@ -100,6 +130,7 @@ struct ExpertGemmQ4Args {
   int32_t splits;           // requested split-K count of the down projection
   int num_sms;
   cudaEvent_t between;      // recorded after the first GEMM if not null
+  bool pdl;                 // launched as dependents of the grouping kernel (no event in between)
 };
 void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits);
 // number of K splits the down projection really uses for a requested count
@@ -160,13 +191,15 @@ struct CombineArgs {
   uint16_t* y;              // [T, d]
   int64_t T;
   int32_t d, k;
+  bool pdl;                 // launched as a dependent of the down-projection GEMM
+  uint32_t* status;         // device status word (debug bounds checks), or nullptr
 };
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
 
 // y_perm[r] = bf16(sum_s partials[s][r]) for r < offsets[E].
 cudaError_t launch_splitk_reduce(const float* partials, int32_t splits, int64_t part_stride,
                                  const int32_t* offsets, int32_t E, uint16_t* y_perm, int64_t S,
-                                 int32_t d, int num_sms, cudaStream_t s);
+                                 int32_t d, int num_sms, cudaStream_t s, uint32_t* status);
 
 // Driver entry point for tensor-map encoding (resolved once through the runtime).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -49,6 +49,8 @@ __global__ void __launch_bounds__(kSelectThreads) capacity_select_kernel(const i
                                                                          const int32_t* __restrict__ counts,
                                                                          uint64_t* __restrict__ thresh,
                                                                          int64_t S, int32_t k, int64_t cap) {
+  pdl_trigger();
+  pdl_wait();  // the router's outputs
   const int e = blockIdx.x;
   const int64_t cnt = counts[e];
   if (cnt <= cap) {
@@ -79,6 +81,10 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
   __shared__ int32_t s_row[kPermuteTile];
   __shared__ int32_t s_tok[kPermuteTile];
 
+  // The expert GEMM that follows may launch at once: before its own wait it
+  // only prefetches weights.
+  pdl_trigger();
+  pdl_wait();  // the router's (or capacity selection's) outputs
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E, k = a.k;
   const int64_t S = a.T * k;
@@ -106,7 +112,7 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
   bool elig = false;
   if (ranker && s < S) {
     e = a.topk_idx[s];
-    elig = e >= 0;  // a negative expert marks a slot dropped before grouping
+    elig = e >= 0 && MOE_DCHECK(a.status, e < E);  // a negative expert marks a slot dropped before grouping
     if (elig && a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
   }
   int rank_w = 0;
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(PermuteArgs a)
     if (elig) {
       const int32_t rank = s_excl[e] + s_wpre[warp][e] + rank_w;
       const bool kept = !(a.cap >= 0 && a.policy == 1 && rank >= a.cap);
-      if (kept) {
+      if (kept && MOE_DCHECK(a.status, s_off[e] + rank < s_off[e + 1] && s_off[e] + rank < S)) {
         row = s_off[e] + rank;
         a.perm_slot[row] = (int32_t)s;
         const int q = atomicAdd(&s_nkept, 1);
@@ -199,6 +205,8 @@ __global__ void __launch_bounds__(256) permute_small_kernel(PermuteArgs a) {
   __shared__ int32_t s_run[32];
   __shared__ int32_t s_row[kSmallSlots];   // row of slot s, or -1
   __shared__ int32_t s_list[kSmallSlots];  // kept slots in row order
+  pdl_trigger();
+  pdl_wait();  // the router's (or capacity selection's) outputs
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E, k = a.k;
   const int S = (int)(a.T * k);
@@ -221,7 +229,7 @@ __global__ void __launch_bounds__(256) permute_small_kernel(PermuteArgs a) {
       bool elig = false;
       if (s < S) {
         e = a.topk_idx[s];
-        elig = e >= 0;  // a negative expert marks a slot dropped before grouping
+        elig = e >= 0 && MOE_DCHECK(a.status, e < E);  // a negative expert marks a slot dropped before grouping
         if (elig && a.cap >= 0 && a.policy == 0) elig = slot_key(a.topk_p[s], s / k) >= a.thresh[e];
       }
       const uint32_t peers = __match_any_sync(0xffffffffu, elig ? e : -1);
@@ -229,7 +237,9 @@ __global__ void __launch_bounds__(256) permute_small_kernel(PermuteArgs a) {
       int32_t row = -1;
       if (elig) {
         const int32_t rank = s_run[e] + before;
-        if (!(a.cap >= 0 && a.policy == 1 && rank >= a.cap)) row = s_off[e] + rank;
+        if (!(a.cap >= 0 && a.policy == 1 && rank >= a.cap) &&
+            MOE_DCHECK(a.status, s_off[e] + rank < s_off[e + 1] && s_off[e] + rank < S))
+          row = s_off[e] + rank;
       }
       __syncwarp();
       if (elig && before == 0) s_run[e] += __popc(peers);
@@ -278,18 +288,15 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zero
   if (a.cap >= 0 && a.policy == 0) {
     err = cudaFuncSetAttribute(capacity_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
     if (err != cudaSuccess) return err;
-    capacity_select_kernel<<<a.E, kSelectThreads, kSelectSmem, s>>>(a.topk_idx, a.topk_p, a.counts, a.thresh, S,
-                                                                    a.k, a.cap);
-    err = cudaGetLastError();
+    err = launch_k(capacity_select_kernel, dim3(a.E), dim3(kSelectThreads), kSelectSmem, s, a.pdl, a.topk_idx,
+                   a.topk_p, a.counts, a.thresh, S, a.k, a.cap);
     if (err != cudaSuccess) return err;
   }
   if (S <= kSmallSlots) {
     const int blocks = (int)(S < kSmallBlocks ? S : kSmallBlocks);
-    permute_small_kernel<<<blocks, 256, 0, s>>>(a);
-  } else {
-    permute_kernel<<<(unsigned)tiles, kPermuteThreads, 0, s>>>(a);
+    return launch_k(permute_small_kernel, dim3(blocks), dim3(256), 0, s, a.pdl, a);
   }
-  return cudaGetLastError();
+  return launch_k(permute_kernel, dim3((unsigned)tiles), dim3(kPermuteThreads), 0, s, a.pdl, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -305,8 +312,7 @@ constexpr size_t kNoAllocBytes = kNoAllocHeader + sizeof(uint32_t) * (kNoAllocMa
 static __device__ __align__(256) unsigned char g_permute_scratch[kNoAllocBytes];
 
 namespace {
-constexpr int kNoAllocMaxDevices = 64;
-void* g_scratch_addr[kNoAllocMaxDevices];  // device address per device, once looked up
+void* g_scratch_addr[kMaxDevices];  // device address per device, once looked up
 }  // namespace
 
 }  // namespace moe
@@ -332,7 +338,8 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* sh, const moe_bf16* x
   st = api_check_device(&sms);
   if (st != MOE_OK) return st;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;  // as api_check_device
   if (!g_scratch_addr[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_permute_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
@@ -364,4 +371,16 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* sh, const moe_bf16* x
   a.cap = cap;
   a.policy = sh->drop_policy;
   return launch_permute(a, s, true) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" moe_status moe_permute_noalloc_status(moe_stream_t stream) {
+  using namespace moe;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!g_scratch_addr[dev]) return MOE_OK;  // no call on this device yet
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, g_scratch_addr[dev], sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  return v == 0 ? MOE_OK : (moe_status)v;
 }

@@ -5,14 +5,27 @@
 // "Mixtral", section "MoE Layer" (bias-free nn.Linear router, topk of the
 // logits, softmax over the k kept logits).
 //
-// Logits are fp32 dot products of a token's bf16 row with the E rows of W_g,
-// read as 16-byte vectors.  A block takes a group of tokens (one token when
-// there are few, so that many SMs share the work) and splits d over its warps;
-// every W_g vector a warp reads serves all tokens of the group.  The top-k
-// (ties to the smaller expert index), the k-way softmax and the full-softmax
-// probability of each chosen expert are computed redundantly per lane and
-// lanes 0..k-1 write one slot each.  The per-expert histogram is aggregated in
-// shared memory and added to global memory once per block.
+// Logits are fp32 dot products of a token's bf16 row with the E rows of W_g.
+// Two kernels compute them:
+//
+// router_reg_kernel (E <= 8, d <= 4096, the Mixtral shape): a persistent
+//   block of d/8 threads holds all of W_g in registers, thread i owning inputs
+//   [8i, 8i+8) of every expert row, so W_g is read once per block instead of
+//   once per token.  Token rows stream through a ring of shared-memory slots
+//   filled by bulk copies (one copy per group of TB consecutive rows), so many
+//   rows are in flight per SM without costing registers.  Each thread forms
+//   its 8 partial logits of a token, a warp reduce-scatter leaves one expert's
+//   warp sum on every fourth lane, and the warp sums are added across warps in
+//   shared memory in warp order.
+// router_group_kernel (any other shape): a block takes a group of tokens and
+//   splits d over its warps; every W_g vector a warp reads (from L2) serves
+//   all tokens of the group.
+//
+// In both, the top-k (ties to the smaller expert index), the k-way softmax
+// and the full-softmax probability of each chosen expert are computed
+// redundantly per lane of one warp and lanes 0..k-1 write one slot each.  The
+// per-expert histogram is aggregated in shared memory and added to global
+// memory once per block.
 #include <cfloat>
 #include <cstdint>
 
@@ -20,8 +33,6 @@
 #include "sm100.cuh"
 
 namespace moe {
-
-constexpr int kMaxK = 8;
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -32,80 +43,50 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
-// All lanes hold all E logits of token t.  Top-k by repeated arg-max over
-// the experts not yet chosen (strict '>' keeps the smaller index on equal
-// logits); softmax over the k kept logits; full softmax over all E at the
-// chosen experts.  Lane j < k writes slot j and counts it in *hist.
+// Lane e < E holds the logit l of expert e for token t (other lanes: any
+// value).  Every lane ranks its expert in the order (logit descending, index
+// ascending), so the experts of rank < k are the top-k, rank 0 first, and
+// ranks k .. 2k-1 are the next-best candidates.  With m the largest logit,
+// the gate of a chosen expert is exp(l - m) over the sum of exp(l' - m) of the
+// k chosen ones, and its full-softmax probability is exp(l - m) over the sum
+// across all E experts.  The sums are butterflies over the first EMAX lanes
+// (a fixed order).  Lane e writes the slot of its rank and counts it in *hist.
 template <int EMAX>
-__device__ __forceinline__ void finish_token(const RouterArgs& a, int64_t t, const float (&acc)[EMAX], int lane,
-                                             int* hist) {
+__device__ __forceinline__ void finish_token(const RouterArgs& a, int64_t t, float l, int lane, int* hist) {
   const int E = a.E, k = a.k;
-  int sel[kMaxK];
-  float sl[kMaxK];
-  uint32_t chosen = 0;
+  const bool valid = lane < E;
+  int rank = 0;
 #pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    sel[j] = 0;
-    sl[j] = 0.f;
-    if (j < k) {
-      int best = -1;
-      float bl = -FLT_MAX;
-#pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-        if (e < E && !((chosen >> e) & 1u) && (best < 0 || acc[e] > bl)) {
-          best = e;
-          bl = acc[e];
-        }
-      }
-      sel[j] = best;
-      sl[j] = bl;
-      chosen |= 1u << best;
-    }
+  for (int e = 0; e < EMAX; ++e) {
+    const float le = __shfl_sync(0xffffffffu, l, e);
+    if (e < E && (le > l || (le == l && e < lane))) ++rank;
   }
-  const float m = sl[0];
-  float zk = 0.f;
+  float m = valid ? l : -FLT_MAX;
 #pragma unroll
-  for (int j = 0; j < kMaxK; ++j)
-    if (j < k) zk += expf(sl[j] - m);
-  float zE = 0.f;
+  for (int off = EMAX / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const float ex = valid ? expf(l - m) : 0.f;
+  float zE = ex, zk = (valid && rank < k) ? ex : 0.f;
 #pragma unroll
-  for (int e = 0; e < EMAX; ++e)
-    if (e < E) zE += expf(acc[e] - m);
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    if (j < k && lane == j) {
-      const float ej = expf(sl[j] - m);
-      a.topk_idx[t * k + j] = sel[j];
-      a.topk_w[t * k + j] = ej / zk;
-      a.topk_p[t * k + j] = ej / zE;
-      atomicAdd(&hist[sel[j]], 1);
-    }
+  for (int off = EMAX / 2; off > 0; off >>= 1) {
+    zE += __shfl_xor_sync(0xffffffffu, zE, off);
+    zk += __shfl_xor_sync(0xffffffffu, zk, off);
   }
-  if (a.logits) {
-#pragma unroll
-    for (int e = 0; e < EMAX; ++e)
-      if (e < E && lane == e) a.logits[t * E + e] = acc[e];
+  if (valid && rank < k) {
+    a.topk_idx[t * k + rank] = lane;
+    a.topk_w[t * k + rank] = ex / zk;
+    a.topk_p[t * k + rank] = ex / zE;
+    atomicAdd(&hist[lane], 1);
   }
+  if (a.logits && valid) a.logits[t * E + lane] = l;
   if (a.next_idx) {
-    // ranks k .. 2k-1 (capacity fallback): continue the same arg-max order
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (j < k) {
-        int best = -1;
-        float bl = -FLT_MAX;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-          if (e < E && !((chosen >> e) & 1u) && (best < 0 || acc[e] > bl)) {
-            best = e;
-            bl = acc[e];
-          }
-        }
-        if (best >= 0) chosen |= 1u << best;
-        if (lane == j) {
-          a.next_idx[t * k + j] = best;
-          a.next_p[t * k + j] = best >= 0 ? expf(bl - m) / zE : 0.f;
-        }
-      }
+    // ranks k .. 2k-1 (capacity fallback); ranks past E - 1 do not exist
+    if (valid && rank >= k && rank < 2 * k) {
+      a.next_idx[t * k + rank - k] = lane;
+      a.next_p[t * k + rank - k] = ex / zE;
+    }
+    if (lane < k && k + lane >= E) {
+      a.next_idx[t * k + lane] = -1;
+      a.next_p[t * k + lane] = 0.f;
     }
   }
 }
@@ -135,6 +116,7 @@ template <int EMAX, int G>
 __global__ void __launch_bounds__(kGroupThreads) router_group_kernel(RouterArgs a) {
   __shared__ float s_part[kGroupWarps][G][EMAX];
   __shared__ int s_count[32];
+  pdl_trigger();  // the grouping kernel may launch now; it waits for this grid
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E, d = a.d;
   const int64_t t0 = (int64_t)blockIdx.x * G;
@@ -180,18 +162,187 @@ __global__ void __launch_bounds__(kGroupThreads) router_group_kernel(RouterArgs 
   }
   __syncthreads();
   if (warp < G && t0 + warp < a.T) {
-    float lg[EMAX];
+    float v = 0.f;
+    if (lane < EMAX) {
 #pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < kGroupWarps; ++w) v += s_part[w][warp][e];
-      lg[e] = v;
+      for (int w = 0; w < kGroupWarps; ++w) v += s_part[w][warp][lane];
     }
-    finish_token<EMAX>(a, t0 + warp, lg, lane, s_count);
+    finish_token<EMAX>(a, t0 + warp, v, lane, s_count);
   }
   __syncthreads();
   if (tid < E && s_count[tid] != 0) atomicAdd(&a.counts[tid], s_count[tid]);
+}
+
+// ---------------------------------------------------------------- W_g in registers
+constexpr int kRegMaxThreads = 512;  // d <= 8 * 512
+constexpr int kRegSlots = 4;         // ring depth, in groups of TB token rows
+constexpr int kRegMaxWarps = kRegMaxThreads / 32;
+
+// acc[8] of every lane -> the warp's sum of expert expert_of_lane(lane), exact
+// on lanes with (lane & 3) == 0.  Halving exchanges (16, 8, 4) hand half of
+// the remaining experts to the partner lane; two more steps finish the sum.
+__device__ __forceinline__ float warp_reduce_scatter8(const float (&acc)[8], int lane) {
+  const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4;
+  float v4[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float send = b16 ? acc[j] : acc[j + 4];
+    const float keep = b16 ? acc[j + 4] : acc[j];
+    v4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+  float v2[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float send = b8 ? v4[j] : v4[j + 2];
+    const float keep = b8 ? v4[j + 2] : v4[j];
+    v2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  const float send = b4 ? v2[0] : v2[1];
+  float v = (b4 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v;
+}
+
+__device__ __forceinline__ int expert_of_lane(int lane) {
+  return ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+}
+
+// Dynamic shared memory of router_reg_kernel<TB> for rows of d bf16.
+__host__ __device__ constexpr size_t reg_ring_bytes(int TB, int d) { return (size_t)kRegSlots * TB * d * 2; }
+__host__ __device__ constexpr size_t reg_smem_bytes(int TB, int d) {
+  return reg_ring_bytes(TB, d) + sizeof(float) * 2 * TB * kRegMaxWarps * 8 + sizeof(uint64_t) * kRegSlots +
+         sizeof(int) * 32;
+}
+
+// Block b takes token groups b, b + gridDim.x, ... (TB consecutive tokens
+// each).  Thread 0 keeps up to kRegSlots groups in flight; a slot is refilled
+// right after the block barrier that follows its last read.
+template <int TB>
+__global__ void __launch_bounds__(kRegMaxThreads, 1) router_reg_kernel(RouterArgs a, int64_t ngroups) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  pdl_trigger();  // the grouping kernel may launch now; it waits for this grid
+  const int d = a.d, E = a.E;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const size_t row_bytes = (size_t)d * 2;
+  uint8_t* ring = smem;
+  float* s_part = reinterpret_cast<float*>(smem + reg_ring_bytes(TB, d));  // [2][TB][kRegMaxWarps][8]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_part + 2 * TB * kRegMaxWarps * 8);
+  int* s_count = reinterpret_cast<int*>(bars + kRegSlots);
+
+  const int64_t g0 = blockIdx.x, gstride = gridDim.x;
+  const int64_t my_groups = g0 < ngroups ? (ngroups - 1 - g0) / gstride + 1 : 0;
+  if (tid < 32) s_count[tid] = 0;
+  if (tid == 0) {
+    for (int i = 0; i < kRegSlots; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int64_t i) {  // this block's i-th group into slot i % kRegSlots
+    const int64_t t0 = (g0 + i * gstride) * TB;
+    const int64_t nt = a.T - t0 < TB ? a.T - t0 : TB;
+    const uint32_t bytes = (uint32_t)(nt * (int64_t)row_bytes);
+    uint64_t* bar = &bars[i % kRegSlots];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(ring + (size_t)(i % kRegSlots) * TB * row_bytes, a.x + t0 * d, bytes, bar);
+  };
+  if (tid == 0)
+    for (int64_t i = 0; i < my_groups && i < kRegSlots; ++i) issue(i);
+
+  // inputs [8 tid, 8 tid + 8) of every expert row as pairs (2i, 2i+1); zero
+  // past E and past d
+  const bool active = tid < (d >> 3);
+  uint64_t w2[8][4];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
+    if (active && e < E) {
+      const float4* src = reinterpret_cast<const float4*>(a.Wg + (int64_t)e * d + tid * 8);
+      w0 = __ldg(src);
+      w1 = __ldg(src + 1);
+    }
+    w2[e][0] = pack_f32x2(w0.x, w0.y);
+    w2[e][1] = pack_f32x2(w0.z, w0.w);
+    w2[e][2] = pack_f32x2(w1.x, w1.y);
+    w2[e][3] = pack_f32x2(w1.z, w1.w);
+  }
+
+  bool ok = true;
+  for (int64_t i = 0; i < my_groups; ++i) {
+    const int slot = (int)(i % kRegSlots);
+    const int64_t t0 = (g0 + i * gstride) * TB;
+    const int nt = (int)(a.T - t0 < TB ? a.T - t0 : TB);
+    if (ok) ok = mbar_wait(&bars[slot], (uint32_t)((i / kRegSlots) & 1), nullptr);
+    float* part = s_part + (i & 1) * TB * kRegMaxWarps * 8;
+    const uint8_t* rows = ring + (size_t)slot * TB * row_bytes;
+#pragma unroll
+    for (int tb = 0; tb < TB; ++tb) {
+      if (tb < nt) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        if (active) {
+          // even and odd inputs accumulate in the two halves of a packed pair
+          const uint4 v = *reinterpret_cast<const uint4*>(rows + tb * row_bytes + tid * 16);
+          const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+          uint64_t acc2[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc2[e] = 0ull;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint64_t x2 = pack_f32x2(__uint_as_float(xw[i] << 16), __uint_as_float(xw[i] & 0xFFFF0000u));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) fma_f32x2(acc2[e], x2, w2[e][i]);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float lo, hi;
+            unpack_f32x2(acc2[e], lo, hi);
+            acc[e] = lo + hi;
+          }
+        }
+        const float r = warp_reduce_scatter8(acc, lane);
+        if ((lane & 3) == 0) part[(tb * kRegMaxWarps + warp) * 8 + expert_of_lane(lane)] = r;
+      }
+    }
+    if (!__syncthreads_and(ok)) {
+      // a row copy never arrived: report, let the copies still in flight land, leave
+      if (tid == 0) {
+        record_status(a.status, kStatusTimeout);
+        for (int64_t j = i; j < my_groups && j < i + kRegSlots; ++j)
+          mbar_wait(&bars[j % kRegSlots], (uint32_t)((j / kRegSlots) & 1), nullptr, kWaitLimitNs / 8);
+      }
+      return;
+    }
+    if (tid == 0 && i + kRegSlots < my_groups) issue(i + kRegSlots);
+    // warp sums -> logits, in warp order: lane (q, e) adds warps q, q+4, q+8, q+12
+    for (int tb = warp; tb < nt; tb += nwarps) {
+      const int e = lane & 7, q = lane >> 3;
+      float v = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < kRegMaxWarps; ww += 4)
+        if (q + ww < nwarps) v += part[(tb * kRegMaxWarps + q + ww) * 8 + e];
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      finish_token<8>(a, t0 + tb, v, lane, s_count);  // lane e < 8 holds logit e
+    }
+  }
+  __syncthreads();
+  if (tid < E && s_count[tid] != 0) atomicAdd(&a.counts[tid], s_count[tid]);
+}
+
+template <int TB>
+static cudaError_t launch_router_reg(const RouterArgs& a, int num_sms, cudaStream_t s) {
+  const size_t smem = reg_smem_bytes(TB, a.d);
+  cudaError_t err = cudaFuncSetAttribute(router_reg_kernel<TB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return err;
+  const int64_t ngroups = (a.T + TB - 1) / TB;
+  const int64_t grid = ngroups < num_sms ? ngroups : num_sms;
+  const int threads = ((a.d / 8 + 31) / 32) * 32;
+  router_reg_kernel<TB><<<(unsigned)grid, threads, smem, s>>>(a, ngroups);
+  return cudaGetLastError();
 }
 
 constexpr int64_t kFewTokens = 512;
@@ -213,7 +364,13 @@ cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s, bool
     cudaError_t err = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
     if (err != cudaSuccess) return err;
   }
-  (void)num_sms;
+  if (a.E <= 8 && a.d <= 8 * kRegMaxThreads) {
+    // tokens per SM decide how many rows one ring slot carries
+    const int64_t per_sm = (a.T + num_sms - 1) / num_sms;
+    if (per_sm >= 16) return launch_router_reg<4>(a, num_sms, s);
+    if (per_sm >= 4) return launch_router_reg<2>(a, num_sms, s);
+    return launch_router_reg<1>(a, num_sms, s);
+  }
   if (a.E <= 8) return launch_router_e<8>(a, s);
   if (a.E <= 16) return launch_router_e<16>(a, s);
   return launch_router_e<32>(a, s);

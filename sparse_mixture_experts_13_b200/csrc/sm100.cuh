@@ -27,6 +27,20 @@ __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code) {
   if (status) atomicCAS(status, kStatusOk, code);
 }
 
+// Debug builds (MOE_DEBUG): MOE_DCHECK(status, cond) is cond, and a false
+// cond records kStatusBounds; the caller skips the access it guards.
+// Release builds: always true, no code.
+constexpr uint32_t kStatusBounds = 6;  // matches MOE_ERR_BOUNDS
+#ifdef MOE_DEBUG
+__device__ __forceinline__ bool dcheck(uint32_t* status, bool cond) {
+  if (!cond) record_status(status, kStatusBounds);
+  return cond;
+}
+#define MOE_DCHECK(status, cond) ::moe::dcheck((status), (cond))
+#else
+#define MOE_DCHECK(status, cond) true
+#endif
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -132,6 +146,34 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
+// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global memory into this CTA's shared memory, counted on an
+// mbarrier of this CTA.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Prefetch one box of a tiled tensor map into L2 (no shared memory is
+// written, nothing is waited for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// ---------------------------------------------------------------- launch chain
+// Programmatic dependent launch.  pdl_wait: block this thread until the
+// kernels this grid depends on have completed and their writes are visible
+// (returns at once if the grid was not launched as a dependent).
+// pdl_trigger: this CTA no longer holds back the launch of the next kernel
+// in the stream (which still waits for this grid before reading its output).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -233,6 +275,22 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 }
 
 // ---------------------------------------------------------------- misc
+// Packed pair of fp32 values (lo in the low word) for the f32x2 instructions.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// acc = a * b + acc on both halves (two IEEE fused multiply-adds, one instruction).
+__device__ __forceinline__ void fma_f32x2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -160,5 +160,16 @@ class MoELayerQ4:
         _lib.check(st, "moe_layer_forward_q4")
         return y
 
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
+        """x_host, y_host: page-locked CPU bf16 [T, d]; queued on the stream."""
+        T = x_host.shape[0]
+        cpu = torch.device("cpu")
+        check_activation(x_host, T, self.d, cpu, "x_host")
+        check_activation(y_host, T, self.d, cpu, "y_host")
+        ws = self.workspace(T)
+        st = _lib.moe_layer_forward_q4_host(self.shape(T), x_host, self.Wg, self.q1, self.q3, self.q2, y_host, ws,
+                                            ws.numel(), stream)
+        _lib.check(st, "moe_layer_forward_q4_host")
+
     def device_status(self, T: int) -> int:
         return _lib.moe_read_device_status(self.workspace(T))

@@ -127,6 +127,12 @@ def test_q4_arguments_rejected_before_device(moe):
     assert moe.moe_layer_forward_q4(sh, ok, ok, q, q, q, ok, None, None, ok, n - 1, 0) == W
     assert moe.moe_grouped_swiglu_q4(sh, ok, ok, q, q, (ok + 8, ok), ok, ok, ok, n, 0) == E
     assert moe.moe_layer_forward_q4_profiled(sh, ok, ok, q, q, q, ok, [ok] * 6, None, n, 0) == W
+    assert moe.moe_layer_forward_q4_host(sh, None, ok, q, q, q, ok, ok, n, 0) == E
+    assert moe.moe_layer_forward_q4_host(sh, ok, ok, q, q, q, None, ok, n, 0) == E
+    assert moe.moe_layer_forward_q4_host(sh, ok, ok, (ok + 4, ok), q, q, ok, ok, n, 0) == E
+    assert moe.moe_layer_forward_q4_host(sh, ok, ok, q, q, q, ok, ok, n - 1, 0) == W
+    assert moe.moe_layer_forward_q4_host(moe.make_shape(0, 128, 448), None, None, (None, None), (None, None),
+                                         (None, None), None, None, 0, 0) == moe.MOE_OK
     for bad in ((0, 64, 128), (2, 60, 128), (2, 64, 96), (33, 64, 128), (2, 64, 65600)):
         assert moe.moe_quantize_q4(ok, *bad, ok, ok, 0) == E
     assert moe.moe_quantize_q4(ok, 2, 64, 128, ok + 4, ok, 0) == E

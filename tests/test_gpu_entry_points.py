@@ -124,3 +124,24 @@ def test_q4_profiled_equals_q4_layer(name):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
     assert np.array_equal(H.bf16_host(y), ref), name
     _check_events(evs)
+
+
+@pytest.mark.parametrize("name", ["tiny", "cap_by_prob"])
+def test_q4_host_buffers_equal_q4_layer(name):
+    """moe_layer_forward_q4_host (x and y in page-locked host memory) gives
+    moe_layer_forward_q4's output bit for bit, on two calls in a row with
+    different tokens on a side stream."""
+    wl = synth.Workload(name, **CASES[name]).generate()
+    dev = H.QDevice(wl, oracle.Oracle())
+    sh = dev.shape(0)
+    n = moe.moe_workspace_size_q4(sh)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    for call, x_bits in enumerate([wl.x, synth.normal_bf16(wl.seed + 100, synth.TID_X, (wl.T, wl.d))]):
+        dev.x = H.to_dev_bf16(x_bits)
+        ref = H.run_layer_q4(dev)["y"]
+        y_host = torch.full((wl.T, wl.d), float("nan"), dtype=torch.bfloat16).pin_memory()
+        moe.check(moe.moe_layer_forward_q4_host(sh, _pinned_bf16(x_bits), dev.Wg, *dev.q, y_host, ws, n, s),
+                  "moe_layer_forward_q4_host")
+        assert moe.moe_read_device_status(ws, s) == moe.MOE_OK
+        assert np.array_equal(_host_bits(y_host), ref), (name, call)

@@ -4,8 +4,14 @@ allocate device memory (its scratch is a fixed array inside the library).
 Through the C ABI, its outputs must equal moe_permute's, bit for bit (they are
 integer and copy results), on two calls in a row, so that the contents the
 first call leaves in the shared scratch cannot leak into the second.  This
-file is collected last on purpose and also runs alone in a fresh process.
+file is collected last on purpose; test_runs_alone_in_a_fresh_process runs
+the rest of it again in a new process, where the first call on the device
+also does the address look-up.
 """
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -45,7 +51,10 @@ def _outputs(wl):
     dict(T=256, d=128, f=256, E=8, k=2, capacity_factor=1.0, skew=True),    # capacity, drop by probability
     dict(T=256, d=128, f=256, E=8, k=2, capacity_factor=0.5, drop_policy=1, skew=True),  # by token order
     dict(T=32768, d=64, f=64, E=32, k=2, seed=4),                            # the size limit: 65536 slots
-], ids=["dropless", "cap_by_prob", "cap_by_order", "max_slots"])
+    # more than 1024 slots: the look-back path, with capacity thresholds and drops by rank
+    dict(T=4096, d=128, f=256, E=8, k=2, capacity_factor=1.0, skew=True, seed=6),
+    dict(T=4096, d=128, f=256, E=8, k=2, capacity_factor=1.0, drop_policy=1, skew=True, seed=6),
+], ids=["dropless", "cap_by_prob", "cap_by_order", "max_slots", "lookback_cap_by_prob", "lookback_cap_by_order"])
 def test_noalloc_matches_workspace_entry_point(case):
     import sparse_mixture_experts_13_b200 as moe
     wl = synth.Workload("noalloc", **case).generate(weights=False)
@@ -62,7 +71,7 @@ def test_noalloc_matches_workspace_entry_point(case):
         got = _outputs(wl)
         moe.check(moe.moe_permute_noalloc(sh, x, idx, p, counts, got["offsets"], got["slot_pos"],
                                           got["perm_slot"], got["x_perm"]), "moe_permute_noalloc")
-        torch.cuda.synchronize()
+        assert moe.moe_permute_noalloc_status() == moe.MOE_OK, call
         assert torch.equal(got["offsets"], ref["offsets"]), call
         assert torch.equal(got["slot_pos"], ref["slot_pos"]), call
         assert torch.equal(got["perm_slot"][:N], ref["perm_slot"][:N]), call
@@ -74,3 +83,14 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     sh = moe.make_shape(32769, 64, 64, 8, 2)          # 65538 slots > 65536
     ok = 1 << 20
     assert moe.moe_permute_noalloc(sh, ok, ok, ok, ok, ok, ok, ok, ok) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_runs_alone_in_a_fresh_process():
+    """The comparisons above, alone in a new process: the first
+    moe_permute_noalloc call there does the per-device set-up."""
+    here = os.path.abspath(__file__)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", here, "-k",
+                        "not fresh_process"], capture_output=True, text=True, timeout=900,
+                       cwd=os.path.dirname(os.path.dirname(here)))
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+    assert " passed" in r.stdout
