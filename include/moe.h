@@ -304,7 +304,8 @@ MOE_API moe_status moe_router_stats(const moe_shape *shape, const int32_t *topk_
 MOE_API moe_status moe_ep_plan(const int32_t *counts_all, int32_t E, int32_t rank, int32_t world,
                                int32_t *recv_off, int32_t *owner_off, moe_stream_t stream);
 
-/* shape: this rank's T, the global E, k (capacity_factor must be <= 0).
+/* shape: this rank's T, the global E, k (capacity_factor must be <= 0; with
+ * a capacity use moe_ep_dispatch_cap).
  * x [T, d], topk_idx [T, k], counts [E] from moe_router_topk; recv_off from
  * moe_ep_plan; peer_x: DEVICE array of `world` device pointers, entry o the
  * receive buffer [rows, d] bf16 of rank o (this rank's own included).
@@ -322,6 +323,63 @@ MOE_API moe_status moe_ep_dispatch(const moe_shape *shape, int32_t world, const 
 MOE_API moe_status moe_ep_combine(const moe_shape *shape, int32_t world, const int32_t *topk_idx,
                                   const float *topk_w, const int32_t *ret_row, const moe_bf16 *const *peer_y,
                                   moe_bf16 *y, moe_stream_t stream);
+
+/* Expert parallelism with a capacity (capacity_factor > 0; policies
+ * MOE_DROP_BY_PROB and MOE_DROP_BY_ORDER).  Sources: "How Mixtral 8x7B uses
+ * mixture of experts", "Routing without auxiliary loss" (each expert keeps at
+ * most cf x (tokens x k / E) slots, the rest are dropped) and "Tensor
+ * parallelism vs expert parallelism".  The ranks' tokens form one batch,
+ * their concatenation in rank order (token t of rank r is token
+ * t_base(r) + t, t_base(r) = the tokens of ranks 0 .. r-1), and the layer is
+ * the single-device layer on that batch: cap = floor(cf * T_all * k / E)
+ * with T_all the tokens of all ranks, and the kept slots of an expert are
+ * the cap of largest full-softmax probability (ties: the smaller batch
+ * index) or the first cap in batch order.  Only the owner of an expert sees
+ * all of its slots, so it decides:
+ *   1. moe_router_topk, counts all-gathered, moe_ep_plan (as dropless);
+ *   2. moe_ep_dispatch_cap: every slot's row to its owner as in
+ *      moe_ep_dispatch, and (by probability) its priority key to the same
+ *      row of the owner's key buffer;
+ *   3. barrier; on the owner, moe_ep_select: row_map [rows] (kept row or -1)
+ *      and kept_off [epr + 1], the kept rows gathered into x_kept; then
+ *      moe_grouped_swiglu on x_kept with kept_off;
+ *   4. barrier; moe_ep_combine_cap: as moe_ep_combine, each slot's row
+ *      passed through its owner's row_map; a dropped slot adds zero and the
+ *      other gates are not renormalised.
+ * Buffers of `rows` rows (the sum over ranks of T*k at most): x_recv, keys,
+ * row_map and the kept-row output y_kept must be reachable by every rank
+ * (peer arrays); x_kept and h are the owner's own. */
+
+/* shape: this rank's T, the global E, k, capacity_factor > 0 and the drop
+ * policy; counts_all [world, E] as for moe_ep_plan; topk_p [T, k] from
+ * moe_router_topk (by probability); peer_keys: DEVICE array of `world`
+ * device pointers to the owners' key buffers [rows] uint64 (by probability;
+ * may be NULL by order).  Other arguments and preconditions as
+ * moe_ep_dispatch.  The next-best fallback policies give
+ * MOE_ERR_UNSUPPORTED. */
+MOE_API moe_status moe_ep_dispatch_cap(const moe_shape *shape, int32_t world, int32_t rank,
+                                       const int32_t *counts_all, const moe_bf16 *x, const int32_t *topk_idx,
+                                       const float *topk_p, const int32_t *counts, const int32_t *recv_off,
+                                       moe_bf16 *const *peer_x, uint64_t *const *peer_keys, int32_t *ret_row,
+                                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Owner side of the capacity (after the dispatch's barrier).  shape: the
+ * global E, k, d_model, capacity_factor and policy (T is not used);
+ * counts_all and owner_off from this step; keys [rows] this rank's key
+ * buffer (by probability); x_recv [rows, d] its receive buffer.  Out:
+ * x_kept [rows, d], kept_off [epr + 1] int32, row_map [rows] int32.
+ * Allocates nothing; 1 + 1 kernels on `stream`. */
+MOE_API moe_status moe_ep_select(const moe_shape *shape, int32_t world, const int32_t *counts_all,
+                                 const int32_t *owner_off, const uint64_t *keys, const moe_bf16 *x_recv,
+                                 moe_bf16 *x_kept, int32_t *kept_off, int32_t *row_map, moe_stream_t stream);
+
+/* peer_map: DEVICE array of `world` device pointers to the owners' row_map;
+ * peer_y: to the owners' outputs of moe_grouped_swiglu on x_kept.  Otherwise
+ * as moe_ep_combine. */
+MOE_API moe_status moe_ep_combine_cap(const moe_shape *shape, int32_t world, const int32_t *topk_idx,
+                                      const float *topk_w, const int32_t *ret_row,
+                                      const int32_t *const *peer_map, const moe_bf16 *const *peer_y,
+                                      moe_bf16 *y, moe_stream_t stream);
 
 /* ---------------------------------------------------------------- 4-bit experts
  * Sources: "How Mixtral 8x7B uses mixture of experts", "Deployment tradeoffs

@@ -13,5 +13,6 @@ from ._lib import (EXPORTED, MOE_ERR_BOUNDS, moe_debug_build, moe_debug_workspac
                    moe_layer_forward_profiled, moe_permute,
                    moe_read_device_status, moe_router_topk, moe_selftest_wait_timeout, moe_shape, moe_workspace_size, status_string,
                    moe_quantize_q4, moe_workspace_size_q4, moe_grouped_swiglu_q4, moe_layer_forward_q4,
-                   moe_layer_forward_q4_profiled, moe_layer_forward_q4_host, moe_router_stats, moe_ep_plan, moe_ep_dispatch, moe_ep_combine)
+                   moe_layer_forward_q4_profiled, moe_layer_forward_q4_host, moe_router_stats, moe_ep_plan, moe_ep_dispatch, moe_ep_combine,
+                   moe_ep_dispatch_cap, moe_ep_select, moe_ep_combine_cap)
 from .layer import MoELayer, MoELayerQ4  # noqa: F401

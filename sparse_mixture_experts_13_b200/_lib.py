@@ -26,7 +26,7 @@ EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped
             "moe_layer_forward", "moe_layer_forward_host", "moe_layer_forward_profiled", "moe_permute_noalloc",
             "moe_permute_noalloc_status",
             "moe_selftest_wait_timeout", "moe_read_device_status", "moe_router_stats", "moe_ep_plan", "moe_ep_dispatch",
-            "moe_ep_combine", "moe_quantize_q4", "moe_workspace_size_q4",
+            "moe_ep_combine", "moe_ep_dispatch_cap", "moe_ep_select", "moe_ep_combine_cap", "moe_quantize_q4", "moe_workspace_size_q4",
             "moe_grouped_swiglu_q4", "moe_layer_forward_q4", "moe_layer_forward_q4_profiled", "moe_layer_forward_q4_host",
             "moe_debug_build", "moe_debug_workspace_arm", "moe_debug_workspace_check", "moe_status_string")
 _SIZE_RETURNING = ("moe_workspace_size", "moe_workspace_size_q4")
@@ -79,6 +79,9 @@ def lib():
         L.moe_ep_plan.argtypes = [P, i32, i32, i32, P, P, P]
         L.moe_ep_dispatch.argtypes = [S, i32, P, P, P, P, P, P, P, sz, P]
         L.moe_ep_combine.argtypes = [S, i32, P, P, P, P, P, P]
+        L.moe_ep_dispatch_cap.argtypes = [S, i32, i32, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_ep_select.argtypes = [S, i32, P, P, P, P, P, P, P, P]
+        L.moe_ep_combine_cap.argtypes = [S, i32, P, P, P, P, P, P, P]
         L.moe_quantize_q4.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P]
         L.moe_workspace_size_q4.argtypes = [S]
         L.moe_grouped_swiglu_q4.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, sz, P]
@@ -212,6 +215,23 @@ def moe_ep_dispatch(shape, world, x, topk_idx, counts, recv_off, peer_x, ret_row
 def moe_ep_combine(shape, world, topk_idx, topk_w, ret_row, peer_y, y, stream=None) -> int:
     return lib().moe_ep_combine(ctypes.byref(shape), int(world), _p(topk_idx), _p(topk_w), _p(ret_row), _p(peer_y),
                                 _p(y), _stream(stream))
+
+
+def moe_ep_dispatch_cap(shape, world, rank, counts_all, x, topk_idx, topk_p, counts, recv_off, peer_x, peer_keys,
+                        ret_row, ws, ws_bytes, stream=None) -> int:
+    return lib().moe_ep_dispatch_cap(ctypes.byref(shape), int(world), int(rank), _p(counts_all), _p(x), _p(topk_idx),
+                                     _p(topk_p), _p(counts), _p(recv_off), _p(peer_x), _p(peer_keys), _p(ret_row),
+                                     _p(ws), int(ws_bytes), _stream(stream))
+
+
+def moe_ep_select(shape, world, counts_all, owner_off, keys, x_recv, x_kept, kept_off, row_map, stream=None) -> int:
+    return lib().moe_ep_select(ctypes.byref(shape), int(world), _p(counts_all), _p(owner_off), _p(keys), _p(x_recv),
+                               _p(x_kept), _p(kept_off), _p(row_map), _stream(stream))
+
+
+def moe_ep_combine_cap(shape, world, topk_idx, topk_w, ret_row, peer_map, peer_y, y, stream=None) -> int:
+    return lib().moe_ep_combine_cap(ctypes.byref(shape), int(world), _p(topk_idx), _p(topk_w), _p(ret_row),
+                                    _p(peer_map), _p(peer_y), _p(y), _stream(stream))
 
 
 # ------------------------------------------------------------ 4-bit experts

@@ -655,6 +655,85 @@ moe_status moe_ep_combine(const moe_shape* sh, int32_t world, const int32_t* top
                                        y, sh->T, sh->k, sh->d_model, sh->E / world, sms, (cudaStream_t)stream));
 }
 
+moe_status moe_ep_dispatch_cap(const moe_shape* sh, int32_t world, int32_t rank, const int32_t* counts_all,
+                               const moe_bf16* x, const int32_t* topk_idx, const float* topk_p, const int32_t* counts,
+                               const int32_t* recv_off, moe_bf16* const* peer_x, uint64_t* const* peer_keys,
+                               int32_t* ret_row, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (world < 1 || world > 32 || sh->E % world || rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+  if (!(sh->capacity_factor > 0.f)) return MOE_ERR_INVALID_ARG;              // the dropless path is moe_ep_dispatch
+  if (sh->drop_policy > MOE_DROP_BY_ORDER) return MOE_ERR_UNSUPPORTED;       // no next-best fallback here
+  if (sh->T == 0) return MOE_OK;
+  const bool by_prob = sh->drop_policy == MOE_DROP_BY_PROB;
+  MOE_TRY(check_bf16(x));
+  MOE_TRY(check_i32(topk_idx));
+  MOE_TRY(check_i32(counts));
+  MOE_TRY(check_i32(counts_all));
+  MOE_TRY(check_i32(recv_off));
+  MOE_TRY(check_bf16(peer_x));
+  MOE_TRY(check_i32(ret_row));
+  if (by_prob) {
+    MOE_TRY(check_i32(topk_p));
+    MOE_TRY(check_bf16(peer_keys));
+  }
+  MOE_TRY(check_ws(sh, ws, ws_bytes));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  moe_shape dropless = *sh;  // every slot is sent; the owners select
+  dropless.capacity_factor = 0.f;
+  const Layout L = layout_of(&dropless);
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, 8, s)));
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* slot_pos = at<int32_t>(ws, L.slot_pos);
+  MOE_TRY(run_permute(&dropless, L, x, topk_idx, nullptr, counts, offsets, slot_pos, at<int32_t>(ws, L.perm_slot),
+                      nullptr, ws, s, false));
+  const EpKeys keys{topk_p, counts_all, sh->E, rank, peer_keys};
+  return cuda_status(launch_ep_dispatch(x, topk_idx, offsets, slot_pos, recv_off,
+                                        reinterpret_cast<uint16_t* const*>(peer_x), ret_row, sh->T * sh->k, sh->k,
+                                        sh->d_model, sh->E / world, sms, s, by_prob ? &keys : nullptr));
+}
+
+moe_status moe_ep_select(const moe_shape* sh, int32_t world, const int32_t* counts_all, const int32_t* owner_off,
+                         const uint64_t* keys, const moe_bf16* x_recv, moe_bf16* x_kept, int32_t* kept_off,
+                         int32_t* row_map, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (world < 1 || world > 32 || sh->E % world) return MOE_ERR_INVALID_ARG;
+  if (!(sh->capacity_factor > 0.f)) return MOE_ERR_INVALID_ARG;
+  if (sh->drop_policy > MOE_DROP_BY_ORDER) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(check_i32(counts_all));
+  MOE_TRY(check_i32(owner_off));
+  MOE_TRY(check_bf16(x_recv));
+  MOE_TRY(check_bf16(x_kept));
+  MOE_TRY(check_i32(kept_off));
+  MOE_TRY(check_i32(row_map));
+  if (sh->drop_policy == MOE_DROP_BY_PROB) MOE_TRY(check_bf16(keys));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return cuda_status(launch_ep_select(counts_all, world, sh->E, sh->k, sh->capacity_factor, sh->drop_policy, owner_off,
+                                      keys, sh->E / world, kept_off, row_map, x_recv, x_kept, sh->d_model, sms,
+                                      (cudaStream_t)stream));
+}
+
+moe_status moe_ep_combine_cap(const moe_shape* sh, int32_t world, const int32_t* topk_idx, const float* topk_w,
+                              const int32_t* ret_row, const int32_t* const* peer_map, const moe_bf16* const* peer_y,
+                              moe_bf16* y, moe_stream_t stream) {
+  MOE_TRY(check_shape(sh));
+  if (world < 1 || world > 32 || sh->E % world) return MOE_ERR_INVALID_ARG;
+  if (sh->T == 0) return MOE_OK;
+  MOE_TRY(check_i32(topk_idx));
+  MOE_TRY(check_i32(topk_w));
+  MOE_TRY(check_i32(ret_row));
+  MOE_TRY(check_bf16(peer_map));
+  MOE_TRY(check_bf16(peer_y));
+  MOE_TRY(check_bf16(y));
+  int sms = 0;
+  MOE_TRY(check_device(&sms));
+  return cuda_status(launch_ep_combine(topk_idx, topk_w, ret_row, reinterpret_cast<const uint16_t* const*>(peer_y),
+                                       y, sh->T, sh->k, sh->d_model, sh->E / world, sms, (cudaStream_t)stream,
+                                       peer_map));
+}
+
 moe_status moe_router_stats(const moe_shape* sh, const int32_t* topk_idx, int32_t* slot_counts, int32_t* pair_counts,
                             int32_t accumulate, moe_stream_t stream) {
   MOE_TRY(check_shape(sh));

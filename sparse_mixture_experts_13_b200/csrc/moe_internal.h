@@ -173,13 +173,25 @@ cudaError_t launch_fallback(const FallbackArgs& a, int num_sms, cudaStream_t s);
 // Expert parallelism (csrc/ep.cu).
 cudaError_t launch_ep_plan(const int32_t* counts_all, int32_t E, int32_t rank, int32_t world, int32_t* recv_off,
                            int32_t* owner_off, cudaStream_t s);
+// Capacity with expert parallelism: what the dispatch needs to store each
+// slot's priority key in its owner's key buffer.
+struct EpKeys {
+  const float* topk_p;        // [S] full-softmax probabilities of this rank's slots
+  const int32_t* counts_all;  // [world, E] routed counts of every rank
+  int32_t E, rank;
+  uint64_t* const* peer_keys; // [world] device pointers to the owners' key buffers
+};
 cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, const int32_t* offsets,
                                const int32_t* slot_pos, const int32_t* recv_off, uint16_t* const* peer_x,
                                int32_t* ret_row, int64_t S, int32_t k, int32_t d, int32_t epr, int num_sms,
-                               cudaStream_t s);
+                               cudaStream_t s, const EpKeys* keys = nullptr);
 cudaError_t launch_ep_combine(const int32_t* topk_idx, const float* topk_w, const int32_t* ret_row,
                               const uint16_t* const* peer_y, uint16_t* y, int64_t T, int32_t k, int32_t d, int32_t epr,
-                              int num_sms, cudaStream_t s);
+                              int num_sms, cudaStream_t s, const int32_t* const* peer_map = nullptr);
+cudaError_t launch_ep_select(const int32_t* counts_all, int32_t world, int32_t E, int32_t k, float cf, int32_t policy,
+                             const int32_t* owner_off, const uint64_t* keys, int32_t epr, int32_t* kept_off,
+                             int32_t* row_map, const uint16_t* x_recv, uint16_t* x_kept, int32_t d, int num_sms,
+                             cudaStream_t s);
 
 struct CombineArgs {
   const uint16_t* y_perm;   // [S, d] bf16, or nullptr when reading partials

@@ -36,21 +36,28 @@ def _ptrs(tensors, device) -> torch.Tensor:
     return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
 
 
-def ep_forward_emulated(xs, Wg, W1, W3, W2, world: int, k: int = 2):
+def ep_forward_emulated(xs, Wg, W1, W3, W2, world: int, k: int = 2, capacity_factor: float = 0.0,
+                        drop_policy: int = _lib.MOE_DROP_BY_PROB, info: dict | None = None):
     """Expert-parallel forward of `world` emulated ranks on one GPU.
 
     xs: list of `world` bf16 [T_r, d] token batches; Wg fp32 [E, d]; W1, W3
     [E, f, d] and W2 [E, d, f] bf16 (rank o uses experts o*E/world ..).
-    Returns (list of y [T_r, d], list of topk_idx [T_r*k], list of counts [E]).
+    With capacity_factor > 0 the ranks' tokens are one batch (their
+    concatenation) and each owner keeps its experts' slots under the capacity
+    (moe_ep_dispatch_cap, moe_ep_select, moe_ep_combine_cap).
+    Returns (list of y [T_r, d], list of topk_idx [T_r*k], list of counts [E]);
+    `info`, if given, receives the routers' probabilities, ret_row of every
+    rank and row_map of every owner.
     """
     dev = xs[0].device
     E, f, d = W1.shape
     assert E % world == 0 and len(xs) == world
     epr = E // world
+    cap_mode = capacity_factor > 0
     cu = lambda *shape, dt: torch.empty(*shape, dtype=dt, device=dev)
     # 1. routers
-    shapes = [_lib.make_shape(x.shape[0], d, f, E, k) for x in xs]
-    idx, w, counts = [], [], []
+    shapes = [_lib.make_shape(x.shape[0], d, f, E, k, capacity_factor, drop_policy) for x in xs]
+    idx, w, probs, counts = [], [], [], []
     for r, x in enumerate(xs):
         T = x.shape[0]
         i, ww, p, c = cu(T * k, dt=torch.int32), cu(T * k, dt=torch.float32), cu(T * k, dt=torch.float32), \
@@ -58,6 +65,7 @@ def ep_forward_emulated(xs, Wg, W1, W3, W2, world: int, k: int = 2):
         _check(_lib.moe_router_topk(shapes[r], x, Wg, None, i, ww, p, c), "moe_router_topk")
         idx.append(i)
         w.append(ww)
+        probs.append(p)
         counts.append(c)
     # 2. all-gather of the counts
     counts_all = torch.stack(counts).contiguous()
@@ -71,29 +79,50 @@ def ep_forward_emulated(xs, Wg, W1, W3, W2, world: int, k: int = 2):
     owner_off = [cu(epr + 1, dt=torch.int32) for _ in range(world)]
     for r in range(world):
         _check(_lib.moe_ep_plan(counts_all, E, r, world, recv_off[r], owner_off[r]), "moe_ep_plan")
+    if cap_mode:
+        keys = [cu(max(rows, 1), dt=torch.int64) for _ in range(world)]
+        row_map = [cu(max(rows, 1), dt=torch.int32) for _ in range(world)]
+        x_kept = [cu(rows, d, dt=torch.bfloat16) for _ in range(world)]
+        kept_off = [cu(epr + 1, dt=torch.int32) for _ in range(world)]
+        peer_keys, peer_map = _ptrs(keys, dev), _ptrs(row_map, dev)
     # 4. dispatch
     ret_row = []
     for r, x in enumerate(xs):
         rr = cu(x.shape[0] * k, dt=torch.int32)
         n = _lib.moe_workspace_size(shapes[r])
         ws = cu(n, dt=torch.uint8)
-        _check(_lib.moe_ep_dispatch(shapes[r], world, x, idx[r], counts[r], recv_off[r], peer_x, rr, ws, n),
-               "moe_ep_dispatch")
+        if cap_mode:
+            _check(_lib.moe_ep_dispatch_cap(shapes[r], world, r, counts_all, x, idx[r], probs[r], counts[r],
+                                            recv_off[r], peer_x, peer_keys, rr, ws, n), "moe_ep_dispatch_cap")
+        else:
+            _check(_lib.moe_ep_dispatch(shapes[r], world, x, idx[r], counts[r], recv_off[r], peer_x, rr, ws, n),
+                   "moe_ep_dispatch")
         ret_row.append(rr)
-    # 5. owners' expert GEMMs on their receive buffers
+    # 5. owners: the capacity (with one) and the expert GEMMs
     osh = _lib.make_shape(rows, d, f, epr, 1)
     n = _lib.moe_workspace_size(osh)
     for o in range(world):
         ws = cu(n, dt=torch.uint8)
         sl = slice(o * epr, (o + 1) * epr)
-        _check(_lib.moe_grouped_swiglu(osh, x_recv[o], owner_off[o], W1[sl].contiguous(), W3[sl].contiguous(),
+        a_in, a_off = x_recv[o], owner_off[o]
+        if cap_mode:
+            _check(_lib.moe_ep_select(shapes[0], world, counts_all, owner_off[o], keys[o], x_recv[o], x_kept[o],
+                                      kept_off[o], row_map[o]), "moe_ep_select")
+            a_in, a_off = x_kept[o], kept_off[o]
+        _check(_lib.moe_grouped_swiglu(osh, a_in, a_off, W1[sl].contiguous(), W3[sl].contiguous(),
                                        W2[sl].contiguous(), h_recv[o], y_recv[o], ws, n), "moe_grouped_swiglu")
     # 6. combine
     ys = []
     for r, x in enumerate(xs):
         y = cu(x.shape[0], d, dt=torch.bfloat16)
-        _check(_lib.moe_ep_combine(shapes[r], world, idx[r], w[r], ret_row[r], peer_y, y), "moe_ep_combine")
+        if cap_mode:
+            _check(_lib.moe_ep_combine_cap(shapes[r], world, idx[r], w[r], ret_row[r], peer_map, peer_y, y),
+                   "moe_ep_combine_cap")
+        else:
+            _check(_lib.moe_ep_combine(shapes[r], world, idx[r], w[r], ret_row[r], peer_y, y), "moe_ep_combine")
         ys.append(y)
+    if info is not None:
+        info.update(p=probs, ret_row=ret_row, row_map=row_map if cap_mode else None, epr=epr)
     return ys, idx, counts
 
 
@@ -106,7 +135,8 @@ class EPLayer:
     same sequence of layers (it contains collectives).
     """
 
-    def __init__(self, Wg, W1_local, W3_local, W2_local, E: int, k: int, max_tokens: int, group=None):
+    def __init__(self, Wg, W1_local, W3_local, W2_local, E: int, k: int, max_tokens: int, group=None,
+                 capacity_factor: float = 0.0, drop_policy: int = _lib.MOE_DROP_BY_PROB):
         import torch.distributed as dist
         import torch.distributed._symmetric_memory as symm_mem
         self.dist, self.group = dist, group
@@ -131,13 +161,29 @@ class EPLayer:
         self.peer_y = torch.tensor([p_ + oy for p_ in hy.buffer_ptrs], dtype=torch.int64, device=dev)
         self._handles = (hx, hy)
         self.h_recv = torch.empty(self.rows, self.f, dtype=torch.bfloat16, device=dev)
+        self.capacity_factor, self.drop_policy = capacity_factor, drop_policy
+        if capacity_factor > 0:
+            # the owner's key buffer and row map are written / read by the
+            # other ranks, so they live in symmetric memory too
+            self.keys = symm_mem.empty(self.rows, dtype=torch.int64, device=dev)
+            self.row_map = symm_mem.empty(self.rows, dtype=torch.int32, device=dev)
+            hk = symm_mem.rendezvous(self.keys, group=g)
+            hm = symm_mem.rendezvous(self.row_map, group=g)
+            ok_ = self.keys.data_ptr() - hk.buffer_ptrs[self.rank]
+            om = self.row_map.data_ptr() - hm.buffer_ptrs[self.rank]
+            self.peer_keys = torch.tensor([p_ + ok_ for p_ in hk.buffer_ptrs], dtype=torch.int64, device=dev)
+            self.peer_map = torch.tensor([p_ + om for p_ in hm.buffer_ptrs], dtype=torch.int64, device=dev)
+            self._handles = self._handles + (hk, hm)
+            self.x_kept = torch.empty(self.rows, self.d, dtype=torch.bfloat16, device=dev)
+            self.kept_off = torch.empty(self.epr + 1, dtype=torch.int32, device=dev)
         self.owner_shape = _lib.make_shape(self.rows, self.d, self.f, self.epr, 1)
         self.owner_ws = torch.empty(_lib.moe_workspace_size(self.owner_shape), dtype=torch.uint8, device=dev)
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         dist, dev = self.dist, x.device
         T, d, E, k = x.shape[0], self.d, self.E, self.k
-        sh = _lib.make_shape(T, d, self.f, E, k)
+        cap_mode = self.capacity_factor > 0
+        sh = _lib.make_shape(T, d, self.f, E, k, self.capacity_factor, self.drop_policy)
         cu = lambda *shape, dt: torch.empty(*shape, dtype=dt, device=dev)
         idx, w, p, counts = cu(T * k, dt=torch.int32), cu(T * k, dt=torch.float32), cu(T * k, dt=torch.float32), \
             cu(E, dt=torch.int32)
@@ -149,15 +195,28 @@ class EPLayer:
         ret_row = cu(T * k, dt=torch.int32)
         n = _lib.moe_workspace_size(sh)
         ws = cu(n, dt=torch.uint8)
-        _check(_lib.moe_ep_dispatch(sh, self.world, x, idx, counts, recv_off, self.peer_x, ret_row, ws, n),
-               "moe_ep_dispatch")
-        dist.barrier(group=self.group)  # every rank's rows have landed
-        _check(_lib.moe_grouped_swiglu(self.owner_shape, self.x_recv, owner_off, self.W1, self.W3, self.W2,
+        if cap_mode:
+            _check(_lib.moe_ep_dispatch_cap(sh, self.world, self.rank, counts_all, x, idx, p, counts, recv_off,
+                                            self.peer_x, self.peer_keys, ret_row, ws, n), "moe_ep_dispatch_cap")
+        else:
+            _check(_lib.moe_ep_dispatch(sh, self.world, x, idx, counts, recv_off, self.peer_x, ret_row, ws, n),
+                   "moe_ep_dispatch")
+        dist.barrier(group=self.group)  # every rank's rows (and keys) have landed
+        a_in, a_off = self.x_recv, owner_off
+        if cap_mode:
+            _check(_lib.moe_ep_select(sh, self.world, counts_all, owner_off, self.keys, self.x_recv, self.x_kept,
+                                      self.kept_off, self.row_map), "moe_ep_select")
+            a_in, a_off = self.x_kept, self.kept_off
+        _check(_lib.moe_grouped_swiglu(self.owner_shape, a_in, a_off, self.W1, self.W3, self.W2,
                                        self.h_recv, self.y_recv, self.owner_ws, self.owner_ws.numel()),
                "moe_grouped_swiglu")
-        dist.barrier(group=self.group)  # every owner's results are written
+        dist.barrier(group=self.group)  # every owner's results (and row map) are written
         y = cu(T, d, dt=torch.bfloat16)
-        _check(_lib.moe_ep_combine(sh, self.world, idx, w, ret_row, self.peer_y, y), "moe_ep_combine")
+        if cap_mode:
+            _check(_lib.moe_ep_combine_cap(sh, self.world, idx, w, ret_row, self.peer_map, self.peer_y, y),
+                   "moe_ep_combine_cap")
+        else:
+            _check(_lib.moe_ep_combine(sh, self.world, idx, w, ret_row, self.peer_y, y), "moe_ep_combine")
         dist.barrier(group=self.group)  # the buffers may be reused by the next call
         return y
 

@@ -133,3 +133,108 @@ def test_ep_plan_kernel_equals_host_plan(world, E):
         want_recv, want_owner = ep_plan_host(counts_all.tolist(), rank, world)
         assert recv_off.cpu().tolist() == want_recv, rank
         assert owner_off.cpu().tolist() == want_owner, rank
+
+
+def run_ep_capacity(o, world, Ts, d, f, cf, policy, E=8, k=2, seed=11, rows=None, weights=None):
+    """Expert parallelism with a capacity, emulated: the ranks' tokens are one
+    batch (their concatenation), so the reference is the oracle's layer on
+    that batch.  The kept slots must be exactly the oracle's (up to slots
+    within the comparison tolerance of an expert's threshold probability),
+    and each rank's y must match the oracle's rows for its tokens."""
+    T_all = sum(Ts)
+    base = synth.Workload("epcap", T_all, d, f, E=E, k=k, capacity_factor=cf, drop_policy=policy, skew=True,
+                          seed=seed)
+    base.generate(weights=weights is None)
+    if weights is not None:
+        base.W1, base.W3, base.W2 = weights
+    starts = np.concatenate([[0], np.cumsum(Ts)])
+    xs = [H.to_dev_bf16(base.x[starts[r]:starts[r + 1]]) for r in range(world)]
+    dev_w = [H.to_dev_bf16(W) for W in (base.W1, base.W3, base.W2)]
+    info = {}
+    ys, idx, counts = ep.ep_forward_emulated(xs, torch.from_numpy(base.Wg).cuda(), *dev_w, world=world, k=k,
+                                            capacity_factor=cf, drop_policy=policy, info=info)
+    torch.cuda.synchronize()
+    epr = info["epr"]
+    maps = [m.cpu().numpy() for m in info["row_map"]]
+    gpu_idx = np.concatenate([i.cpu().numpy() for i in idx])
+    gpu_p = np.concatenate([p.cpu().numpy() for p in info["p"]])
+    ret = [r.cpu().numpy() for r in info["ret_row"]]
+    kept = np.concatenate([np.array([maps[e // epr][row] >= 0 for e, row in zip(i.cpu().numpy(), rr)], bool)
+                           for i, rr in zip(idx, ret)])
+    rt = H.conditional_route(o, base, gpu_idx, gpu_p, np.where(kept, 0, -1))
+    assert rt["cap"] is not None
+    assert np.array_equal(gpu_idx.reshape(T_all, k), rt["idx"])
+    assert np.array_equal(kept, rt["slot_pos"] >= 0), "kept slots differ from the oracle's"
+    assert (~kept).any(), "the case should drop slots"
+    toks = np.arange(T_all) if rows is None else H.sample_tokens(base, rt, rows)
+    ref = o.layer_rows(base.x, base.W1, base.W3, base.W2, rt, toks)
+    y_all = np.concatenate([H.bf16_f64(H.bf16_host(y)) for y in ys])
+    H.assert_close(y_all[toks], ref["y"], f"y (expert parallel, {world} ranks, cf {cf}, policy {policy})")
+    fully = np.nonzero((rt["slot_pos"].reshape(T_all, k) < 0).all(1))[0]
+    if fully.size:
+        assert not y_all[fully].any()
+    return rt
+
+
+@pytest.mark.parametrize("policy", [0, 1], ids=["by_prob", "by_order"])
+@pytest.mark.parametrize("cf", [1.0, 1.25])
+@pytest.mark.parametrize("world", [2, 8])
+def test_ep_capacity(o, world, cf, policy):
+    run_ep_capacity(o, world, [61 + 29 * r for r in range(world)], 128, 256, cf, policy)
+
+
+def test_ep_capacity_uneven_ranks_sixteen_experts(o):
+    """Four ranks of 1, 300, 64 and 129 tokens, 16 experts (4 per rank)."""
+    for policy in (0, 1):
+        run_ep_capacity(o, 4, [1, 300, 64, 129], 128, 192, 1.0, policy, E=16, seed=12)
+
+
+def test_ep_capacity_mixtral_eight_ranks(o):
+    """Mixtral shapes, one expert per rank, skewed routing, cf 1.25."""
+    wl = synth.workload("decode")
+    wl.generate()
+    run_ep_capacity(o, 8, [256] * 8, synth.MIXTRAL_D, synth.MIXTRAL_F, 1.25, 0, rows=12,
+                    weights=(wl.W1, wl.W3, wl.W2))
+
+
+def test_ep_capacity_entry_points_refuse():
+    z = torch.zeros(64, dtype=torch.int32, device="cuda")
+    x = torch.zeros(16, 128, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    nb = moe.make_shape(16, 128, 256, E=8, k=2, capacity_factor=1.0, drop_policy=moe.MOE_DROP_BY_PROB_NEXT_BEST)
+    assert moe.moe_ep_dispatch_cap(nb, 2, 0, z, x, z, z, z, z, z, z, z, ws, ws.numel()) == moe.MOE_ERR_UNSUPPORTED
+    assert moe.moe_ep_select(nb, 2, z, z, z, x, x, z, z) == moe.MOE_ERR_UNSUPPORTED
+    dl = moe.make_shape(16, 128, 256, E=8, k=2)
+    assert moe.moe_ep_dispatch_cap(dl, 2, 0, z, x, z, z, z, z, z, z, z, ws, ws.numel()) == moe.MOE_ERR_INVALID_ARG
+    cap = moe.make_shape(16, 128, 256, E=8, k=2, capacity_factor=1.0)
+    assert moe.moe_ep_dispatch_cap(cap, 2, 2, z, x, z, z, z, z, z, z, z, ws, ws.numel()) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_ep_dispatch_cap(cap, 2, 0, z, x, z, None, z, z, z, z, z, ws, ws.numel()) == \
+        moe.MOE_ERR_INVALID_ARG        # by probability needs the probabilities
+
+
+def test_ep_layer_capacity_one_process_group_of_one(o):
+    """EPLayer with a capacity in a group of one rank: the owner (this rank)
+    selects over its slots, which is the single-GPU layer's capacity."""
+    import socket
+    import torch.distributed as dist
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        for policy in (0, 1):
+            wl = synth.Workload("eplcap", 96, 128, 256, seed=6, capacity_factor=1.0, drop_policy=policy,
+                                skew=True).generate()
+            dev = H.Device(wl)
+            layer = ep.EPLayer(dev.Wg, dev.W1, dev.W3, dev.W2, E=wl.E, k=wl.k, max_tokens=wl.T,
+                               capacity_factor=wl.capacity_factor, drop_policy=policy)
+            y = layer.forward(dev.x)
+            torch.cuda.synchronize()
+            single = H.bf16_f64(H.run_layer(dev, 1)["y"])
+            got = H.bf16_f64(H.bf16_host(y))
+            assert H.rel_fro(got, single) < 2e-3, policy       # same routing, same kept slots
+            assert np.array_equal(got == 0, single == 0), policy  # the same fully dropped tokens
+            del layer
+    finally:
+        dist.destroy_process_group()
