@@ -343,6 +343,7 @@ class Run:
                                                 self.layer.W2, self.y, evs[i], ws, ws.numel())
             moe.check(st, "moe_layer_forward_profiled")
         torch.cuda.synchronize()
+        self.clock_mhz = gemm_clocks(ws)
         for i in range(steps):
             sums += [evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
         return dict(zip(["router", "capacity_and_permute", "gemm1_swiglu", "gemm2", "combine"],
@@ -448,6 +449,7 @@ class RunQ4(Run):
             moe.check(moe.moe_layer_forward_q4_profiled(sh, self.x, L.Wg, L.q1, L.q3, L.q2, self.y, evs[i], ws,
                                                         ws.numel()), "moe_layer_forward_q4_profiled")
         torch.cuda.synchronize()
+        self.clock_mhz = gemm_clocks(ws)
         for i in range(steps):
             sums += [evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
         return dict(zip(["router", "capacity_and_permute", "gemm1_swiglu", "gemm2", "combine"],
@@ -457,6 +459,22 @@ class RunQ4(Run):
         wl, L = self.wl, self.layer
         return self.moe.MoELayerQ4(L.Wg, L.q1, L.q3, L.q2, k=wl.k, capacity_factor=wl.capacity_factor,
                                    drop_policy=wl.drop_policy)
+
+
+def gemm_clocks(ws) -> dict:
+    """SM clock (MHz) each expert GEMM of the last profiled call ran at: the
+    profiled entry points store {clock64, globaltimer ns} of CTA 0 at entry
+    and exit of both GEMMs in bytes 64 .. 127 of the workspace."""
+    rec = ws[64:128].view(dtype=__import__("torch").int64).cpu().numpy().astype(np.float64)
+    out = {}
+    for name, (c0, n0, c1, n1) in (("gemm1", rec[0:4]), ("gemm2", rec[4:8])):
+        out[name] = (c1 - c0) / (n1 - n0) * 1e3 if n1 > n0 else None
+    return out
+
+
+def clock_peak_tflops(mhz, sms=148, flop_per_clk_sm=8192):
+    """Dense bf16 tensor peak at a given SM clock (TFLOP/s)."""
+    return sms * flop_per_clk_sm * mhz * 1e-6 if mhz else None
 
 
 def expert_bytes(d, f):
@@ -607,7 +625,7 @@ def stage_report(wl, q, world, peaks, kernel, traffic_kernel, workload_key, q4=F
                          entry_point=q["entry"]),
                 e2e_pipelined=dict(value=weak_scaling_value(world, wl.T, q["e2e_pipe_ms"]), unit="tokens/s",
                                    note="two streams, consecutive steps overlap"),
-                experts_touched=q["touched"])
+                experts_touched=q["touched"], gemm_clock_mhz=q["gemm_clock_mhz"])
 
 
 def run_ours(args):
@@ -663,6 +681,7 @@ def run_ours(args):
             e2e_pipe_ms, _, _ = run.e2e_pipelined(args.steps, dist)
         ms_flushed = flushed_median_ms(run.step, max(args.steps, 20), torch, flush, dist)
         out[name] = dict(wl=wl, ms=ms, stages=stages, N=N, touched=touched, e2e_ms=e2e_ms / args.steps,
+                         gemm_clock_mhz=run.clock_mhz,
                          e2e_pipe_ms=e2e_pipe_ms / args.steps, h2d=h2d, d2h=d2h, ms_flushed=ms_flushed,
                          entry="moe_layer_forward_q4_host" if name == "decode_q4" else "moe_layer_forward_host")
         del run
@@ -684,7 +703,8 @@ def run_ours(args):
         tr = traffic_record("expert_gemm_pair_kernel<0,2>", "prefill")
         value = weak_scaling_value(world, wl.T, p["ms"])
         tflops = flops_layer / (p["ms"] * 1e-3) / 1e12
-        pre_clk = (clocks.get("by_region") or {}).get("prefill", {}).get("sm_mhz")
+        # the SM clock the gate/up GEMM ran at (in-kernel records), else NVML's median
+        pre_clk = p["gemm_clock_mhz"].get("gemm1") or (clocks.get("by_region") or {}).get("prefill", {}).get("sm_mhz")
         dec = stage_report(out["decode"]["wl"], out["decode"], world, peaks,
                            "gate/up-projection GEMM (SwiGLU fused)", "expert_gemm_kernel<2,16>", "decode")
         dec_q4 = stage_report(out["decode_q4"]["wl"], out["decode_q4"], world, peaks,
@@ -703,7 +723,9 @@ def run_ours(args):
             stage_ms=p["stages"],
             roofline=dict(bound="tensor", kernel="gate/up-projection GEMM (SwiGLU fused)", achieved=achieved_tf,
                           peak=peak_tf, unit="TFLOP/s", frac=achieved_tf / peak_tf, traffic=tr,
-                          achieved_per_ghz=achieved_tf / (pre_clk / 1000.0) if pre_clk else None,
+                          sm_mhz_in_kernel=p["gemm_clock_mhz"].get("gemm1"),
+                          frac_of_peak_at_that_clock=(achieved_tf / clock_peak_tflops(p["gemm_clock_mhz"]["gemm1"])
+                                                      if p["gemm_clock_mhz"].get("gemm1") else None),
                           peak_source=f"{peaks['source']} bf16 dense "
                                       f"({'sustained' if long_run else 'burst'})"),
             e2e=dict(value=weak_scaling_value(world, wl.T, p["e2e_ms"]), unit="tokens/s", h2d_bytes_per_step=p["h2d"],
@@ -761,6 +783,7 @@ def run_sweep(args):
             ms = time_steps(run.step, args.steps, torch) / args.steps
         stages = run.profiled(args.steps)
         flops = 6.0 * N * wl.d * wl.f + 2.0 * wl.T * wl.d * wl.E
+        g1_mhz = run.clock_mhz.get("gemm1")
         wbytes = touched * 3 * wl.d * wl.f * 2
         bytes_ = wbytes + 2 * wl.T * wl.d * 2 + wl.E * wl.d * 4 + 2 * N * wl.f * 2 + 2 * N * wl.d * 2
         tfs = flops / (ms * 1e-3) / 1e12
@@ -768,7 +791,9 @@ def run_sweep(args):
         line = dict(workload=workload_desc(wl), T=wl.T, kept_slots=N, experts_touched=touched,
                     ms_per_step=ms, tokens_per_s=wl.T / (ms * 1e-3), tflops=tfs, gbs=gbs,
                     frac_bf16_burst=tfs / peaks["bf16"], frac_hbm=gbs / peaks["hbm"], stage_ms=stages,
-                    peaks_source=peaks["source"])
+                    gemm_clock_mhz=run.clock_mhz, peaks_source=peaks["source"],
+                    gemm1_frac_of_peak_at_its_clock=(4.0 * N * wl.d * wl.f / (stages["gemm1_swiglu"] * 1e-3) / 1e12
+                                                     / clock_peak_tflops(g1_mhz)) if g1_mhz else None)
         if hasattr(sampler, "samples"):
             rows = [r for r in sampler.samples if r[0] == tag]
             line["clocks"] = sampler._summary(rows)

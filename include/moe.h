@@ -237,7 +237,13 @@ MOE_API moe_status moe_layer_forward(const moe_shape *shape, const moe_bf16 *x, 
  *   [2] after capacity selection and grouping by expert
  *   [3] after the gate/up-projection GEMM (SiLU * mul fused)
  *   [4] after the down-projection GEMM    [5] after the combine.
- * Same arguments and results as moe_layer_forward otherwise. */
+ * The two expert GEMMs also record, from their first CTA, the SM cycle
+ * counter and the global nanosecond timer at entry and exit: 64-bit words
+ * at byte 64 of ws, {cycles, ns} at entry then at exit for the gate/up GEMM
+ * (bytes 64 .. 95) and for the down GEMM (96 .. 127); (cycles difference) /
+ * (ns difference) is the SM clock in GHz the GEMM ran at.  The kernels after
+ * the router are not chained by programmatic launch here (the events sit
+ * between them).  Same arguments and results as moe_layer_forward otherwise. */
 MOE_API moe_status moe_layer_forward_profiled(const moe_shape *shape, const moe_bf16 *x,
                                               const float *Wg, const moe_bf16 *W1,
                                               const moe_bf16 *W3, const moe_bf16 *W2, moe_bf16 *y,
@@ -444,7 +450,8 @@ MOE_API moe_status moe_layer_forward_q4_host(const moe_shape *shape, const moe_b
                                              size_t ws_bytes, moe_stream_t stream);
 
 /* moe_layer_forward_q4 recording six CUDA events (cudaEvent_t) on `stream`
- * between its stages, as moe_layer_forward_profiled. */
+ * between its stages and the GEMMs' clock records in ws, as
+ * moe_layer_forward_profiled. */
 MOE_API moe_status moe_layer_forward_q4_profiled(const moe_shape *shape, const moe_bf16 *x,
                                                  const float *Wg, const uint8_t *W1c,
                                                  const moe_bf16 *W1s, const uint8_t *W3c,

@@ -64,6 +64,7 @@ struct GemmParams {
   int32_t kb_per_split;
   uint32_t* tile_counter;  // CTA-pair kernels: next tile id (zero before the launch)
   int64_t S;               // rows of the activation and output buffers (T * k)
+  uint64_t* clock_probe;   // profiled calls: CTA 0 writes {clock64, globaltimer} at entry and exit, else nullptr
   int32_t prefetch_kb;     // streaming kernels launched as dependents: K chunks of the
                            // first tile's weights to prefetch into L2 before waiting (0: none)
 };
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = bars + 2 * STAGES + 4;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (p.clock_probe && blockIdx.x == 0 && tid == 0) probe_clock(p.clock_probe);
 
   if (tid == 0) {
     tma_prefetch_desc(&map_act);
@@ -443,6 +445,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (p.clock_probe && blockIdx.x == 0 && tid == 0) probe_clock(p.clock_probe + 2);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
@@ -541,6 +544,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* ring_empty = ring_full + kRing;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (p.clock_probe && blockIdx.x == 0 && tid == 0) probe_clock(p.clock_probe);
   const uint32_t rank = cluster_ctarank();
 
   if (tid == 0) {
@@ -815,6 +819,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   cluster_sync();
+  if (p.clock_probe && blockIdx.x == 0 && tid == 0) probe_clock(p.clock_probe + 2);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, 512);
@@ -963,6 +968,7 @@ static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.splits = 1;
   p1.kb_per_split = p1.num_kb;
   p1.prefetch_kb = a.pdl ? prefetch_chunks(a.num_sms) : 0;
+  p1.clock_probe = a.clock_probe;
   cudaError_t err = launch_one<EPI_STREAM_SWIGLU, BN>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl);
   if (err != cudaSuccess) return err;
   if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
@@ -981,6 +987,7 @@ static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
   p2.splits = (p2.num_kb + p2.kb_per_split - 1) / p2.kb_per_split;
   const bool pdl2 = a.pdl && !a.between;
   p2.prefetch_kb = pdl2 ? prefetch_chunks(a.num_sms) : 0;
+  p2.clock_probe = a.clock_probe ? a.clock_probe + 4 : nullptr;
   return launch_one<EPI_STREAM_PARTIAL, BN>(mh, mw2, mw2, p2, a.num_sms, s, pdl2);
 }
 
@@ -1004,6 +1011,7 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.splits = 1;
   p1.kb_per_split = p1.num_kb;
   p1.tile_counter = a.tile_counters;
+  p1.clock_probe = a.clock_probe;
   // two 64-element K chunks per pipeline stage (3 stages): half the handshakes
   cudaError_t err = a.pair ? launch_pair<EPI_TILED_SWIGLU, 2>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl)
                            : launch_one<EPI_TILED_SWIGLU, 256>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl);
@@ -1022,6 +1030,7 @@ static cudaError_t launch_tiled(const ExpertGemmArgs& a, cudaStream_t s) {
   p2.splits = 1;
   p2.kb_per_split = p2.num_kb;
   p2.tile_counter = a.tile_counters + 1;
+  p2.clock_probe = a.clock_probe ? a.clock_probe + 4 : nullptr;
   const bool pdl2 = a.pdl && !a.between;
   return a.pair ? launch_pair<EPI_TILED_STORE, 2>(mh, mw2, mw2, p2, a.num_sms, s, pdl2)
                 : launch_one<EPI_TILED_STORE, 256>(mh, mw2, mw2, p2, a.num_sms, s, pdl2);

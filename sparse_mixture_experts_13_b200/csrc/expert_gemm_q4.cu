@@ -97,6 +97,7 @@ struct Q4Params {
   int32_t splits;
   int32_t kq_per_split;
   int64_t S;            // rows of the activation and output buffers (T * k)
+  uint64_t* clock_probe;  // profiled calls: CTA 0 writes {clock64, globaltimer} at entry and exit
 };
 
 struct Q4Tile {
@@ -186,6 +187,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
   uint64_t* drain_bar = tfull_bar + 4;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (p.clock_probe && blockIdx.x == 0 && tid == 0) probe_clock(p.clock_probe);
 
   if (tid == 0) {
     tma_prefetch_desc(&map_act);
@@ -482,6 +484,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (p.clock_probe && blockIdx.x == 0 && tid == 0) probe_clock(p.clock_probe + 2);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
@@ -596,6 +599,7 @@ cudaError_t launch_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
   p1.offsets = a.offsets;
   p1.status = a.status;
   p1.S = a.S;
+  p1.clock_probe = a.clock_probe;
   p1.out = a.h;
   p1.out_ld = a.f;
   p1.E = a.E;
@@ -611,6 +615,7 @@ cudaError_t launch_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
   p2.offsets = a.offsets;
   p2.status = a.status;
   p2.S = a.S;
+  p2.clock_probe = a.clock_probe ? a.clock_probe + 4 : nullptr;
   p2.out = a.partials;
   p2.out_ld = a.d;
   p2.part_stride = a.S * (int64_t)a.d;

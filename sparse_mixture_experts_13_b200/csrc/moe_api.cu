@@ -23,6 +23,10 @@ constexpr bool kDebugBuild = true;
 #else
 constexpr bool kDebugBuild = false;
 #endif
+// Profiled calls: the two expert GEMMs each write {clock64, globaltimer} of
+// CTA 0 at entry and exit here (bytes 64 .. 127 of the control header, which
+// the layer clears at the start of every call).
+constexpr size_t kClockProbeOffset = 64;
 constexpr size_t kGuard = 256;        // debug build: guard bytes after each region past the control region
 constexpr int kMaxGuards = 32;
 #ifdef MOE_DEBUG
@@ -251,6 +255,9 @@ moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_per
                      void* ws, int num_sms, cudaStream_t s, cudaEvent_t between = nullptr, bool pdl = false) {
   ExpertGemmArgs a{};
   a.pdl = pdl;
+  // profiled calls (events between the kernels): clock records in the
+  // control header's spare bytes 64 .. 127
+  a.clock_probe = between ? at<uint64_t>(ws, L.status + kClockProbeOffset) : nullptr;
   a.offsets = offsets;
   a.x_perm = x_perm;
   a.W1 = W1;
@@ -286,6 +293,7 @@ moe_status run_gemms_q4(const moe_shape* sh, const Layout& L, const moe_bf16* x_
                         cudaEvent_t between = nullptr, bool pdl = false) {
   ExpertGemmQ4Args a{};
   a.pdl = pdl;
+  a.clock_probe = between ? at<uint64_t>(ws, L.status + kClockProbeOffset) : nullptr;
   a.offsets = offsets;
   a.x_perm = x_perm;
   a.W1c = W.W1c;

@@ -103,6 +103,7 @@ struct ExpertGemmArgs {
   bool pair;                // tiled variant: CTA-pair (cta_group::2) kernels
   uint32_t* tile_counters;  // [2] tile counters of the pair kernels, zeroed by the caller
   bool pdl;                 // launched as dependents of the grouping kernel (no event in between)
+  uint64_t* clock_probe;    // profiled calls: [8] clock records of the two GEMMs, else nullptr
 };
 // Streaming-variant parameters chosen from host-known sizes.
 void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,
@@ -131,6 +132,7 @@ struct ExpertGemmQ4Args {
   int num_sms;
   cudaEvent_t between;      // recorded after the first GEMM if not null
   bool pdl;                 // launched as dependents of the grouping kernel (no event in between)
+  uint64_t* clock_probe;    // profiled calls: [8] clock records of the two GEMMs, else nullptr
 };
 void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits);
 // number of K splits the down projection really uses for a requested count

@@ -178,34 +178,28 @@ constexpr int kRegMaxThreads = 512;  // d <= 8 * 512
 constexpr int kRegSlots = 4;         // ring depth, in groups of TB token rows
 constexpr int kRegMaxWarps = kRegMaxThreads / 32;
 
-// acc[8] of every lane -> the warp's sum of expert expert_of_lane(lane), exact
-// on lanes with (lane & 3) == 0.  Halving exchanges (16, 8, 4) hand half of
-// the remaining experts to the partner lane; two more steps finish the sum.
-__device__ __forceinline__ float warp_reduce_scatter8(const float (&acc)[8], int lane) {
-  const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4;
-  float v4[4];
+// a[V] (V a power of two, 8 <= V <= 32) of every lane -> the warp's sum of
+// value lane >> log2(32 / V), exact on every lane.  Halving exchanges with
+// masks 16, 8, ... (log2 V of them) hand the partner the half of the values
+// this lane gives up; each step's V / 2^s exchanges are independent, so the
+// steps pipeline.  Masks left below the last halving step are plain sums.
+template <int V>
+__device__ __forceinline__ float warp_transpose_reduce(float (&a)[V], int lane) {
+  int m = 16;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float send = b16 ? acc[j] : acc[j + 4];
-    const float keep = b16 ? acc[j + 4] : acc[j];
-    v4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-  }
-  float v2[2];
+  for (int n = V / 2; n >= 1; n /= 2, m /= 2) {
+    const bool up = lane & m;
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const float send = b8 ? v4[j] : v4[j + 2];
-    const float keep = b8 ? v4[j + 2] : v4[j];
-    v2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    for (int j = 0; j < n; ++j) {
+      const float send = up ? a[j] : a[j + n];
+      const float keep = up ? a[j + n] : a[j];
+      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
   }
-  const float send = b4 ? v2[0] : v2[1];
-  float v = (b4 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
-  v += __shfl_xor_sync(0xffffffffu, v, 2);
-  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  float v = a[0];
+#pragma unroll
+  for (; m >= 1; m /= 2) v += __shfl_xor_sync(0xffffffffu, v, m);
   return v;
-}
-
-__device__ __forceinline__ int expert_of_lane(int lane) {
-  return ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
 }
 
 // Dynamic shared memory of router_reg_kernel<TB> for rows of d bf16.
@@ -276,13 +270,14 @@ __global__ void __launch_bounds__(kRegMaxThreads, 1) router_reg_kernel(RouterArg
     if (ok) ok = mbar_wait(&bars[slot], (uint32_t)((i / kRegSlots) & 1), nullptr);
     float* part = s_part + (i & 1) * TB * kRegMaxWarps * 8;
     const uint8_t* rows = ring + (size_t)slot * TB * row_bytes;
+    // this thread's partial logits of the group's tokens: value tb * 8 + e
+    float acc[8 * TB];
 #pragma unroll
-    for (int tb = 0; tb < TB; ++tb) {
-      if (tb < nt) {
-        float acc[8];
+    for (int j = 0; j < 8 * TB; ++j) acc[j] = 0.f;
+    if (active) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        if (active) {
+      for (int tb = 0; tb < TB; ++tb) {
+        if (tb < nt) {
           // even and odd inputs accumulate in the two halves of a packed pair
           const uint4 v = *reinterpret_cast<const uint4*>(rows + tb * row_bytes + tid * 16);
           const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
@@ -299,12 +294,17 @@ __global__ void __launch_bounds__(kRegMaxThreads, 1) router_reg_kernel(RouterArg
           for (int e = 0; e < 8; ++e) {
             float lo, hi;
             unpack_f32x2(acc2[e], lo, hi);
-            acc[e] = lo + hi;
+            acc[tb * 8 + e] = lo + hi;
           }
         }
-        const float r = warp_reduce_scatter8(acc, lane);
-        if ((lane & 3) == 0) part[(tb * kRegMaxWarps + warp) * 8 + expert_of_lane(lane)] = r;
       }
+    }
+    // the warp's sums of all TB x 8 values at once; value j on lanes j << shift
+    {
+      constexpr int kShift = TB == 4 ? 0 : (TB == 2 ? 1 : 2);
+      const float r = warp_transpose_reduce<8 * TB>(acc, lane);
+      const int j = lane >> kShift, tb = j >> 3;
+      if ((lane & ((1 << kShift) - 1)) == 0 && tb < nt) part[(tb * kRegMaxWarps + warp) * 8 + (j & 7)] = r;
     }
     if (!__syncthreads_and(ok)) {
       // a row copy never arrived: report, let the copies still in flight land, leave

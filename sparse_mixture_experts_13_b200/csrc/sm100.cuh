@@ -19,6 +19,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// p[0] = this SM's cycle counter, p[1] = the global nanosecond timer: two
+// such records around a kernel give the SM clock it ran at.
+__device__ __forceinline__ void probe_clock(uint64_t* p) {
+  p[0] = (uint64_t)clock64();
+  p[1] = globaltimer_ns();
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

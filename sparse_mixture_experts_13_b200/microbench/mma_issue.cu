@@ -1,11 +1,12 @@
 // Issue cost of tcgen05.mma at the small N of the decode GEMMs.
 //
-// One CTA of 16 warps on one SM.  Thread 0 issues `iters` MMAs back to back
-// into one accumulator (M = 128 rows, N token columns), with a
-// tcgen05.commit after every `commit_every` of them, and reads clock64 before
-// and after issuing and once the last commit has arrived.  Optional busy
-// warps run a fused multiply-add loop at the same time, each on the
-// scheduler of warp (index % 4); warp 4k shares the issuing thread's.
+// One CTA of 16 warps on one SM.  Thread 0 (warp 0, scheduler 0) issues
+// `iters` MMAs back to back into one accumulator (M = 128 rows, N token
+// columns), with a tcgen05.commit after every `commit_every` of them (to one
+// mbarrier, or to a ring of four), and reads clock64 before and after issuing
+// and once the last commit has arrived.  Optional busy warps run a fused
+// multiply-add loop meanwhile: `busy` of them on each scheduler whose bit is
+// set in `smsp_mask` (warp w runs on scheduler w % 4).
 //
 // Kinds: 0 = kind::f16 with bf16 A and B (K = 16 per instruction),
 //        1 = kind::i8 with signed 8-bit A and B (K = 32 per instruction).
@@ -73,9 +74,11 @@ struct Result {
 };
 
 template <int KIND, bool A_TMEM>
-__global__ void __launch_bounds__(kThreads, 1) issue_kernel(int n, int iters, int commit_every, int busy, Result* out) {
+__global__ void __launch_bounds__(kThreads, 1) issue_kernel(int n, int iters, int commit_every, int busy,
+                                                             int smsp_mask, int ring, Result* out) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bars[4];
+  __shared__ uint64_t fin;  // warm-up and final drain only: exactly two phases
   __shared__ uint32_t tbase_s;
   __shared__ volatile int done;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -83,7 +86,8 @@ __global__ void __launch_bounds__(kThreads, 1) issue_kernel(int n, int iters, in
   uint8_t* sb = smem + kSmemA;
   for (int i = tid; i < (kSmemA + kSmemB) / 16; i += kThreads) reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
   if (tid == 0) {
-    mbar_init(&bar, 1);
+    for (int b = 0; b < 4; ++b) mbar_init(&bars[b], 1);
+    mbar_init(&fin, 1);
     fence_barrier_init();
     done = 0;
   }
@@ -119,28 +123,31 @@ __global__ void __launch_bounds__(kThreads, 1) issue_kernel(int n, int iters, in
         else mma_i8_ss(tbase, ad + koff, bd + koff, idesc, acc);
       }
     };
+    uint32_t uses[4] = {0, 0, 0, 0};
+    auto commit = [&](int b) {
+      umma_commit(&bars[b]);
+      ++uses[b];
+      ++commits;
+    };
     for (int i = 0; i < 64; ++i) one(i);  // warm-up
-    umma_commit(&bar);
-    ++commits;
-    bool ok = mbar_wait(&bar, (commits - 1) & 1, nullptr);
+    umma_commit(&fin);
+    bool ok = mbar_wait(&fin, 0, nullptr);
     const long long t0 = clock64();
     for (int i = 0; i < iters; ++i) {
       one(i + 1);
-      if (commit_every > 0 && (i + 1) % commit_every == 0) {
-        umma_commit(&bar);
-        ++commits;
-      }
+      if (commit_every > 0 && (i + 1) % commit_every == 0) commit(ring ? (int)(commits % 4) : 0);
     }
     const long long t1 = clock64();
-    umma_commit(&bar);
-    ++commits;
-    ok = mbar_wait(&bar, (commits - 1) & 1, nullptr) && ok;
+    // commits complete in order, so this one arriving means every MMA is done
+    // (the loop's barriers may be several phases behind and are not waited on)
+    umma_commit(&fin);
+    ok = mbar_wait(&fin, 1, nullptr) && ok;
     const long long t2 = clock64();
     out->issue = t1 - t0;
     out->total = t2 - t0;
     out->status = ok ? 0u : kStatusTimeout;
     done = 1;
-  } else if (warp >= 4 && warp < 4 + busy) {
+  } else if (warp >= 4 && ((smsp_mask >> (warp & 3)) & 1) && (warp - 4) / 4 < busy) {
     // fused multiply-adds until the issuing thread is done (bounded)
     float a0 = tid, a1 = tid + 1, a2 = tid + 2, a3 = tid + 3;
     long long it = 0;
@@ -163,20 +170,20 @@ __global__ void __launch_bounds__(kThreads, 1) issue_kernel(int n, int iters, in
 }
 
 template <int KIND, bool A_TMEM>
-int run(int n, int iters, int commit_every, int busy, Result* dres) {
+int run(int n, int iters, int commit_every, int busy, Result* dres, int smsp_mask = 0xF, int ring = 0) {
   const int smem = kSmemA + kSmemB + 1024;
   if (cudaFuncSetAttribute(issue_kernel<KIND, A_TMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
   cudaMemset(dres, 0, sizeof(Result));
-  issue_kernel<KIND, A_TMEM><<<1, kThreads, smem>>>(n, iters, commit_every, busy, dres);
+  issue_kernel<KIND, A_TMEM><<<1, kThreads, smem>>>(n, iters, commit_every, busy, smsp_mask, ring, dres);
   if (cudaDeviceSynchronize() != cudaSuccess) return 2;
   Result r;
   cudaMemcpy(&r, dres, sizeof(r), cudaMemcpyDeviceToHost);
   const int K = KIND == 0 ? 16 : 32;
   printf("{\"kind\": \"%s\", \"a\": \"%s\", \"M\": 128, \"N\": %d, \"K\": %d, \"iters\": %d, \"commit_every\": %d, "
-         "\"busy_warps\": %d, \"issue_cycles_per_mma\": %.2f, \"cycles_per_mma\": %.2f, \"weights_per_kcycle\": %.1f, "
-         "\"status\": %u}\n",
-         KIND == 0 ? "f16(bf16)" : "i8(s8)", A_TMEM ? "tmem" : "smem", n, K, iters, commit_every, busy,
+         "\"commit_ring\": %d, \"busy_per_scheduler\": %d, \"busy_scheduler_mask\": %d, "
+         "\"issue_cycles_per_mma\": %.2f, \"cycles_per_mma\": %.2f, \"weights_per_kcycle\": %.1f, \"status\": %u}\n",
+         KIND == 0 ? "f16(bf16)" : "i8(s8)", A_TMEM ? "tmem" : "smem", n, K, iters, commit_every, ring, busy, smsp_mask,
          (double)r.issue / iters, (double)r.total / iters, 128.0 * K * 1000.0 / ((double)r.total / iters), r.status);
   return r.status != 0 ? 3 : 0;
 }
@@ -195,11 +202,18 @@ int main(int argc, char** argv) {
     rc |= run<1, false>(n, iters, 0, 0, d);
     rc |= run<1, true>(n, iters, 0, 0, d);
   }
-  // the decode kernels' situation: one commit per stage, busy warps beside the issuer
-  for (int busy : {0, 4, 12}) {
-    rc |= run<0, true>(16, iters, 8, busy, d);
-    rc |= run<1, true>(32, iters, 4, busy, d);
-    rc |= run<1, true>(16, iters, 4, busy, d);
+  // commits: one barrier, or a ring of four barriers
+  for (int ce : {1, 4, 16, 64}) {
+    rc |= run<1, true>(32, iters, ce, 0, d, 0xF, 0);
+    rc |= run<1, true>(32, iters, ce, 0, d, 0xF, 1);
+  }
+  // busy warps: on every scheduler, or only on the three the issuer does not use
+  for (int busy : {1, 3}) {
+    for (int mask : {0xF, 0xE}) {
+      rc |= run<1, true>(32, iters, 0, busy, d, mask, 0);
+      rc |= run<1, true>(32, iters, 4, busy, d, mask, 1);
+      rc |= run<0, true>(16, iters, 8, busy, d, mask, 1);
+    }
   }
   cudaFree(d);
   return rc;

@@ -83,6 +83,17 @@ def test_host_buffers_tiny_against_oracle():
     H.assert_close(H.bf16_f64(_host_bits(y_host)), ref, "y (host buffers)")
 
 
+def _check_clock_records(ws):
+    """The two expert GEMMs' {cycles, ns} records at entry and exit (bytes
+    64 .. 127 of the workspace) give a plausible SM clock."""
+    rec = ws[64:128].view(torch.int64).cpu().numpy()
+    for g in (0, 4):
+        c0, n0, c1, n1 = (int(v) for v in rec[g:g + 4])
+        assert c1 > c0 and n1 > n0, rec
+        mhz = (c1 - c0) / (n1 - n0) * 1e3
+        assert 300.0 < mhz < 3000.0, mhz
+
+
 def _check_events(evs):
     torch.cuda.synchronize()
     gaps = [evs[i].elapsed_time(evs[i + 1]) for i in range(5)]
@@ -107,6 +118,7 @@ def test_profiled_equals_layer(name, variant):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
     assert np.array_equal(H.bf16_host(y), ref), (name, variant)
     _check_events(evs)
+    _check_clock_records(ws)
 
 
 @pytest.mark.parametrize("name", ["tiny", "cap_by_prob"])
@@ -124,6 +136,7 @@ def test_q4_profiled_equals_q4_layer(name):
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
     assert np.array_equal(H.bf16_host(y), ref), name
     _check_events(evs)
+    _check_clock_records(ws)
 
 
 @pytest.mark.parametrize("name", ["tiny", "cap_by_prob"])
