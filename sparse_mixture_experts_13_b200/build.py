@@ -19,7 +19,7 @@ LIB = os.path.join(PKG, "libmoe.so")
 # debug build: -DMOE_DEBUG (device-side bounds checks, workspace guards,
 # stage-failure hook), objects in _build/debug
 LIB_DEBUG = os.path.join(PKG, "libmoe_debug.so")
-SOURCES = ["router.cu", "permute.cu", "expert_gemm.cu", "expert_gemm_q4.cu", "router_stats.cu", "fallback.cu", "ep.cu", "combine.cu", "moe_api.cu", "selftest.cu"]
+SOURCES = ["router.cu", "permute.cu", "expert_gemm.cu", "expert_gemm_q4.cu", "expert_gemm_q4i8.cu", "router_stats.cu", "fallback.cu", "ep.cu", "combine.cu", "moe_api.cu", "selftest.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -146,7 +146,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // (code - 8) * s for the two codes in bits 0..3 and 16..19 of `bits`.
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t bits, __nv_bfloat162 s2) {
@@ -536,6 +535,8 @@ __global__ void __launch_bounds__(256) quantize_q4_kernel(const uint4* __restric
   }
 }
 
+}  // namespace
+
 // codes [E, R, K/2] as a 3-D uint8 map, box {64 bytes, box_rows, 1}, 64-byte swizzle
 bool encode_codes(CUtensorMap* m, const void* base, int64_t E, int64_t R, int64_t K, int box_rows) {
   EncodeTiledFn enc = get_encode_tiled();
@@ -563,6 +564,8 @@ bool encode_scales(CUtensorMap* m, const void* base, int64_t E, int64_t R, int64
 }
 
 // token tile [S, K] bf16, box {64, box_rows}, 128-byte swizzle
+namespace {
+
 bool encode_tokens(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return false;
@@ -665,6 +668,8 @@ int32_t q4_effective_splits(int32_t f, int32_t splits) {
 }
 
 cudaError_t launch_expert_gemms_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
+  // token tiles of 16 and 32: the integer-MMA kernels (expert_gemm_q4i8.cu)
+  if (a.act_q && a.bn <= 32) return launch_expert_gemms_q4i8(a, s);
   switch (a.bn) {
     case 16: return launch_q4<16>(a, s);
     case 32: return launch_q4<32>(a, s);

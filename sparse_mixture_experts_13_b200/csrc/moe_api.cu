@@ -80,6 +80,7 @@ struct Layout {
   bool q4;                 // 4-bit expert weights (always the streaming schedule)
   int32_t bn, splits;      // streaming schedule: token tile, requested split-K count
   int32_t eff_splits;      // split-K partial buffers the down projection writes
+  size_t act_q, act_scale; // 4-bit, token tiles <= 32: quantised activations [2][S][max(d, f)] and scales [S]
   size_t guards[kMaxGuards];  // debug build: offsets of the guards
   int nguards;
 };
@@ -169,6 +170,12 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
     o = next_region(L, o + 4 * S);
     L.thresh2 = o;
     o = next_region(L, o + 8 * E);
+  }
+  if (L.q4 && L.bn <= 32) {
+    L.act_q = o;
+    o = next_region(L, o + 2 * (size_t)S * (size_t)(d > f ? d : f));
+    L.act_scale = o;
+    o = next_region(L, o + 4 * (size_t)S);
   }
   L.total = o;
   return L;
@@ -313,6 +320,10 @@ moe_status run_gemms_q4(const moe_shape* sh, const Layout& L, const moe_bf16* x_
   a.splits = L.splits;
   a.num_sms = num_sms;
   a.between = between;
+  if (L.act_q) {
+    a.act_q = at<int8_t>(ws, L.act_q);
+    a.act_scale = at<float>(ws, L.act_scale);
+  }
   return cuda_status(launch_expert_gemms_q4(a, s));
 }
 

@@ -133,7 +133,14 @@ struct ExpertGemmQ4Args {
   cudaEvent_t between;      // recorded after the first GEMM if not null
   bool pdl;                 // launched as dependents of the grouping kernel (no event in between)
   uint64_t* clock_probe;    // profiled calls: [8] clock records of the two GEMMs, else nullptr
+  int8_t* act_q;            // token tiles <= 32: quantised activations [2][S][max(d, f)] (high, low bytes)
+  float* act_scale;         // and their per-row scales [S]; nullptr: the bf16-dequantising kernels
 };
+// The integer-MMA 4-bit GEMMs (token tiles of 16 and 32).
+cudaError_t launch_expert_gemms_q4i8(const ExpertGemmQ4Args& a, cudaStream_t s);
+// Tensor maps of the 4-bit format (expert_gemm_q4.cu).
+bool encode_codes(CUtensorMap* m, const void* base, int64_t E, int64_t R, int64_t K, int box_rows);
+bool encode_scales(CUtensorMap* m, const void* base, int64_t E, int64_t R, int64_t K, int box_rows);
 void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits);
 // number of K splits the down projection really uses for a requested count
 int32_t q4_effective_splits(int32_t f, int32_t splits);

@@ -29,6 +29,8 @@
 #include <cfloat>
 #include <cstdint>
 
+#include <cuda_bf16.h>
+
 #include "moe_internal.h"
 #include "sm100.cuh"
 
@@ -345,6 +347,195 @@ static cudaError_t launch_router_reg(const RouterArgs& a, int num_sms, cudaStrea
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- tensor-core router
+// router_mma_kernel (E <= 8, d a multiple of 256 up to 4096): the logits of a
+// tile of 8 tokens by mma.sync m16n8k16 (bf16 operands, fp32 accumulation).
+// x is exact in bf16, and every fp32 weight is split exactly into three bf16
+// terms, w = hi + mid + lo (hi = bf16(w), mid = bf16(w - hi), lo = w - hi -
+// mid, which bf16 holds exactly: 8 + 8 + 8 significant bits), so the three
+// MMAs per 16 inputs multiply exactly by the fp32 weights and the products
+// add up in fp32.  Each of the 16 warps owns d/16 inputs and keeps its slice
+// of the three weight terms as MMA B fragments for the whole launch (hi and
+// mid in registers, lo in shared memory); the token rows arrive by TMA, boxes
+// of 64 inputs x 8 tokens with a
+// 128-byte swizzle read by ldmatrix, into a ring of two tiles.  The MMA's
+// rows 8..15 repeat rows 0..7 (ignored).  Per tile each warp leaves its 8 x 8
+// partial logits in shared memory; the partials are added in warp order and
+// warp t finishes token t.
+constexpr int kMmaTile = 8;     // tokens per tile
+constexpr int kMmaWarps = 16;
+constexpr int kMmaSlots = 2;
+constexpr int kMmaMaxSteps = 16;  // 16-input steps per warp (d <= 4096)
+
+__device__ __forceinline__ uint32_t bf16_bits(float v) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// w -> (hi, mid, lo) bf16 bits with hi + mid + lo == w exactly
+__device__ __forceinline__ void split3(float w, uint32_t& h, uint32_t& m, uint32_t& l) {
+  h = bf16_bits(w);
+  const float r1 = w - __uint_as_float(h << 16);
+  m = bf16_bits(r1);
+  const float r2 = r1 - __uint_as_float(m << 16);
+  l = bf16_bits(r2);
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__host__ __device__ constexpr size_t mma_slot_bytes(int d) { return (size_t)(d / 64) * 1024; }
+// lo fragments: [warp][step][lane] uint2
+__host__ __device__ constexpr size_t mma_lo_bytes(int d) { return (size_t)kMmaWarps * (d / (16 * kMmaWarps)) * 32 * 8; }
+__host__ __device__ constexpr size_t mma_smem_bytes(int d) {
+  return 1024 + kMmaSlots * mma_slot_bytes(d) + mma_lo_bytes(d) + sizeof(float) * 2 * kMmaWarps * kMmaTile * 8 +
+         sizeof(uint64_t) * kMmaSlots + sizeof(int) * 32;
+}
+
+__global__ void __launch_bounds__(kMmaWarps * 32, 1)
+    router_mma_kernel(const __grid_constant__ CUtensorMap map_x, RouterArgs a, int64_t ntiles) {
+  extern __shared__ uint8_t smem_raw[];
+  pdl_trigger();  // the grouping kernel may launch now; it waits for this grid
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int d = a.d, E = a.E;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t slot_bytes = mma_slot_bytes(d);
+  uint2* s_lo = reinterpret_cast<uint2*>(smem + kMmaSlots * slot_bytes);     // [warps][steps][32]
+  float* s_part = reinterpret_cast<float*>(smem + kMmaSlots * slot_bytes + mma_lo_bytes(d));  // [2][warps][8][8]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_part + 2 * kMmaWarps * kMmaTile * 8);
+  int* s_count = reinterpret_cast<int*>(bars + kMmaSlots);
+
+  const int64_t g0 = blockIdx.x, gstride = gridDim.x;
+  const int64_t my_tiles = g0 < ntiles ? (ntiles - 1 - g0) / gstride + 1 : 0;
+  const int nbox = d / 64;
+  if (tid < 32) s_count[tid] = 0;
+  if (tid == 0) {
+    tma_prefetch_desc(&map_x);
+    for (int i = 0; i < kMmaSlots; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int64_t j) {  // this block's j-th tile into slot j % 2
+    const int32_t t0 = (int32_t)((g0 + j * gstride) * kMmaTile);
+    uint8_t* dst = smem + (size_t)(j % kMmaSlots) * slot_bytes;
+    uint64_t* bar = &bars[j % kMmaSlots];
+    mbar_arrive_expect_tx(bar, (uint32_t)slot_bytes);  // rows past T are zero-filled and counted
+    for (int b = 0; b < nbox; ++b) tma_load_2d(&map_x, bar, dst + (size_t)b * 1024, b * 64, t0);
+  };
+  if (tid == 0)
+    for (int64_t j = 0; j < my_tiles && j < kMmaSlots; ++j) issue(j);
+
+  // B fragments of this warp's inputs: lane l holds expert l / 4 at inputs
+  // 2 (l % 4) + {0, 1} and + {8, 9} of each 16-input step
+  const int steps = d / (16 * kMmaWarps);
+  const int n = lane >> 2, kq = 2 * (lane & 3);
+  uint32_t bh[kMmaMaxSteps][2], bm[kMmaMaxSteps][2];
+  uint2* my_lo = s_lo + (size_t)warp * steps * 32 + lane;
+#pragma unroll
+  for (int ks = 0; ks < kMmaMaxSteps; ++ks) {
+    float w[4] = {0.f, 0.f, 0.f, 0.f};
+    if (ks < steps && n < E) {
+      const float* row = a.Wg + (int64_t)n * d + warp * (steps * 16) + ks * 16 + kq;
+      const float2 u = *reinterpret_cast<const float2*>(row);
+      const float2 v = *reinterpret_cast<const float2*>(row + 8);
+      w[0] = u.x; w[1] = u.y; w[2] = v.x; w[3] = v.y;
+    }
+    uint32_t h[4], m[4], lo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) split3(w[q], h[q], m[q], lo[q]);
+    bh[ks][0] = h[0] | (h[1] << 16);
+    bh[ks][1] = h[2] | (h[3] << 16);
+    bm[ks][0] = m[0] | (m[1] << 16);
+    bm[ks][1] = m[2] | (m[3] << 16);
+    if (ks < steps) my_lo[ks * 32] = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+  }
+  __syncwarp();
+  // ldmatrix rows: thread l addresses row l % 8 of matrix l / 8 (matrices 0, 1:
+  // inputs 0..7 of the step, 2, 3: inputs 8..15; rows 8..15 of the MMA repeat
+  // rows 0..7)
+  const int lr = lane & 7, lhalf = (lane >> 4) & 1;
+
+  bool ok = true;
+  for (int64_t j = 0; j < my_tiles; ++j) {
+    const int slot = (int)(j % kMmaSlots);
+    const int64_t t0 = (g0 + j * gstride) * kMmaTile;
+    if (ok) ok = mbar_wait(&bars[slot], (uint32_t)((j / kMmaSlots) & 1), nullptr);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    if (ok) {
+      const uint32_t base = smem_u32(smem + (size_t)slot * slot_bytes);
+#pragma unroll
+      for (int ks = 0; ks < kMmaMaxSteps; ++ks) {
+        if (ks < steps) {
+          const int k0 = warp * (steps * 16) + ks * 16;     // first input of the step
+          const int chunk = ((k0 & 63) >> 3) + lhalf;       // 16-byte chunk within the 128-byte row
+          const uint32_t addr = base + (uint32_t)((k0 >> 6) * 1024 + lr * 128 + ((chunk ^ lr) << 4));
+          uint32_t af[4];
+          ldmatrix_x4(addr, af);
+          mma_bf16_16816(c, af, bh[ks][0], bh[ks][1]);
+          mma_bf16_16816(c, af, bm[ks][0], bm[ks][1]);
+          const uint2 bl = my_lo[ks * 32];
+          mma_bf16_16816(c, af, bl.x, bl.y);
+        }
+      }
+    }
+    // c[0], c[1]: token lane / 4, experts kq, kq + 1
+    float* part = s_part + (j & 1) * kMmaWarps * kMmaTile * 8;
+    *reinterpret_cast<float2*>(part + (warp * kMmaTile + n) * 8 + kq) = make_float2(c[0], c[1]);
+    if (!__syncthreads_and(ok)) {
+      // a tile never arrived: report, let the copies still in flight land, leave
+      if (tid == 0) {
+        record_status(a.status, kStatusTimeout);
+        for (int64_t q = j; q < my_tiles && q < j + kMmaSlots; ++q)
+          mbar_wait(&bars[q % kMmaSlots], (uint32_t)((q / kMmaSlots) & 1), nullptr, kWaitLimitNs / 8);
+      }
+      return;
+    }
+    if (tid == 0 && j + kMmaSlots < my_tiles) issue(j + kMmaSlots);
+    // warp w < 8 finishes token t0 + w: lane e < 8 adds the 16 warps' partials in warp order
+    if (warp < kMmaTile && t0 + warp < a.T) {
+      float v = 0.f;
+      if (lane < 8) {
+#pragma unroll
+        for (int ww = 0; ww < kMmaWarps; ++ww) v += part[(ww * kMmaTile + warp) * 8 + lane];
+      }
+      finish_token<8>(a, t0 + warp, v, lane, s_count);
+    }
+  }
+  __syncthreads();
+  if (tid < E && s_count[tid] != 0) atomicAdd(&a.counts[tid], s_count[tid]);
+}
+
+static cudaError_t launch_router_mma(const RouterArgs& a, int num_sms, cudaStream_t s) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return cudaErrorInvalidValue;
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)a.d, (cuuint64_t)a.T};
+  cuuint64_t strides[1] = {(cuuint64_t)a.d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kMmaTile};
+  cuuint32_t estr[2] = {1, 1};
+  if (enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = mma_smem_bytes(a.d);
+  cudaError_t err = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const int64_t ntiles = (a.T + kMmaTile - 1) / kMmaTile;
+  const int64_t grid = ntiles < num_sms ? ntiles : num_sms;
+  router_mma_kernel<<<(unsigned)grid, kMmaWarps * 32, smem, s>>>(m, a, ntiles);
+  return cudaGetLastError();
+}
+
 constexpr int64_t kFewTokens = 512;
 
 template <int EMAX>
@@ -364,6 +555,8 @@ cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s, bool
     cudaError_t err = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
     if (err != cudaSuccess) return err;
   }
+  if (a.E <= 8 && a.d % (16 * kMmaWarps) == 0 && a.d <= 16 * kMmaWarps * kMmaMaxSteps)
+    return launch_router_mma(a, num_sms, s);
   if (a.E <= 8 && a.d <= 8 * kRegMaxThreads) {
     // tokens per SM decide how many rows one ring slot carries
     const int64_t per_sm = (a.T + num_sms - 1) / num_sms;

@@ -76,10 +76,15 @@ def test_streaming_layout_adds_splitk_planes(moe, T, d, f):
     assert _splits(extra, T * 2, d) is not None, extra
 
 
-@pytest.mark.parametrize("T", [16, 300])
+@pytest.mark.parametrize("T", [16, 32, 33, 300])
 def test_q4_layout_always_has_splitk_planes(moe, T):
+    """The 4-bit layout adds split-K planes and, for token tiles of 16 and 32
+    (T <= 32, the integer-MMA kernels), the quantised activations [2][S][max(d,
+    f)] signed bytes and their scales [S] fp32 at the end."""
     sh = moe.make_shape(T, 4096, 14336)
     extra = moe.moe_workspace_size_q4(sh) - expected(T, 4096, 14336, 8, 2)
+    if T <= 32:
+        extra -= al(2 * T * 2 * 14336) + al(4 * T * 2)
     assert _splits(extra, T * 2, 4096) is not None, extra
 
 
