@@ -356,10 +356,10 @@ static cudaError_t launch_router_reg(const RouterArgs& a, int num_sms, cudaStrea
 // MMAs per 16 inputs multiply exactly by the fp32 weights and the products
 // add up in fp32.  Each of the 16 warps owns d/16 inputs and keeps its slice
 // of the three weight terms as MMA B fragments for the whole launch (hi and
-// mid in registers, lo in shared memory); the token rows arrive by TMA, boxes
-// of 64 inputs x 8 tokens with a
-// 128-byte swizzle read by ldmatrix, into a ring of two tiles.  The MMA's
-// rows 8..15 repeat rows 0..7 (ignored).  Per tile each warp leaves its 8 x 8
+// mid in registers, lo in shared memory); the token rows arrive by bulk
+// copies, one per row, into a ring of two tiles with rows 16 bytes further
+// apart than their length, and are read by ldmatrix.  The MMA's rows 8..15
+// repeat rows 0..7 (ignored).  Per tile each warp leaves its 8 x 8
 // partial logits in shared memory; the partials are added in warp order and
 // warp t finishes token t.
 constexpr int kMmaTile = 8;     // tokens per tile
@@ -394,7 +394,10 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__host__ __device__ constexpr size_t mma_slot_bytes(int d) { return (size_t)(d / 64) * 1024; }
+// a tile's rows in shared memory, 16 bytes more apart than a row, so the 8
+// rows that one ldmatrix reads fall in distinct bank groups
+__host__ __device__ constexpr size_t mma_row_pitch(int d) { return (size_t)d * 2 + 16; }
+__host__ __device__ constexpr size_t mma_slot_bytes(int d) { return (((size_t)kMmaTile * mma_row_pitch(d)) + 127) / 128 * 128; }
 // lo fragments: [warp][step][lane] uint2
 __host__ __device__ constexpr size_t mma_lo_bytes(int d) { return (size_t)kMmaWarps * (d / (16 * kMmaWarps)) * 32 * 8; }
 __host__ __device__ constexpr size_t mma_smem_bytes(int d) {
@@ -403,7 +406,7 @@ __host__ __device__ constexpr size_t mma_smem_bytes(int d) {
 }
 
 __global__ void __launch_bounds__(kMmaWarps * 32, 1)
-    router_mma_kernel(const __grid_constant__ CUtensorMap map_x, RouterArgs a, int64_t ntiles) {
+    router_mma_kernel(RouterArgs a, int64_t ntiles) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();  // the grouping kernel may launch now; it waits for this grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -417,20 +420,20 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
 
   const int64_t g0 = blockIdx.x, gstride = gridDim.x;
   const int64_t my_tiles = g0 < ntiles ? (ntiles - 1 - g0) / gstride + 1 : 0;
-  const int nbox = d / 64;
   if (tid < 32) s_count[tid] = 0;
   if (tid == 0) {
-    tma_prefetch_desc(&map_x);
     for (int i = 0; i < kMmaSlots; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
   }
   __syncthreads();
-  auto issue = [&](int64_t j) {  // this block's j-th tile into slot j % 2
-    const int32_t t0 = (int32_t)((g0 + j * gstride) * kMmaTile);
+  const size_t row_pitch = mma_row_pitch(d);
+  auto issue = [&](int64_t j) {  // this block's j-th tile into slot j % 2: one bulk copy per token row
+    const int64_t t0 = (g0 + j * gstride) * kMmaTile;
+    const int rows = (int)(a.T - t0 < kMmaTile ? a.T - t0 : kMmaTile);
     uint8_t* dst = smem + (size_t)(j % kMmaSlots) * slot_bytes;
     uint64_t* bar = &bars[j % kMmaSlots];
-    mbar_arrive_expect_tx(bar, (uint32_t)slot_bytes);  // rows past T are zero-filled and counted
-    for (int b = 0; b < nbox; ++b) tma_load_2d(&map_x, bar, dst + (size_t)b * 1024, b * 64, t0);
+    mbar_arrive_expect_tx(bar, (uint32_t)(rows * d * 2));
+    for (int r = 0; r < rows; ++r) bulk_load(dst + r * row_pitch, a.x + (t0 + r) * d, (uint32_t)(d * 2), bar);
   };
   if (tid == 0)
     for (int64_t j = 0; j < my_tiles && j < kMmaSlots; ++j) issue(j);
@@ -470,23 +473,27 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     const int slot = (int)(j % kMmaSlots);
     const int64_t t0 = (g0 + j * gstride) * kMmaTile;
     if (ok) ok = mbar_wait(&bars[slot], (uint32_t)((j / kMmaSlots) & 1), nullptr);
+    // three independent accumulators (one per weight term) keep the MMAs of
+    // a step from waiting on each other; they are added at the end
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     if (ok) {
+      float ch[4] = {}, cm[4] = {}, cl[4] = {};
       const uint32_t base = smem_u32(smem + (size_t)slot * slot_bytes);
 #pragma unroll
       for (int ks = 0; ks < kMmaMaxSteps; ++ks) {
         if (ks < steps) {
           const int k0 = warp * (steps * 16) + ks * 16;     // first input of the step
-          const int chunk = ((k0 & 63) >> 3) + lhalf;       // 16-byte chunk within the 128-byte row
-          const uint32_t addr = base + (uint32_t)((k0 >> 6) * 1024 + lr * 128 + ((chunk ^ lr) << 4));
+          const uint32_t addr = base + (uint32_t)(lr * row_pitch + k0 * 2 + lhalf * 16);
           uint32_t af[4];
           ldmatrix_x4(addr, af);
-          mma_bf16_16816(c, af, bh[ks][0], bh[ks][1]);
-          mma_bf16_16816(c, af, bm[ks][0], bm[ks][1]);
           const uint2 bl = my_lo[ks * 32];
-          mma_bf16_16816(c, af, bl.x, bl.y);
+          mma_bf16_16816(ch, af, bh[ks][0], bh[ks][1]);
+          mma_bf16_16816(cm, af, bm[ks][0], bm[ks][1]);
+          mma_bf16_16816(cl, af, bl.x, bl.y);
         }
       }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) c[q] = (ch[q] + cm[q]) + cl[q];
     }
     // c[0], c[1]: token lane / 4, experts kq, kq + 1
     float* part = s_part + (j & 1) * kMmaWarps * kMmaTile * 8;
@@ -516,23 +523,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
 }
 
 static cudaError_t launch_router_mma(const RouterArgs& a, int num_sms, cudaStream_t s) {
-  EncodeTiledFn enc = get_encode_tiled();
-  if (!enc) return cudaErrorInvalidValue;
-  CUtensorMap m;
-  cuuint64_t dims[2] = {(cuuint64_t)a.d, (cuuint64_t)a.T};
-  cuuint64_t strides[1] = {(cuuint64_t)a.d * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kMmaTile};
-  cuuint32_t estr[2] = {1, 1};
-  if (enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
   const size_t smem = mma_smem_bytes(a.d);
   cudaError_t err = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int64_t ntiles = (a.T + kMmaTile - 1) / kMmaTile;
   const int64_t grid = ntiles < num_sms ? ntiles : num_sms;
-  router_mma_kernel<<<(unsigned)grid, kMmaWarps * 32, smem, s>>>(m, a, ntiles);
+  router_mma_kernel<<<(unsigned)grid, kMmaWarps * 32, smem, s>>>(a, ntiles);
   return cudaGetLastError();
 }
 
