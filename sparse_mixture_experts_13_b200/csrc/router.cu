@@ -29,7 +29,6 @@
 #include <cfloat>
 #include <cstdint>
 
-#include <cuda_bf16.h>
 
 #include "moe_internal.h"
 #include "sm100.cuh"
@@ -351,8 +350,7 @@ static cudaError_t launch_router_reg(const RouterArgs& a, int num_sms, cudaStrea
 // router_mma_kernel (E <= 8, d a multiple of 256 up to 4096): the logits of a
 // tile of 8 tokens by mma.sync m16n8k16 (bf16 operands, fp32 accumulation).
 // x is exact in bf16, and every fp32 weight is split exactly into three bf16
-// terms, w = hi + mid + lo (hi = bf16(w), mid = bf16(w - hi), lo = w - hi -
-// mid, which bf16 holds exactly: 8 + 8 + 8 significant bits), so the three
+// terms, w = hi + mid + lo (8 + 8 + 8 significant bits, by truncation), so the three
 // MMAs per 16 inputs multiply exactly by the fp32 weights and the products
 // add up in fp32.  Each of the 16 warps owns d/16 inputs and keeps its slice
 // of the three weight terms as MMA B fragments for the whole launch (hi and
@@ -366,18 +364,19 @@ constexpr int kMmaTile = 8;     // tokens per tile
 constexpr int kMmaWarps = 16;
 constexpr int kMmaSlots = 2;
 constexpr int kMmaMaxSteps = 16;  // 16-input steps per warp (d <= 4096)
+constexpr int64_t kMmaMinTokens = 1024;
 
-__device__ __forceinline__ uint32_t bf16_bits(float v) {
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-
-// w -> (hi, mid, lo) bf16 bits with hi + mid + lo == w exactly
+// w -> (hi, mid, lo) bf16 bits with hi + mid + lo == w exactly: hi keeps the
+// top 8 significant bits of w (truncation), mid the next 8 of the remainder,
+// lo the rest (at most 8 bits, so bf16 holds it); both subtractions are exact
 __device__ __forceinline__ void split3(float w, uint32_t& h, uint32_t& m, uint32_t& l) {
-  h = bf16_bits(w);
-  const float r1 = w - __uint_as_float(h << 16);
-  m = bf16_bits(r1);
-  const float r2 = r1 - __uint_as_float(m << 16);
-  l = bf16_bits(r2);
+  const uint32_t wb = __float_as_uint(w);
+  h = wb >> 16;
+  const float r1 = w - __uint_as_float(wb & 0xFFFF0000u);
+  const uint32_t rb = __float_as_uint(r1);
+  m = rb >> 16;
+  const float r2 = r1 - __uint_as_float(rb & 0xFFFF0000u);
+  l = __float_as_uint(r2) >> 16;
 }
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -444,23 +443,36 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
   const int n = lane >> 2, kq = 2 * (lane & 3);
   uint32_t bh[kMmaMaxSteps][2], bm[kMmaMaxSteps][2];
   uint2* my_lo = s_lo + (size_t)warp * steps * 32 + lane;
+  // W_g comes from HBM at every launch: the loads of half the steps are
+  // issued together before any is split, so the warp waits for two memory
+  // round trips rather than one per step
+  constexpr int kHalf = kMmaMaxSteps / 2;
 #pragma unroll
-  for (int ks = 0; ks < kMmaMaxSteps; ++ks) {
-    float w[4] = {0.f, 0.f, 0.f, 0.f};
-    if (ks < steps && n < E) {
-      const float* row = a.Wg + (int64_t)n * d + warp * (steps * 16) + ks * 16 + kq;
-      const float2 u = *reinterpret_cast<const float2*>(row);
-      const float2 v = *reinterpret_cast<const float2*>(row + 8);
-      w[0] = u.x; w[1] = u.y; w[2] = v.x; w[3] = v.y;
+  for (int ph = 0; ph < 2; ++ph) {
+    float2 u[kHalf], v[kHalf];
+#pragma unroll
+    for (int q = 0; q < kHalf; ++q) {
+      const int ks = ph * kHalf + q;
+      u[q] = v[q] = make_float2(0.f, 0.f);
+      if (ks < steps && n < E) {
+        const float* row = a.Wg + (int64_t)n * d + warp * (steps * 16) + ks * 16 + kq;
+        u[q] = *reinterpret_cast<const float2*>(row);
+        v[q] = *reinterpret_cast<const float2*>(row + 8);
+      }
     }
-    uint32_t h[4], m[4], lo[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) split3(w[q], h[q], m[q], lo[q]);
-    bh[ks][0] = h[0] | (h[1] << 16);
-    bh[ks][1] = h[2] | (h[3] << 16);
-    bm[ks][0] = m[0] | (m[1] << 16);
-    bm[ks][1] = m[2] | (m[3] << 16);
-    if (ks < steps) my_lo[ks * 32] = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+    for (int q = 0; q < kHalf; ++q) {
+      const int ks = ph * kHalf + q;
+      const float w[4] = {u[q].x, u[q].y, v[q].x, v[q].y};
+      uint32_t h[4], m[4], lo[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) split3(w[c], h[c], m[c], lo[c]);
+      bh[ks][0] = h[0] | (h[1] << 16);
+      bh[ks][1] = h[2] | (h[3] << 16);
+      bm[ks][0] = m[0] | (m[1] << 16);
+      bm[ks][1] = m[2] | (m[3] << 16);
+      if (ks < steps) my_lo[ks * 32] = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+    }
   }
   __syncwarp();
   // ldmatrix rows: thread l addresses row l % 8 of matrix l / 8 (matrices 0, 1:
@@ -551,7 +563,9 @@ cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s, bool
     cudaError_t err = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
     if (err != cudaSuccess) return err;
   }
-  if (a.E <= 8 && a.d % (16 * kMmaWarps) == 0 && a.d <= 16 * kMmaWarps * kMmaMaxSteps)
+  // Many tokens: tensor cores (fewer instructions per token); few tokens: the
+  // register kernel, whose set-up (W_g into registers) is shorter.
+  if (a.T >= kMmaMinTokens && a.E <= 8 && a.d % (16 * kMmaWarps) == 0 && a.d <= 16 * kMmaWarps * kMmaMaxSteps)
     return launch_router_mma(a, num_sms, s);
   if (a.E <= 8 && a.d <= 8 * kRegMaxThreads) {
     // tokens per SM decide how many rows one ring slot carries

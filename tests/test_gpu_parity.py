@@ -184,6 +184,24 @@ def test_exact_logit_ties(o, variant):
     check_everything(o, wl, variant)
 
 
+def test_tensor_core_router_ties(o):
+    """1100 tokens at d=256 take the tensor-core router (T >= 1024, d a
+    multiple of 256), with a ragged last tile of 4 tokens: experts 2 and 3
+    tie exactly for many tokens (the smaller index wins), and zero rows pick
+    experts 0 and 1 with gates 1/2, as in the oracle."""
+    wl = synth.Workload("ties_mma", 1100, 256, 256, seed=9).generate()
+    wl.Wg[2] += 3.0 * np.abs(wl.Wg[2]).max()
+    wl.Wg[3] = wl.Wg[2]
+    wl.x[:10] = 0
+    g = H.run_stages(H.Device(wl), 1)
+    idx = g["idx"].cpu().numpy().reshape(1100, 2)
+    both = (idx == 2).any(1) & (idx == 3).any(1)
+    assert both.sum() > 100
+    assert np.all(idx[both, 0] == 2) and np.all(idx[both, 1] == 3)
+    assert np.all(idx[:10] == [0, 1]) and np.all(g["w"].cpu().numpy().reshape(1100, 2)[:10] == 0.5)
+    check_everything(o, wl, 1)
+
+
 def test_zero_input_ties():
     """x = 0: all logits are 0, the experts 0..k-1 are chosen, gates are 1/k
     and the output is exactly zero."""
@@ -248,7 +266,7 @@ def test_sweep(o, T):
 
 @pytest.mark.parametrize("E", [8, 16, 32])
 def test_router_many_tokens(o, E):
-    """More than 512 tokens take the shared-memory router (several tokens
-    per warp); cover it for each expert-count template."""
+    """700 tokens at d=128: the register router for E=8, the grouped router
+    with several tokens per block for E=16 and 32."""
     wl = synth.Workload(f"many{E}", 700, 128, 192, E=E, k=2, seed=E).generate()
     check_everything(o, wl, 1)
