@@ -641,8 +641,10 @@ void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sm
   else if (b > 16) b = 32;
   *bn = (int32_t)b;
   // split K of the down projection so that (experts x 128-row blocks x
-  // splits) tiles fill whole waves of the SMs as evenly as possible
-  const int32_t num_kq = (f + KQ - 1) / KQ;
+  // splits) tiles fill whole waves of the SMs as evenly as possible; K goes
+  // in stages of the kernel the token tile selects
+  const int32_t kq_inputs = b <= 32 ? q4i8_stage_inputs((int32_t)b) : KQ;
+  const int32_t num_kq = (f + kq_inputs - 1) / kq_inputs;
   const int64_t touched = T * k < E ? T * k : E;
   const int64_t base = touched * ((d + 127) / 128);
   int32_t best = 1;
@@ -661,8 +663,9 @@ void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sm
   *splits = best;
 }
 
-int32_t q4_effective_splits(int32_t f, int32_t splits) {
-  const int32_t num_kq = (f + KQ - 1) / KQ;
+int32_t q4_effective_splits(int32_t f, int32_t splits, int32_t bn) {
+  const int32_t kq_inputs = bn <= 32 ? q4i8_stage_inputs(bn) : KQ;
+  const int32_t num_kq = (f + kq_inputs - 1) / kq_inputs;
   const int32_t kps = (num_kq + splits - 1) / splits;
   return (num_kq + kps - 1) / kps;
 }

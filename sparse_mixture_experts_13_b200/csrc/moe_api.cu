@@ -80,7 +80,7 @@ struct Layout {
   bool q4;                 // 4-bit expert weights (always the streaming schedule)
   int32_t bn, splits;      // streaming schedule: token tile, requested split-K count
   int32_t eff_splits;      // split-K partial buffers the down projection writes
-  size_t act_q, act_scale; // 4-bit, token tiles <= 32: quantised activations [2][S][max(d, f)] and scales [S]
+  size_t act_q, act_scale; // 4-bit, token tiles <= 32: tiled quantised activations and their scales [S]
   size_t guards[kMaxGuards];  // debug build: offsets of the guards
   int nguards;
 };
@@ -108,7 +108,7 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
   L.eff_splits = 1;
   if (q4) {
     q4_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
-    L.eff_splits = q4_effective_splits(sh->d_ff, L.splits);
+    L.eff_splits = q4_effective_splits(sh->d_ff, L.splits, L.bn);
   } else if (L.variant == MOE_VARIANT_STREAM) {
     stream_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
     const int32_t num_kb = sh->d_ff / 64;
@@ -173,7 +173,7 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
   }
   if (L.q4 && L.bn <= 32) {
     L.act_q = o;
-    o = next_region(L, o + 2 * (size_t)S * (size_t)(d > f ? d : f));
+    o = next_region(L, o + q4i8_act_bytes(S, E, d, f, L.bn));
     L.act_scale = o;
     o = next_region(L, o + 4 * (size_t)S);
   }
@@ -321,7 +321,7 @@ moe_status run_gemms_q4(const moe_shape* sh, const Layout& L, const moe_bf16* x_
   a.num_sms = num_sms;
   a.between = between;
   if (L.act_q) {
-    a.act_q = at<int8_t>(ws, L.act_q);
+    a.act_q = at<uint8_t>(ws, L.act_q);
     a.act_scale = at<float>(ws, L.act_scale);
   }
   return cuda_status(launch_expert_gemms_q4(a, s));

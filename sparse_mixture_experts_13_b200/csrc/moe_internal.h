@@ -133,17 +133,22 @@ struct ExpertGemmQ4Args {
   cudaEvent_t between;      // recorded after the first GEMM if not null
   bool pdl;                 // launched as dependents of the grouping kernel (no event in between)
   uint64_t* clock_probe;    // profiled calls: [8] clock records of the two GEMMs, else nullptr
-  int8_t* act_q;            // token tiles <= 32: quantised activations [2][S][max(d, f)] (high, low bytes)
-  float* act_scale;         // and their per-row scales [S]; nullptr: the bf16-dequantising kernels
+  uint8_t* act_q;           // token tiles <= 32: the quantised activations as the tiled token operand
+  float* act_scale;         // (q4i8_act_bytes) and their per-row scales [S]; nullptr: the bf16-dequantising kernels
 };
 // The integer-MMA 4-bit GEMMs (token tiles of 16 and 32).
 cudaError_t launch_expert_gemms_q4i8(const ExpertGemmQ4Args& a, cudaStream_t s);
+// inputs per pipeline stage of those kernels for a token tile, and the bytes
+// of their tiled token operand
+int32_t q4i8_stage_inputs(int32_t bn);
+size_t q4i8_act_bytes(int64_t S, int32_t E, int32_t d, int32_t f, int32_t bn);
 // Tensor maps of the 4-bit format (expert_gemm_q4.cu).
 bool encode_codes(CUtensorMap* m, const void* base, int64_t E, int64_t R, int64_t K, int box_rows);
 bool encode_scales(CUtensorMap* m, const void* base, int64_t E, int64_t R, int64_t K, int box_rows);
 void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits);
 // number of K splits the down projection really uses for a requested count
-int32_t q4_effective_splits(int32_t f, int32_t splits);
+// (token tile bn decides the kernel and its K granularity)
+int32_t q4_effective_splits(int32_t f, int32_t splits, int32_t bn);
 cudaError_t launch_expert_gemms_q4(const ExpertGemmQ4Args& a, cudaStream_t s);
 // W [E, R, K] bf16 -> codes and scales (K a multiple of 64, R a multiple of 8)
 cudaError_t launch_quantize_q4(const uint16_t* W, int32_t E, int32_t R, int32_t K, uint8_t* codes,

@@ -79,13 +79,20 @@ def test_streaming_layout_adds_splitk_planes(moe, T, d, f):
 @pytest.mark.parametrize("T", [16, 32, 33, 300])
 def test_q4_layout_always_has_splitk_planes(moe, T):
     """The 4-bit layout adds split-K planes and, for token tiles of 16 and 32
-    (T <= 32, the integer-MMA kernels), the quantised activations [2][S][max(d,
-    f)] signed bytes and their scales [S] fp32 at the end."""
+    (T <= 32, the integer-MMA kernels), the quantised activations as their
+    tiled token operand and their scales [S] fp32 at the end.  The operand
+    holds, per token tile (at most S / bn + E of them) and stage of ks inputs
+    (256 for 16-token tiles, 128 for 32), the high and low bytes of the
+    tile's bn rows: 2 bn x ks bytes."""
     sh = moe.make_shape(T, 4096, 14336)
     extra = moe.moe_workspace_size_q4(sh) - expected(T, 4096, 14336, 8, 2)
+    S = T * 2
     if T <= 32:
-        extra -= al(2 * T * 2 * 14336) + al(4 * T * 2)
-    assert _splits(extra, T * 2, 4096) is not None, extra
+        bn = 16 if T <= 16 else 32
+        ks = 256 if bn == 16 else 128
+        tiles = -(-S // bn) + 8
+        extra -= al(tiles * -(-14336 // ks) * 2 * bn * ks) + al(4 * S)
+    assert _splits(extra, S, 4096) is not None, extra
 
 
 def test_quoted_sizes(moe):
