@@ -28,9 +28,10 @@ __device__ __forceinline__ void bf16x8_unpack(const uint4& v, float (&f)[8]) {
 }
 
 // One warp per (token, chunk of 32 * CPL columns); lane l owns CPL
-// consecutive columns.  From bf16 rows (CPL = 16) every row load of a lane is
-// issued before the sums; from fp32 split-K partials (CPL = 8) the split loads
-// are unrolled by four.
+// consecutive columns.  The launch picks CPL = 16 for bf16 rows of y_perm and
+// CPL = 4 for fp32 split-K partials.  From bf16 rows every row load of a lane is
+// issued before the sums; from partials (narrow chunks, so that more warps
+// share a token) up to 8 splits of every slot are in flight at once.
 template <int CPL, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   constexpr int kCols = 32 * CPL;
@@ -61,7 +62,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     float acc[CPL];
 #pragma unroll
     for (int i = 0; i < CPL; ++i) acc[i] = 0.f;
-    if (a.y_perm) {
+    if constexpr (CPL >= 8) {  // bf16 rows of y_perm
       uint4 raw[KMAX][NV];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j)
@@ -82,55 +83,65 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
         }
       }
     } else {
+      // Every slot's splits are loaded before any is added (SPR splits per
+      // round), so the loads of a token overlap; each slot's splits are still
+      // summed in split order.
+      constexpr int SPR = KMAX <= 2 ? 8 : 2;
+      constexpr int NQ = CPL / 4;
+      float o[KMAX][CPL];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (pos[j] < 0) continue;
-        const float* base = a.partials + (int64_t)pos[j] * a.d + col;
-        float o[CPL];
+      for (int j = 0; j < KMAX; ++j)
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) o[i] = 0.f;
-        int sp = 0;
-        for (; sp + 4 <= a.splits; sp += 4) {
-          float4 q[4][CPL / 4];
+        for (int i = 0; i < CPL; ++i) o[j][i] = 0.f;
+      for (int sp0 = 0; sp0 < a.splits; sp0 += SPR) {
+        float4 qv[KMAX][SPR][NQ];
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
+        for (int j = 0; j < KMAX; ++j)
 #pragma unroll
-            for (int c = 0; c < CPL / 4; ++c)
-              q[u][c] = reinterpret_cast<const float4*>(base + (sp + u) * a.part_stride)[c];
+          for (int u = 0; u < SPR; ++u)
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int c = 0; c < CPL / 4; ++c) {
-              o[4 * c] += q[u][c].x;
-              o[4 * c + 1] += q[u][c].y;
-              o[4 * c + 2] += q[u][c].z;
-              o[4 * c + 3] += q[u][c].w;
+            for (int c = 0; c < NQ; ++c) {
+              qv[j][u][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (pos[j] >= 0 && sp0 + u < a.splits)
+                qv[j][u][c] = reinterpret_cast<const float4*>(a.partials + (int64_t)(sp0 + u) * a.part_stride +
+                                                              (int64_t)pos[j] * a.d + col)[c];
             }
-        }
-        for (; sp < a.splits; ++sp) {
 #pragma unroll
-          for (int c = 0; c < CPL / 4; ++c) {
-            const float4 v = reinterpret_cast<const float4*>(base + sp * a.part_stride)[c];
-            o[4 * c] += v.x;
-            o[4 * c + 1] += v.y;
-            o[4 * c + 2] += v.z;
-            o[4 * c + 3] += v.w;
-          }
-        }
+        for (int j = 0; j < KMAX; ++j)
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) acc[i] = fmaf(w[j], o[i], acc[i]);
+          for (int u = 0; u < SPR; ++u)
+            if (sp0 + u < a.splits) {
+#pragma unroll
+              for (int c = 0; c < NQ; ++c) {
+                o[j][4 * c] += qv[j][u][c].x;
+                o[j][4 * c + 1] += qv[j][u][c].y;
+                o[j][4 * c + 2] += qv[j][u][c].z;
+                o[j][4 * c + 3] += qv[j][u][c].w;
+              }
+            }
       }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(a.y + t * a.d + col);
 #pragma unroll
-    for (int h = 0; h < NV; ++h)
-      dst[h] = make_uint4(pack_bf16x2(acc[8 * h], acc[8 * h + 1]), pack_bf16x2(acc[8 * h + 2], acc[8 * h + 3]),
-                          pack_bf16x2(acc[8 * h + 4], acc[8 * h + 5]), pack_bf16x2(acc[8 * h + 6], acc[8 * h + 7]));
+      for (int j = 0; j < KMAX; ++j)
+        if (pos[j] >= 0) {
+#pragma unroll
+          for (int i = 0; i < CPL; ++i) acc[i] = fmaf(w[j], o[j][i], acc[i]);
+        }
+    }
+    if constexpr (CPL >= 8) {
+      uint4* dst = reinterpret_cast<uint4*>(a.y + t * a.d + col);
+#pragma unroll
+      for (int h = 0; h < NV; ++h)
+        dst[h] = make_uint4(pack_bf16x2(acc[8 * h], acc[8 * h + 1]), pack_bf16x2(acc[8 * h + 2], acc[8 * h + 3]),
+                            pack_bf16x2(acc[8 * h + 4], acc[8 * h + 5]), pack_bf16x2(acc[8 * h + 6], acc[8 * h + 7]));
+    } else {
+      *reinterpret_cast<uint2*>(a.y + t * a.d + col) =
+          make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+    }
   }
 }
 
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
-  const int cpl = a.y_perm ? 16 : 8;
+  const int cpl = a.y_perm ? 16 : 4;
   const int64_t warps_needed = a.T * ((a.d + 32 * cpl - 1) / (32 * cpl));
   int64_t blocks = (warps_needed + 7) / 8;
   const int64_t cap = (int64_t)num_sms * 16;
@@ -139,10 +150,10 @@ cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
   const dim3 g((unsigned)blocks), b(256);
   if (a.k <= 2) {
     if (cpl == 16) return launch_k(combine_kernel<16, 2>, g, b, 0, s, a.pdl, a);
-    return launch_k(combine_kernel<8, 2>, g, b, 0, s, a.pdl, a);
+    return launch_k(combine_kernel<4, 2>, g, b, 0, s, a.pdl, a);
   }
   if (cpl == 16) return launch_k(combine_kernel<16, 8>, g, b, 0, s, a.pdl, a);
-  return launch_k(combine_kernel<8, 8>, g, b, 0, s, a.pdl, a);
+  return launch_k(combine_kernel<4, 8>, g, b, 0, s, a.pdl, a);
 }
 
 // y_perm[r] = bf16(sum over splits of partials[sp][r]) for rows r < offsets[E].

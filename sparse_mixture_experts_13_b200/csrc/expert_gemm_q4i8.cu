@@ -565,26 +565,28 @@ __global__ void __launch_bounds__(kI8Threads, 1)
   }
 }
 
-// One warp per row r < offsets[E] of `in` [S, K] bf16: a = max |x[r]|,
-// q = clamp(rint(x * 32639 / a), -32639, 32639), low byte ((q + 128) & 255) - 128,
-// high byte (q - low) / 256, in the MMA's K order (0 4 1 5 2 6 3 7 per group
-// of 8), written into the tiled token operand (layout at the top of this
-// file; inputs from K up to the last stage's end are zero); scale[r] = a / 32639.
-__global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ in,
-                                                           const int32_t* __restrict__ offsets, int32_t E, int32_t K,
-                                                           int32_t bn, int32_t ks, int32_t num_kq,
-                                                           uint8_t* __restrict__ q8, float* __restrict__ scale) {
+// One block per row r < offsets[E] of `in` [S, K] bf16 (8 warps share the
+// row): a = max |x[r]|, q = clamp(rint(x * 32639 / a), -32639, 32639), low
+// byte ((q + 128) & 255) - 128, high byte (q - low) / 256, in the MMA's K
+// order (0 4 1 5 2 6 3 7 per group of 8), written into the tiled token
+// operand (layout at the top of this file; inputs from K up to the last
+// stage's end are zero); scale[r] = a / 32639.
+constexpr int kQuantThreads = 256;
+__global__ void __launch_bounds__(kQuantThreads) quantize_act_kernel(const uint16_t* __restrict__ in,
+                                                                     const int32_t* __restrict__ offsets, int32_t E,
+                                                                     int32_t K, int32_t bn, int32_t ks, int32_t num_kq,
+                                                                     uint8_t* __restrict__ q8,
+                                                                     float* __restrict__ scale) {
+  __shared__ float s_amax[kQuantThreads / 32];
   pdl_wait();  // the rows (and offsets) of the kernels before this one
   pdl_trigger();
-  const int lane = threadIdx.x & 31;
-  const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t rows = offsets[E];
   const int nvec = K >> 3;
   const int nvec_all = (num_kq * ks) >> 3;
   const int n_rows = 2 * bn;  // rows of a 128-byte slice: high bytes, then low bytes
   const int64_t tile_bytes = (int64_t)(ks / 128) * n_rows * 128;
-  for (int64_t row = w0; row < rows; row += nw) {
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     // token tile of the row: its expert's tiles follow those of the experts before it
     int e = 0;
     int64_t tau = 0;
@@ -600,7 +602,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
 
     const uint4* src = reinterpret_cast<const uint4*>(in + row * (int64_t)K);
     float amax = 0.f;
-    for (int v = lane; v < nvec; v += 32) {
+    for (int v = tid; v < nvec; v += kQuantThreads) {
       const uint4 x = src[v];
       const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -609,9 +611,15 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) s_amax[warp] = amax;
+    __syncthreads();
+    amax = s_amax[0];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, s_amax[w]);
+    __syncthreads();  // s_amax is rewritten for the next row
     const float inv = amax > 0.f ? (float)kQMax / amax : 0.f;
-    if (lane == 0) scale[row] = amax / (float)kQMax;
-    for (int v = lane; v < nvec_all; v += 32) {
+    if (tid == 0) scale[row] = amax / (float)kQMax;
+    for (int v = tid; v < nvec_all; v += kQuantThreads) {
       uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
       if (v < nvec) {
         const uint4 x = src[v];
@@ -672,13 +680,13 @@ bool encode_scales_i8(CUtensorMap* m, const void* base, int64_t E, int64_t R, in
 
 cudaError_t launch_quantize_act(const uint16_t* in, const int32_t* offsets, int32_t E, int64_t S, int32_t K, int bn,
                                 uint8_t* q8, float* scale, int num_sms, cudaStream_t s, bool pdl) {
-  int64_t blocks = (S + 7) / 8;  // 8 warps per block
+  int64_t blocks = S;  // a block per row
   if (blocks > 8 * (int64_t)num_sms) blocks = 8 * (int64_t)num_sms;
   if (blocks < 1) blocks = 1;
   const int ks = i8_stage_inputs(bn);
   const int num_kq = (K + ks - 1) / ks;
-  return launch_k(quantize_act_kernel, dim3((unsigned)blocks), dim3(256), 0, s, pdl, in, offsets, E, K, bn, ks,
-                  num_kq, q8, scale);
+  return launch_k(quantize_act_kernel, dim3((unsigned)blocks), dim3(kQuantThreads), 0, s, pdl, in, offsets, E, K, bn,
+                  ks, num_kq, q8, scale);
 }
 
 template <int EPI, int BN>
