@@ -925,22 +925,23 @@ void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int nu
   else if (b > 32) b = 64;
   else if (b > 16) b = 32;
   *bn = (int32_t)b;
-  // Split K of the down projection so that (experts x 128-row blocks x
-  // splits) tiles fill whole waves of the SMs as evenly as possible.  At most
-  // T * k experts receive tokens, which bounds the tile count for few tokens.
+  // Split K of the down projection: the count that minimises the waves of
+  // (experts x 128-row blocks x splits) tiles times the K chunks of a tile
+  // plus one (a tile's start-up and epilogue), plus one chunk per split for
+  // the partial plane the combine reads.  At most T * k experts receive
+  // tokens, which bounds the tile count for few tokens.
   const int32_t num_kb = f / BK;
   const int64_t touched = T * k < E ? T * k : E;
   const int64_t base = touched * ((d + 127) / 128);
   int32_t best = 1;
-  double best_eff = 0.0;
+  int64_t best_cost = INT64_MAX;
   for (int32_t sp = 1; sp <= 16 && sp <= num_kb; ++sp) {
     const int32_t kbps = (num_kb + sp - 1) / sp;
     const int32_t real = (num_kb + kbps - 1) / kbps;
-    const int64_t tiles = base * real;
-    const int64_t waves = (tiles + num_sms - 1) / num_sms;
-    const double eff = (double)(base * num_kb) / (double)(waves * num_sms * kbps);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
+    const int64_t waves = (base * real + num_sms - 1) / num_sms;
+    const int64_t cost = waves * (kbps + 1) + real;
+    if (cost < best_cost) {
+      best_cost = cost;
       best = real;
     }
   }

@@ -640,23 +640,22 @@ void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sm
   else if (b > 32) b = 64;
   else if (b > 16) b = 32;
   *bn = (int32_t)b;
-  // split K of the down projection so that (experts x 128-row blocks x
-  // splits) tiles fill whole waves of the SMs as evenly as possible; K goes
-  // in stages of the kernel the token tile selects
+  // split K of the down projection as the bf16 streaming schedule does
+  // (fewest waves x (stages per tile + 1) + one stage per partial plane); K
+  // goes in stages of the kernel the token tile selects
   const int32_t kq_inputs = b <= 32 ? q4i8_stage_inputs((int32_t)b) : KQ;
   const int32_t num_kq = (f + kq_inputs - 1) / kq_inputs;
   const int64_t touched = T * k < E ? T * k : E;
   const int64_t base = touched * ((d + 127) / 128);
   int32_t best = 1;
-  double best_eff = 0.0;
+  int64_t best_cost = INT64_MAX;
   for (int32_t sp = 1; sp <= 16 && sp <= num_kq; ++sp) {
     const int32_t kps = (num_kq + sp - 1) / sp;
     const int32_t real = (num_kq + kps - 1) / kps;
-    const int64_t tiles = base * real;
-    const int64_t waves = (tiles + num_sms - 1) / num_sms;
-    const double eff = (double)(base * num_kq) / (double)(waves * num_sms * kps);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
+    const int64_t waves = (base * real + num_sms - 1) / num_sms;
+    const int64_t cost = waves * (kps + 1) + real;
+    if (cost < best_cost) {
+      best_cost = cost;
       best = real;
     }
   }
