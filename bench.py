@@ -805,6 +805,83 @@ def run_sweep(args):
     sampler.stop()
 
 
+# Peer copy bandwidth per direction measured on this machine's B200s over
+# NVLink 5 (nominal 900 GB/s): the reference for the dispatch and return.
+NVLINK_PEER_GBS = 770.0
+
+
+def run_ep(args):
+    """Expert-parallel arm: the E experts are split over the ranks (E / world
+    each, same seed-0 weights as the other arms), every rank routes its own T
+    tokens (prefill shape, seed 1 + rank), stores each row straight into the
+    receive buffer of its expert's owner (peer stores into symmetric memory),
+    runs its experts and reads the results back from the owners.  One JSON
+    line: tokens/s over all ranks, the phase times, and the bytes that cross
+    between GPUs per step against the peer-copy bandwidth."""
+    import datetime
+    import torch
+    import torch.distributed as tdist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks")
+    torch.cuda.set_device(local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    if "MASTER_PORT" not in os.environ:
+        os.environ["MASTER_PORT"] = str(free_port())
+    tdist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=300),
+                             device_id=torch.device("cuda", local))
+    import sparse_mixture_experts_13_b200 as moe
+    from sparse_mixture_experts_13_b200.ep import EPLayer
+    moe.lib()
+    wl0 = synth.workload("prefill")
+    E, d, f, k, T = wl0.E, wl0.d, wl0.f, wl0.k, args.ep_tokens
+    if E % world:
+        raise SystemExit(f"{E} experts do not split over {world} ranks")
+    epr = E // world
+    lo_e = rank * epr
+    W1 = synth.normal_bf16(0, synth.TID_W1, (E, f, d), 0.0, 1.0 / np.sqrt(d))[lo_e:lo_e + epr]
+    W3 = synth.normal_bf16(0, synth.TID_W3, (E, f, d), 0.0, 1.0 / np.sqrt(d))[lo_e:lo_e + epr]
+    W2 = synth.normal_bf16(0, synth.TID_W2, (E, d, f), 0.0, 1.0 / np.sqrt(f))[lo_e:lo_e + epr]
+    Wg = torch.from_numpy(synth.normal_f32(0, synth.TID_WG, (E, d), 0.0, 1.0 / np.sqrt(d))).cuda()
+    x = to_dev_bf16(synth.normal_bf16(1 + rank, synth.TID_X, (T, d)), torch)
+    layer = EPLayer(Wg, to_dev_bf16(W1, torch), to_dev_bf16(W3, torch), to_dev_bf16(W2, torch), E, k, T)
+    for _ in range(args.warmup):
+        layer.forward(x)
+    ms = time_steps(lambda: layer.forward(x), args.steps, torch, tdist)
+    # phases of one more step, and the rows that left this rank
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    torch.cuda.synchronize()
+    layer.forward(x, events=evs)
+    torch.cuda.synchronize()
+    names = ["route_and_plan", "dispatch", "expert_gemms", "combine"]
+    phases = {n: max_over_ranks(evs[i].elapsed_time(evs[i + 1]), torch, tdist) for i, n in enumerate(names)}
+    counts = layer.last_counts_all.view(world, E).cpu().numpy()
+    remote_rows = int(sum(counts[rank, e] for e in range(E) if e // epr != rank))
+    remote = torch.tensor([remote_rows], dtype=torch.int64, device="cuda")
+    tdist.all_reduce(remote, op=tdist.ReduceOp.MAX)
+    bytes_out = int(remote.item()) * d * 2  # the busiest rank's rows sent (and read back)
+    tdist.barrier()
+    if rank == 0:
+        def link(phase):
+            gbs = bytes_out / (phases[phase] * 1e-3) / 1e9 if phases[phase] > 0 else 0.0
+            return dict(bytes_per_rank=bytes_out, gbs=gbs, peak=NVLINK_PEER_GBS, unit="GB/s",
+                        frac=gbs / NVLINK_PEER_GBS, peak_source="measured peer copy per direction on this pool")
+        line = dict(metric="expert-parallel MoE-layer tokens/s", value=weak_scaling_value(world, T, ms),
+                    unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup, ms_per_step=ms,
+                    higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+                    config=dict(workload=f"expert-parallel: T={T} tokens per rank d_model={d} d_ff={f} E={E} "
+                                         f"({epr} per rank) top-{k} dropless",
+                                parallelism=f"ep{world}",
+                                l2="inputs larger than L2: expert weights streamed every step"),
+                    phases_ms=phases, dispatch=link("dispatch"), return_=link("combine"))
+        line["return"] = line.pop("return_")
+        print(json.dumps(line), flush=True)
+    del layer
+    tdist.destroy_process_group()
+
+
 def free_port() -> int:
     import socket
     with socket.socket() as s_:
@@ -830,6 +907,9 @@ def main():
                     help="one JSON line per workload (tiny, decode, prefill, skew, T sweep) instead of the contract line")
     ap.add_argument("--dry-run", action="store_true",
                     help="check the rank launcher and plumbing on CPU (gloo): no GPU work")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert-parallel arm: the experts split over the --gpus ranks (one JSON line)")
+    ap.add_argument("--ep-tokens", type=int, default=4096, help="tokens per rank of the expert-parallel arm")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -839,6 +919,8 @@ def main():
         sys.exit(launch_ranks(args))
     if args.dry_run:
         run_dry(args)
+    elif args.ep:
+        run_ep(args)
     elif args.impl == "reference":
         run_reference(args)
     elif args.sweep:

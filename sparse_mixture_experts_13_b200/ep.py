@@ -179,8 +179,13 @@ class EPLayer:
         self.owner_shape = _lib.make_shape(self.rows, self.d, self.f, self.epr, 1)
         self.owner_ws = torch.empty(_lib.moe_workspace_size(self.owner_shape), dtype=torch.uint8, device=dev)
 
-    def forward(self, x: torch.Tensor) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, events=None) -> torch.Tensor:
+        """`events`, if given, is a list of 5 CUDA events recorded on the
+        current stream before the router and after the plan, the dispatch,
+        the owner's GEMMs and the combine (phase times for benchmarks)."""
         dist, dev = self.dist, x.device
+        mark = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        mark(0)
         T, d, E, k = x.shape[0], self.d, self.E, self.k
         cap_mode = self.capacity_factor > 0
         sh = _lib.make_shape(T, d, self.f, E, k, self.capacity_factor, self.drop_policy)
@@ -192,6 +197,8 @@ class EPLayer:
         dist.all_gather_into_tensor(counts_all, counts, group=self.group)
         recv_off, owner_off = cu(E, dt=torch.int32), cu(self.epr + 1, dt=torch.int32)
         _check(_lib.moe_ep_plan(counts_all, E, self.rank, self.world, recv_off, owner_off), "moe_ep_plan")
+        self.last_counts_all = counts_all
+        mark(1)
         ret_row = cu(T * k, dt=torch.int32)
         n = _lib.moe_workspace_size(sh)
         ws = cu(n, dt=torch.uint8)
@@ -201,6 +208,7 @@ class EPLayer:
         else:
             _check(_lib.moe_ep_dispatch(sh, self.world, x, idx, counts, recv_off, self.peer_x, ret_row, ws, n),
                    "moe_ep_dispatch")
+        mark(2)
         dist.barrier(group=self.group)  # every rank's rows (and keys) have landed
         a_in, a_off = self.x_recv, owner_off
         if cap_mode:
@@ -210,6 +218,7 @@ class EPLayer:
         _check(_lib.moe_grouped_swiglu(self.owner_shape, a_in, a_off, self.W1, self.W3, self.W2,
                                        self.h_recv, self.y_recv, self.owner_ws, self.owner_ws.numel()),
                "moe_grouped_swiglu")
+        mark(3)
         dist.barrier(group=self.group)  # every owner's results (and row map) are written
         y = cu(T, d, dt=torch.bfloat16)
         if cap_mode:
@@ -217,6 +226,7 @@ class EPLayer:
                    "moe_ep_combine_cap")
         else:
             _check(_lib.moe_ep_combine(sh, self.world, idx, w, ret_row, self.peer_y, y), "moe_ep_combine")
+        mark(4)
         dist.barrier(group=self.group)  # the buffers may be reused by the next call
         return y
 
