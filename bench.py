@@ -849,7 +849,7 @@ def run_ep(args):
     layer = EPLayer(Wg, to_dev_bf16(W1, torch), to_dev_bf16(W3, torch), to_dev_bf16(W2, torch), E, k, T)
     for _ in range(args.warmup):
         layer.forward(x)
-    ms = time_steps(lambda: layer.forward(x), args.steps, torch, tdist)
+    ms = time_steps(lambda: layer.forward(x), args.steps, torch, tdist) / args.steps
     # phases of one more step, and the rows that left this rank
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
     torch.cuda.synchronize()

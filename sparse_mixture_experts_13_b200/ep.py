@@ -137,8 +137,12 @@ class EPLayer:
 
     def __init__(self, Wg, W1_local, W3_local, W2_local, E: int, k: int, max_tokens: int, group=None,
                  capacity_factor: float = 0.0, drop_policy: int = _lib.MOE_DROP_BY_PROB):
+        import os
         import torch.distributed as dist
         import torch.distributed._symmetric_memory as symm_mem
+        # The kernels use plain peer loads and stores; the buffers need no
+        # NVLink multicast object (none is bound to them).
+        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
         self.dist, self.group = dist, group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
