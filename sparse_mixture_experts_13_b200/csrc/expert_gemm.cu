@@ -48,7 +48,19 @@ constexpr int BK = 64;   // K elements per stage: 128 bytes of bf16, one swizzle
 constexpr int kGemmThreads = 192;
 constexpr int A_BYTES = BM * BK * 2;
 
-enum : int { EPI_TILED_SWIGLU = 0, EPI_TILED_STORE = 1, EPI_STREAM_SWIGLU = 2, EPI_STREAM_PARTIAL = 3 };
+// EPI_STREAM_GU_PARTIAL: the gate/up GEMM split along K (few tokens): fp32
+// partials of both projections, [splits][S][2 f] (W1 columns, then W3),
+// summed and passed through SiLU * mul by swiglu_splitk_kernel.
+enum : int {
+  EPI_TILED_SWIGLU = 0,
+  EPI_TILED_STORE = 1,
+  EPI_STREAM_SWIGLU = 2,
+  EPI_STREAM_PARTIAL = 3,
+  EPI_STREAM_GU_PARTIAL = 4
+};
+__host__ __device__ constexpr bool epi_is_gate_up(int epi) {
+  return epi == EPI_STREAM_SWIGLU || epi == EPI_STREAM_GU_PARTIAL;
+}
 
 struct GemmParams {
   const int32_t* offsets;
@@ -84,7 +96,7 @@ struct GemmCfg {
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + XBUF_BYTES + BAR_BYTES;
   // rows of the weight operand per tile (n-extent of one weight block)
-  static constexpr int W_ROWS = (EPI == EPI_TILED_SWIGLU) ? 128 : (EPI == EPI_TILED_STORE) ? 256 : (EPI == EPI_STREAM_SWIGLU) ? 64 : 128;
+  static constexpr int W_ROWS = (EPI == EPI_TILED_SWIGLU) ? 128 : (EPI == EPI_TILED_STORE) ? 256 : epi_is_gate_up(EPI) ? 64 : 128;
   static constexpr uint32_t IDESC = make_idesc_bf16(BM, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -159,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (tid == 0) {
     tma_prefetch_desc(&map_act);
     tma_prefetch_desc(&map_wa);
-    if (EPI == EPI_TILED_SWIGLU || EPI == EPI_STREAM_SWIGLU) tma_prefetch_desc(&map_wb);
+    if (EPI == EPI_TILED_SWIGLU || epi_is_gate_up(EPI)) tma_prefetch_desc(&map_wb);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
@@ -189,7 +201,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int32_t kb1 = min(p.num_kb, kb0 + min(p.kb_per_split, p.prefetch_kb));
       for (int32_t kb = kb0; kb < kb1; ++kb) {
         tma_prefetch_l2_3d(&map_wa, kb * BK, n0, e);
-        if (EPI == EPI_STREAM_SWIGLU) tma_prefetch_l2_3d(&map_wb, kb * BK, n0, e);
+        if (epi_is_gate_up(EPI)) tma_prefetch_l2_3d(&map_wb, kb * BK, n0, e);
       }
     }
   }
@@ -254,7 +266,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else if (EPI == EPI_TILED_STORE) {
             tma_load_2d(&map_act, &full_bar[stage], a_dst, kx, t.row0);
             tma_load_3d(&map_wa, &full_bar[stage], b_dst, kx, t.n0, t.e);
-          } else if (EPI == EPI_STREAM_SWIGLU) {
+          } else if (epi_is_gate_up(EPI)) {
             tma_load_3d(&map_wa, &full_bar[stage], a_dst, kx, t.n0, t.e);
             tma_load_3d(&map_wb, &full_bar[stage], a_dst + 64 * 128, kx, t.n0, t.e);
             tma_load_2d(&map_act, &full_bar[stage], b_dst, kx, t.row0);
@@ -419,9 +431,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           named_bar_sync(1, 128);
         }
       } else {
-        // fp32 split-K partial: lane r is output column n0 + r; TMEM columns are tokens.
-        float* out = reinterpret_cast<float*>(p.out) + (int64_t)t.split * p.part_stride;
-        const bool col_ok = t.n0 + r < p.n_out;
+        // fp32 split-K partial; TMEM columns are tokens.  Down projection:
+        // lane r is output column n0 + r.  Gate/up: lanes 0..63 are W1
+        // column n0 + r, lanes 64..127 W3 column n0 + r - 64, stored f later.
+        float* out = reinterpret_cast<float*>(p.out) + (int64_t)t.split * p.part_stride +
+                     (EPI == EPI_STREAM_GU_PARTIAL && r >= 64 ? (int64_t)p.n_out - 64 : 0);
+        const bool col_ok = t.n0 + (EPI == EPI_STREAM_GU_PARTIAL ? (r & 63) : r) < p.n_out;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           uint32_t v[16];
@@ -917,7 +932,8 @@ static int32_t prefetch_chunks(int num_sms) {
   return (int32_t)(n < 1 ? 1 : n);
 }
 
-void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
+void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits,
+                   int32_t* splits1) {
   int64_t b = ((T + 15) / 16) * 16;
   if (b < 16) b = 16;
   if (b > 128) b = 128;
@@ -946,7 +962,59 @@ void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int nu
     }
   }
   *splits = best;
+  // Split K of the gate/up projection only where it shortens the last,
+  // partly filled wave of (experts x 64-row blocks) tiles enough (by 3 %)
+  // to pay for its fp32 partials and the extra reduction launch (counted
+  // as 8 chunk-waves).
+  const int32_t num_kb1 = d / BK;
+  const int64_t base1 = touched * (f / 64);
+  const int64_t plane = (T * k * 2 * (int64_t)f * 8 + 16384LL * num_sms - 1) / (16384LL * num_sms);
+  const int64_t cost1 = ((base1 + num_sms - 1) / num_sms) * (num_kb1 + 1);
+  int32_t best1 = 1;
+  int64_t best1_cost = cost1;
+  for (int32_t sp = 2; sp <= 8 && sp <= num_kb1; sp *= 2) {
+    const int32_t kbps = (num_kb1 + sp - 1) / sp;
+    const int32_t real = (num_kb1 + kbps - 1) / kbps;
+    const int64_t waves = (base1 * real + num_sms - 1) / num_sms;
+    const int64_t c = waves * (kbps + 1) + real * plane + 8;
+    if (c * 100 <= cost1 * 97 && c < best1_cost) {
+      best1_cost = c;
+      best1 = real;
+    }
+  }
+  *splits1 = best1;
 }
+
+// h[r, c] = bf16(SiLU(a) * b), a and b the sums over splits (in split order)
+// of the gate/up partials of row r < offsets[E]: columns c and f + c.
+__global__ void __launch_bounds__(256) swiglu_splitk_kernel(const float* __restrict__ partials, int32_t splits,
+                                                            int64_t part_stride, const int32_t* __restrict__ offsets,
+                                                            int32_t E, int32_t f, uint16_t* __restrict__ h, int64_t S,
+                                                            uint32_t* status) {
+  pdl_wait();  // the gate/up partials
+  pdl_trigger();
+  int64_t rows = offsets[E];
+  if (!MOE_DCHECK(status, rows >= 0 && rows <= S)) rows = 0;
+  const int nvec = f >> 2;
+  const int64_t total = rows * nvec;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / nvec;
+    const int v = (int)(i % nvec);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    for (int sp = 0; sp < splits; ++sp) {
+      const float* row = partials + sp * part_stride + r * 2 * (int64_t)f;
+      const float4 pa = reinterpret_cast<const float4*>(row)[v];
+      const float4 pb = reinterpret_cast<const float4*>(row + f)[v];
+      a.x += pa.x; a.y += pa.y; a.z += pa.z; a.w += pa.w;
+      b.x += pb.x; b.y += pb.y; b.z += pb.z; b.w += pb.w;
+    }
+    reinterpret_cast<uint2*>(h + r * (int64_t)f)[v] =
+        make_uint2(pack_bf16x2(silu_f32(a.x) * b.x, silu_f32(a.y) * b.y),
+                   pack_bf16x2(silu_f32(a.z) * b.z, silu_f32(a.w) * b.w));
+  }
+}
+
+
 
 template <int BN>
 static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
@@ -970,7 +1038,24 @@ static cudaError_t launch_stream(const ExpertGemmArgs& a, cudaStream_t s) {
   p1.kb_per_split = p1.num_kb;
   p1.prefetch_kb = a.pdl ? prefetch_chunks(a.num_sms) : 0;
   p1.clock_probe = a.clock_probe;
-  cudaError_t err = launch_one<EPI_STREAM_SWIGLU, BN>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl);
+  cudaError_t err;
+  if (a.splits1 > 1) {
+    // gate/up split along K: fp32 partials, then their sum through SiLU * mul
+    p1.out = a.partials1;
+    p1.out_ld = 2 * (int64_t)a.f;
+    p1.part_stride = a.S * 2 * (int64_t)a.f;
+    p1.kb_per_split = (p1.num_kb + a.splits1 - 1) / a.splits1;
+    p1.splits = (p1.num_kb + p1.kb_per_split - 1) / p1.kb_per_split;
+    err = launch_one<EPI_STREAM_GU_PARTIAL, BN>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl);
+    if (err != cudaSuccess) return err;
+    int64_t blocks = (a.S * (a.f / 4) + 255) / 256;
+    if (blocks > 4 * (int64_t)a.num_sms) blocks = 4 * (int64_t)a.num_sms;
+    if (blocks < 1) blocks = 1;
+    err = launch_k(swiglu_splitk_kernel, dim3((unsigned)blocks), dim3(256), 0, s, a.pdl, (const float*)a.partials1,
+                   p1.splits, p1.part_stride, a.offsets, a.E, a.f, a.h, a.S, a.status);
+  } else {
+    err = launch_one<EPI_STREAM_SWIGLU, BN>(mx, mw1, mw3, p1, a.num_sms, s, a.pdl);
+  }
   if (err != cudaSuccess) return err;
   if (a.between && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
   GemmParams p2{};

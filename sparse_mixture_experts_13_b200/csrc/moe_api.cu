@@ -79,6 +79,8 @@ struct Layout {
   int variant;
   bool q4;                 // 4-bit expert weights (always the streaming schedule)
   int32_t bn, splits;      // streaming schedule: token tile, requested split-K count
+  int32_t splits1;         // streaming schedule: gate/up split-K count (1: none)
+  size_t partials1;        // gate/up partials [splits1, S, 2 f] when splits1 > 1
   int32_t eff_splits;      // split-K partial buffers the down projection writes
   size_t act_q, act_scale; // 4-bit, token tiles <= 32: tiled quantised activations and their scales [S]
   size_t guards[kMaxGuards];  // debug build: offsets of the guards
@@ -105,12 +107,13 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
   L.q4 = q4;
   L.bn = 128;
   L.splits = 1;
+  L.splits1 = 1;
   L.eff_splits = 1;
   if (q4) {
     q4_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
     L.eff_splits = q4_effective_splits(sh->d_ff, L.splits, L.bn);
   } else if (L.variant == MOE_VARIANT_STREAM) {
-    stream_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits);
+    stream_params(T, sh->k, sh->d_model, sh->d_ff, sh->E, kPlanSms, &L.bn, &L.splits, &L.splits1);
     const int32_t num_kb = sh->d_ff / 64;
     const int32_t kbps = (num_kb + L.splits - 1) / L.splits;
     L.eff_splits = (num_kb + kbps - 1) / kbps;
@@ -133,6 +136,8 @@ Layout layout_of(const moe_shape* sh, bool q4 = false) {
   o = next_region(L, o + 8 * E);
   L.partials = o;
   if (L.variant == MOE_VARIANT_STREAM) o = next_region(L, o + 4 * (size_t)L.eff_splits * S * d);
+  L.partials1 = o;
+  if (L.splits1 > 1) o = next_region(L, o + 4 * (size_t)L.splits1 * S * 2 * f);
   L.topk_idx = o;
   o = next_region(L, o + 4 * S);
   L.topk_w = o;
@@ -282,6 +287,8 @@ moe_status run_gemms(const moe_shape* sh, const Layout& L, const moe_bf16* x_per
   a.pair = L.variant == MOE_VARIANT_TILED;
   a.stream_bn = L.bn;
   a.splits = L.splits;
+  a.splits1 = L.splits1;
+  a.partials1 = L.splits1 > 1 ? at<float>(ws, L.partials1) : nullptr;
   a.num_sms = num_sms;
   a.between = between;
   a.tile_counters = at<uint32_t>(ws, L.status) + 2;  // words 2 and 3 of the control header

@@ -98,6 +98,8 @@ struct ExpertGemmArgs {
   int32_t variant;          // 1 tiled, 2 streaming
   int32_t stream_bn;        // streaming variant: token tile (16..128)
   int32_t splits;           // streaming variant: split-K count of the down projection
+  int32_t splits1;          // streaming variant: split-K count of the gate/up projection (1: none)
+  float* partials1;         // [splits1, S, 2 f] gate/up partials when splits1 > 1
   int num_sms;
   cudaEvent_t between;      // recorded after the first GEMM if not null
   bool pair;                // tiled variant: CTA-pair (cta_group::2) kernels
@@ -107,7 +109,7 @@ struct ExpertGemmArgs {
 };
 // Streaming-variant parameters chosen from host-known sizes.
 void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn,
-                   int32_t* splits);
+                   int32_t* splits, int32_t* splits1);
 cudaError_t launch_expert_gemms(const ExpertGemmArgs& a, cudaStream_t s);
 
 // Expert GEMMs with 4-bit weights (codes [E, R, K/2], scales [E, K/64, R]

@@ -264,6 +264,13 @@ def test_sweep(o, T):
     check_everything(o, full_workload("sweep", T=T), 0, rows=64 if T >= 4096 else 16)
 
 
+def test_gate_up_split_along_k(o):
+    """Two Mixtral tokens: the streaming gate/up GEMM is split 4 ways along K
+    (fp32 partials, then their sum through SiLU * mul); T = 1 in the sweep
+    takes the same path."""
+    check_everything(o, full_workload("sweep", T=2), 0, rows=16)
+
+
 @pytest.mark.parametrize("E", [8, 16, 32])
 def test_router_many_tokens(o, E):
     """700 tokens at d=128: the register router for E=8, the grouped router
