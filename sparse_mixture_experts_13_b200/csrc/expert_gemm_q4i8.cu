@@ -179,6 +179,19 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
       : "memory");
 }
 
+// Position in a ring of N barrier-guarded slots: the slot and the parity of
+// its current use (32-bit counters instead of divisions of a 64-bit index).
+template <int N>
+struct RingPos {
+  uint32_t slot = 0, phase = 0;
+  __device__ __forceinline__ void next() {
+    if (++slot == (uint32_t)N) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 // 32 lanes x W consecutive columns into registers (W = 8 or 16).
 template <int W>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
@@ -304,14 +317,15 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     if (lane == 0) {
       // ------------------------------------------------ loads
       int64_t i = 0;
+      RingPos<STAGES> sp;
       bool ok = true;
       for (int32_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         I8Tile t;
         i8_decode_tile<EPI, BN>(p, s_off, s_base, s_tau, tile, t);
-        for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i) {
-          const int stage = (int)(i % STAGES);
-          const int64_t use = i / STAGES;
-          if (use >= 1 && !mbar_wait(&free_bar[stage], (uint32_t)((use - 1) & 1), &s_abort)) {
+        for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i, sp.next()) {
+          const int stage = (int)sp.slot;
+          // the slot's previous use (parity phase ^ 1) must have been read
+          if (i >= STAGES && !mbar_wait(&free_bar[stage], sp.phase ^ 1u, &s_abort)) {
             ok = false;
             break;
           }
@@ -350,16 +364,18 @@ __global__ void __launch_bounds__(kI8Threads, 1)
       // per stage: block b's two K = 32 MMAs into accumulator columns
       // (i % DBUFS) DCOLS + b N, then one commit
       int64_t i = 0;
+      RingPos<STAGES> sp;
+      RingPos<ABUFS> ap;
+      RingPos<DBUFS> dp;
       bool ok = true;
       for (int32_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         I8Tile t;
         i8_decode_tile<EPI, BN>(p, s_off, s_base, s_tau, tile, t);
-        for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i) {
-          const int stage = (int)(i % STAGES);
-          const int ab = (int)(i % ABUFS), db = (int)(i % DBUFS);
-          ok = mbar_wait(&full_bar[stage], (uint32_t)((i / STAGES) & 1), &s_abort) &&
-               mbar_wait(&afull_bar[ab], (uint32_t)((i / ABUFS) & 1), &s_abort) &&
-               (i < DBUFS || mbar_wait(&dfree_bar[db], (uint32_t)(((i / DBUFS) - 1) & 1), &s_abort));
+        for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i, sp.next(), ap.next(), dp.next()) {
+          const int stage = (int)sp.slot;
+          const int ab = (int)ap.slot, db = (int)dp.slot;
+          ok = mbar_wait(&full_bar[stage], sp.phase, &s_abort) && mbar_wait(&afull_bar[ab], ap.phase, &s_abort) &&
+               (i < DBUFS || mbar_wait(&dfree_bar[db], dp.phase ^ 1u, &s_abort));
           if (!ok) break;
           tc_fence_after();
           const uint32_t d = tmem_base + (uint32_t)(db * C::DCOLS);
@@ -395,20 +411,22 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     const uint32_t cx = CHUNKS == 8 ? (uint32_t)(r & 7) : (uint32_t)((r >> 1) & 3);
     const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
     int64_t i = 0;
+    RingPos<STAGES> sp, lag;  // lag: the stage ABUFS before this one
+    RingPos<ABUFS> ap;
     bool ok = true;
     for (int32_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       I8Tile t;
       i8_decode_tile<EPI, BN>(p, s_off, s_base, s_tau, tile, t);
-      for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i) {
-        const int stage = (int)(i % STAGES);
-        // A buffer i % ABUFS is free once stage i - ABUFS's MMAs are done
-        ok = mbar_wait(&full_bar[stage], (uint32_t)((i / STAGES) & 1), &s_abort) &&
-             (i < ABUFS ||
-              mbar_wait(&mma_bar[(i - ABUFS) % STAGES], (uint32_t)(((i - ABUFS) / STAGES) & 1), &s_abort));
+      for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i, sp.next(), ap.next()) {
+        const int stage = (int)sp.slot;
+        // A buffer ap.slot is free once stage i - ABUFS's MMAs are done
+        ok = mbar_wait(&full_bar[stage], sp.phase, &s_abort) &&
+             (i < ABUFS || mbar_wait(&mma_bar[lag.slot], lag.phase, &s_abort));
+        if (i >= ABUFS) lag.next();
         if (!ok) break;  // the issuer then stops at its own wait for this buffer
         tc_fence_after();
         const uint8_t* codes = smem + stage * C::STAGE_BYTES + C::B_BYTES + row_base;
-        const uint32_t acol = lane_base + kI8ACol0 + (uint32_t)((i % ABUFS) * C::ACOLS);
+        const uint32_t acol = lane_base + kI8ACol0 + ap.slot * (uint32_t)C::ACOLS;
 #pragma unroll
         for (int half = 0; half < CHUNKS / 2; ++half) {
           // chunks 2 half, 2 half + 1: 64 inputs -> 16 columns
@@ -429,7 +447,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&afull_bar[i % ABUFS]);
+        if (lane == 0) mbar_arrive(&afull_bar[ap.slot]);
       }
     }
     if (!ok) {
@@ -452,7 +470,8 @@ __global__ void __launch_bounds__(kI8Threads, 1)
 #pragma unroll
     for (int j = 0; j < TPW / 2; ++j) acc[j] = 0ull;
     bool ok = true;
-    int64_t i = 0;
+    RingPos<STAGES> sp;
+    RingPos<DBUFS> dp;
 
     // The tile's outputs: a[t] * acc / 16, SiLU * mul or fp32 partials.
     auto epilogue = [&](const I8Tile& t) {
@@ -514,10 +533,10 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     for (int32_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
       I8Tile t;
       i8_decode_tile<EPI, BN>(p, s_off, s_base, s_tau, tile, t);
-      for (int32_t kq = t.kq0; kq < t.kq1; ++kq, ++i) {
-        const int stage = (int)(i % STAGES);
-        const int db = (int)(i % DBUFS);
-        ok = ok && mbar_wait(&mma_bar[stage], (uint32_t)((i / STAGES) & 1), &s_abort);
+      for (int32_t kq = t.kq0; kq < t.kq1; ++kq, sp.next(), dp.next()) {
+        const int stage = (int)sp.slot;
+        const int db = (int)dp.slot;
+        ok = ok && mbar_wait(&mma_bar[stage], sp.phase, &s_abort);
         tc_fence_after();
         if (ok) {
           const uint8_t* st = smem + stage * C::STAGE_BYTES;
