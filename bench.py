@@ -708,7 +708,7 @@ def run_ours(args):
         dec = stage_report(out["decode"]["wl"], out["decode"], world, peaks,
                            "gate/up-projection GEMM (SwiGLU fused)", "expert_gemm_kernel<2,16>", "decode")
         dec_q4 = stage_report(out["decode_q4"]["wl"], out["decode_q4"], world, peaks,
-                              "4-bit gate/up-projection GEMM (SwiGLU fused)", "expert_gemm_q4_kernel<0,16>",
+                              "4-bit gate/up-projection GEMM (integer MMA, SwiGLU fused)", "expert_gemm_q4i8_kernel<0,16>",
                               "decode_q4", q4=True)
         kernels_per_step = 5 + (1 if (wl.capacity_factor > 0 and wl.drop_policy == 0) else 0)
         line = dict(

@@ -37,8 +37,9 @@
 //   warp 0       loads: the token operand (one bulk copy), the codes of 128
 //                weight rows (TMA, rows of KS / 2 bytes, swizzled to match)
 //                and their scales;
-//   warp 1       MMA issue: per scale block two K = 32 MMAs (A from tensor
-//                memory) into the block's own accumulator columns, then one
+//   warps 1, 14  MMA issue, each for half of a stage's scale blocks (on
+//                different schedulers): per block two K = 32 MMAs (A from
+//                tensor memory) into its own accumulator columns, then one
 //                commit per stage;
 //   warps 2-5    expanders, one per tensor-memory lane quarter (warp w owns
 //                rows 32 (w % 4) .. +31): the row's codes -> 16 (c - 8) into
@@ -62,11 +63,14 @@ namespace moe {
 
 namespace {
 
-// warps: 0 loads, 1 MMA issuer, 2-5 expanders, 6-13 scalers (two per lane
-// quarter, one per half of the token tile); warp w runs on scheduler w % 4
-// and reaches tensor-memory lanes 32 (w % 4) .. +31
-constexpr int kI8Threads = 448;
+// warps: 0 loads, 1 and 14 MMA issuers (the first and the second half of a
+// stage's scale blocks), 2-5 expanders, 6-13 scalers (two per lane quarter,
+// one per half of the token tile); warp w runs on scheduler w % 4 and
+// reaches tensor-memory lanes 32 (w % 4) .. +31.  Measured slower at
+// 16-token tiles: one issuer per block (four, twice the commits per stage)
+// and two expanders per lane quarter (four more warps on the schedulers).
 constexpr int kI8FirstScaler = 6;
+constexpr int kI8FirstExtraIssuer = 14;
 constexpr int kI8Scalers = 256;
 constexpr int kI8ACol0 = 256;               // A buffers start here; accumulators below
 constexpr int kI8TmemCols = 512;
@@ -89,6 +93,8 @@ struct I8Cfg {
   static constexpr int KS = i8_stage_inputs(BN);         // inputs per stage
   static constexpr int NB = KS / 64;                     // scale blocks per stage
   static constexpr int KH = KS / 128;                    // 128-byte slices of a token row per stage
+  static constexpr int ISSUERS = 2;
+  static constexpr int THREADS = 32 * (kI8FirstExtraIssuer + ISSUERS - 1);
   static constexpr int N = 2 * BN;                       // MMA N: the tokens' high bytes, then low bytes
   static constexpr int B_BYTES = KH * N * 128;           // token operand of a stage
   static constexpr int ROW_BYTES = KS / 2;               // codes of one weight row per stage
@@ -229,7 +235,7 @@ __device__ __forceinline__ uint32_t codes_lo_s8x16(uint32_t x) { return ((x << 4
 __device__ __forceinline__ uint32_t codes_hi_s8x16(uint32_t x) { return (x & 0xF0F0F0F0u) ^ 0x80808080u; }
 
 template <int EPI, int BN>
-__global__ void __launch_bounds__(kI8Threads, 1)
+__global__ void __launch_bounds__(I8Cfg<EPI, BN>::THREADS, 1)
     expert_gemm_q4i8_kernel(const __grid_constant__ CUtensorMap map_ca,   // codes: W1 or W2
                             const __grid_constant__ CUtensorMap map_cb,   // codes: W3
                             const __grid_constant__ CUtensorMap map_sa,   // scales: W1 or W2
@@ -253,7 +259,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
   float* xbuf = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES + C::XBUF_BYTES);
   uint64_t* full_bar = bars;                  // the loads of a stage
-  uint64_t* mma_bar = bars + STAGES;          // the stage's MMAs completed (one commit)
+  uint64_t* mma_bar = bars + STAGES;          // the stage's MMAs completed (one commit per issuer)
   uint64_t* free_bar = bars + 2 * STAGES;     // the 8 scalers read the stage's scales
   uint64_t* afull_bar = bars + 3 * STAGES;    // the 4 expanders wrote an A buffer
   uint64_t* dfree_bar = afull_bar + ABUFS;    // the 8 scalers read an accumulator set
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&mma_bar[s], 1);
+      mbar_init(&mma_bar[s], C::ISSUERS);
       mbar_init(&free_bar[s], 8);
     }
     for (int a = 0; a < ABUFS; ++a) mbar_init(&afull_bar[a], 4);
@@ -358,11 +364,13 @@ __global__ void __launch_bounds__(kI8Threads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp >= kI8FirstExtraIssuer) {
     if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
+      // ------------------------------------------------ MMA issuers
       // per stage: block b's two K = 32 MMAs into accumulator columns
-      // (i % DBUFS) DCOLS + b N, then one commit
+      // (i % DBUFS) DCOLS + b N, then one commit; the two issuers (on
+      // different schedulers) take the first and the second half of the blocks
+      const int b_lo = warp == 1 ? 0 : NB / 2, b_hi = warp == 1 ? NB / 2 : NB;
       int64_t i = 0;
       RingPos<STAGES> sp;
       RingPos<ABUFS> ap;
@@ -383,6 +391,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
           const uint32_t b0 = smem_u32(smem + stage * C::STAGE_BYTES);
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
+            if (b < b_lo || b >= b_hi) continue;
             // block b: 128-byte slice b / 2 of the token rows, 64 bytes into it
             const uint64_t b_desc = make_sdesc_sw128(b0 + (uint32_t)((b >> 1) * N * 128));
             umma_i8_ts(d + b * N, a0 + b * 16, b_desc + (uint64_t)(((b & 1) * 64) >> 4), C::IDESC, 0u);
@@ -715,7 +724,7 @@ cudaError_t launch_i8_one(const CUtensorMap& ca, const CUtensorMap& cb, const CU
   cudaError_t err =
       cudaFuncSetAttribute(expert_gemm_q4i8_kernel<EPI, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  return launch_k(expert_gemm_q4i8_kernel<EPI, BN>, dim3(num_sms), dim3(kI8Threads), C::SMEM_BYTES, s, pdl, ca, cb,
+  return launch_k(expert_gemm_q4i8_kernel<EPI, BN>, dim3(num_sms), dim3(C::THREADS), C::SMEM_BYTES, s, pdl, ca, cb,
                   sa, sb, p);
 }
 
