@@ -402,8 +402,14 @@ MOE_API moe_status moe_ep_combine_cap(const moe_shape *shape, int32_t world, con
  *          inputs of a row, stored block-major.
  *   w = (code - 8) * scale, code in 0 .. 15.
  * The expert matrices are W1, W3 [E, d_ff, d_model] and W2 [E, d_model, d_ff]
- * as in the bf16 entry points; the router stays fp32.  The GPU rounds each
- * dequantised weight to bf16 and accumulates in fp32. */
+ * as in the bf16 entry points; the router stays fp32.  Arithmetic on the
+ * GPU: for T <= 32 (token tiles of 16 and 32 slots per expert tile) the
+ * weights stay exact integers (code - 8) and each token slot's
+ * activations are rounded to 16-bit integers with one fp32 scale per slot
+ * (error at most half a step, 1.5e-5 of the slot's largest value); the
+ * per-64-input integer sums are exact and are scaled and added in fp32.  For
+ * larger tiles each dequantised weight is rounded to bf16 and the GEMM
+ * accumulates in fp32. */
 
 /* Quantises W [E, R, K] bf16 (device) into codes and scales (device, out):
  * per 64-input block s = bf16(absmax / 7) and code = 8 + clamp(round half to
@@ -415,7 +421,8 @@ MOE_API moe_status moe_quantize_q4(const moe_bf16 *W, int32_t E, int32_t R, int3
                                    moe_bf16 *scales, moe_stream_t stream);
 
 /* Workspace bytes the 4-bit entry points need for `shape` (0 if the shape is
- * invalid).  gemm_variant is ignored: the 4-bit GEMMs have one schedule. */
+ * invalid); for token tiles of 16 and 32 it includes the quantised
+ * activations.  gemm_variant is ignored: the 4-bit GEMMs stream the weights. */
 MOE_API size_t moe_workspace_size_q4(const moe_shape *shape);
 
 /* moe_grouped_swiglu with 4-bit expert weights (W1c/W1s, W3c/W3s, W2c/W2s
