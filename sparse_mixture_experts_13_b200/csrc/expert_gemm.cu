@@ -934,7 +934,10 @@ static int32_t prefetch_chunks(int num_sms) {
 
 void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits,
                    int32_t* splits1) {
-  int64_t b = ((T + 15) / 16) * 16;
+  // token tile: twice the mean slots per expert, rounded up to 16 (an
+  // expert's slots usually fit one tile; smaller tiles mean smaller stages,
+  // more of them in flight, and a shorter epilogue)
+  int64_t b = ((2 * ((T * k + E - 1) / E) + 15) / 16) * 16;
   if (b < 16) b = 16;
   if (b > 128) b = 128;
   if (b > 64) b = 128;

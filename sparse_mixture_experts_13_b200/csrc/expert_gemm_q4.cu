@@ -634,7 +634,11 @@ cudaError_t launch_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
 }  // namespace
 
 void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
-  int64_t b = ((T + 15) / 16) * 16;
+  // token tile: twice the mean slots per expert, so that an expert's slots
+  // usually fit one tile (a second tile streams the expert's weights again)
+  // while the integer-MMA kernels' per-token work is not spent on empty
+  // columns (T = 32 with 8 experts and top-2: 16, not 32)
+  int64_t b = ((2 * ((T * k + E - 1) / E) + 15) / 16) * 16;
   if (b < 16) b = 16;
   if (b > 64) b = 128;
   else if (b > 32) b = 64;

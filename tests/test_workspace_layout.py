@@ -83,19 +83,20 @@ def test_streaming_layout_adds_splitk_planes(moe, T, d, f):
     assert _splits(extra, T * 2, d) is not None, extra
 
 
-@pytest.mark.parametrize("T", [16, 32, 33, 300])
+@pytest.mark.parametrize("T", [16, 32, 33, 64, 65, 300])
 def test_q4_layout_always_has_splitk_planes(moe, T):
     """The 4-bit layout adds split-K planes and, for token tiles of 16 and 32
-    (T <= 32, the integer-MMA kernels), the quantised activations as their
-    tiled token operand and their scales [S] fp32 at the end.  The operand
+    (twice the mean slots per expert, up to T = 64 for 8 experts and top-2:
+    the integer-MMA kernels), the quantised activations as their tiled token
+    operand and their scales [S] fp32 at the end.  The operand
     holds, per token tile (at most S / bn + E of them) and stage of ks inputs
     (256 for 16-token tiles, 128 for 32), the high and low bytes of the
     tile's bn rows: 2 bn x ks bytes."""
     sh = moe.make_shape(T, 4096, 14336)
     extra = moe.moe_workspace_size_q4(sh) - expected(T, 4096, 14336, 8, 2)
     S = T * 2
-    if T <= 32:
-        bn = 16 if T <= 16 else 32
+    bn = -(-2 * -(-S // 8) // 16) * 16    # token tile: twice the mean slots per expert, rounded up to 16
+    if bn <= 32:
         ks = 256 if bn == 16 else 128
         tiles = -(-S // bn) + 8
         extra -= al(tiles * -(-14336 // ks) * 2 * bn * ks) + al(4 * S)
