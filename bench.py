@@ -767,6 +767,10 @@ def run_sweep(args):
     cases = [("tiny", None), ("decode", None), ("prefill", None), ("skew", None)] + \
             [("sweep", T) for T in synth.SWEEP_T]
     for name, T in cases:
+        # a second of idle between workloads, so that one workload's power-capped
+        # clock does not carry into the next
+        torch.cuda.synchronize()
+        time.sleep(1.0)
         wl = synth.workload(name, T=T)
         wl.generate(weights=(name == "tiny"))
         if name == "tiny":
