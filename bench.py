@@ -82,15 +82,20 @@ def strip_c_comments(text: str) -> str:
     return " ".join("".join(out).split())
 
 
-def kernel_source_sha(root: str = None) -> str:
-    """Hash of the CUDA sources (comments and layout ignored)."""
+def kernel_source_sha(root: str = None, files=None) -> str:
+    """Hash of the CUDA sources (comments and layout ignored): the named
+    files of the source folder, else all of them."""
     import hashlib
     src = os.path.join(root or ROOT, "sparse_mixture_experts_13_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(src)):
+    names = sorted(files) if files else sorted(os.listdir(src))
+    for name in names:
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(src, name), encoding="utf-8") as fh:
-                h.update(strip_c_comments(fh.read()).encode())
+            try:
+                with open(os.path.join(src, name), encoding="utf-8") as fh:
+                    h.update(strip_c_comments(fh.read()).encode())
+            except OSError:
+                h.update(b"\0missing:" + name.encode())
     return h.hexdigest()[:16]
 
 
@@ -104,9 +109,11 @@ def traffic_record(kernel: str, workload: str):
             recs = json.load(fh)
     except (OSError, ValueError):
         return None
-    sha = kernel_source_sha(ROOT)
     for r in recs:
-        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
+        if r.get("kernel") != kernel or r.get("workload") != workload:
+            continue
+        # a record names the files its kernel is built from; the others may change
+        if r.get("source_sha") == kernel_source_sha(ROOT, r.get("source_files")):
             return r.get("dram_bytes_per_launch")
     return None
 

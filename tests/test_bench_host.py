@@ -89,6 +89,25 @@ def test_traffic_record_only_for_unchanged_kernels(tmp_path, monkeypatch):
     assert bench.traffic_record("k", "w") is None   # the kernel changed since the capture
 
 
+def test_traffic_record_scoped_to_its_files(tmp_path, monkeypatch):
+    code = "__global__ void k(int* p) { p[0] = 1; }\n"
+    _fake_tree(tmp_path, code)
+    csrc = tmp_path / "sparse_mixture_experts_13_b200" / "csrc"
+    (csrc / "other.cu").write_text("__global__ void o(int* p) { p[0] = 3; }\n")
+    sha = bench.kernel_source_sha(str(tmp_path), ["k.cu"])
+    assert sha != bench.kernel_source_sha(str(tmp_path))
+    rec = [dict(kernel="k", workload="w", source_sha=sha, source_files=["k.cu"], dram_bytes_per_launch=77)]
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_record("k", "w") == 77
+    (csrc / "other.cu").write_text("__global__ void o(int* p) { p[0] = 4; }\n")
+    assert bench.traffic_record("k", "w") == 77     # a file the kernel is not built from changed
+    (csrc / "k.cu").write_text(code.replace("p[0] = 1", "p[0] = 2"))
+    assert bench.traffic_record("k", "w") is None   # its own source changed
+    (csrc / "k.cu").unlink()
+    assert bench.traffic_record("k", "w") is None   # or went away
+
+
 def test_traffic_record_missing_file(tmp_path, monkeypatch):
     _fake_tree(tmp_path, "x")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
