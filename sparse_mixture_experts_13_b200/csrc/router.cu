@@ -44,34 +44,40 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
-// Lane e < E holds the logit l of expert e for token t (other lanes: any
-// value).  Every lane ranks its expert in the order (logit descending, index
-// ascending), so the experts of rank < k are the top-k, rank 0 first, and
-// ranks k .. 2k-1 are the next-best candidates.  With m the largest logit,
-// the gate of a chosen expert is exp(l - m) over the sum of exp(l' - m) of the
-// k chosen ones, and its full-softmax probability is exp(l - m) over the sum
-// across all E experts.  The sums are butterflies over the first EMAX lanes
-// (a fixed order).  Lane e writes the slot of its rank and counts it in *hist.
-template <int EMAX>
-__device__ __forceinline__ void finish_token(const RouterArgs& a, int64_t t, float l, int lane, int* hist) {
+// Lane e < E of a segment of SEG lanes holds the logit l of expert e for
+// token t (other lanes of the segment: any value; `lane` is the index within
+// the segment).  Every lane ranks its expert in the order (logit
+// descending, index ascending), so the experts of rank < k are the top-k,
+// rank 0 first, and ranks k .. 2k-1 are the next-best candidates.  With m
+// the largest logit, the gate of a chosen expert is exp(l - m) over the sum
+// of exp(l' - m) of the k chosen ones, and its full-softmax probability is
+// exp(l - m) over the sum across all E experts.  The sums are butterflies
+// over the first EMAX lanes of the segment (a fixed order).  Lane e writes
+// the slot of its rank and counts it in *hist.  Every lane of the warp calls
+// this (the shuffles span it); a segment with `active` false writes nothing.
+template <int EMAX, int SEG = 32>
+__device__ __forceinline__ void finish_token(const RouterArgs& a, int64_t t, float l, int lane, int* hist,
+                                             bool active = true) {
+  static_assert(EMAX <= SEG, "the experts of a token fit its segment");
   const int E = a.E, k = a.k;
   const bool valid = lane < E;
   int rank = 0;
 #pragma unroll
   for (int e = 0; e < EMAX; ++e) {
-    const float le = __shfl_sync(0xffffffffu, l, e);
+    const float le = __shfl_sync(0xffffffffu, l, e, SEG);
     if (e < E && (le > l || (le == l && e < lane))) ++rank;
   }
   float m = valid ? l : -FLT_MAX;
 #pragma unroll
-  for (int off = EMAX / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int off = EMAX / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off, SEG));
   const float ex = valid ? expf(l - m) : 0.f;
   float zE = ex, zk = (valid && rank < k) ? ex : 0.f;
 #pragma unroll
   for (int off = EMAX / 2; off > 0; off >>= 1) {
-    zE += __shfl_xor_sync(0xffffffffu, zE, off);
-    zk += __shfl_xor_sync(0xffffffffu, zk, off);
+    zE += __shfl_xor_sync(0xffffffffu, zE, off, SEG);
+    zk += __shfl_xor_sync(0xffffffffu, zk, off, SEG);
   }
+  if (!active) return;
   if (valid && rank < k) {
     a.topk_idx[t * k + rank] = lane;
     a.topk_w[t * k + rank] = ex / zk;
@@ -347,24 +353,46 @@ static cudaError_t launch_router_reg(const RouterArgs& a, int num_sms, cudaStrea
 }
 
 // ---------------------------------------------------------------- tensor-core router
-// router_mma_kernel (E <= 8, d a multiple of 256 up to 4096): the logits of a
-// tile of 8 tokens by mma.sync m16n8k16 (bf16 operands, fp32 accumulation).
-// x is exact in bf16, and every fp32 weight is split exactly into three bf16
-// terms, w = hi + mid + lo (8 + 8 + 8 significant bits, by truncation), so the three
-// MMAs per 16 inputs multiply exactly by the fp32 weights and the products
-// add up in fp32.  Each of the 16 warps owns d/16 inputs and keeps its slice
-// of the three weight terms as MMA B fragments for the whole launch (hi and
-// mid in registers, lo in shared memory); the token rows arrive by bulk
-// copies, one per row, into a ring of two tiles with rows 16 bytes further
-// apart than their length, and are read by ldmatrix.  The MMA's rows 8..15
-// repeat rows 0..7 (ignored).  Per tile each warp leaves its 8 x 8
-// partial logits in shared memory; the partials are added in warp order and
-// warp t finishes token t.
-constexpr int kMmaTile = 8;     // tokens per tile
-constexpr int kMmaWarps = 16;
-constexpr int kMmaSlots = 2;
-constexpr int kMmaMaxSteps = 16;  // 16-input steps per warp (d <= 4096)
+// router_mma_kernel (E <= 8, d a multiple of 512 up to 4096): the logits of a
+// tile of 16 tokens by mma.sync m16n8k16 (bf16 operands, fp32 accumulation),
+// computed by a cluster of 4 CTAs that split d four ways.  x is exact in bf16,
+// and every fp32 weight is split exactly into three bf16 terms, w = hi + mid
+// + lo (8 + 8 + 8 significant bits, by truncation), so the three MMAs per 16
+// inputs multiply exactly by the fp32 weights and the products add up in fp32.
+//
+// CTA c of a cluster owns inputs [c d/4, (c+1) d/4) and reads only that
+// quarter of W_g; each of its 8 MMA warps owns d/32 of those inputs and keeps
+// its slice of the three weight terms in registers as MMA B fragments for the
+// whole launch.  The CTAs of a cluster walk the same token tiles.  A producer
+// warp brings a CTA's quarter of each tile's 16 rows into a ring of
+// shared-memory slots with one TMA load, viewed as (64 inputs, 16 rows, d/256
+// chunks of 64) so that the slot holds chunk-major 128-byte rows with the
+// 128-byte swizzle: the 8 token rows one ldmatrix reads fall in distinct bank
+// groups.  Each MMA warp pushes its partial logits of tokens 4c' .. 4c'+3
+// straight into CTA c''s receive ring with asynchronous remote stores
+// counted on that CTA's mbarrier, and frees the slot.  Four finishing warps
+// take the tiles in turn: for each of the CTA's four tokens of a tile (one
+// 8-lane segment each) they add the 32 partials (CTA order, then warp order),
+// finish the token and tell the senders that the ring entry was read (a
+// relaxed remote arrive).  No step needs a cluster-wide fence, and loads,
+// MMAs and finishing overlap across tiles.
+constexpr int kMmaCtas = 4;       // cluster size: d split four ways
+constexpr int kMmaWarps = 8;      // MMA warps
+constexpr int kMmaTile = 16;      // tokens per tile (the MMA's M)
+constexpr int kMmaSlots = 4;      // ring of token tiles per CTA
+constexpr int kMmaMaxSteps = 8;   // 16-input steps per MMA warp (d <= 4096)
+constexpr int kMmaRecv = 8;       // receive ring of a CTA's partial logits (tiles)
+constexpr int kMmaPerCta = kMmaTile / kMmaCtas;  // tokens each CTA finishes per tile
+constexpr int kMmaProducer = kMmaWarps;          // the warp that issues the tile loads
+constexpr int kMmaFinishers = 4;                 // finishing warps, tiles in turn
+constexpr int kMmaFinisher0 = kMmaProducer + 1;
+constexpr int kMmaThreads = 32 * (kMmaFinisher0 + kMmaFinishers);
+// one tile's partials into one CTA: [sender CTA][MMA warp][token][expert] fp32
+constexpr uint32_t kMmaRecvFloats = kMmaCtas * kMmaWarps * kMmaPerCta * 8;
+constexpr uint32_t kMmaRecvBytes = kMmaRecvFloats * 4;
 constexpr int64_t kMmaMinTokens = 1024;
+static_assert(kMmaPerCta * 8 == 32, "a finishing warp holds one CTA's tokens of a tile, 8 lanes per token");
+static_assert(kMmaRecv % kMmaFinishers == 0, "a ring entry is always finished by the same warp");
 
 // w -> (hi, mid, lo) bf16 bits with hi + mid + lo == w exactly: hi keeps the
 // top 8 significant bits of w (truncation), mid the next 8 of the remainder,
@@ -393,155 +421,294 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// a tile's rows in shared memory, 16 bytes more apart than a row, so the 8
-// rows that one ldmatrix reads fall in distinct bank groups
-__host__ __device__ constexpr size_t mma_row_pitch(int d) { return (size_t)d * 2 + 16; }
-__host__ __device__ constexpr size_t mma_slot_bytes(int d) { return (((size_t)kMmaTile * mma_row_pitch(d)) + 127) / 128 * 128; }
-// lo fragments: [warp][step][lane] uint2
-__host__ __device__ constexpr size_t mma_lo_bytes(int d) { return (size_t)kMmaWarps * (d / (16 * kMmaWarps)) * 32 * 8; }
-__host__ __device__ constexpr size_t mma_smem_bytes(int d) {
-  return 1024 + kMmaSlots * mma_slot_bytes(d) + mma_lo_bytes(d) + sizeof(float) * 2 * kMmaWarps * kMmaTile * 8 +
-         sizeof(uint64_t) * kMmaSlots + sizeof(int) * 32;
+// 8-byte asynchronous store into a cluster peer's shared memory, counted (as
+// transaction bytes) on the peer's mbarrier at `bar`
+__device__ __forceinline__ void st_async_f32x2(uint32_t cluster_addr, float v0, float v1, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+                   cluster_addr),
+               "f"(v0), "f"(v1), "r"(bar)
+               : "memory");
+}
+// arrive on named barrier `id` (of `nthreads` threads) without waiting
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// split-phase cluster barrier: a relaxed arrive (no ordering of this thread's
+// memory operations) and an acquiring wait
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// arrive on a (possibly remote) mbarrier without ordering this thread's
+// earlier memory operations: the reads it reports have been consumed already
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-__global__ void __launch_bounds__(kMmaWarps * 32, 1)
-    router_mma_kernel(RouterArgs a, int64_t ntiles) {
+// a slot: a CTA's quarter of 16 token rows, chunk-major rows of 64 inputs
+__host__ __device__ constexpr size_t mma_slot_bytes(int d) { return (size_t)kMmaTile * (d / kMmaCtas) * 2; }
+__host__ __device__ constexpr size_t mma_smem_bytes(int d) {
+  return 1024 + kMmaSlots * mma_slot_bytes(d) + (size_t)kMmaRecv * kMmaRecvBytes +
+         sizeof(uint64_t) * 2 * (kMmaSlots + kMmaRecv) + sizeof(int) * 32;
+}
+
+__global__ void __launch_bounds__(kMmaThreads, 1)
+    router_mma_kernel(const __grid_constant__ CUtensorMap xmap, RouterArgs a, int64_t ntiles, int64_t nclusters) {
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();  // the grouping kernel may launch now; it waits for this grid
+  // the 128-byte swizzle repeats every 1024 bytes: slots start on that boundary
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int d = a.d, E = a.E;
+  const int dq = d / kMmaCtas;                 // inputs of this CTA
+  const int chunks = dq / 64;                  // 64-input chunks of this CTA
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int crank = (int)cluster_ctarank();
+  const int64_t cl = blockIdx.x / kMmaCtas;    // the cluster (its CTAs are consecutive blocks)
   const size_t slot_bytes = mma_slot_bytes(d);
-  uint2* s_lo = reinterpret_cast<uint2*>(smem + kMmaSlots * slot_bytes);     // [warps][steps][32]
-  float* s_part = reinterpret_cast<float*>(smem + kMmaSlots * slot_bytes + mma_lo_bytes(d));  // [2][warps][8][8]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_part + 2 * kMmaWarps * kMmaTile * 8);
-  int* s_count = reinterpret_cast<int*>(bars + kMmaSlots);
+  float* s_recv = reinterpret_cast<float*>(smem + kMmaSlots * slot_bytes);    // [ring][kMmaRecvFloats]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_recv + kMmaRecv * kMmaRecvFloats);  // a slot is loaded
+  uint64_t* empty = full + kMmaSlots;           // the MMA warps have read a slot
+  uint64_t* recv_full = empty + kMmaSlots;      // a ring entry holds every partial of its tile
+  uint64_t* recv_empty = recv_full + kMmaRecv;  // every CTA has read what this CTA sent to an entry
+  int* s_count = reinterpret_cast<int*>(recv_empty + kMmaRecv);
 
-  const int64_t g0 = blockIdx.x, gstride = gridDim.x;
-  const int64_t my_tiles = g0 < ntiles ? (ntiles - 1 - g0) / gstride + 1 : 0;
+  // every CTA of a cluster has the same tiles: cl, cl + nclusters, ...
+  const int64_t my_tiles = cl < ntiles ? (ntiles - 1 - cl) / nclusters + 1 : 0;
   if (tid < 32) s_count[tid] = 0;
-  if (tid == 0) {
-    for (int i = 0; i < kMmaSlots; ++i) mbar_init(&bars[i], 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
-  const size_t row_pitch = mma_row_pitch(d);
-  auto issue = [&](int64_t j) {  // this block's j-th tile into slot j % 2: one bulk copy per token row
-    const int64_t t0 = (g0 + j * gstride) * kMmaTile;
-    const int rows = (int)(a.T - t0 < kMmaTile ? a.T - t0 : kMmaTile);
-    uint8_t* dst = smem + (size_t)(j % kMmaSlots) * slot_bytes;
-    uint64_t* bar = &bars[j % kMmaSlots];
-    mbar_arrive_expect_tx(bar, (uint32_t)(rows * d * 2));
-    for (int r = 0; r < rows; ++r) bulk_load(dst + r * row_pitch, a.x + (t0 + r) * d, (uint32_t)(d * 2), bar);
+  auto issue = [&](int64_t j) {  // this CTA's quarter of tile j's rows into slot j % kMmaSlots
+    uint64_t* bar = &full[j % kMmaSlots];
+    mbar_arrive_expect_tx(bar, (uint32_t)slot_bytes);  // rows past T are zero-filled and counted
+    tma_load_3d(&xmap, bar, smem + (size_t)(j % kMmaSlots) * slot_bytes, 0,
+                (int32_t)((cl + j * nclusters) * kMmaTile), crank * chunks);
   };
-  if (tid == 0)
-    for (int64_t j = 0; j < my_tiles && j < kMmaSlots; ++j) issue(j);
 
   // B fragments of this warp's inputs: lane l holds expert l / 4 at inputs
-  // 2 (l % 4) + {0, 1} and + {8, 9} of each 16-input step
-  const int steps = d / (16 * kMmaWarps);
+  // 2 (l % 4) + {0, 1} and + {8, 9} of each 16-input step.  All of the
+  // warp's W_g loads are issued before the first token tile is requested
+  // (so they do not queue behind it) and before any is split.
+  const int steps = dq / (16 * kMmaWarps);
   const int n = lane >> 2, kq = 2 * (lane & 3);
-  uint32_t bh[kMmaMaxSteps][2], bm[kMmaMaxSteps][2];
-  uint2* my_lo = s_lo + (size_t)warp * steps * 32 + lane;
-  // W_g comes from HBM at every launch: the loads of half the steps are
-  // issued together before any is split, so the warp waits for two memory
-  // round trips rather than one per step
-  constexpr int kHalf = kMmaMaxSteps / 2;
+  uint32_t bh[kMmaMaxSteps][2], bm[kMmaMaxSteps][2], bl[kMmaMaxSteps][2];
+  float2 u[kMmaMaxSteps], v[kMmaMaxSteps];
+  if (warp < kMmaWarps) {
+    const int k_warp = crank * dq + warp * steps * 16;  // first input of this warp
 #pragma unroll
-  for (int ph = 0; ph < 2; ++ph) {
-    float2 u[kHalf], v[kHalf];
-#pragma unroll
-    for (int q = 0; q < kHalf; ++q) {
-      const int ks = ph * kHalf + q;
+    for (int q = 0; q < kMmaMaxSteps; ++q) {
       u[q] = v[q] = make_float2(0.f, 0.f);
-      if (ks < steps && n < E) {
-        const float* row = a.Wg + (int64_t)n * d + warp * (steps * 16) + ks * 16 + kq;
+      if (q < steps && n < E) {
+        const float* row = a.Wg + (int64_t)n * d + k_warp + q * 16 + kq;
         u[q] = *reinterpret_cast<const float2*>(row);
         v[q] = *reinterpret_cast<const float2*>(row + 8);
       }
     }
+  }
+  // the producer requests the first tiles once the W_g loads are out
+  if (warp < kMmaWarps) named_bar_arrive(2, 32 * (kMmaWarps + 1));
+  else if (warp == kMmaProducer) named_bar_sync(2, 32 * (kMmaWarps + 1));
+  int64_t issued = 0;  // producer lane 0: tiles whose loads were issued
+  if (warp == kMmaProducer && lane == 0) {
+    tma_prefetch_desc(&xmap);
+    for (int i = 0; i < kMmaSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kMmaWarps);
+    }
+    for (int i = 0; i < kMmaRecv; ++i) {
+      mbar_init(&recv_full[i], 1);
+      mbar_init(&recv_empty[i], kMmaCtas);
+      if (i < my_tiles) mbar_arrive_expect_tx(&recv_full[i], kMmaRecvBytes);
+    }
+    fence_barrier_init();
+    for (; issued < my_tiles && issued < kMmaSlots; ++issued) issue(issued);
+  }
+  if (warp < kMmaWarps) {
 #pragma unroll
-    for (int q = 0; q < kHalf; ++q) {
-      const int ks = ph * kHalf + q;
+    for (int q = 0; q < kMmaMaxSteps; ++q) {
       const float w[4] = {u[q].x, u[q].y, v[q].x, v[q].y};
       uint32_t h[4], m[4], lo[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) split3(w[c], h[c], m[c], lo[c]);
-      bh[ks][0] = h[0] | (h[1] << 16);
-      bh[ks][1] = h[2] | (h[3] << 16);
-      bm[ks][0] = m[0] | (m[1] << 16);
-      bm[ks][1] = m[2] | (m[3] << 16);
-      if (ks < steps) my_lo[ks * 32] = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+      bh[q][0] = h[0] | (h[1] << 16);
+      bh[q][1] = h[2] | (h[3] << 16);
+      bm[q][0] = m[0] | (m[1] << 16);
+      bm[q][1] = m[2] | (m[3] << 16);
+      bl[q][0] = lo[0] | (lo[1] << 16);
+      bl[q][1] = lo[2] | (lo[3] << 16);
     }
   }
-  __syncwarp();
-  // ldmatrix rows: thread l addresses row l % 8 of matrix l / 8 (matrices 0, 1:
-  // inputs 0..7 of the step, 2, 3: inputs 8..15; rows 8..15 of the MMA repeat
-  // rows 0..7)
-  const int lr = lane & 7, lhalf = (lane >> 4) & 1;
+  __syncthreads();  // this CTA's barrier inits and zeroed counts are visible to its threads
+  // every CTA's mbarriers are initialised (and the init fenced) before any
+  // peer stores or arrives on them; nothing else needs ordering here
+  cluster_arrive_relaxed();
+  cluster_wait();
 
   bool ok = true;
-  for (int64_t j = 0; j < my_tiles; ++j) {
-    const int slot = (int)(j % kMmaSlots);
-    const int64_t t0 = (g0 + j * gstride) * kMmaTile;
-    if (ok) ok = mbar_wait(&bars[slot], (uint32_t)((j / kMmaSlots) & 1), nullptr);
-    // three independent accumulators (one per weight term) keep the MMAs of
-    // a step from waiting on each other; they are added at the end
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
-    if (ok) {
-      float ch[4] = {}, cm[4] = {}, cl[4] = {};
-      const uint32_t base = smem_u32(smem + (size_t)slot * slot_bytes);
+  if (warp < kMmaWarps) {
+    // ldmatrix rows: thread l addresses row l % 8 of matrix l / 8; matrices
+    // 0..3 are (tokens 0-7, inputs 0-7), (tokens 8-15, inputs 0-7), (tokens
+    // 0-7, inputs 8-15), (tokens 8-15, inputs 8-15): the A fragment's order.
+    // Token row r of chunk c is the 128-byte row 16 c + r of the slot, whose
+    // 16-byte pieces are permuted by r % 8 (the swizzle).
+    const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8, lpiece = lane >> 4;
+    // this lane's partials: tokens n and n + 8 (finished by CTAs n / 4 and
+    // n / 4 + 2, as their token n % 4), experts kq and kq + 1
+    const uint32_t dst_off =
+        (uint32_t)(((crank * kMmaWarps + warp) * kMmaPerCta + (n % kMmaPerCta)) * 8 + kq) * 4;
+    const uint32_t dst_rank0 = (uint32_t)(n / kMmaPerCta), dst_rank1 = dst_rank0 + 2;
+    for (int64_t j = 0; j < my_tiles; ++j) {
+      const int slot = (int)(j % kMmaSlots);
+      if (ok) ok = mbar_wait(&full[slot], (uint32_t)((j / kMmaSlots) & 1), nullptr);
+      // six independent accumulators (one per weight term and step parity)
+      // keep the MMAs of consecutive steps from waiting on each other
+      float acc[6][4];
 #pragma unroll
-      for (int ks = 0; ks < kMmaMaxSteps; ++ks) {
-        if (ks < steps) {
-          const int k0 = warp * (steps * 16) + ks * 16;     // first input of the step
-          const uint32_t addr = base + (uint32_t)(lr * row_pitch + k0 * 2 + lhalf * 16);
-          uint32_t af[4];
-          ldmatrix_x4(addr, af);
-          const uint2 bl = my_lo[ks * 32];
-          mma_bf16_16816(ch, af, bh[ks][0], bh[ks][1]);
-          mma_bf16_16816(cm, af, bm[ks][0], bm[ks][1]);
-          mma_bf16_16816(cl, af, bl.x, bl.y);
+      for (int q = 0; q < 6; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+      if (ok) {
+        const uint32_t base = smem_u32(smem + (size_t)slot * slot_bytes);
+#pragma unroll
+        for (int ks = 0; ks < kMmaMaxSteps; ++ks) {
+          if (ks < steps) {
+            const int k0 = warp * steps * 16 + ks * 16;  // first input of the step in this CTA's quarter
+            const uint32_t row = (uint32_t)((k0 >> 6) * kMmaTile + lrow);
+            const uint32_t piece = (uint32_t)(((k0 & 63) >> 3) + lpiece);
+            uint32_t af[4];
+            ldmatrix_x4(base + row * 128 + ((piece ^ (row & 7)) << 4), af);
+            float (&ch)[4] = acc[(ks & 1) * 3], (&cm)[4] = acc[(ks & 1) * 3 + 1], (&cq)[4] = acc[(ks & 1) * 3 + 2];
+            mma_bf16_16816(ch, af, bh[ks][0], bh[ks][1]);
+            mma_bf16_16816(cm, af, bm[ks][0], bm[ks][1]);
+            mma_bf16_16816(cq, af, bl[ks][0], bl[ks][1]);
+          }
         }
       }
+      __syncwarp();  // the warp's reads of the slot are done
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      float c[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) c[q] = (ch[q] + cm[q]) + cl[q];
+      for (int q = 0; q < 4; ++q)
+        c[q] = ((acc[0][q] + acc[3][q]) + (acc[1][q] + acc[4][q])) + (acc[2][q] + acc[5][q]);
+      // into the finishing CTAs' ring entry, once every CTA has read tile j - ring from it
+      const int b = (int)(j % kMmaRecv);
+      if (j >= kMmaRecv && !mbar_wait(&recv_empty[b], (uint32_t)(((j / kMmaRecv) + 1) & 1), nullptr)) ok = false;
+      const uint32_t dst = smem_u32(s_recv + (size_t)b * kMmaRecvFloats) + dst_off;
+      const uint32_t bar = smem_u32(&recv_full[b]);
+      st_async_f32x2(map_to_rank(dst, dst_rank0), c[0], c[1], map_to_rank(bar, dst_rank0));
+      st_async_f32x2(map_to_rank(dst, dst_rank1), c[2], c[3], map_to_rank(bar, dst_rank1));
     }
-    // c[0], c[1]: token lane / 4, experts kq, kq + 1
-    float* part = s_part + (j & 1) * kMmaWarps * kMmaTile * 8;
-    *reinterpret_cast<float2*>(part + (warp * kMmaTile + n) * 8 + kq) = make_float2(c[0], c[1]);
-    if (!__syncthreads_and(ok)) {
-      // a tile never arrived: report, let the copies still in flight land, leave
-      if (tid == 0) {
-        record_status(a.status, kStatusTimeout);
-        for (int64_t q = j; q < my_tiles && q < j + kMmaSlots; ++q)
-          mbar_wait(&bars[q % kMmaSlots], (uint32_t)((q / kMmaSlots) & 1), nullptr, kWaitLimitNs / 8);
+    if (!ok && lane == 0) record_status(a.status, kStatusTimeout);
+  } else if (warp == kMmaProducer) {
+    if (lane == 0) {
+      // refill each slot once all MMA warps have read it
+      for (; issued < my_tiles; ++issued) {
+        const int64_t prev = issued - kMmaSlots;
+        if (!mbar_wait(&empty[prev % kMmaSlots], (uint32_t)((prev / kMmaSlots) & 1), nullptr)) {
+          record_status(a.status, kStatusTimeout);
+          break;
+        }
+        issue(issued);
       }
-      return;
+      // a CTA leaves only with no load in flight (the MMA warps wait for
+      // every load, but may have given up on one)
+      for (int64_t q = issued - kMmaSlots > 0 ? issued - kMmaSlots : 0; q < issued; ++q)
+        mbar_wait(&full[q % kMmaSlots], (uint32_t)((q / kMmaSlots) & 1), nullptr, kWaitLimitNs / 8);
     }
-    if (tid == 0 && j + kMmaSlots < my_tiles) issue(j + kMmaSlots);
-    // warp w < 8 finishes token t0 + w: lane e < 8 adds the 16 warps' partials in warp order
-    if (warp < kMmaTile && t0 + warp < a.T) {
+  } else {
+    // finishing warp f: tiles f, f + 4, ...; segment s (lanes 8s .. 8s+7)
+    // finishes token 4 crank + s of the tile, lane e of the segment the logit
+    // of expert e: the partials of the four CTAs' eight warps, CTA order,
+    // warp order within a CTA
+    const int f = warp - kMmaFinisher0, seg = lane >> 3, e = lane & 7;
+    for (int64_t jj = f; jj < my_tiles; jj += kMmaFinishers) {
+      const int b = (int)(jj % kMmaRecv);
+      const int64_t t = (cl + jj * nclusters) * kMmaTile + crank * kMmaPerCta + seg;
+      const bool okf = mbar_wait(&recv_full[b], (uint32_t)((jj / kMmaRecv) & 1), nullptr);
+      // the entry's next use (tile jj + ring, this warp's too) expects its
+      // bytes again; they come only after this warp reports the entry read
+      if (lane == 0 && okf && jj + kMmaRecv < my_tiles) mbar_arrive_expect_tx(&recv_full[b], kMmaRecvBytes);
       float v = 0.f;
-      if (lane < 8) {
+      if (okf) {
+        const float* r = s_recv + (size_t)b * kMmaRecvFloats + seg * 8 + e;
 #pragma unroll
-        for (int ww = 0; ww < kMmaWarps; ++ww) v += part[(ww * kMmaTile + warp) * 8 + lane];
+        for (int c = 0; c < kMmaCtas; ++c) {
+          float sc = 0.f;
+#pragma unroll
+          for (int w = 0; w < kMmaWarps; ++w) sc += r[(c * kMmaWarps + w) * kMmaPerCta * 8];
+          v += sc;
+        }
       }
-      finish_token<8>(a, t0 + warp, v, lane, s_count);
+      __syncwarp();  // v holds the sums: the senders may reuse the entry
+      // (only entries that are used again are reported, so that every arrive
+      // on a peer is awaited by that peer before it exits)
+      if (lane < kMmaCtas && jj + kMmaRecv < my_tiles)
+        mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&recv_empty[b]), (uint32_t)lane));
+      if (!okf && lane == 0) record_status(a.status, kStatusTimeout);
+      finish_token<8, 8>(a, t, v, e, s_count, okf && t < a.T);
     }
   }
+  // A CTA may leave now: every store a peer makes into it (a ring entry) and
+  // every arrive on it (an entry read, reported only for entries in use
+  // again) is awaited before this point.
   __syncthreads();
   if (tid < E && s_count[tid] != 0) atomicAdd(&a.counts[tid], s_count[tid]);
 }
 
-static cudaError_t launch_router_mma(const RouterArgs& a, int num_sms, cudaStream_t s) {
+// clusters of 4 router CTAs that can be resident at once on this device
+static int router_mma_clusters(const cudaLaunchConfig_t& cfg) {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = -1;
+  if (dev >= 0 && cached[dev] > 0) return cached[dev];
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, router_mma_kernel, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    clusters = 0;
+  }
+  if (dev >= 0 && clusters > 0) cached[dev] = clusters;
+  return clusters;
+}
+
+// x as (64 inputs, T rows, d / 64 chunks): strides 2 bytes, d * 2 bytes, 128
+// bytes; a box is a CTA's quarter of 16 rows, stored chunk-major with the
+// 128-byte swizzle.  False if the driver refuses the map.
+static bool encode_router_map(CUtensorMap* m, const uint16_t* x, int64_t T, int d) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)(d / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)kMmaTile, (cuuint32_t)(d / kMmaCtas / 64)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// false: the tensor-core router cannot take this launch (the caller uses another)
+static bool launch_router_mma(const RouterArgs& a, int num_sms, cudaStream_t s, cudaError_t* err) {
+  CUtensorMap xmap;
+  if (!encode_router_map(&xmap, a.x, a.T, a.d)) return false;
   const size_t smem = mma_smem_bytes(a.d);
-  cudaError_t err = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
+  *err = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (*err != cudaSuccess) return true;
   const int64_t ntiles = (a.T + kMmaTile - 1) / kMmaTile;
-  const int64_t grid = ntiles < num_sms ? ntiles : num_sms;
-  router_mma_kernel<<<(unsigned)grid, kMmaWarps * 32, smem, s>>>(a, ntiles);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kMmaCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kMmaThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // as many clusters as fit at once (each walks several tiles), at most one per tile
+  int64_t nclusters = num_sms / kMmaCtas;
+  cfg.gridDim = dim3((unsigned)(nclusters * kMmaCtas), 1, 1);
+  const int fit = router_mma_clusters(cfg);
+  if (fit > 0 && fit < nclusters) nclusters = fit;
+  if (ntiles < nclusters) nclusters = ntiles;
+  if (nclusters < 1) nclusters = 1;
+  cfg.gridDim = dim3((unsigned)(nclusters * kMmaCtas), 1, 1);
+  *err = cudaLaunchKernelEx(&cfg, router_mma_kernel, xmap, a, ntiles, nclusters);
+  return true;
 }
 
 constexpr int64_t kFewTokens = 512;
@@ -565,8 +732,11 @@ cudaError_t launch_router(const RouterArgs& a, int num_sms, cudaStream_t s, bool
   }
   // Many tokens: tensor cores (fewer instructions per token); few tokens: the
   // register kernel, whose set-up (W_g into registers) is shorter.
-  if (a.T >= kMmaMinTokens && a.E <= 8 && a.d % (16 * kMmaWarps) == 0 && a.d <= 16 * kMmaWarps * kMmaMaxSteps)
-    return launch_router_mma(a, num_sms, s);
+  if (a.T >= kMmaMinTokens && a.E <= 8 && a.d % (16 * kMmaWarps * kMmaCtas) == 0 &&
+      a.d <= 16 * kMmaWarps * kMmaCtas * kMmaMaxSteps && (reinterpret_cast<uintptr_t>(a.x) & 15) == 0) {
+    cudaError_t err = cudaSuccess;
+    if (launch_router_mma(a, num_sms, s, &err)) return err;
+  }
   if (a.E <= 8 && a.d <= 8 * kRegMaxThreads) {
     // tokens per SM decide how many rows one ring slot carries
     const int64_t per_sm = (a.T + num_sms - 1) / num_sms;

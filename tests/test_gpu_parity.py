@@ -185,11 +185,11 @@ def test_exact_logit_ties(o, variant):
 
 
 def test_tensor_core_router_ties(o):
-    """1100 tokens at d=256 take the tensor-core router (T >= 1024, d a
-    multiple of 256), with a ragged last tile of 4 tokens: experts 2 and 3
+    """1100 tokens at d=512 take the tensor-core router (T >= 1024, d a
+    multiple of 512), with a ragged last tile of 12 tokens: experts 2 and 3
     tie exactly for many tokens (the smaller index wins), and zero rows pick
     experts 0 and 1 with gates 1/2, as in the oracle."""
-    wl = synth.Workload("ties_mma", 1100, 256, 256, seed=9).generate()
+    wl = synth.Workload("ties_mma", 1100, 512, 256, seed=9).generate()
     wl.Wg[2] += 3.0 * np.abs(wl.Wg[2]).max()
     wl.Wg[3] = wl.Wg[2]
     wl.x[:10] = 0
@@ -257,6 +257,15 @@ def test_skew_T8192_capacity(o, policy):
     share = float((H.run_layer(device_inputs(wl), 0)["counts"][0])) / (wl.T * wl.k)
     assert 0.37 < share < 0.43, share
     wl.drop_policy = 0
+
+
+@pytest.mark.parametrize("E,d,T", [(5, 1024, 2051), (8, 2048, 1024), (2, 4096, 1031)])
+def test_tensor_core_router_shapes(o, E, d, T):
+    """The tensor-core router with fewer than 8 experts (unused MMA columns),
+    a quarter of d per CTA of 1 to 8 MMA steps per warp, and tiles that the
+    clusters share unevenly, the last one ragged; every row is compared."""
+    wl = synth.Workload(f"mma_router{E}_{d}", T, d, 128, E=E, k=2, seed=E + d).generate()
+    check_everything(o, wl, 1)
 
 
 @pytest.mark.parametrize("T", [1, 8, 64, 512, 32768])
