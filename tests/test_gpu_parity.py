@@ -259,12 +259,14 @@ def test_skew_T8192_capacity(o, policy):
     wl.drop_policy = 0
 
 
-@pytest.mark.parametrize("E,d,T", [(5, 1024, 2051), (8, 2048, 1024), (2, 4096, 1031)])
-def test_tensor_core_router_shapes(o, E, d, T):
-    """The tensor-core router with fewer than 8 experts (unused MMA columns),
-    a quarter of d per CTA of 1 to 8 MMA steps per warp, and tiles that the
-    clusters share unevenly, the last one ragged; every row is compared."""
-    wl = synth.Workload(f"mma_router{E}_{d}", T, d, 128, E=E, k=2, seed=E + d).generate()
+@pytest.mark.parametrize("E,d,T,k", [(5, 1024, 2051, 2), (8, 2048, 1024, 2), (2, 4096, 1031, 2), (1, 512, 1030, 1),
+                                     (8, 1024, 1100, 3)])
+def test_tensor_core_router_shapes(o, E, d, T, k):
+    """The tensor-core router with fewer than 8 experts (unused MMA columns,
+    down to a single expert), top-1 and top-3, a quarter of d per CTA of 1
+    to 8 MMA steps per warp, and tiles that the clusters share unevenly, the
+    last one ragged; every row is compared."""
+    wl = synth.Workload(f"mma_router{E}_{d}_{k}", T, d, 128, E=E, k=k, seed=E + d + k).generate()
     check_everything(o, wl, 1)
 
 
