@@ -366,7 +366,9 @@ class Run:
         """Tokens/s through the host-buffer entry point (moe_layer_forward_host
         here) with page-locked host x and y, one call after another on one
         stream: every step copies its x in, runs the layer and copies its y out
-        before the next step starts."""
+        before the next step starts (from 4096 dropless tokens the call itself
+        overlaps its groups' copies with the other groups' kernels, on the
+        library's copy streams; its work ends on this stream)."""
         torch, moe = self.torch, self.moe
         wl, L = self.wl, self.layer
         s_ = torch.cuda.Stream()
@@ -737,7 +739,7 @@ def run_ours(args):
                                       f"({'sustained' if long_run else 'burst'})"),
             e2e=dict(value=weak_scaling_value(world, wl.T, p["e2e_ms"]), unit="tokens/s", h2d_bytes_per_step=p["h2d"],
                      d2h_bytes_per_step=p["d2h"], entry_point=p["entry"],
-                     note="one stream; each step copies x in and y out around the layer"),
+                     note="one call after another on one stream; each call copies x in and y out around the layer (in token groups whose copies overlap the other groups' kernels from 4096 dropless tokens)"),
             e2e_pipelined=dict(value=weak_scaling_value(world, wl.T, p["e2e_pipe_ms"]), unit="tokens/s",
                                note="two streams, consecutive steps overlap"),
             gpu_launches=kernels_per_step * args.steps,

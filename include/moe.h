@@ -252,9 +252,18 @@ MOE_API moe_status moe_layer_forward_profiled(const moe_shape *shape, const moe_
 
 /* The whole layer with the activations in HOST memory: copies x_host
  * [T, d] to the device (inside the workspace), runs moe_layer_forward and
- * copies y back to y_host [T, d], all queued on `stream`.  Weights are
- * device pointers.  Use page-locked host buffers for asynchronous copies;
- * y_host is valid once the stream has been synchronised. */
+ * copies y back to y_host [T, d].  Weights are device pointers.  Use
+ * page-locked host buffers for asynchronous copies; y_host is valid once
+ * `stream` has been synchronised.
+ * Dropless calls (capacity_factor <= 0) with T >= 4096 on the CTA-pair
+ * schedule run the layer on 2 to 8 consecutive groups of at least 2048
+ * tokens.  Each group's copies run on two copy streams that the library
+ * creates once per device (kept for the process; invalid after a device
+ * reset) and overlap the other groups' kernels.  y is the same, bit for
+ * bit: in dropless mode no token's result depends on the others.  All of
+ * the call's work is ordered before later work on `stream`, and it waits
+ * for earlier work on `stream`.  Otherwise everything is queued on
+ * `stream`. */
 MOE_API moe_status moe_layer_forward_host(const moe_shape *shape, const moe_bf16 *x_host,
                                   const float *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
                                   const moe_bf16 *W2, moe_bf16 *y_host, void *ws,

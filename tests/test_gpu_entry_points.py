@@ -1,8 +1,10 @@
 """The whole-layer entry points other than moe_layer_forward, on the GPU.
 
 * moe_layer_forward_host takes x and y in host memory and queues the two
-  copies and the layer on one stream: the call of a caller whose activations
-  live on the host, and the one the end-to-end figure of the benchmark times.
+  copies and the layer: the call of a caller whose activations live on the
+  host, and the one the end-to-end figure of the benchmark times.  From 4096
+  dropless tokens on it runs the layer on groups of tokens whose copies
+  overlap the other groups' kernels (the "chunked" case).
 * moe_layer_forward_profiled and moe_layer_forward_q4_profiled record six
   CUDA events between the kernels: the benchmark's per-kernel timings.
 
@@ -31,6 +33,7 @@ CASES = {
     "ragged": dict(T=300, d=256, f=512, seed=3),                                   # CTA pairs, ragged tiles
     "cap_by_prob": dict(T=256, d=128, f=256, capacity_factor=1.0, skew=True),      # capacity select kernel
     "next_best": dict(T=256, d=128, f=256, capacity_factor=1.0, drop_policy=2, skew=True),  # fallback kernels
+    "chunked": dict(T=6000, d=128, f=256, seed=4),  # host buffers in 2 groups of 3000 tokens, copies overlapped
 }
 
 
