@@ -258,8 +258,9 @@ MOE_API moe_status moe_layer_forward_profiled(const moe_shape *shape, const moe_
  * Dropless calls (capacity_factor <= 0) with T >= 4096 on the CTA-pair
  * schedule run the layer on 2 to 8 consecutive groups of at least 2048
  * tokens.  Each group's copies run on two copy streams that the library
- * creates once per device (kept for the process; invalid after a device
- * reset) and overlap the other groups' kernels.  y is the same, bit for
+ * creates once per device and calling stream (up to 8 calling streams per
+ * device; further ones share; kept for the process and invalid after a
+ * device reset) and overlap the other groups' kernels.  y is the same, bit for
  * bit: in dropless mode no token's result depends on the others.  All of
  * the call's work is ordered before later work on `stream`, and it waits
  * for earlier work on `stream`.  Otherwise everything is queued on

@@ -628,20 +628,41 @@ static int64_t host_chunks(const moe_shape* sh) {
 }
 
 // The two copy streams (host to device, device to host) of chunked
-// host-buffer calls on a device, created on first use and kept for the
-// process (invalid after the device is reset).
-static moe_status copy_streams(cudaStream_t* in, cudaStream_t* out) {
-  static cudaStream_t streams[kMaxDevices][2];
+// host-buffer calls made on `user` (a stream of the current device): one
+// pair per user stream, so that calls on different streams do not queue
+// behind each other's copies; created on first use and kept for the
+// process (invalid after the device is reset).  Past kCopyPairs user
+// streams on a device, the pairs are shared (still correct, less overlap).
+constexpr int kCopyPairs = 8;
+static moe_status copy_streams(cudaStream_t user, cudaStream_t* in, cudaStream_t* out) {
+  struct Pair {
+    cudaStream_t user, in, out;
+    bool used;
+  };
+  static Pair pairs[kMaxDevices][kCopyPairs];
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < 2; ++i)
-    if (!streams[dev][i] && cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  *in = streams[dev][0];
-  *out = streams[dev][1];
+  Pair* row = pairs[dev];
+  int slot = -1;
+  for (int i = 0; i < kCopyPairs && slot < 0; ++i)
+    if (row[i].used && row[i].user == user) slot = i;
+  for (int i = 0; i < kCopyPairs && slot < 0; ++i)
+    if (!row[i].used) {
+      if (cudaStreamCreateWithFlags(&row[i].in, cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaStreamCreateWithFlags(&row[i].out, cudaStreamNonBlocking) != cudaSuccess) {
+        cudaStreamDestroy(row[i].in);
+        return MOE_ERR_CUDA;
+      }
+      row[i].user = user;
+      row[i].used = true;
+      slot = i;
+    }
+  if (slot < 0) slot = (int)((reinterpret_cast<uintptr_t>(user) >> 4) % kCopyPairs);
+  *in = row[slot].in;
+  *out = row[slot].out;
   return MOE_OK;
 }
 
@@ -652,7 +673,7 @@ static moe_status layer_forward_host_chunked(const moe_shape* sh, int64_t C, con
                                              const ExpertWeights& Wt, moe_bf16* y_host, moe_bf16* xd, moe_bf16* yd,
                                              void* ws, int sms, cudaStream_t s) {
   cudaStream_t cin = nullptr, cout = nullptr;
-  MOE_TRY(copy_streams(&cin, &cout));
+  MOE_TRY(copy_streams(s, &cin, &cout));
   constexpr int kMaxEvents = 2 * 8 + 2;
   cudaEvent_t ev[kMaxEvents] = {};
   const int nev = (int)(2 * C + 2);
