@@ -102,7 +102,7 @@ typedef enum {
 
 /* Expert-GEMM schedule.  Both compute the same function. */
 typedef enum {
-  MOE_VARIANT_AUTO = 0,         /* STREAM when T <= 128, TILED otherwise */
+  MOE_VARIANT_AUTO = 0,         /* STREAM when T <= 128, TILED_SINGLE while T*k/E <= 112, TILED above */
   MOE_VARIANT_TILED = 1,        /* 256-token x 256-column tiles on CTA pairs
                                    (one MMA over two SMs): compute-bound sizes */
   MOE_VARIANT_STREAM = 2,       /* weights as the 128-row MMA operand, tokens as N,

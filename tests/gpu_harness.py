@@ -257,12 +257,15 @@ def sample_tokens(wl: synth.Workload, r: dict, n: int, seed: int = 1, block_rows
     return np.array(sorted(pick), np.int64)
 
 
-def schedule_block_rows(T: int, variant: int) -> int:
-    """Token rows per tile of the expert GEMMs: the streaming schedule's
-    token tile (T <= 128 under AUTO), 256 for CTA pairs, 128 for single-CTA
-    tiles."""
-    if variant == 2 or (variant == 0 and T <= 128):
-        b = max(16, ((T + 15) // 16) * 16)
+def schedule_block_rows(T: int, variant: int, k: int = 2, E: int = 8) -> int:
+    """Token rows per tile of the expert GEMMs, as the library chooses them:
+    the streaming schedule's token tile (twice the mean slots per expert,
+    rounded up to 16; AUTO takes it for T <= 128), 128 for single-CTA tiles
+    (AUTO while T k / E <= 112), 256 for CTA pairs."""
+    if variant == 0:
+        variant = 2 if T <= 128 else 3 if T * k <= 112 * E else 1
+    if variant == 2:
+        b = max(16, ((2 * ((T * k + E - 1) // E) + 15) // 16) * 16)
         return 16 if b <= 16 else 32 if b <= 32 else 64 if b <= 64 else 128
     return 128 if variant == 3 else 256
 

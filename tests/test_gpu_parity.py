@@ -83,7 +83,7 @@ def check_everything(o, wl, variant, rows=None, stages=True):
     assert np.array_equal(lay["idx"].reshape(wl.T, wl.k), r["idx"]), "layer topk_idx"
     assert np.array_equal(lay["counts"], r["counts"]), "layer counts"
     toks = np.arange(wl.T) if rows is None else \
-        H.sample_tokens(wl, r, rows, block_rows=H.schedule_block_rows(wl.T, variant))
+        H.sample_tokens(wl, r, rows, block_rows=H.schedule_block_rows(wl.T, variant, wl.k, wl.E))
     ref = o.layer_rows(wl.x, wl.W1, wl.W3, wl.W2, r, toks, want_h=stages, want_o=stages)
     y_gpu = H.bf16_f64(lay["y"])[toks]
     H.assert_close(y_gpu, ref["y"], f"y (layer, {VNAME[variant]})")
