@@ -83,11 +83,12 @@ def test_streaming_layout_adds_splitk_planes(moe, T, d, f):
     assert _splits(extra, T * 2, d) is not None, extra
 
 
-@pytest.mark.parametrize("T", [16, 32, 33, 64, 65, 300])
+@pytest.mark.parametrize("T", [16, 32, 33, 64, 65, 79, 80, 300])
 def test_q4_layout_always_has_splitk_planes(moe, T):
     """The 4-bit layout adds split-K planes and, for token tiles of 16 and 32
-    (twice the mean slots per expert, up to T = 64 for 8 experts and top-2:
-    the integer-MMA kernels), the quantised activations as their tiled token
+    (the integer-MMA kernels; the tile is 16 while the mean slots per expert
+    fit it, else twice the mean: 16 up to T = 64 for 8 experts and top-2,
+    64 from T = 65), the quantised activations as their tiled token
     operand and their scales [S] fp32 at the end.  The operand
     holds, per token tile (at most S / bn + E of them) and stage of ks inputs
     (256 for 16-token tiles, 128 for 32), the high and low bytes of the
@@ -95,7 +96,8 @@ def test_q4_layout_always_has_splitk_planes(moe, T):
     sh = moe.make_shape(T, 4096, 14336)
     extra = moe.moe_workspace_size_q4(sh) - expected(T, 4096, 14336, 8, 2)
     S = T * 2
-    bn = -(-2 * -(-S // 8) // 16) * 16    # token tile: twice the mean slots per expert, rounded up to 16
+    mean = -(-S // 8)
+    bn = 16 if mean <= 16 else -(-2 * mean // 16) * 16    # token tile, rounded up to 16
     if bn <= 32:
         ks = 256 if bn == 16 else 128
         tiles = -(-S // bn) + 8
