@@ -185,7 +185,7 @@ def test_exact_logit_ties(o, variant):
 
 
 def test_tensor_core_router_ties(o):
-    """1100 tokens at d=512 take the tensor-core router (T >= 1024, d a
+    """1100 tokens at d=512 take the tensor-core router (T >= 192, d a
     multiple of 512), with a ragged last tile of 12 tokens: experts 2 and 3
     tie exactly for many tokens (the smaller index wins), and zero rows pick
     experts 0 and 1 with gates 1/2, as in the oracle."""
@@ -260,12 +260,13 @@ def test_skew_T8192_capacity(o, policy):
 
 
 @pytest.mark.parametrize("E,d,T,k", [(5, 1024, 2051, 2), (8, 2048, 1024, 2), (2, 4096, 1031, 2), (1, 512, 1030, 1),
-                                     (8, 1024, 1100, 3)])
+                                     (8, 1024, 1100, 3), (8, 512, 192, 2), (6, 1024, 777, 2)])
 def test_tensor_core_router_shapes(o, E, d, T, k):
-    """The tensor-core router with fewer than 8 experts (unused MMA columns,
-    down to a single expert), top-1 and top-3, a quarter of d per CTA of 1
-    to 8 MMA steps per warp, and tiles that the clusters share unevenly, the
-    last one ragged; every row is compared."""
+    """The tensor-core router (from 192 tokens) with fewer than 8 experts
+    (unused MMA columns, down to a single expert), top-1 and top-3, a
+    quarter of d per CTA of 1 to 8 MMA steps per warp, and tiles that the
+    clusters share unevenly (or one tile per cluster), the last one ragged;
+    every row is compared."""
     wl = synth.Workload(f"mma_router{E}_{d}_{k}", T, d, 128, E=E, k=k, seed=E + d + k).generate()
     check_everything(o, wl, 1)
 
