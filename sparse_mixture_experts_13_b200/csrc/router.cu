@@ -6,8 +6,11 @@
 // logits, softmax over the k kept logits).
 //
 // Logits are fp32 dot products of a token's bf16 row with the E rows of W_g.
-// Two kernels compute them:
+// Three kernels compute them:
 //
+// router_mma_kernel (from 192 tokens, E <= 8, d a multiple of 512 up to
+//   4096): tensor-core MMAs on W_g split exactly into three bf16 terms, in
+//   clusters of 4 CTAs that split d (described at the kernel below).
 // router_reg_kernel (E <= 8, d <= 4096, the Mixtral shape): a persistent
 //   block of d/8 threads holds all of W_g in registers, thread i owning inputs
 //   [8i, 8i+8) of every expert row, so W_g is read once per block instead of
@@ -21,9 +24,10 @@
 //   splits d over its warps; every W_g vector a warp reads (from L2) serves
 //   all tokens of the group.
 //
-// In both, the top-k (ties to the smaller expert index), the k-way softmax
-// and the full-softmax probability of each chosen expert are computed
-// redundantly per lane of one warp and lanes 0..k-1 write one slot each.  The
+// In all three, the top-k (ties to the smaller expert index), the k-way
+// softmax and the full-softmax probability of each chosen expert are
+// computed redundantly per lane of one warp (or of an 8-lane segment) and
+// lanes 0..k-1 write one slot each.  The
 // per-expert histogram is aggregated in shared memory and added to global
 // memory once per block.
 #include <cfloat>
