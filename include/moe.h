@@ -30,14 +30,16 @@
  *   - All pointers are DEVICE pointers unless the name ends in _host.  The
  *     caller allocates every buffer, including the workspace; the library
  *     allocates no memory and keeps no state between calls apart from cached
- *     device attributes and driver entry points.
+ *     device attributes, driver entry points and the copy streams of
+ *     moe_layer_forward_host's chunked calls.
  *   - Calls are asynchronous on `stream`; none synchronises except
  *     moe_read_device_status.  A workspace may serve one call in flight at a
  *     time.
  *   - Host threads: the first call on each device fills a small per-device
  *     cache (compute capability and SM count; for moe_permute_noalloc also
- *     its scratch address).  Make one call on each device from a single
- *     thread before calling from several threads at once; afterwards calls
+ *     its scratch address; moe_layer_forward_host's copy streams are created
+ *     under a lock).  Make one call on each device from a single thread
+ *     before calling from several threads at once; afterwards calls
  *     from different threads are independent if their buffers, workspaces
  *     and streams are (not moe_permute_noalloc: all its calls share one
  *     scratch array).
