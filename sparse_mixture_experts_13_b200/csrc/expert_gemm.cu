@@ -965,17 +965,18 @@ void stream_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int nu
     }
   }
   *splits = best;
-  // Split K of the gate/up projection only where it shortens the last,
-  // partly filled wave of (experts x 64-row blocks) tiles enough (by 3 %)
-  // to pay for its fp32 partials and the extra reduction launch (counted
-  // as 8 chunk-waves).
+  // Split K of the gate/up projection (2 ways) only where it shortens the
+  // last, partly filled wave of (experts x 64-row blocks) tiles enough (by
+  // 3 %) to pay for its fp32 partials and the extra reduction launch
+  // (counted as 8 chunk-waves).  4 ways was measured 1 % slower than 2 at
+  // one and two Mixtral tokens, where the model preferred it.
   const int32_t num_kb1 = d / BK;
   const int64_t base1 = touched * (f / 64);
   const int64_t plane = (T * k * 2 * (int64_t)f * 8 + 16384LL * num_sms - 1) / (16384LL * num_sms);
   const int64_t cost1 = ((base1 + num_sms - 1) / num_sms) * (num_kb1 + 1);
   int32_t best1 = 1;
   int64_t best1_cost = cost1;
-  for (int32_t sp = 2; sp <= 8 && sp <= num_kb1; sp *= 2) {
+  for (int32_t sp = 2; sp <= 2 && sp <= num_kb1; sp *= 2) {
     const int32_t kbps = (num_kb1 + sp - 1) / sp;
     const int32_t real = (num_kb1 + kbps - 1) / kbps;
     const int64_t waves = (base1 * real + num_sms - 1) / num_sms;

@@ -277,7 +277,7 @@ def test_sweep(o, T):
 
 
 def test_gate_up_split_along_k(o):
-    """Two Mixtral tokens: the streaming gate/up GEMM is split 4 ways along K
+    """Two Mixtral tokens: the streaming gate/up GEMM is split 2 ways along K
     (fp32 partials, then their sum through SiLU * mul); T = 1 in the sweep
     takes the same path."""
     check_everything(o, full_workload("sweep", T=2), 0, rows=16)

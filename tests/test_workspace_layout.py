@@ -74,12 +74,12 @@ def _splits(extra, S, d):
 def test_streaming_layout_adds_splitk_planes(moe, T, d, f):
     """The streaming schedule adds the down projection's split-K planes
     [splits, S, d] fp32; at one or two Mixtral tokens (2 or 4 experts' tiles
-    fill the last wave of 148 SMs poorly) the gate/up projection is split 4
-    ways along K too, adding [4, S, 2 f] fp32 partials."""
+    fill the last wave of 148 SMs poorly) the gate/up projection is split 2
+    ways along K too, adding [2, S, 2 f] fp32 partials."""
     sh = moe.make_shape(T, d, f)                 # AUTO: streaming schedule for T <= 128
     extra = moe.moe_workspace_size(sh) - expected(T, d, f, 8, 2)
     if T <= 2 and f == 14336:
-        extra -= al(4 * 4 * T * 2 * 2 * f)
+        extra -= al(4 * 2 * T * 2 * 2 * f)
     assert _splits(extra, T * 2, d) is not None, extra
 
 
