@@ -415,9 +415,9 @@ MOE_API moe_status moe_ep_combine_cap(const moe_shape *shape, int32_t world, con
  *   w = (code - 8) * scale, code in 0 .. 15.
  * The expert matrices are W1, W3 [E, d_ff, d_model] and W2 [E, d_model, d_ff]
  * as in the bf16 entry points; the router stays fp32.  Arithmetic on the
- * GPU: at token tiles of 16 and 32 (the tile is 16 while the mean slots per
- * expert, T k / E, fit it, else twice the mean rounded up to 16: T <= 64
- * for 8 experts and top-2), the weights stay
+ * GPU: at token tiles of 16 and 32 (16 while the mean slots per expert,
+ * T k / E, fit it, 32 up to a mean of 22, else twice the mean rounded up
+ * to 16: T <= 88 for 8 experts and top-2), the weights stay
  * exact integers (code - 8) and each token slot's
  * activations are rounded to 16-bit integers with one fp32 scale per slot
  * (error at most half a step, 1.5e-5 of the slot's largest value); the

@@ -634,15 +634,16 @@ cudaError_t launch_q4(const ExpertGemmQ4Args& a, cudaStream_t s) {
 }  // namespace
 
 void q4_params(int64_t T, int32_t k, int32_t d, int32_t f, int32_t E, int num_sms, int32_t* bn, int32_t* splits) {
-  // token tile: 16 while the mean slots per expert fit it, else twice the
-  // mean, so that an expert's slots usually fit one tile (a second tile
-  // streams the expert's weights again).  The integer-MMA kernel costs far
-  // less per weight byte at 16 tokens than at 32, enough that re-reading the
-  // weights of experts that spill into a second 16-token tile still wins:
-  // 0.371 -> 0.227 ms at T = 40, 0.371 -> 0.320 ms at T = 64 (8 experts,
-  // top-2); from about 96 tokens the wide tiles win again.
+  // token tile: 16 while the mean slots per expert fit it, 32 up to a mean
+  // of 22, else twice the mean, so that an expert's slots usually fit one
+  // tile (a second tile streams the expert's weights again).  The
+  // integer-MMA kernel costs far less per weight byte at 16 tokens than at
+  // 32, enough that re-reading the weights of experts that spill into a
+  // second 16-token tile still wins: 0.371 -> 0.227 ms at T = 40, 0.371 ->
+  // 0.320 ms at T = 64 (8 experts, top-2); 32-token integer-MMA tiles beat
+  // 64-token dequantising ones by 2-3 % from T = 65 to 88 and lose at 96.
   const int64_t mean = (T * k + E - 1) / E;
-  int64_t b = mean <= 16 ? 16 : ((2 * mean + 15) / 16) * 16;
+  int64_t b = mean <= 16 ? 16 : mean <= 22 ? 32 : ((2 * mean + 15) / 16) * 16;
   if (b < 16) b = 16;
   if (b > 64) b = 128;
   else if (b > 32) b = 64;

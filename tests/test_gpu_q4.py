@@ -164,11 +164,11 @@ def full_q4(o, T):
     return wl, _FULL["q"]
 
 
-@pytest.mark.parametrize("T", [16, 1, 32, 64, 512])
+@pytest.mark.parametrize("T", [16, 1, 32, 64, 72, 512])
 def test_q4_mixtral_sizes(o, T):
-    """Integer-MMA kernels at T = 1 and 16 (16-token tiles, 256-input stages)
-    and 32 (32-token tiles, 128-input stages); the dequantising kernels at
-    64 and 512."""
+    """Integer-MMA kernels at T = 1, 16, 32 and 64 (16-token tiles,
+    256-input stages; at 64 some experts spill into a second tile) and 72
+    (32-token tiles, 128-input stages); the dequantising kernels at 512."""
     wl, q = full_q4(o, T)
     check_q4(o, wl, rows=16, q=q)
 

@@ -83,12 +83,13 @@ def test_streaming_layout_adds_splitk_planes(moe, T, d, f):
     assert _splits(extra, T * 2, d) is not None, extra
 
 
-@pytest.mark.parametrize("T", [16, 32, 33, 64, 65, 79, 80, 300])
+@pytest.mark.parametrize("T", [16, 32, 33, 64, 65, 88, 89, 300])
 def test_q4_layout_always_has_splitk_planes(moe, T):
     """The 4-bit layout adds split-K planes and, for token tiles of 16 and 32
     (the integer-MMA kernels; the tile is 16 while the mean slots per expert
-    fit it, else twice the mean: 16 up to T = 64 for 8 experts and top-2,
-    64 from T = 65), the quantised activations as their tiled token
+    fit it, 32 up to a mean of 22, else twice the mean: for 8 experts and
+    top-2, 16 up to T = 64, 32 up to 88, then 64), the quantised activations
+    as their tiled token
     operand and their scales [S] fp32 at the end.  The operand
     holds, per token tile (at most S / bn + E of them) and stage of ks inputs
     (256 for 16-token tiles, 128 for 32), the high and low bytes of the
@@ -97,7 +98,7 @@ def test_q4_layout_always_has_splitk_planes(moe, T):
     extra = moe.moe_workspace_size_q4(sh) - expected(T, 4096, 14336, 8, 2)
     S = T * 2
     mean = -(-S // 8)
-    bn = 16 if mean <= 16 else -(-2 * mean // 16) * 16    # token tile, rounded up to 16
+    bn = 16 if mean <= 16 else 32 if mean <= 22 else -(-2 * mean // 16) * 16    # token tile
     if bn <= 32:
         ks = 256 if bn == 16 else 128
         tiles = -(-S // bn) + 8
