@@ -23,7 +23,10 @@
 //   2 = inclusive prefix) until it meets an inclusive prefix.  The row of a
 //   kept slot is offsets[e] + (eligible slots of e before it).  All of the
 //   block's warps then copy the kept tokens' rows of x into x_perm with
-//   16-byte vector loads and stores.
+//   16-byte vector loads and stores -- except when launch_permute runs the
+//   row copy as gather_rows_kernel (a warp per row over every SM), which it
+//   does for the look-back path: same rows, 3-13 us per step less at T =
+//   4096-8192.
 #include <cstdint>
 
 #include "moe_internal.h"
@@ -275,6 +278,45 @@ __global__ void __launch_bounds__(256) permute_small_kernel(PermuteArgs a) {
   }
 }
 
+// Row copy of the grouping with many slots: x_perm[r] = x[perm_slot[r] / k]
+// for the grouped rows r < offsets[E], apart from the ranking so that every
+// SM copies (the ranking kernel has one block per 64 slots).  A warp copies
+// a row with up to 8 KB of loads in flight (16-byte vectors).
+constexpr int kGatherThreads = 256;
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint16_t* __restrict__ x,
+                                                                     const int32_t* __restrict__ perm_slot,
+                                                                     const int32_t* __restrict__ offsets, int32_t E,
+                                                                     int32_t k, int32_t d, int64_t T, int64_t S,
+                                                                     uint16_t* __restrict__ x_perm, uint32_t* status) {
+  pdl_wait();     // the grouping's rows
+  pdl_trigger();  // the expert GEMM may start its weight prefetch
+  int64_t rows = offsets[E];
+  if (!MOE_DCHECK(status, rows >= 0 && rows <= S)) rows = 0;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int nvec = d >> 3;
+  for (int64_t r = warp; r < rows; r += nwarps) {
+    const int64_t tok = perm_slot[r] / k;
+    if (!MOE_DCHECK(status, tok >= 0 && tok < T)) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(x + tok * d);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + r * d);
+    for (int v0 = 0; v0 < nvec; v0 += 512) {
+      uint4 q[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int v = v0 + lane + 32 * u;
+        if (v < nvec) q[u] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int v = v0 + lane + 32 * u;
+        if (v < nvec) dst[v] = q[u];
+      }
+    }
+  }
+}
+
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zeroed) {
   const int64_t S = a.T * a.k;
   const int64_t tiles = permute_tiles(S);
@@ -296,7 +338,16 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool state_zero
     const int blocks = (int)(S < kSmallBlocks ? S : kSmallBlocks);
     return launch_k(permute_small_kernel, dim3(blocks), dim3(256), 0, s, a.pdl, a);
   }
-  return launch_k(permute_kernel, dim3((unsigned)tiles), dim3(kPermuteThreads), 0, s, a.pdl, a);
+  // ranking and rows; the row copy follows as its own kernel
+  PermuteArgs rank_only = a;
+  rank_only.x_perm = nullptr;
+  err = launch_k(permute_kernel, dim3((unsigned)tiles), dim3(kPermuteThreads), 0, s, a.pdl, rank_only);
+  if (err != cudaSuccess || !a.x_perm) return err;
+  // a warp per row, up to 1024 blocks (grid-stride beyond)
+  int64_t blocks = (S + (kGatherThreads / 32) - 1) / (kGatherThreads / 32);
+  if (blocks > 1024) blocks = 1024;
+  return launch_k(gather_rows_kernel, dim3((unsigned)blocks), dim3(kGatherThreads), 0, s, a.pdl, a.x, a.perm_slot,
+                  a.offsets, a.E, a.k, a.d, a.T, S, a.x_perm, a.status);
 }
 
 // ---------------------------------------------------------------------------
