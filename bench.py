@@ -719,7 +719,11 @@ def run_ours(args):
         dec_q4 = stage_report(out["decode_q4"]["wl"], out["decode_q4"], world, peaks,
                               "4-bit gate/up-projection GEMM (integer MMA, SwiGLU fused)", "expert_gemm_q4i8_kernel<0,16>",
                               "decode_q4", q4=True)
-        kernels_per_step = 5 + (1 if (wl.capacity_factor > 0 and wl.drop_policy == 0) else 0)
+        # router, grouping, gate/up GEMM, down GEMM, combine; the grouping's
+        # row copy runs as its own kernel above 1024 slots; capacity by
+        # probability adds its select kernel
+        kernels_per_step = (5 + (1 if wl.T * wl.k > 1024 else 0) +
+                            (1 if (wl.capacity_factor > 0 and wl.drop_policy == 0) else 0))
         line = dict(
             metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
             ms_per_step=p["ms"], ms_per_step_median_l2_flushed=p["ms_flushed"], higher_is_better=True,
