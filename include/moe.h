@@ -266,7 +266,8 @@ MOE_API moe_status moe_layer_forward_profiled(const moe_shape *shape, const moe_
  * bit: in dropless mode no token's result depends on the others.  All of
  * the call's work is ordered before later work on `stream`, and it waits
  * for earlier work on `stream`.  Otherwise everything is queued on
- * `stream`. */
+ * `stream`.  To capture such a call in a CUDA graph, make one call on the
+ * same stream outside the capture first (it creates the copy streams). */
 MOE_API moe_status moe_layer_forward_host(const moe_shape *shape, const moe_bf16 *x_host,
                                   const float *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
                                   const moe_bf16 *W2, moe_bf16 *y_host, void *ws,
