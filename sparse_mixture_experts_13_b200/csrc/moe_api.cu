@@ -710,9 +710,13 @@ static moe_status layer_forward_host_chunked(const moe_shape* sh, int64_t C, con
     if (st == MOE_OK)
       st = cuda_status(cudaMemcpyAsync(y_host + r0 * d, yd + r0 * d, 2 * (size_t)n * d, cudaMemcpyDeviceToHost, cout));
   }
-  // the call's last copy is ordered before whatever follows on s
-  if (st == MOE_OK) st = cuda_status(cudaEventRecord(ev[nev - 1], cout));
-  if (st == MOE_OK) st = cuda_status(cudaStreamWaitEvent(s, ev[nev - 1], 0));
+  // the call's last copy is ordered before whatever follows on s, also when
+  // a step above failed (copies already queued still finish before it)
+  if (ev[nev - 1]) {
+    const moe_status j = cuda_status(cudaEventRecord(ev[nev - 1], cout));
+    const moe_status w = j == MOE_OK ? cuda_status(cudaStreamWaitEvent(s, ev[nev - 1], 0)) : j;
+    if (st == MOE_OK) st = w;
+  }
   for (int i = 0; i < nev; ++i)
     if (ev[i]) cudaEventDestroy(ev[i]);
   return st;
